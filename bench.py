@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed-KV hot path on B200.
+
+One step = the whole path for one decode token of every sequence of the 32K GQA
+workload (batch 8, 32 query heads over 8 KV heads, d=128, context 32768, bf16,
+16-token ring, 3-bit keys b1=2 + m=128, 2-bit values g=32):
+    tq_append (1 new token per sequence: the oldest ring token is quantised
+               into the packed cache, the new one enters the ring)
+    tq_decode_prep -> tq_decode_partial (split-K) -> tq_decode_combine.
+Inputs are resident in HBM before timing; L2 is flushed (256 MB write) between
+steps, outside the timed events.  `value` is algorithmic bytes (packed cache +
+ring + append traffic) per second.  Also reported: the dominant kernel's
+roofline, end-to-end (host buffers, copies inside the timed region), the key
+quantise throughput of the 131072-token x 8-head append workload, the CPU
+oracle baseline, clocks, and the number of library kernel launches.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed decode-attn HBM GB/s (% of 8 TB/s) and tokens/s; key-quantize Mkeys/s"
+NOMINAL_HBM = 8000.0      # GB/s, the metric's reference figure
+FALLBACK_HBM = 6650.0     # GB/s, used only when MEASURED_PEAKS.json is absent
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quantize", action="store_true")
+    ap.add_argument("--workload", default="gqa32k")
+    return ap.parse_args()
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "compressed_attention_turboquantprod_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file: str, src_hash: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", kernel_file)
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("source_hash") == src_hash:
+            return d.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.t0 = time.time()
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names[1:], parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_decode_sample(w, K1, V1, Q_steps, Kn, Vn, budget_s=12.0, min_reps=2, max_reps=None):
+    """Time the oracle on one (batch, KV head) unit at full context: untimed prefill
+    quantisation, then timed steps of append-one-token + decode of its G query heads.
+    Returns (seconds per step, algorithmic bytes per step, reps, threads)."""
+    import numpy as np
+    from oracle import cache as ocache
+    from oracle import codebook as ocb
+    from oracle import projections as oproj
+    po = oproj.make_projections(w.d, w.m, 0, with_rotation=w.b1 > 0)
+    cb = ocb.build(w.d, w.b1) if w.b1 else None
+    cap = w.T + 4096
+    oc = ocache.OracleCache(1, 1, w.d, w.b1, w.m, w.vbits, w.group, w.W, cap, w.dtype, po, cb)
+    oc.append(K1[None, None], V1[None, None])
+    G = w.Hq // w.Hkv
+    times, nbytes = [], []
+    i = 0
+    t_start = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oc.append(Kn[i % Kn.shape[0]][None, None, None], Vn[i % Vn.shape[0]][None, None, None])
+        oc.decode(Q_steps[i % Q_steps.shape[0]][None, :G])
+        times.append(time.perf_counter() - t0)
+        nbytes.append(oc.n_comp * oc.lay.token_bytes + 2 * oc.n_ring * w.d * (4 if w.dtype == "f32" else 2))
+        i += 1
+        el = time.perf_counter() - t_start
+        if (i >= min_reps and el >= budget_s) or (max_reps and i >= max_reps):
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    return statistics.mean(times), statistics.mean(nbytes), i, threads
+
+
+def _host_unit(w, device):
+    """K, V of unit (b=0, h=0) at full context and per-step inputs, as float64 numpy."""
+    import numpy as np
+    import synth
+    import torch
+    K, V = synth.keys_values(w.scaled(B=1, Hkv=1), device=device)
+    Q, Kn, Vn = synth.decode_stream(w.scaled(B=1, Hkv=1, Hq=w.Hq // w.Hkv), 8, device=device)
+    f = lambda t: t.to("cpu", torch.float32).numpy().astype(np.float64)
+    return f(K[0, 0]), f(V[0, 0]), f(Q[:, 0]), f(Kn[:, 0, 0, 0]), f(Vn[:, 0, 0, 0])
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    dev = "cpu"
+    units = w.B * w.Hkv
+    # Size the per-step sample so that the whole run stays within ~150 s: one
+    # (batch, KV head) unit, at full context when that fits, else at a shorter one.
+    K1, V1, Qs, Kn, Vn = _host_unit(w, dev)
+    t_full, _, _, _ = oracle_decode_sample(w, K1, V1, Qs, Kn, Vn, budget_s=0.0, min_reps=1, max_reps=1)
+    n_total = max(1, args.warmup + args.steps)
+    ctx = w.T
+    if n_total * t_full > 150.0:
+        ctx = max(1024, int(w.T * 150.0 / (n_total * t_full)) // 64 * 64)
+    ws = w.scaled(T=ctx)
+    K1, V1 = K1[:ctx], V1[:ctx]
+    if args.warmup:
+        oracle_decode_sample(ws, K1, V1, Qs, Kn, Vn, budget_s=0.0, min_reps=args.warmup,
+                             max_reps=args.warmup)
+    sec, nbytes, reps, threads = oracle_decode_sample(ws, K1, V1, Qs, Kn, Vn, budget_s=0.0,
+                                                      min_reps=max(1, args.steps),
+                                                      max_reps=max(1, args.steps))
+    gbs = nbytes / sec / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w, args),
+        "cpu_baseline": {"kind": "oracle", "value": gbs, "unit": "GB/s", "cores": threads,
+                         "sample": f"1 of {units} (batch, KV-head) units per step at context {ctx} "
+                                   f"(of {w.T}): append one token + decode its query heads, NumPy float64"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "tokens_per_s": 1.0 / sec / units,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, args):
+    return {"workload": f"{w.name}: batch {w.B}, {w.Hq} query heads over {w.Hkv} KV heads, d={w.d}, "
+                        f"context {w.T} ({w.W}-token {w.dtype} ring), keys b1={w.b1} + QJL m={w.m}, "
+                        f"values {w.vbits}-bit group {w.group}",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.T, "ring": w.W,
+            "b1": w.b1, "m": w.m, "vbits": w.vbits, "group": w.group, "input_dtype": w.dtype,
+            "l2": "flushed between timed steps (256 MB write, outside the events)",
+            "parallelism": f"independent replicas per GPU (weak scaling)" if args.gpus > 1 else "1 GPU"}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    world, rank, local = dist_setup(args)
+    import synth
+    from compressed_attention_turboquantprod_b200 import (Codebook, CompressedKVCache, Projections,
+                                                           native)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload].scaled(seed=rank)
+    G = w.Hq // w.Hkv
+    n_steps = args.warmup + args.steps
+    pj, cb = Projections(w.d, w.m, 0, rotation=w.b1 > 0, device=dev), (
+        Codebook(w.d, w.b1, device=dev) if w.b1 else None)
+    cap = w.T - w.W + 2 * n_steps + 128
+    cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, cap,
+                              dtype=w.torch_dtype, device=dev)
+    K, V = synth.keys_values(w, device=dev)
+    cache.append(K, V, pj, cb)
+    del K, V
+    Qs, Kn, Vn = synth.decode_stream(w, n_steps, device=dev)
+    ws = cache.workspace(w.Hq, args.splits)
+    out = torch.empty(w.B, w.Hq, w.d, dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(w.d)
+    cent = cb.centroids if cb else None
+    bnd = cb.boundaries if cb else None
+    es = 4 if w.dtype == "f32" else 2
+    tb = cache.state.token_bytes
+
+    def step_bytes():
+        n_comp, n_ring = cache.n_comp, cache.n_ring
+        dec = w.B * w.Hkv * (n_comp * tb + 2 * n_ring * w.d * es)
+        app = w.B * w.Hkv * (2 * w.d * es + tb + 2 * w.d * es)   # read ring token + new token, write record + ring
+        return dec, dec + app
+
+    def step(i, evs=None):
+        if evs:
+            evs[0].record(stream)
+        native.tq_append(cache.state, Kn[i], Vn[i], pj.Pi, pj.T, cent, bnd)
+        native.tq_decode_prep(cache.state, Qs[i], pj.Pi, pj.S, args.splits, ws)
+        if evs:
+            evs[1].record(stream)
+        native.tq_decode_partial(cache.state, w.Hq, scale, cent, None, args.splits, ws)
+        if evs:
+            evs[2].record(stream)
+        native.tq_decode_combine(cache.state, w.Hq, out, args.splits, ws)
+        if evs:
+            evs[3].record(stream)
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    clocks.start()
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dec_bytes, all_bytes = [], []
+    for k in range(args.steps):
+        flush.zero_()
+        step(args.warmup + k, events[k])
+        db, ab = step_bytes()          # host state: the context the decode just read
+        dec_bytes.append(db)
+        all_bytes.append(ab)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t_step = [e[0].elapsed_time(e[3]) for e in events]             # ms
+    t_part = [e[1].elapsed_time(e[2]) for e in events]
+    tot_ms = sum(t_step)
+    tot_ms_max = reduce_max(tot_ms, world)
+    bytes_all = reduce_sum(float(sum(all_bytes)), world)
+    value = bytes_all / (tot_ms_max * 1e-3) / 1e9
+    tokens_s = reduce_sum(float(w.B * args.steps), world) / (tot_ms_max * 1e-3)
+    part_avg_ms = sum(t_part) / len(t_part)
+    part_bytes = sum(dec_bytes) / len(dec_bytes)
+    peak, peak_kind = measured_peak()
+    src_hash = source_hash("decode_kernels.cu")
+    traffic = profiled_traffic("decode_partial_gqa32k.json", src_hash)
+    achieved = part_bytes / (part_avg_ms * 1e-3) / 1e9
+
+    # end to end: per step, H2D of the step's Q / new K / new V from pinned host
+    # buffers and D2H of the output inside the timed region
+    e2e = None
+    if args.steps > 0:
+        n_e2e = min(args.steps, 100)
+        Qh = Qs[:n_e2e].cpu().pin_memory()
+        Kh = Kn[:n_e2e].cpu().pin_memory()
+        Vh = Vn[:n_e2e].cpu().pin_memory()
+        outh = torch.empty(n_e2e, *out.shape, dtype=out.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(Qs[0]), torch.empty_like(Kn[0]), torch.empty_like(Vn[0])
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
+        e2e_bytes = 0
+        torch.cuda.synchronize()
+        for k in range(n_e2e):
+            flush.zero_()
+            ev[k][0].record(stream)
+            qd.copy_(Qh[k], non_blocking=True)
+            kd.copy_(Kh[k], non_blocking=True)
+            vd.copy_(Vh[k], non_blocking=True)
+            native.tq_append(cache.state, kd, vd, pj.Pi, pj.T, cent, bnd)
+            native.tq_decode_attention(cache.state, qd, scale, pj.Pi, pj.S, cent, out, None,
+                                       args.splits, ws)
+            outh[k].copy_(out, non_blocking=True)
+            ev[k][1].record(stream)
+            e2e_bytes += step_bytes()[1]
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ev), world)
+        e2e_val = reduce_sum(float(e2e_bytes), world) / (e2e_ms * 1e-3) / 1e9
+        e2e = {"value": e2e_val, "unit": "GB/s",
+               "h2d_bytes_per_step": int(Qh[0].numel() * Qh.element_size() + 2 * Kh[0].numel() * Kh.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+               "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e}
+
+    # key/value quantise throughput: 131072 tokens x 8 KV heads in chunks of 4096
+    quant = None
+    if not args.no_quantize:
+        quant = bench_quantize(dev, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        K1, V1, Q1, Kn1, Vn1 = _host_unit(w, dev)
+        sec, nb, reps, threads = oracle_decode_sample(w, K1, V1, Q1, Kn1, Vn1)
+        cpu = {"kind": "oracle", "value": nb / sec / 1e9, "unit": "GB/s", "cores": threads,
+               "sample": f"1 of {w.B * w.Hkv} (batch, KV-head) units at full context, {reps} steps "
+                         "(append one token + decode its query heads), NumPy float64; GB/s of "
+                         "that unit's packed bytes"}
+
+    launches = 5 * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": _config(w, args),
+        "pct_of_8TBps": 100.0 * value / NOMINAL_HBM,
+        "tokens_per_s": tokens_s,
+        "roofline": {"bound": "hbm", "kernel": "k_decode_partial", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": part_bytes,
+                     "avg_launch_ms": part_avg_ms, "source_hash": src_hash},
+        "e2e": e2e,
+        "quantize": quant,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_quantize(dev, world, reps=3):
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import Codebook, CompressedKVCache, Projections
+    w = synth.WORKLOADS["quant"]
+    pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)
+    K, V = synth.keys_values(w, device=dev)
+    chunks = [(K[:, :, t:t + w.chunk].contiguous(), V[:, :, t:t + w.chunk].contiguous())
+              for t in range(0, w.T, w.chunk)]
+    del K, V
+    cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
+                              dtype=w.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for r in range(reps + 1):
+        cache.state.n_total = 0
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k, v in chunks:
+            cache.append(k, v, pj, cb)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if r > 0:
+            times.append(e0.elapsed_time(e1))
+    ms = reduce_max(min(times), world)
+    keys = reduce_sum(float(w.T * w.Hkv * w.B), world)
+    tb = cache.state.token_bytes
+    nbytes = w.T * w.Hkv * w.B * (2 * w.d * 2 + tb)
+    return {"Mkeys_per_s": keys / (ms * 1e-3) / 1e6, "ms": ms, "keys": int(keys),
+            "GB_per_s": reduce_sum(float(nbytes), world) / (ms * 1e-3) / 1e9,
+            "workload": "quant: 131072 tokens x 8 KV heads, d=128, bf16, appended in chunks of 4096; "
+                        "keys b1=2 + m=128, values 2-bit g=32 (key + value per key)"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

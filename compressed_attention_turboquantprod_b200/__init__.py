@@ -1,0 +1,122 @@
+"""TurboQuant-prod / QJL compressed KV cache and decode attention on B200 (sm_100a).
+
+The compute lives in ``libtq.so`` (hand-written CUDA kernels behind the C ABI
+of ``include/tq.h``); ``native`` is its ctypes binding and this module adds
+small owners of the device buffers (allocated with PyTorch) around it.
+``native`` is loaded on first use (so that ``build`` can run before the library
+exists); using any class here without a built ``libtq.so`` raises ImportError.
+"""
+from __future__ import annotations
+
+import importlib
+import math
+from typing import Optional
+
+import torch
+
+__all__ = ["native", "TQError", "Codebook", "Projections", "CompressedKVCache", "LayerGroups"]
+
+
+def __getattr__(name):
+    if name == "TQError":
+        return importlib.import_module(".native", __name__).TQError
+    raise AttributeError(name)
+
+
+class _Native:
+    def __getattr__(self, name):
+        return getattr(importlib.import_module(".native", __package__), name)
+
+
+native = _Native()
+
+
+class Codebook:
+    """Lloyd-Max centroids/boundaries for head dim d and b1 bits, built on the GPU."""
+
+    def __init__(self, d: int, bits: int, device="cuda"):
+        self.d, self.bits = d, bits
+        L = 1 << bits
+        self.centroids = torch.empty(L, dtype=torch.float32, device=device)
+        self.boundaries = torch.empty(max(L - 1, 1), dtype=torch.float32, device=device)
+        native.tq_codebook_build(d, bits, self.centroids, self.boundaries)
+
+
+class Projections:
+    """Per-layer Pi (d x d), S (m x d) and T = S Pi^T, generated on the GPU."""
+
+    def __init__(self, d: int, m: int, layer: int, rotation: bool = True, device="cuda",
+                 base_seed: int = 42, stride: int = 7):
+        self.d, self.m, self.layer = d, m, layer
+        f32 = dict(dtype=torch.float32, device=device)
+        self.Pi = torch.empty(d, d, **f32) if rotation else None
+        self.S = torch.empty(m, d, **f32)
+        self.T = torch.empty(m, d, **f32)
+        ws = None
+        if rotation:
+            ws = torch.empty(native.tq_projections_workspace_bytes(d), dtype=torch.uint8, device=device)
+        native.tq_make_projections(d, m, layer, self.Pi, self.S, self.T, ws, base_seed, stride)
+
+
+class LayerGroups:
+    """A-QJL per-layer-group sketch dims from the config strings ("8,16,24", "512,384,256,192")."""
+
+    def __init__(self, boundaries: str, sketch_dims: str):
+        self._g = native.tq_layer_groups_parse(boundaries, sketch_dims)
+
+    def m_for_layer(self, layer: int) -> int:
+        return native.tq_m_for_layer(self._g, layer)
+
+
+class CompressedKVCache:
+    """A packed cache of B x Hkv sequences plus its full-precision ring."""
+
+    def __init__(self, B, Hkv, d, b1, m, vbits, group, W, capacity, dtype=torch.bfloat16,
+                 device="cuda"):
+        self.desc = native.make_desc(B, Hkv, d, b1, m, vbits, group, W, capacity, dtype)
+        self.dtype = dtype
+        nbytes = native.tq_cache_bytes(self.desc)
+        if nbytes == 0:
+            native.tq_cache_layout(self.desc)      # raises with the reason
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.state = native.tq_cache()
+        native.tq_cache_init(self.state, self.desc, self.buffer)
+        self._ws = None
+
+    @property
+    def n_total(self) -> int:
+        return self.state.n_total
+
+    @property
+    def n_comp(self) -> int:
+        return native.lib.tq_cache_compressed_tokens(self.state)
+
+    @property
+    def n_ring(self) -> int:
+        return native.lib.tq_cache_ring_tokens(self.state)
+
+    def append(self, K: torch.Tensor, V: torch.Tensor, proj: Projections, cb: Optional[Codebook]):
+        native.tq_append(self.state, K, V, proj.Pi, proj.T,
+                         cb.centroids if cb is not None else None,
+                         cb.boundaries if cb is not None else None)
+
+    def workspace(self, Hq: int, num_splits: int = 0) -> torch.Tensor:
+        need = native.tq_decode_workspace_bytes(self.state, Hq, num_splits)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.buffer.device)
+        return self._ws
+
+    def decode(self, Q: torch.Tensor, proj: Projections, cb: Optional[Codebook],
+               softmax_scale: Optional[float] = None, want_logits: bool = False,
+               num_splits: int = 0, out: Optional[torch.Tensor] = None):
+        B, Hq, d = Q.shape
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+        out = torch.empty_like(Q) if out is None else out
+        logits = None
+        if want_logits:
+            logits = torch.empty(B, Hq, self.n_comp + self.n_ring, dtype=torch.float32, device=Q.device)
+        ws = self.workspace(Hq, num_splits)
+        native.tq_decode_attention(self.state, Q, scale, proj.Pi, proj.S,
+                                   cb.centroids if cb is not None else None, out, logits,
+                                   num_splits, ws)
+        return (out, logits) if want_logits else out

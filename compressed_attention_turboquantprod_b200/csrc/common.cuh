@@ -1,0 +1,58 @@
+// Device helpers shared by the kernel files.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+__device__ __forceinline__ float load_f(const void* p, int64_t i, int dtype) {
+  if (dtype == TQ_F32) return reinterpret_cast<const float*>(p)[i];
+  if (dtype == TQ_F16) return __half2float(reinterpret_cast<const __half*>(p)[i]);
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ void store_f(void* p, int64_t i, int dtype, float v) {
+  if (dtype == TQ_F32) {
+    reinterpret_cast<float*>(p)[i] = v;
+  } else if (dtype == TQ_F16) {
+    reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  } else {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  }
+}
+
+__device__ __forceinline__ int dtype_size(int dtype) { return dtype == TQ_F32 ? 4 : 2; }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Byte address of field `off`/`size` of absolute compressed token t in region (b, h).
+__device__ __forceinline__ uint8_t* field_ptr(uint8_t* base, const Geom& g, int bh, int64_t t,
+                                              int off, int size) {
+  return base + (int64_t)bh * g.region_bytes + (t / kBlockTokens) * g.block_bytes + off +
+         (t % kBlockTokens) * size;
+}
+
+}  // namespace tq

@@ -1,0 +1,432 @@
+// Key/value quantisation and append ([TQ] 二 three-stage pipeline, 五
+// ProdQuantized, 六 store + ring, 七 value group quantisation).
+//
+// One CTA quantises a tile of 64 tokens of one (b, kv head):
+//   keys   rho = ||x|| (float64 sum of exact fp32 squares)
+//          Y = X Pi^T (fp32 FMA), y = Y / rho, idx_j = #{k : beta_k < y_j},
+//          e = y - c[idx], ||r|| = rho ||e||, z = rho (T e) with T = S Pi^T,
+//          sign bit = [z >= 0]; bit-planes and signs packed with warp ballots
+//          (lane i -> bit i, so words are LSB-first / little-endian).
+//          Pure QJL (b1 = 0): z = S x.
+//   values per (token, group): mn, mx, s = (mx - mn)/(2^vb - 1),
+//          code = clamp(rint((v - mn)/s)) in IEEE fp32 (__fsub_rn/__fdiv_rn/rintf).
+// The contractions run as a register-tiled fp32 SGEMM (64 tokens x 128 columns
+// per pass, 4x8 outputs per thread).
+#include <cfloat>
+
+#include "common.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int NT = 64;        // tokens per tile
+constexpr int THREADS = 256;
+constexpr int NC = 128;       // output columns per GEMM pass
+constexpr int KC = 32;        // k-chunk staged in shared memory
+constexpr int SBS = NC + 4;   // row stride of the staged B chunk / Z tile
+
+struct QParams {
+  // source
+  const void* K;
+  const void* V;
+  int dtype;
+  int64_t n, t_first, n_old, n_new;
+  bool cache_mode;
+  const void* ringK;
+  const void* ringV;
+  // shapes
+  int d, b1, m, vbits, group;
+  bool do_keys, do_values;
+  const float* Pi;
+  const float* T;
+  const float* cent;
+  const float* bnd;
+  // outputs
+  QuantDst arr;
+  uint8_t* base;
+  Geom g;
+};
+
+struct Smem {
+  float* X;      // [NT][d+4]
+  float* Y;      // [NT][d+4]
+  float* B;      // [KC][SBS]
+  float* Z;      // [NT][SBS]
+  double* rho64; // [NT]
+  float* rho;    // [NT]
+  float* inv;    // [NT]
+  float* cb;     // [16] centroids, [16] boundaries
+  float* vs;     // [NT * 16] value scales
+  float* vm;     // [NT * 16] value minima
+};
+
+__host__ __device__ inline size_t smem_bytes(int d) {
+  const int sx = d + 4;
+  return sizeof(float) * (2 * NT * sx + KC * SBS + NT * SBS) + sizeof(double) * NT +
+         sizeof(float) * (2 * NT + 32 + 2 * NT * 16);
+}
+
+__device__ Smem carve(unsigned char* raw, int d) {
+  Smem s;
+  const int sx = d + 4;
+  double* dp = reinterpret_cast<double*>(raw);
+  s.rho64 = dp;
+  float* f = reinterpret_cast<float*>(dp + NT);
+  s.X = f;
+  f += NT * sx;
+  s.Y = f;
+  f += NT * sx;
+  s.B = f;
+  f += KC * SBS;
+  s.Z = f;
+  f += NT * SBS;
+  s.rho = f;
+  f += NT;
+  s.inv = f;
+  f += NT;
+  s.cb = f;
+  f += 32;
+  s.vs = f;
+  f += NT * 16;
+  s.vm = f;
+  return s;
+}
+
+// Element pointer base + index of row i (token t_first + i) of (b, h) in the source.
+__device__ __forceinline__ const void* src_row(const QParams& p, bool values, int bh, int64_t i,
+                                               int64_t& elem) {
+  const int d = p.d;
+  const void* chunk = values ? p.V : p.K;
+  if (!p.cache_mode) {
+    elem = i * d;
+    return chunk;
+  }
+  const int64_t t = p.t_first + i;
+  if (t < p.n_old) {
+    elem = ((int64_t)bh * p.g.W + t % p.g.W) * d;
+    return values ? p.ringV : p.ringK;
+  }
+  elem = ((int64_t)bh * p.n_new + (t - p.n_old)) * d;
+  return chunk;
+}
+
+__device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t i, int which) {
+  // which: 0 idx, 1 sign, 2 rho, 3 rnorm, 4 vcode, 5 vscale, 6 vmin
+  if (p.cache_mode) {
+    const Geom& g = p.g;
+    const int64_t t = p.t_first + i;
+    switch (which) {
+      case 0: return field_ptr(p.base, g, bh, t, g.o_idx, g.f_idx);
+      case 1: return field_ptr(p.base, g, bh, t, g.o_sign, g.f_sign);
+      case 2: return field_ptr(p.base, g, bh, t, g.o_rho, 4);
+      case 3: return field_ptr(p.base, g, bh, t, g.o_rnorm, 4);
+      case 4: return field_ptr(p.base, g, bh, t, g.o_vcode, g.f_vcode);
+      case 5: return field_ptr(p.base, g, bh, t, g.o_vscale, g.f_vmeta);
+      default: return field_ptr(p.base, g, bh, t, g.o_vmin, g.f_vmeta);
+    }
+  }
+  const int d = p.d;
+  const int64_t ti = p.t_first + i;
+  switch (which) {
+    case 0: return p.arr.idx + ti * (p.b1 * d / 8);
+    case 1: return p.arr.signs + ti * (p.m / 8);
+    case 2: return reinterpret_cast<uint8_t*>(p.arr.rho + ti);
+    case 3: return reinterpret_cast<uint8_t*>(p.arr.rnorm + ti);
+    case 4: return p.arr.codes + ti * (d * p.vbits / 8);
+    case 5: return reinterpret_cast<uint8_t*>(p.arr.vscale + ti * (d / p.group));
+    default: return reinterpret_cast<uint8_t*>(p.arr.vmin + ti * (d / p.group));
+  }
+}
+
+// Load rows [row0, row0+NT) of the key or value source into X (fp32, zero past n).
+__device__ void load_tile(const QParams& p, bool values, int bh, int64_t row0, float* X) {
+  const int d = p.d, sx = d + 4;
+  for (int idx = threadIdx.x; idx < NT * d; idx += THREADS) {
+    const int r = idx / d, c = idx % d;
+    float v = 0.f;
+    if (row0 + r < p.n) {
+      int64_t e;
+      const void* src = src_row(p, values, bh, row0 + r, e);
+      v = load_f(src, e + c, p.dtype);
+    }
+    X[r * sx + c] = v;
+  }
+}
+
+// acc[r][c] = sum_k A[4ty+r][k] * Bg[col0 + tx + 16c][k], k < kdim; Bg row-major
+// [ncols][kdim], rows past ncols read as zero.
+__device__ void gemm_pass(const float* A, int sa, const float* Bg, int kdim, int col0, int ncols,
+                          float* sB, float acc[4][8]) {
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+  for (int k0 = 0; k0 < kdim; k0 += KC) {
+    for (int idx = tid; idx < KC * NC; idx += THREADS) {
+      const int kk = idx % KC, c = idx / KC;
+      const int col = col0 + c;
+      sB[kk * SBS + c] = (col < ncols) ? Bg[(int64_t)col * kdim + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < KC; ++kk) {
+      float a[4], b[8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a[r] = A[(4 * ty + r) * sa + k0 + kk];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) b[c] = sB[kk * SBS + tx + 16 * c];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+    }
+    __syncthreads();
+  }
+}
+
+__device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int64_t row0) {
+  const int d = p.d, sx = d + 4, b1 = p.b1, m = p.m;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ty = tid / 16, tx = tid % 16;
+  load_tile(p, false, bh, row0, s.X);
+  __syncthreads();
+  for (int r = warp; r < NT; r += THREADS / 32) {
+    double ss = 0.0;
+    for (int c = lane; c < d; c += 32) {
+      const double x = s.X[r * sx + c];
+      ss += x * x;
+    }
+    ss = warp_sum_d(ss);
+    if (lane == 0) {
+      const double rho = sqrt(ss);
+      s.rho64[r] = rho;
+      s.rho[r] = (float)rho;
+      s.inv[r] = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
+    }
+  }
+  __syncthreads();
+  const float* E = s.X;
+  if (b1 > 0) {
+    for (int col0 = 0; col0 < d; col0 += NC) {
+      float acc[4][8];
+      gemm_pass(s.X, sx, p.Pi, d, col0, d, s.B, acc);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int col = col0 + tx + 16 * c;
+          if (col < d) s.Y[(4 * ty + r) * sx + col] = acc[r][c] * s.inv[4 * ty + r];
+        }
+    }
+    __syncthreads();
+    const int L = 1 << b1;
+    for (int r = warp; r < NT; r += THREADS / 32) {
+      const bool valid = row0 + r < p.n;
+      double se = 0.0;
+      uint8_t* idx_dst = valid ? dst_field(p, bh, row0 + r, 0) : nullptr;
+      for (int jb = 0; jb < d; jb += 32) {
+        const float y = s.Y[r * sx + jb + lane];
+        int idx = 0;
+        for (int k = 0; k + 1 < L; ++k) idx += (s.cb[16 + k] < y) ? 1 : 0;
+        const float e = y - s.cb[idx];
+        s.Y[r * sx + jb + lane] = e;
+        se += (double)e * (double)e;
+        for (int pl = 0; pl < b1; ++pl) {
+          const unsigned word = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
+          if (lane == 0 && valid)
+            *reinterpret_cast<uint32_t*>(idx_dst + pl * (d / 8) + jb / 8) = word;
+        }
+      }
+      se = warp_sum_d(se);
+      if (lane == 0 && valid)
+        *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 3)) = (float)(s.rho64[r] * sqrt(se));
+    }
+    __syncthreads();
+    E = s.Y;
+  }
+  for (int col0 = 0; col0 < m; col0 += NC) {
+    float acc[4][8];
+    gemm_pass(E, sx, p.T, d, col0, m, s.B, acc);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float z = (b1 > 0) ? acc[r][c] * s.rho[4 * ty + r] : acc[r][c];
+        s.Z[(4 * ty + r) * SBS + tx + 16 * c] = z;
+      }
+    __syncthreads();
+    for (int r = warp; r < NT; r += THREADS / 32) {
+      const bool valid = row0 + r < p.n;
+      uint8_t* sdst = valid ? dst_field(p, bh, row0 + r, 1) : nullptr;
+      for (int cb = 0; cb < NC && col0 + cb < m; cb += 32) {
+        const unsigned word = __ballot_sync(0xffffffffu, s.Z[r * SBS + cb + lane] >= 0.f);
+        if (lane == 0 && valid) *reinterpret_cast<uint32_t*>(sdst + (col0 + cb) / 8) = word;
+      }
+    }
+    __syncthreads();
+  }
+  for (int r = tid; r < NT; r += THREADS)
+    if (row0 + r < p.n) *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = s.rho[r];
+}
+
+__device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, int64_t row0) {
+  const int d = p.d, sx = d + 4, g = p.group, ng = d / g, vb = p.vbits;
+  const float levels = (float)((1 << vb) - 1);
+  const int tid = threadIdx.x;
+  load_tile(p, true, bh, row0, s.X);
+  __syncthreads();
+  for (int pr = tid; pr < NT * ng; pr += THREADS) {
+    const int r = pr / ng, gi = pr % ng;
+    float mn = FLT_MAX, mx = -FLT_MAX;
+    for (int k = 0; k < g; ++k) {
+      const float v = s.X[r * sx + gi * g + k];
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+    const float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
+    s.vs[pr] = sc;
+    s.vm[pr] = mn;
+    if (row0 + r < p.n) {
+      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 5))[gi] = sc;
+      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 6))[gi] = mn;
+    }
+  }
+  __syncthreads();
+  const int per_word = 32 / vb;
+  const int wpr = d / per_word;
+  for (int pw = tid; pw < NT * wpr; pw += THREADS) {
+    const int r = pw / wpr, w = pw % wpr;
+    if (row0 + r >= p.n) continue;
+    uint32_t word = 0;
+    for (int k = 0; k < per_word; ++k) {
+      const int ch = w * per_word + k;
+      const int gi = ch / g;
+      const float sc = s.vs[r * ng + gi], mn = s.vm[r * ng + gi];
+      uint32_t code = 0;
+      if (sc != 0.f) {
+        float q = rintf(__fdiv_rn(__fsub_rn(s.X[r * sx + ch], mn), sc));
+        q = fminf(fmaxf(q, 0.f), levels);
+        code = (uint32_t)q;
+      }
+      word |= code << (k * vb);
+    }
+    reinterpret_cast<uint32_t*>(dst_field(p, bh, row0 + r, 4))[w] = word;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(THREADS) k_quantize(QParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Smem s = carve(smem_raw, p.d);
+  const int bh = blockIdx.y;
+  const int64_t row0 = (int64_t)blockIdx.x * NT;
+  if (threadIdx.x < 16) {
+    const int L = p.b1 > 0 ? (1 << p.b1) : 0;
+    s.cb[threadIdx.x] = (threadIdx.x < L) ? p.cent[threadIdx.x] : 0.f;
+    s.cb[16 + threadIdx.x] = (threadIdx.x + 1 < L) ? p.bnd[threadIdx.x] : 0.f;
+  }
+  __syncthreads();
+  if (p.do_keys) quantize_keys_tile(p, s, bh, row0);
+  __syncthreads();
+  if (p.do_values) quantize_values_tile(p, s, bh, row0);
+}
+
+__global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V, int64_t n_old,
+                             int64_t n_new) {
+  const int bh = blockIdx.x;
+  const int es = (g.dtype == TQ_F32) ? 4 : 2;
+  const int64_t n_tot = n_old + n_new;
+  const int64_t t0 = (n_tot - g.W > n_old) ? n_tot - g.W : n_old;
+  const int row_words = g.d * es / 4;
+  const int64_t rows = n_tot - t0;
+  for (int64_t idx = threadIdx.x; idx < rows * row_words * 2; idx += blockDim.x) {
+    const int which = (int)(idx / (rows * row_words));      // 0 = K, 1 = V
+    const int64_t rem = idx % (rows * row_words);
+    const int64_t t = t0 + rem / row_words;
+    const int w = (int)(rem % row_words);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(which ? V : K) +
+                          ((int64_t)bh * n_new + (t - n_old)) * row_words;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(base + (which ? g.ring_v_off : g.ring_k_off)) +
+                    ((int64_t)bh * g.W + t % g.W) * row_words;
+    dst[w] = src[w];
+  }
+}
+
+}  // namespace
+
+static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
+  if (p.n <= 0) return cudaSuccess;
+  const size_t smem = smem_bytes(p.d);
+  cudaError_t e = cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((p.n + NT - 1) / NT), (unsigned)bh_count);
+  k_quantize<<<grid, THREADS, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1, int m,
+                                   int vbits, int group, bool do_keys, bool do_values,
+                                   const float* Pi, const float* T, const float* cent,
+                                   const float* bnd, const QuantDst& dst, cudaStream_t s) {
+  QParams p{};
+  p.K = src.K;
+  p.V = src.V;
+  p.dtype = dtype;
+  p.n = src.n;
+  p.t_first = 0;
+  p.cache_mode = false;
+  p.d = d;
+  p.b1 = b1;
+  p.m = m;
+  p.vbits = vbits;
+  p.group = group;
+  p.do_keys = do_keys;
+  p.do_values = do_values;
+  p.Pi = Pi;
+  p.T = T;
+  p.cent = cent;
+  p.bnd = bnd;
+  p.arr = dst;
+  return run_quantize(p, 1, s);
+}
+
+cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* base,
+                                  const float* Pi, const float* T, const float* cent,
+                                  const float* bnd, cudaStream_t s) {
+  QParams p{};
+  p.K = src.K;
+  p.V = src.V;
+  p.dtype = g.dtype;
+  p.n = src.n;
+  p.t_first = src.t_first;
+  p.n_old = src.n_old;
+  p.n_new = src.n_new;
+  p.cache_mode = true;
+  p.ringK = base + g.ring_k_off;
+  p.ringV = base + g.ring_v_off;
+  p.d = g.d;
+  p.b1 = g.b1;
+  p.m = g.m;
+  p.vbits = g.vbits;
+  p.group = g.group;
+  p.do_keys = true;
+  p.do_values = true;
+  p.Pi = Pi;
+  p.T = T;
+  p.cent = cent;
+  p.bnd = bnd;
+  p.base = base;
+  p.g = g;
+  return run_quantize(p, g.B * g.Hkv, s);
+}
+
+cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,
+                              int64_t n_old, int64_t n_new, cudaStream_t s) {
+  if (g.W == 0 || n_new == 0) return cudaSuccess;
+  k_ring_write<<<g.B * g.Hkv, 256, 0, s>>>(g, base, K, V, n_old, n_new);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,81 @@
+// Internal declarations shared by the ABI layer (abi.cu) and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kBlockTokens = TQ_BLOCK_TOKENS;
+constexpr int kMaxG = 8;          // query heads per KV head
+constexpr int kMaxLevels = 16;    // 2^b1 for b1 <= 4 (codebook build)
+
+// Geometry of the packed cache, as plain values for kernels.
+struct Geom {
+  int B, Hkv, d, b1, m, vbits, group, W, dtype;
+  int64_t capacity;
+  int64_t block_bytes, region_bytes, ring_k_off, ring_v_off;
+  int f_idx, f_sign, f_rnorm, f_vcode, f_vmeta;        // bytes per token per field
+  int o_idx, o_sign, o_rho, o_rnorm, o_vcode, o_vscale, o_vmin;  // field offsets in a block
+};
+
+Geom geom_of(const tq_cache* c);
+
+// ---- setup (setup_kernels.cu) ----
+cudaError_t launch_codebook(int d, int bits, float* cent, float* bnd, cudaStream_t s);
+cudaError_t launch_projections(int d, int m, uint64_t seed, float* Pi, float* S, float* T,
+                               double* ws, cudaStream_t s);
+
+// ---- quantisation / append (quant_kernels.cu) ----
+struct QuantSrc {
+  // Token i of (b, h) in this launch is absolute token t = t_first + i.
+  // Cache mode: t < n_old reads ring slot t mod W, else chunk row t - n_old.
+  const void* K;
+  const void* V;
+  int64_t n;          // tokens per (b, h) in this launch
+  int64_t t_first;
+  int64_t n_old;      // cache mode only
+  int64_t n_new;      // cache mode only (rows of the chunk)
+};
+struct QuantDst {  // token-major arrays (standalone calls)
+  uint8_t* idx;
+  uint8_t* signs;
+  float* rho;
+  float* rnorm;
+  uint8_t* codes;
+  float* vscale;
+  float* vmin;
+};
+cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1, int m,
+                                   int vbits, int group, bool do_keys, bool do_values,
+                                   const float* Pi, const float* T, const float* cent,
+                                   const float* bnd, const QuantDst& dst, cudaStream_t s);
+cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* base,
+                                  const float* Pi, const float* T, const float* cent,
+                                  const float* bnd, cudaStream_t s);
+cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,
+                              int64_t n_old, int64_t n_new, cudaStream_t s);
+
+// ---- decode (decode_kernels.cu) ----
+struct DecodeWs {
+  float* qf;      // [B*Hq, d]   query in fp32
+  float* qr;      // [B*Hq, d]   Pi q
+  float* qs;      // [B*Hq, m]   sqrt(pi/2)/m * S q
+  float* part_o;  // [B*Hq, splits, d]
+  float* part_ml; // [B*Hq, splits, 2]
+};
+size_t decode_ws_bytes(const Geom& g, int Hq, int splits);
+DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits);
+int decode_auto_splits(const Geom& g, int64_t n_comp);
+
+cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float* Pi,
+                               const float* S, const DecodeWs& ws, cudaStream_t s);
+cudaError_t launch_decode_partial(const Geom& g, const uint8_t* base, int64_t n_total,
+                                  int Hq, float scale, const float* cent, float* logits,
+                                  int splits, const DecodeWs& ws, cudaStream_t s);
+cudaError_t launch_decode_combine(const Geom& g, int Hq, void* out, int splits,
+                                  const DecodeWs& ws, cudaStream_t s);
+
+}  // namespace tq

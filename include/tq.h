@@ -1,0 +1,302 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant-prod / QJL compressed KV cache and decode
+ * attention computed directly on the compressed cache, for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (cited per call below):
+ *   [TQ]   TurboQuant KV-cache quantization article (kwkr.cn/news/562855),
+ *          sections 二 (three-stage pipeline), 四 (QJL unbiasedness),
+ *          五 (two-stage estimator, ProdQuantized), 六 (scoring kernels, store,
+ *          ring buffer), 七 (value quantization, known limits).
+ *   [AQJL] A-QJL adaptive layer-wise KV compression article
+ *          (zingnex.cn/forum/thread/a-qjl-kv): QJL, A-QJL, deployment config.
+ *
+ * Conventions shared by every call:
+ *   - Every call returns an int status (enum tq_status).  On failure a
+ *     thread-local message is available from tq_last_error().
+ *   - All argument checks happen on the host before any launch; a call that
+ *     fails a check launches nothing and writes nothing.
+ *   - Device buffers are owned by the caller.  The library never allocates
+ *     device memory and never synchronises, except where a call says so.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued on it; results are ready when the stream reaches them.
+ *   - A CUDA error seen at launch (or left pending by earlier work) is
+ *     returned as TQ_ERR_CUDA.
+ *   - No kernel uses a device-side assert or trap.
+ *   - Device pointers must be 16-byte aligned unless stated otherwise.
+ *   - Supported sizes: head_dim d in {64, 128, 256}; Lloyd-Max bits b1 in
+ *     {0 (pure QJL), 1, 2, 3}; sketch dim m a multiple of 32 in [32, 1024];
+ *     value bits vbits in {2, 4}; value group g in {16, 32, 64, 128} dividing d;
+ *     query heads per KV head G = Hq / Hkv in [1, 8].
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum tq_status {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* a pointer, size or shape is invalid            */
+  TQ_ERR_UNSUPPORTED = 2,   /* a valid but unsupported size / bit width        */
+  TQ_ERR_CAPACITY = 3,      /* append would exceed the cache capacity          */
+  TQ_ERR_CUDA = 4,          /* a CUDA runtime error                            */
+  TQ_ERR_NOT_CONVERGED = 5  /* codebook iteration did not converge             */
+};
+
+enum tq_dtype { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 };
+
+/* Number of tokens per packed block of the cache layout. */
+#define TQ_BLOCK_TOKENS 64
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* tq_last_error(void);
+
+/* ABI version of this header: 1. */
+int tq_version(void);
+
+/*
+ * Host-side fault injection for testing callers' error paths: after
+ * tq_debug_fail_next(name), the next call of the ABI function `name` on any
+ * thread returns TQ_ERR_CUDA with message "injected fault" without launching
+ * anything.  name == NULL clears it.  The environment variable TQ_FAULT, read
+ * on the first call, has the same effect.
+ */
+int tq_debug_fail_next(const char* name);
+
+/* ------------------------------------------------------------------------ */
+/* Setup: codebook and projections                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * tq_codebook_build -- Lloyd-Max codebook for one coordinate of a rotated unit
+ * vector in dimension d ([TQ] 二: continuous 1-D k-means for the Beta law of
+ * the rotated coordinates).  The law is f(t) ~ (1 - t^2)^((d-3)/2) on [-1, 1];
+ * the fixed point beta_k = (c_k + c_{k+1})/2, c_k = E[t | cell k] is iterated in
+ * float64 from Gaussian quantiles until max |delta c| < 1e-13 max |c|, then
+ * made exactly antisymmetric.
+ *   d            head dimension, any value in [16, 4096] (not only 64/128/256)
+ *   bits         b1 in [1, 4]; 2^bits centroids
+ *   centroids    device, float[2^bits], ascending (written)
+ *   boundaries   device, float[2^bits - 1], fp32 midpoints (written)
+ * SYNCHRONOUS: waits for the stream to read the convergence flag.
+ * Errors: INVALID_ARG (null/misaligned pointers, d out of range),
+ *         UNSUPPORTED (bits), NOT_CONVERGED, CUDA.
+ */
+int tq_codebook_build(int d, int bits, float* centroids, float* boundaries, void* stream);
+
+/* Bytes of device workspace tq_make_projections needs for head dimension d. */
+size_t tq_projections_workspace_bytes(int d);
+
+/*
+ * tq_make_projections -- per-layer random rotation Pi and Gaussian sketch S
+ * ([TQ] 二: Pi from a QR factorisation, S Gaussian; [TQ] 六: seed
+ * base_seed + stride * layer, i.e. 42 + 7 * layer).  Generator: Philox4x64-10
+ * (Salmon et al., SC'11), draw k of a row-major matrix = counter (k,0,0,0),
+ * key (seed, stream) with stream 0 for Pi's Gaussian source G and 1 for S;
+ * u = ((w >> 11) + 0.5) 2^-53, z = sqrt(-2 ln u0) cos(2 pi u1).
+ * Pi = Q diag(sign diag R) for G = QR (Householder, float64); y = Pi u.
+ *   Pi      device float[d*d] row-major (written); NULL = pure QJL (no rotation)
+ *   S       device float[m*d] row-major (written)
+ *   T       device float[m*d] row-major (written): T = S Pi^T, the sketch in
+ *           rotated coordinates used by the key quantiser (T = S if Pi == NULL);
+ *           may be NULL
+ *   workspace / ws_bytes  device scratch of tq_projections_workspace_bytes(d)
+ *           bytes (needed only when Pi != NULL)
+ * Errors: INVALID_ARG, UNSUPPORTED (d, m), CUDA.
+ */
+int tq_make_projections(int d, int m, int layer, uint64_t base_seed, uint64_t stride,
+                        float* Pi, float* S, float* T, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Quantisation of keys and values (token-major output arrays)              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * tq_quantize_keys -- [TQ] 二 / 五: rho = ||x||, y = Pi x / rho,
+ * idx_j = #{k : beta_k < y_j} (b1 bits), residual r = x - rho Pi^T c[idx],
+ * sign bits [S r >= 0] (computed as [rho T (y - c[idx]) >= 0]), ||r||.
+ * b1 == 0 is pure QJL ([AQJL] QJL): bits [S x >= 0] and rho only.
+ *   K           device, [n, d] of dtype, row-major
+ *   Pi, T       device, from tq_make_projections (Pi unused when b1 == 0; then
+ *               T must be S)
+ *   centroids, boundaries  device, from tq_codebook_build(d, b1) (unused if b1 == 0)
+ *   idx_planes  device uint8[n * b1*d/8]: per key, b1 bit-planes of d bits,
+ *               plane p byte j>>3 bit j&7 = bit p of idx_j   (NULL if b1 == 0)
+ *   signs       device uint8[n * m/8], bit i at byte i>>3, bit i&7
+ *   norm_x      device float[n] (rho)
+ *   norm_r      device float[n] (||r||; NULL if b1 == 0)
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+int tq_quantize_keys(const void* K, int dtype, int64_t n, int d, int b1, int m,
+                     const float* Pi, const float* T, const float* centroids,
+                     const float* boundaries, uint8_t* idx_planes, uint8_t* signs,
+                     float* norm_x, float* norm_r, void* stream);
+
+/*
+ * tq_quantize_values -- [TQ] 二 table / 七: min-max group quantisation, per
+ * token and per contiguous group of g channels, IEEE fp32 in this order:
+ * mn, mx, s = (mx - mn)/(2^vb - 1), code = clamp(rint((v - mn)/s), 0, 2^vb - 1)
+ * (round half to even; 0 when s == 0).  Dequantised value: mn + code * s.
+ *   V       device [n, d] of dtype
+ *   codes   device uint8[n * d*vbits/8], code j at byte (j*vb)>>3, bit (j*vb)&7
+ *   scale   device float[n * d/g];  vmin  device float[n * d/g]
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+int tq_quantize_values(const void* V, int dtype, int64_t n, int d, int vbits, int group,
+                       uint8_t* codes, float* scale, float* vmin, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* The packed cache                                                          */
+/* ------------------------------------------------------------------------ */
+
+typedef struct tq_cache_desc {
+  int32_t B;          /* batch (sequences advance together)                  */
+  int32_t Hkv;        /* KV heads                                            */
+  int32_t d;          /* head dim                                            */
+  int32_t b1;         /* Lloyd-Max bits (0 = pure QJL)                       */
+  int32_t m;          /* sketch dim                                          */
+  int32_t vbits;      /* value bits                                          */
+  int32_t group;      /* value group size                                    */
+  int32_t W;          /* full-precision ring size, 0..1024                    */
+  int64_t capacity;   /* max compressed tokens per (b, kv head)              */
+  int32_t dtype;      /* dtype of K, V, Q, the ring and the output           */
+  int32_t reserved;
+} tq_cache_desc;
+
+/*
+ * Cache state.  Layout of the device buffer (also defined by the CPU oracle):
+ * for each (b, h) a region of ceil(capacity/64) blocks of 64 tokens; a block
+ * stores, field after field, the 64 tokens' idx planes (b1*d/8 B each), sign
+ * bits (m/8 B), rho (fp32), ||r|| (fp32, absent if b1 == 0), value codes
+ * (d*vbits/8 B), value scales (d/g fp32) and value minima (d/g fp32).  After the
+ * regions, 256-byte aligned: ring keys [B, Hkv, W, d] then ring values, in dtype.
+ * Token t (counting every token ever appended) sits in ring slot t mod W.
+ * After each append the ring holds the last min(W, n_total) tokens and every
+ * older token is compressed exactly once, in order ([TQ] 六 store and ring).
+ */
+typedef struct tq_cache {
+  tq_cache_desc desc;
+  void* base;            /* caller-owned device buffer                        */
+  size_t bytes;
+  int64_t n_total;       /* tokens appended so far                            */
+  int64_t block_bytes, region_bytes, ring_k_off, ring_v_off;
+  int32_t token_bytes;
+  int32_t o_idx, o_sign, o_rho, o_rnorm, o_vcode, o_vscale, o_vmin;
+} tq_cache;
+
+/* Bytes of device memory a cache with this descriptor needs (0 if invalid). */
+size_t tq_cache_bytes(const tq_cache_desc* desc);
+
+/*
+ * tq_cache_layout -- host only: fill `out` with the layout of a cache with
+ * this descriptor (offsets, sizes; base = NULL, n_total = 0).  No CUDA call.
+ * Errors: INVALID_ARG, UNSUPPORTED.
+ */
+int tq_cache_layout(const tq_cache_desc* desc, tq_cache* out);
+
+/*
+ * tq_cache_init -- bind a caller-owned device buffer of at least
+ * tq_cache_bytes(desc) bytes (256-byte aligned) to `c`, zero it on `stream`,
+ * and set n_total = 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+int tq_cache_init(tq_cache* c, const tq_cache_desc* desc, void* dev_mem, size_t bytes,
+                  void* stream);
+
+/* Compressed / ring token counts of a cache (host values). */
+int64_t tq_cache_compressed_tokens(const tq_cache* c);
+int64_t tq_cache_ring_tokens(const tq_cache* c);
+
+/*
+ * tq_append -- append n_new tokens per (b, kv head) ([TQ] 六: chunked append
+ * into a flat cache; recent tokens kept at full precision in a ring).  Tokens
+ * leaving the ring and tokens of the chunk older than the last W are quantised
+ * (keys as tq_quantize_keys, values as tq_quantize_values) straight into the
+ * packed blocks; the last W go to the ring.  Two kernels, in stream order.
+ *   K, V     device [B, Hkv, n_new, d] of desc.dtype, contiguous
+ *   Pi, T, centroids, boundaries  as for tq_quantize_keys
+ * Errors: INVALID_ARG, CAPACITY (nothing written), CUDA.
+ */
+int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const float* Pi,
+              const float* T, const float* centroids, const float* boundaries,
+              void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Number of split-K partitions tq_decode_attention uses when num_splits == 0. */
+int tq_decode_auto_splits(const tq_cache* c, int Hq);
+
+/* Bytes of device workspace for a decode with Hq query heads and num_splits
+ * partitions (0 = automatic). */
+size_t tq_decode_workspace_bytes(const tq_cache* c, int Hq, int num_splits);
+
+/*
+ * tq_decode_attention -- one decode step for every (b, query head)
+ * ([TQ] 四-六; [AQJL] QJL).  Logit of compressed token t for query q:
+ *   b1 > 0: rho_t <Pi q, c[idx_t]> + ||r_t|| sqrt(pi/2)/m <S q, 2 bits_t - 1>
+ *   b1 = 0: rho_t sqrt(pi/2)/m <S q, 2 bits_t - 1>
+ * and <q, k_t> exactly for the ring tokens; p = softmax(softmax_scale * logits);
+ * out = sum_t p_t v_t with v = mn + code * s for compressed tokens and the exact
+ * v for ring tokens.  Query head hq uses KV head hq / (Hq / Hkv) (GQA).
+ * The query is rotated forward and sketched once; keys are never dequantised.
+ * Three kernels: query preparation, split-K partial attention, combine.
+ *   Q        device [B, Hq, d] of desc.dtype
+ *   Pi, S    device, from tq_make_projections (Pi unused when b1 == 0)
+ *   centroids device, from tq_codebook_build (unused when b1 == 0)
+ *   out      device [B, Hq, d] of desc.dtype (written)
+ *   logits   device float[B, Hq, n_comp + n_ring] (unscaled logits, compressed
+ *            tokens in order then ring tokens oldest first) or NULL
+ *   num_splits  0 = automatic
+ *   workspace   device, tq_decode_workspace_bytes() bytes
+ * With no tokens at all the output is zero.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                        const float* Pi, const float* S, const float* centroids, void* out,
+                        float* logits, int num_splits, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* The three stages of tq_decode_attention, for callers that time or overlap
+ * them separately.  Same arguments and workspace as tq_decode_attention. */
+int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, const float* Pi, const float* S,
+                   int num_splits, void* workspace, size_t ws_bytes, void* stream);
+int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const float* centroids,
+                      float* logits, int num_splits, void* workspace, size_t ws_bytes,
+                      void* stream);
+int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive per-layer-group sketch dimension ([AQJL] A-QJL, deployment)     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct tq_layer_groups {
+  int32_t n;          /* number of groups, 1..8                              */
+  int32_t bound[8];   /* bound[i], i < n-1: first layer of group i+1          */
+  int32_t m[8];       /* sketch dim of group i                               */
+} tq_layer_groups;
+
+/*
+ * Parse the A-QJL config strings, e.g. boundaries "8,16,24" and sketch dims
+ * "512,384,256,192" ([AQJL] deployment: "layer_group_boundaries" and
+ * "key_quantization_bits_per_group").  Boundaries must increase; there must be
+ * one more sketch dim than boundaries; every m is a multiple of 32 in
+ * [32, 1024].  Errors: INVALID_ARG.
+ */
+int tq_layer_groups_parse(const char* boundaries, const char* sketch_dims, tq_layer_groups* out);
+
+/* Sketch dim of `layer`: m of the group containing it (-1 if g is invalid). */
+int tq_m_for_layer(const tq_layer_groups* g, int layer);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -165,3 +165,16 @@ def queries(w: Workload, layer: int = 0, device="cpu"):
     """Decode queries [B, Hq, d] in the workload's dtype."""
     x = _draw(w, layer, TENSOR_Q, (w.B, w.Hq, w.d), device)
     return x.to(w.torch_dtype)
+
+
+def decode_stream(w: Workload, n_steps: int, layer: int = 0, device="cpu"):
+    """Per-step decode inputs: Q [n, B, Hq, d] and one new token per sequence,
+    K_new / V_new [n, B, Hkv, 1, d] (contiguous per step), same distributions as
+    the workload's cache (drawn under layer id ``1000 + layer``)."""
+    ws = w.scaled(T=n_steps)
+    K, V = keys_values(ws, layer=1000 + layer, device=device)
+    Kn = K.permute(2, 0, 1, 3).unsqueeze(3).contiguous()
+    Vn = V.permute(2, 0, 1, 3).unsqueeze(3).contiguous()
+    g = _generator(w.seed, 1000 + layer, TENSOR_Q, device)
+    Q = torch.randn(n_steps, w.B, w.Hq, w.d, generator=g, device=device).to(w.torch_dtype)
+    return Q, Kn, Vn

@@ -1,0 +1,97 @@
+"""Shared pieces of the GPU parity tests: the library under test, and helpers
+that run the oracle on the very tensors given to the library and compare."""
+import math
+
+import numpy as np
+import torch
+
+from oracle import codebook as ocb
+from oracle import layout as olayout
+from oracle import projections as oproj
+from oracle import quantize as oq
+
+# Tolerances (stated once, used by every parity test):
+#  - codes, sign bits, value codes/scales/minima: bit-exact (key codes and signs
+#    except elements within 1e-5 relative of a decision boundary or zero);
+#  - rho: 4 ulp; ||r||: 2e-6 relative (fp32 rounding of y = Pi x / rho feeds
+#    e = y - c[idx]; ~1e-8 absolute on entries of size ~3e-2 over d terms);
+#  - logits given identical codes: 1e-3 relative or 1e-4 absolute;
+#  - attention outputs: 2e-3 max-abs.
+RHO_ULP = 4
+RNORM_REL = 2e-6
+LOGIT_REL, LOGIT_ABS = 1e-3, 1e-4
+OUT_ABS = 2e-3
+
+TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def nat():
+    from compressed_attention_turboquantprod_b200 import build
+    build.build()
+    from compressed_attention_turboquantprod_b200 import native
+    return native
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+
+
+def oracle_setup(d, b1, m, layer=0):
+    """The oracle's own stored projections and codebook (numpy fp32)."""
+    p = oproj.make_projections(d, m, layer, with_rotation=b1 > 0)
+    cb = ocb.build(d, b1) if b1 > 0 else (None, None)
+    return p, cb
+
+
+def to_dev(a, device="cuda"):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def unpack_bits_dev(packed: torch.Tensor, nbits: int) -> np.ndarray:
+    return olayout.unpack_bits(packed.cpu().numpy(), nbits)
+
+
+def compare_keys(gpu: dict, ref: dict, d: int, b1: int, m: int, beta32):
+    """gpu: dict of host numpy arrays (idx planes bytes, signs bytes, rho, rnorm);
+    ref: oracle quantize_keys output.  Asserts parity; returns counts."""
+    n = ref["rho"].shape[0]
+    bits_g = olayout.unpack_bits(gpu["signs"], m)
+    skip_tok = np.zeros(n, bool)
+    n_code_mis = n_code_ex = 0
+    if b1 > 0:
+        idx_g = np.zeros((n, d), np.uint8)
+        nb = d // 8
+        for p in range(b1):
+            idx_g |= olayout.unpack_bits(gpu["idx"][:, p * nb:(p + 1) * nb], d) << p
+        ex = oq.code_exempt(ref["y32"], beta32)
+        mis = idx_g != ref["idx"]
+        n_code_ex = int(ex.sum())
+        n_code_mis = int(mis.sum())
+        assert not np.any(mis & ~ex), f"{int((mis & ~ex).sum())} non-exempt code mismatches"
+        skip_tok = np.any(mis, axis=1)
+    sex = oq.sign_exempt(ref["z"])
+    smis = (bits_g != ref["bits"]) & ~skip_tok[:, None]
+    assert not np.any(smis & ~sex), f"{int((smis & ~sex).sum())} non-exempt sign mismatches"
+    rho_g = gpu["rho"].astype(np.float32)
+    ulp = np.spacing(np.abs(ref["rho"]).astype(np.float32))
+    assert np.all(np.abs(rho_g - ref["rho"]) <= RHO_ULP * ulp + 0.0)
+    if b1 > 0:
+        rn_g = gpu["rnorm"].astype(np.float64)
+        rn_r = ref["rnorm"].astype(np.float64)
+        ok = np.abs(rn_g - rn_r) <= RNORM_REL * np.abs(rn_r) + 1e-30
+        assert np.all(ok | skip_tok), f"rnorm max rel err {np.max(np.abs(rn_g - rn_r)[~skip_tok] / rn_r[~skip_tok])}"
+    return {"code_mismatch": n_code_mis, "code_exempt": n_code_ex,
+            "sign_mismatch": int(smis.sum()), "sign_exempt": int(sex.sum()),
+            "skipped_tokens": int(skip_tok.sum())}
+
+
+def check_logits(got: np.ndarray, want: np.ndarray):
+    err = np.abs(got - want)
+    ok = (err <= LOGIT_REL * np.abs(want)) | (err <= LOGIT_ABS)
+    assert np.all(ok), f"logit mismatch: worst {np.max(err)} at |want| {np.abs(want).flat[np.argmax(err)]}"
+
+
+def check_out(got: np.ndarray, want: np.ndarray):
+    err = np.max(np.abs(got - want)) if got.size else 0.0
+    assert err <= OUT_ABS, f"output max-abs error {err} (max |o| {np.max(np.abs(want))})"
+    return err

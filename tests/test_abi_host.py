@@ -1,0 +1,165 @@
+"""The C-ABI library loads, exports every call of include/tq.h, and its host-side
+logic (layout, argument checks, capacity, fault injection, layer groups) works
+without a GPU.  No call here reaches a CUDA API."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT, page_figures
+from oracle import layout as olayout
+
+pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
+                                reason="host-only checks use fake device pointers")
+
+
+@pytest.fixture(scope="module")
+def nat():
+    from compressed_attention_turboquantprod_b200 import build
+    build.build()
+    from compressed_attention_turboquantprod_b200 import native
+    return native
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(nat):
+    names = _declared()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(nat.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert nat.lib.tq_version() == 1
+
+
+@pytest.mark.parametrize("cfg", [
+    (8, 8, 128, 2, 128, 2, 32, 16, 32768, "bf16"),
+    (4, 4, 256, 3, 256, 4, 64, 16, 262144, "bf16"),
+    (16, 8, 128, 0, 512, 2, 32, 16, 65536, "f16"),
+    (1, 1, 128, 2, 128, 2, 32, 0, 512, "f32"),
+    (2, 3, 64, 1, 96, 4, 16, 5, 100, "f32"),
+])
+def test_layout_matches_oracle_format(nat, cfg):
+    B, Hkv, d, b1, m, vb, g, W, cap, dt = cfg
+    code = {"f32": 0, "f16": 1, "bf16": 2}[dt]
+    c = nat.tq_cache_layout(nat.make_desc(B, Hkv, d, b1, m, vb, g, W, cap, code))
+    o = olayout.Layout(B, Hkv, d, b1, m, vb, g, W, cap, dt)
+    assert c.block_bytes == o.block_bytes and c.token_bytes == o.token_bytes
+    assert c.region_bytes == o.region_bytes
+    assert (c.o_idx, c.o_sign, c.o_rho, c.o_rnorm, c.o_vcode, c.o_vscale, c.o_vmin) == \
+        (o.o_idx, o.o_sign, o.o_rho, o.o_rnorm, o.o_vcode, o.o_vscale, o.o_vmin)
+    assert (c.ring_k_off, c.ring_v_off, c.bytes) == (o.ring_k_off, o.ring_v_off, o.total_bytes)
+    assert nat.tq_cache_bytes(nat.make_desc(B, Hkv, d, b1, m, vb, g, W, cap, code)) == o.total_bytes
+
+
+def _status(nat, fn, *args):
+    return fn(*args)
+
+
+FAKE = ctypes.c_void_p(1 << 20)    # 16/256-byte aligned, never dereferenced
+
+
+def test_argument_checks_return_before_any_launch(nat):
+    L = nat.lib
+    S = None
+    # unsupported head dim / bit widths / sketch dims
+    assert L.tq_quantize_keys(FAKE, 2, 10, 100, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert "head dim" in L.tq_last_error().decode()
+    assert L.tq_quantize_keys(FAKE, 2, 10, 128, 4, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_quantize_keys(FAKE, 2, 10, 128, 2, 48, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_quantize_keys(FAKE, 7, 10, 128, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_quantize_keys(None, 2, 10, 128, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_quantize_keys(FAKE, 2, 10, 128, 2, 128, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_quantize_keys(ctypes.c_void_p((1 << 20) + 4), 2, 10, 128, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_quantize_keys(FAKE, 2, -1, 128, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    # n == 0 is a no-op success without touching CUDA
+    assert L.tq_quantize_keys(FAKE, 2, 0, 128, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S) == nat.TQ_OK
+    assert L.tq_quantize_values(FAKE, 2, 10, 128, 3, 32, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_quantize_values(FAKE, 2, 10, 128, 2, 24, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_quantize_values(FAKE, 2, 10, 64, 2, 128, FAKE, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_codebook_build(128, 5, FAKE, FAKE, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_codebook_build(8, 2, FAKE, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_codebook_build(128, 2, None, FAKE, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_make_projections(96, 128, 0, 42, 7, FAKE, FAKE, FAKE, FAKE, 1 << 30, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_make_projections(128, 100, 0, 42, 7, FAKE, FAKE, FAKE, FAKE, 1 << 30, S) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_make_projections(128, 128, 0, 42, 7, FAKE, FAKE, FAKE, FAKE, 16, S) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_make_projections(128, 128, -1, 42, 7, FAKE, FAKE, FAKE, FAKE, 1 << 30, S) == nat.TQ_ERR_INVALID_ARG
+
+
+def _fake_cache(nat, **kw):
+    p = dict(B=2, Hkv=2, d=128, b1=2, m=128, vbits=2, group=32, W=16, capacity=100, dtype=2)
+    p.update(kw)
+    desc = nat.make_desc(p["B"], p["Hkv"], p["d"], p["b1"], p["m"], p["vbits"], p["group"],
+                         p["W"], p["capacity"], p["dtype"])
+    c = nat.tq_cache_layout(desc)
+    c.base = 1 << 20
+    return c
+
+
+def test_append_capacity_checked_before_launch(nat):
+    c = _fake_cache(nat)
+    st = nat.lib.tq_append(ctypes.byref(c), FAKE, FAKE, 117, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == nat.TQ_ERR_CAPACITY and c.n_total == 0
+    assert "capacity" in nat.lib.tq_last_error().decode()
+    c.n_total = 100      # 84 compressed + 16 ring; 17 more would need 101 slots
+    st = nat.lib.tq_append(ctypes.byref(c), FAKE, FAKE, 17, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == nat.TQ_ERR_CAPACITY and c.n_total == 100
+    assert nat.lib.tq_append(ctypes.byref(c), FAKE, FAKE, 0, None, None, None, None, None) == nat.TQ_OK
+    assert nat.lib.tq_append(ctypes.byref(c), None, FAKE, 3, FAKE, FAKE, FAKE, FAKE, None) == nat.TQ_ERR_INVALID_ARG
+    assert nat.lib.tq_append(None, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, None) == nat.TQ_ERR_INVALID_ARG
+    bad = _fake_cache(nat)
+    bad.block_bytes += 16        # struct not produced by init/layout
+    assert nat.lib.tq_append(ctypes.byref(bad), FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, None) == nat.TQ_ERR_INVALID_ARG
+
+
+def test_decode_checks(nat):
+    c = _fake_cache(nat)
+    c.n_total = 90
+    L = nat.lib
+    need = L.tq_decode_workspace_bytes(ctypes.byref(c), 8, 0)
+    assert need > 0
+    assert L.tq_decode_workspace_bytes(ctypes.byref(c), 7, 0) == 0
+    assert L.tq_decode_attention(ctypes.byref(c), FAKE, 7, 0.1, FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, need, None) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_decode_attention(ctypes.byref(c), FAKE, 18, 0.1, FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, need, None) == nat.TQ_ERR_UNSUPPORTED
+    assert L.tq_decode_attention(ctypes.byref(c), FAKE, 8, 0.1, FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, 64, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_decode_attention(ctypes.byref(c), None, 8, 0.1, FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, need, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_decode_attention(ctypes.byref(c), FAKE, 8, float("nan"), FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, need, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_decode_attention(ctypes.byref(c), FAKE, 8, 0.1, FAKE, FAKE, FAKE, FAKE, None, -2, FAKE, need, None) == nat.TQ_ERR_INVALID_ARG
+    # the automatic split count stays within the workspace sized for the capacity
+    for n in (0, 1, 16, 17, 80, 116):
+        c.n_total = n
+        s = L.tq_decode_auto_splits(ctypes.byref(c), 8)
+        assert 1 <= s
+        assert L.tq_decode_workspace_bytes(ctypes.byref(c), 8, 0) == need
+
+
+def test_fault_injection_is_host_side_and_one_shot(nat):
+    c = _fake_cache(nat)
+    nat.tq_debug_fail_next("tq_append")
+    st = nat.lib.tq_append(ctypes.byref(c), FAKE, FAKE, 1000, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == nat.TQ_ERR_CUDA and nat.lib.tq_last_error().decode() == "injected fault"
+    st = nat.lib.tq_append(ctypes.byref(c), FAKE, FAKE, 1000, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == nat.TQ_ERR_CAPACITY          # armed once only
+    nat.tq_debug_fail_next("tq_decode_attention")
+    nat.tq_debug_fail_next(None)              # cleared
+    assert nat.lib.tq_decode_attention(ctypes.byref(c), FAKE, 7, 0.1, FAKE, FAKE, FAKE, FAKE, None, 0, FAKE, 1, None) == nat.TQ_ERR_UNSUPPORTED
+
+
+def test_layer_groups_from_page_config(nat):
+    figs = page_figures()
+    g = nat.tq_layer_groups_parse(figs["aqjl_layer_group_boundaries"], figs["aqjl_key_bits_per_group"])
+    want = [512] * 8 + [384] * 8 + [256] * 8 + [192] * 8
+    assert [nat.tq_m_for_layer(g, l) for l in range(32)] == want
+    assert nat.tq_m_for_layer(g, 1000) == 192
+    for bad in (("8,16", "512,384,256,192"), ("16,8,24", "512,384,256,192"),
+                ("8,16,24", "512,384,256,100"), ("8,x,24", "512,384,256,192"), ("", "")):
+        with pytest.raises(nat.TQError):
+            nat.tq_layer_groups_parse(*bad)
+    one = nat.tq_layer_groups_parse("", "256")
+    assert nat.tq_m_for_layer(one, 7) == 256

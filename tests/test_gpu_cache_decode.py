@@ -1,0 +1,209 @@
+"""GPU parity of append (packed bytes) and decode attention against the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_common import (TORCH_DT, check_logits, check_out, compare_keys, host, nat, oracle_setup,
+                        to_dev)
+from oracle import cache as ocache
+from oracle import layout as olayout
+
+pytestmark = pytest.mark.gpu
+
+
+def _workload(**kw):
+    base = dict(name="t", B=2, Hq=8, Hkv=2, d=128, T=300, W=16, b1=2, m=128, vbits=2, group=32,
+                dtype="bf16", seed=11, k_outlier_frac=0.02, v_outlier_frac=0.02, outlier_scale=8.0)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+def _gpu_cache(w, capacity):
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache
+    return CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, capacity,
+                             dtype=TORCH_DT[w.dtype])
+
+
+class _Proj:
+    def __init__(self, po):
+        self.Pi, self.S, self.T = to_dev(po["Pi"]), to_dev(po["S"]), to_dev(po["T"])
+
+
+class _Cb:
+    def __init__(self, cb):
+        self.centroids, self.boundaries = to_dev(cb[0]), to_dev(cb[1])
+
+
+def _oracle_cache(w, capacity, po, cb):
+    return ocache.OracleCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, capacity,
+                              w.dtype, po, cb if w.b1 > 0 else None)
+
+
+def _compare_cache_bytes(gpu_buf: np.ndarray, oc: ocache.OracleCache):
+    ref = oc.to_bytes()
+    assert gpu_buf.shape == ref.shape
+    if np.array_equal(gpu_buf, ref):
+        return 0
+    lay = oc.lay
+    # rings and value fields must match exactly; key fields may differ only on exempt elements
+    assert np.array_equal(gpu_buf[lay.ring_k_off:], ref[lay.ring_k_off:])
+    skipped = 0
+    for b in range(oc.B):
+        for h in range(oc.Hkv):
+            r = oc.rec[b][h]
+            if r is None:
+                continue
+            n = r["rho"].shape[0]
+            fg = olayout.read_region(gpu_buf, lay, b, h, n)
+            fr = olayout.read_region(ref, lay, b, h, n)
+            for name in ("vcode", "vscale", "vmin"):
+                assert np.array_equal(fg[name], fr[name]), name
+            got = {"idx": fg["idx"], "signs": fg["sign"],
+                   "rho": np.ascontiguousarray(fg["rho"]).view("<f4").ravel(),
+                   "rnorm": np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel() if oc.b1 else None}
+            st = compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None)
+            skipped += st["skipped_tokens"]
+    return skipped
+
+
+def test_append_packed_bytes_match_oracle_across_chunks():
+    w = _workload(B=2, Hkv=2, d=128, T=540)
+    cap = 600
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda")
+    gc = _gpu_cache(w, cap)
+    oc = _oracle_cache(w, cap, po, cb)
+    t = 0
+    for n in (5, 11, 1, 100, 64, 300, 1, 58):
+        k = K[:, :, t:t + n].contiguous()
+        v = V[:, :, t:t + n].contiguous()
+        gc.append(k, v, _Proj(po), _Cb(cb))
+        oc.append(host(k), host(v))
+        t += n
+        torch.cuda.synchronize()
+        assert gc.n_total == oc.n_total and gc.n_comp == oc.n_comp and gc.n_ring == oc.n_ring
+        _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("b1,m,vb,g,dt", [(2, 128, 2, 32, "f32"), (0, 256, 2, 32, "f16"),
+                                          (3, 256, 4, 64, "bf16"), (1, 64, 4, 16, "bf16")])
+def test_append_quantize_variants(b1, m, vb, g, dt):
+    w = _workload(B=1, Hkv=3, d=256 if b1 == 3 else 128, b1=b1, m=m, vbits=vb, group=g, dtype=dt,
+                  W=5, T=200)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda")
+    gc = _gpu_cache(w, 256)
+    oc = _oracle_cache(w, 256, po, cb)
+    for a, b in ((0, 3), (3, 130), (130, 200)):
+        k, v = K[:, :, a:b].contiguous(), V[:, :, a:b].contiguous()
+        gc.append(k, v, _Proj(po), _Cb(cb) if b1 else None)
+        oc.append(host(k), host(v))
+    torch.cuda.synchronize()
+    _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
+
+
+def _decode_identical_codes(w, n_tokens, capacity, num_splits=0, Hq=None):
+    """Oracle-built cache bytes decoded by the GPU with the oracle's projections."""
+    Hq = Hq or w.Hq
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda", T=max(n_tokens, 1))
+    oc = _oracle_cache(w, capacity, po, cb)
+    if n_tokens:
+        oc.append(host(K[:, :, :n_tokens]), host(V[:, :, :n_tokens]))
+    gc = _gpu_cache(w, capacity)
+    gc.buffer.copy_(torch.from_numpy(oc.to_bytes()))
+    gc.state.n_total = oc.n_total
+    Q = synth.queries(w.scaled(Hq=Hq), device="cuda")
+    out, logits = gc.decode(Q, _Proj(po), _Cb(cb) if w.b1 else None, want_logits=True,
+                            num_splits=num_splits)
+    torch.cuda.synchronize()
+    ro, rl = oc.decode(host(Q))
+    G = Hq // w.Hkv
+    lg = logits.cpu().numpy().astype(np.float64)
+    for (b, h), want in rl.items():
+        check_logits(lg[b, h * G:(h + 1) * G], want)
+    err = check_out(host(out), ro)
+    return err
+
+
+@pytest.mark.parametrize("n_tokens,splits", [(300, 0), (300, 1), (300, 3), (17, 0), (64 + 16, 2),
+                                             (1000, 7), (16, 0), (5, 0), (1, 0)])
+def test_decode_identical_codes_lengths_and_splits(n_tokens, splits):
+    _decode_identical_codes(_workload(), n_tokens, 1024, splits)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=64, m=64, group=16, Hq=16, Hkv=2),                       # G = 8
+    dict(d=256, b1=3, m=256, vbits=4, group=64, Hq=4, Hkv=4),        # G = 1
+    dict(b1=0, m=512, dtype="f16", Hq=8, Hkv=2),                    # pure QJL
+    dict(b1=0, m=192, dtype="f16", W=0),
+    dict(b1=1, m=96, vbits=4, dtype="f32"),
+    dict(W=0, dtype="f32", B=1, Hq=4, Hkv=1, k_outlier_count=4, outlier_scale=10.0,
+         k_outlier_frac=0.0, v_outlier_frac=0.0),                  # the tiny workload's shape
+])
+def test_decode_identical_codes_shapes(kw):
+    w = _workload(**kw)
+    _decode_identical_codes(w, 333, 512)
+
+
+def test_decode_empty_cache_is_zero():
+    w = _workload()
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache
+    gc = _gpu_cache(w, 64)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    Q = synth.queries(w, device="cuda")
+    out = gc.decode(Q, _Proj(po), _Cb(cb))
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0
+
+
+def test_tiny_workload_end_to_end_with_library_projections():
+    """The tiny workload (d=128, 512 fp32 tokens, 4 outlier channels x10, 4 queries):
+    library-made projections + codebook, GPU append + decode, vs the oracle run on
+    its own projections from the same seed."""
+    from compressed_attention_turboquantprod_b200 import Codebook, Projections
+    w = synth.WORKLOADS["tiny"]
+    for W in (0, 16):
+        wl = w.scaled(W=W)
+        K, V = synth.keys_values(wl, device="cuda")
+        Q = synth.queries(wl, device="cuda")
+        pg, cbg = Projections(wl.d, wl.m, 0), Codebook(wl.d, wl.b1)
+        gc = _gpu_cache(wl, 512)
+        gc.append(K, V, pg, cbg)
+        out, logits = gc.decode(Q, pg, cbg, want_logits=True)
+        torch.cuda.synchronize()
+        po, cb = oracle_setup(wl.d, wl.b1, wl.m)
+        oc = _oracle_cache(wl, 512, po, cb)
+        oc.append(host(K), host(V))
+        ro, rl = oc.decode(host(Q))
+        check_out(host(out), ro)
+        # logits: identical codes except near-boundary flips, so compare where no flip
+        want = rl[(0, 0)]
+        got = logits.cpu().numpy()[0].astype(np.float64)
+        err = np.abs(got - want)
+        bad = ~((err <= 1e-3 * np.abs(want)) | (err <= 1e-4))
+        assert bad.sum() <= 4 * 2, f"{bad.sum()} logits off"
+
+
+def test_gqa32k_shape_reduced_context_end_to_end():
+    from compressed_attention_turboquantprod_b200 import Codebook, Projections
+    w = synth.WORKLOADS["gqa32k"].scaled(T=2000)
+    K, V = synth.keys_values(w, device="cuda")
+    Q = synth.queries(w, device="cuda")
+    pg, cbg = Projections(w.d, w.m, 0), Codebook(w.d, w.b1)
+    gc = _gpu_cache(w, 2048)
+    gc.append(K[:, :, :1500].contiguous(), V[:, :, :1500].contiguous(), pg, cbg)
+    for t in range(1500, 2000, 100):
+        gc.append(K[:, :, t:t + 100].contiguous(), V[:, :, t:t + 100].contiguous(), pg, cbg)
+    out = gc.decode(Q, pg, cbg)
+    torch.cuda.synchronize()
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    oc = _oracle_cache(w.scaled(B=1, Hkv=1, Hq=4), 2048, po, cb)
+    for b, h in ((0, 0), (7, 5)):
+        oc2 = _oracle_cache(w.scaled(B=1, Hkv=1, Hq=4), 2048, po, cb)
+        oc2.append(host(K[b:b + 1, h:h + 1]), host(V[b:b + 1, h:h + 1]))
+        ro, _ = oc2.decode(host(Q[b:b + 1, 4 * h:4 * h + 4]))
+        check_out(host(out[b:b + 1, 4 * h:4 * h + 4]), ro)
