@@ -16,7 +16,9 @@ from oracle import quantize as oq
 #  - rho: 4 ulp; ||r||: 2e-6 relative (fp32 rounding of y = Pi x / rho feeds
 #    e = y - c[idx]; ~1e-8 absolute on entries of size ~3e-2 over d terms);
 #  - logits given identical codes: 1e-3 relative or 1e-4 absolute;
-#  - attention outputs: 2e-3 max-abs.
+#  - attention outputs: 2e-3 max-abs, plus half an ulp of the output dtype at
+#    |o| (the output is stored in the cache dtype; bf16 alone rounds |o| = 4 by
+#    up to 7.8e-3, which no arithmetic can beat).
 RHO_ULP = 4
 RNORM_REL = 2e-6
 LOGIT_REL, LOGIT_ABS = 1e-3, 1e-4
@@ -91,7 +93,20 @@ def check_logits(got: np.ndarray, want: np.ndarray):
     assert np.all(ok), f"logit mismatch: worst {np.max(err)} at |want| {np.abs(want).flat[np.argmax(err)]}"
 
 
-def check_out(got: np.ndarray, want: np.ndarray):
-    err = np.max(np.abs(got - want)) if got.size else 0.0
-    assert err <= OUT_ABS, f"output max-abs error {err} (max |o| {np.max(np.abs(want))})"
-    return err
+HALF_ULP_BITS = {"f32": 24, "f16": 11, "bf16": 8}    # significand bits of each storage type
+
+
+def storage_half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Half an ulp of |x| in the output dtype (rounding-to-nearest error bound)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 1e-30)))
+    return 0.5 * np.exp2(e - (HALF_ULP_BITS[dtype] - 1))
+
+
+def check_out(got: np.ndarray, want: np.ndarray, dtype: str = "bf16"):
+    if not got.size:
+        return 0.0
+    err = np.abs(got - want)
+    tol = OUT_ABS + storage_half_ulp(want, dtype)
+    assert np.all(err <= tol), (f"output error {np.max(err - tol) + OUT_ABS:.3g} over "
+                                f"{OUT_ABS} + storage rounding (max |o| {np.max(np.abs(want)):.3g})")
+    return float(np.max(err))

@@ -125,7 +125,7 @@ def _decode_identical_codes(w, n_tokens, capacity, num_splits=0, Hq=None):
     lg = logits.cpu().numpy().astype(np.float64)
     for (b, h), want in rl.items():
         check_logits(lg[b, h * G:(h + 1) * G], want)
-    err = check_out(host(out), ro)
+    err = check_out(host(out), ro, w.dtype)
     return err
 
 
@@ -179,7 +179,7 @@ def test_tiny_workload_end_to_end_with_library_projections():
         oc = _oracle_cache(wl, 512, po, cb)
         oc.append(host(K), host(V))
         ro, rl = oc.decode(host(Q))
-        check_out(host(out), ro)
+        check_out(host(out), ro, wl.dtype)
         # logits: identical codes except near-boundary flips, so compare where no flip
         want = rl[(0, 0)]
         got = logits.cpu().numpy()[0].astype(np.float64)
@@ -201,9 +201,8 @@ def test_gqa32k_shape_reduced_context_end_to_end():
     out = gc.decode(Q, pg, cbg)
     torch.cuda.synchronize()
     po, cb = oracle_setup(w.d, w.b1, w.m)
-    oc = _oracle_cache(w.scaled(B=1, Hkv=1, Hq=4), 2048, po, cb)
     for b, h in ((0, 0), (7, 5)):
         oc2 = _oracle_cache(w.scaled(B=1, Hkv=1, Hq=4), 2048, po, cb)
         oc2.append(host(K[b:b + 1, h:h + 1]), host(V[b:b + 1, h:h + 1]))
         ro, _ = oc2.decode(host(Q[b:b + 1, 4 * h:4 * h + 4]))
-        check_out(host(out[b:b + 1, 4 * h:4 * h + 4]), ro)
+        check_out(host(out[b:b + 1, 4 * h:4 * h + 4]), ro, w.dtype)
