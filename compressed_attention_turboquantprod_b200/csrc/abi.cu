@@ -175,6 +175,16 @@ int check_decode_common(const tq_cache* c, int Hq, int num_splits) {
 }  // namespace
 
 namespace tq {
+int set_error(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return status;
+}
+
 Geom geom_of(const tq_cache* c) {
   Geom g;
   const tq_cache_desc& d = c->desc;

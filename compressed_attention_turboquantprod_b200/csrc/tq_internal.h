@@ -23,6 +23,9 @@ struct Geom {
 
 Geom geom_of(const tq_cache* c);
 
+// Record a thread-local error message (printf-style) and return `status`.
+int set_error(int status, const char* fmt, ...);
+
 // ---- setup (setup_kernels.cu) ----
 cudaError_t launch_codebook(int d, int bits, float* cent, float* bnd, cudaStream_t s);
 cudaError_t launch_projections(int d, int m, uint64_t seed, float* Pi, float* S, float* T,

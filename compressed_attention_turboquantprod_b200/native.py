@@ -79,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "tq_decode_auto_splits": (I, [C, I]),
         "tq_decode_workspace_bytes": (SZ, [C, I, I]),
         "tq_decode_attention": (I, [C, P, I, F, P, P, P, P, P, I, P, SZ, P]),
+        "tq_decode_attention_noalloc": (I, [C, P, I, F, P, P, P, P, P, I, P]),
         "tq_decode_prep": (I, [C, P, I, P, P, I, P, SZ, P]),
         "tq_decode_partial": (I, [C, I, F, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
@@ -198,6 +199,15 @@ def tq_decode_attention(cache: tq_cache, Q, softmax_scale: float, Pi, S, centroi
                                    _ptr(S), _ptr(centroids), _ptr(out), _ptr(logits), num_splits,
                                    _ptr(workspace), _ws(workspace), _stream(stream)),
            "tq_decode_attention")
+
+
+def tq_decode_attention_noalloc(cache: tq_cache, Q, softmax_scale: float, Pi, S, centroids, out,
+                                logits=None, num_splits: int = 0, stream=None):
+    Hq = Q.shape[1]
+    _check(lib.tq_decode_attention_noalloc(ctypes.byref(cache), _ptr(Q), Hq, softmax_scale,
+                                           _ptr(Pi), _ptr(S), _ptr(centroids), _ptr(out),
+                                           _ptr(logits), num_splits, _stream(stream)),
+           "tq_decode_attention_noalloc")
 
 
 def tq_decode_prep(cache: tq_cache, Q, Pi, S, num_splits, workspace, stream=None):

@@ -273,6 +273,32 @@ int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const floa
 int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void* workspace,
                       size_t ws_bytes, void* stream);
 
+/*
+ * tq_decode_attention_noalloc -- the same decode as tq_decode_attention, for
+ * callers that cannot allocate device memory or pass a workspace (for example
+ * an inference-engine plugin whose host framework owns all device memory and
+ * gives plugins no scratch buffer).  The pages have no counterpart: this is a
+ * deployment convenience of this library.
+ *   Scratch comes from a statically allocated device array of
+ *   TQ_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU that loads the library
+ *   holds until the process exits.  The call allocates nothing.
+ *   The first call on each device looks up that array's device address
+ *   (cudaGetSymbolAddress) with the device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (different
+ *   streams, or different host threads on one device) race and must be
+ *   serialised by the caller.  Each call overwrites every scratch byte it reads,
+ *   so nothing needs clearing between calls.
+ *   Arguments as tq_decode_attention, without the workspace.
+ * Errors: those of tq_decode_attention; UNSUPPORTED when the decode needs more
+ *   scratch than TQ_NOALLOC_SCRATCH_BYTES (e.g. very large B * Hq); CUDA when
+ *   the address lookup fails.
+ */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+int tq_decode_attention_noalloc(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                                const float* Pi, const float* S, const float* centroids,
+                                void* out, float* logits, int num_splits, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Adaptive per-layer-group sketch dimension ([AQJL] A-QJL, deployment)     */
 /* ------------------------------------------------------------------------ */
