@@ -315,7 +315,7 @@ def run_ours(args):
         if evs:
             evs[0].record(stream)
         native.tq_append(cache.state, Kn[i], Vn[i], pj.Pi, pj.T, cent, bnd)
-        native.tq_decode_prep(cache.state, Qs[i], pj.Pi, pj.S, args.splits, ws)
+        native.tq_decode_prep(cache.state, Qs[i], scale, pj.Pi, pj.S, cent, args.splits, ws)
         if evs:
             evs[1].record(stream)
         native.tq_decode_partial(cache.state, w.Hq, scale, cent, None, args.splits, ws)

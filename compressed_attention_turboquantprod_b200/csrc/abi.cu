@@ -147,19 +147,19 @@ int check_cache(const tq_cache* c) {
 }
 
 // Effective split count and the partition it implies.
-int eff_splits(const tq::Geom& g, int64_t n_comp, int num_splits) {
+int eff_splits(const tq::Geom& g, int G, int64_t n_comp, int num_splits) {
   const int64_t nblk = (n_comp + tq::kBlockTokens - 1) / tq::kBlockTokens;
-  int s = num_splits > 0 ? num_splits : tq::decode_auto_splits(g, n_comp);
+  int s = num_splits > 0 ? num_splits : tq::decode_auto_splits(g, G, n_comp);
   if (nblk == 0) return 1;
   if (s > nblk) s = (int)nblk;
   const int64_t bps = (nblk + s - 1) / s;
   return (int)((nblk + bps - 1) / bps);
 }
 
-int max_splits(const tq_cache* c, int num_splits) {
+int max_splits(const tq_cache* c, int Hq, int num_splits) {
   if (num_splits > 0) return num_splits;
   tq::Geom g = tq::geom_of(c);
-  return tq::decode_auto_splits(g, c->desc.capacity);
+  return tq::decode_auto_splits(g, Hq / c->desc.Hkv, c->desc.capacity);
 }
 
 int check_decode_common(const tq_cache* c, int Hq, int num_splits) {
@@ -398,14 +398,13 @@ int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const fl
 }
 
 int tq_decode_auto_splits(const tq_cache* c, int Hq) {
-  (void)Hq;
-  if (check_cache(c) != TQ_OK) return -1;
-  return eff_splits(tq::geom_of(c), n_comp_of(c), 0);
+  if (check_decode_common(c, Hq, 0) != TQ_OK) return -1;
+  return eff_splits(tq::geom_of(c), Hq / c->desc.Hkv, n_comp_of(c), 0);
 }
 
 size_t tq_decode_workspace_bytes(const tq_cache* c, int Hq, int num_splits) {
   if (check_decode_common(c, Hq, num_splits) != TQ_OK) return 0;
-  return tq::decode_ws_bytes(tq::geom_of(c), Hq, max_splits(c, num_splits));
+  return tq::decode_ws_bytes(tq::geom_of(c), Hq, max_splits(c, Hq, num_splits));
 }
 
 static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
@@ -417,7 +416,9 @@ static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_
   const tq_cache_desc& dsc = c->desc;
   tq::Geom g = tq::geom_of(c);
   const int64_t n_comp = n_comp_of(c);
-  const int splits = eff_splits(g, n_comp, num_splits);
+  const int G = Hq / dsc.Hkv;
+  const int splits = eff_splits(g, G, n_comp, num_splits);
+  const bool mma = tq::decode_mma_supported(g, G);
   const size_t need = tq::decode_ws_bytes(g, Hq, splits);
   if (!workspace || !aligned16(workspace) || ws_bytes < need)
     return fail(TQ_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed", name, need);
@@ -425,7 +426,7 @@ static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_
     if (!Q || !S || !aligned16(S) || (dsc.b1 > 0 && (!Pi || !aligned16(Pi))))
       return fail(TQ_ERR_INVALID_ARG, "%s: Q, S (and Pi when b1>0) needed", name);
   }
-  if (partial) {
+  if (prep || partial) {
     if (!std::isfinite(softmax_scale)) return fail(TQ_ERR_INVALID_ARG, "%s: softmax_scale", name);
     if (dsc.b1 > 0 && !centroids) return fail(TQ_ERR_INVALID_ARG, "%s: centroids needed", name);
   }
@@ -436,12 +437,15 @@ static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_
   tq::DecodeWs ws = tq::decode_ws_carve(workspace, g, Hq, splits);
   cudaError_t e = cudaSuccess;
   if (prep) {
-    e = tq::launch_decode_prep(g, Q, Hq, Pi, S, ws, s);
+    e = mma ? tq::launch_decode_prep_mma(g, Q, Hq, Pi, S, centroids, softmax_scale, ws, s)
+            : tq::launch_decode_prep(g, Q, Hq, Pi, S, ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
   }
   if (partial) {
-    e = tq::launch_decode_partial(g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
-                                  softmax_scale, centroids, logits, splits, ws, s);
+    e = mma ? tq::launch_decode_partial_mma(g, static_cast<const uint8_t*>(c->base), c->n_total,
+                                            Hq, softmax_scale, logits, splits, ws, s)
+            : tq::launch_decode_partial(g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
+                                        softmax_scale, centroids, logits, splits, ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
   }
   if (combine) {
@@ -460,11 +464,12 @@ int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_
                       workspace, ws_bytes, stream, true, true, true, "tq_decode_attention");
 }
 
-int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, const float* Pi, const float* S,
-                   int num_splits, void* workspace, size_t ws_bytes, void* stream) {
+int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                   const float* Pi, const float* S, const float* centroids, int num_splits,
+                   void* workspace, size_t ws_bytes, void* stream) {
   TQ_FAULT_POINT("tq_decode_prep");
-  return decode_stage(c, Q, Hq, 1.f, Pi, S, nullptr, nullptr, nullptr, num_splits, workspace,
-                      ws_bytes, stream, true, false, false, "tq_decode_prep");
+  return decode_stage(c, Q, Hq, softmax_scale, Pi, S, centroids, nullptr, nullptr, num_splits,
+                      workspace, ws_bytes, stream, true, false, false, "tq_decode_prep");
 }
 
 int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const float* centroids,
@@ -481,6 +486,24 @@ int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void
   TQ_FAULT_POINT("tq_decode_combine");
   return decode_stage(c, nullptr, Hq, 1.f, nullptr, nullptr, nullptr, out, nullptr, num_splits,
                       workspace, ws_bytes, stream, false, false, true, "tq_decode_combine");
+}
+
+int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* workspace,
+                    size_t ws_bytes, void* stream) {
+  int st = check_decode_common(c, Hq, num_splits);
+  if (st != TQ_OK) return st;
+  tq::Geom g = tq::geom_of(c);
+  const int splits = eff_splits(g, Hq / c->desc.Hkv, n_comp_of(c), num_splits);
+  if (!workspace || ws_bytes < tq::decode_ws_bytes(g, Hq, splits))
+    return fail(TQ_ERR_INVALID_ARG, "tq_decode_check: workspace too small");
+  tq::DecodeWs ws = tq::decode_ws_carve(const_cast<void*>(workspace), g, Hq, splits);
+  int flag = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&flag, ws.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_check");
+  if (flag) return fail(TQ_ERR_CUDA, "decode: a staged load did not complete within its wait limit");
+  return ok();
 }
 
 static int parse_list(const char* s, int* out, int max_n) {

@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(256) k_decode_prep(Geom g, const void* Q, int 
   __shared__ float sq[256];
   const int bq = blockIdx.x, d = g.d, m = g.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (bq == 0 && tid == 0) *ws.err = 0;
   for (int i = tid; i < d; i += blockDim.x) {
     const float v = load_f(Q, (int64_t)bq * d + i, g.dtype);
     sq[i] = v;
@@ -290,19 +291,27 @@ size_t partial_smem(const Geom& g, int G) {
 
 static inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+static size_t frag_words(const Geom& g) {
+  const int F = g.b1 > 0 ? 1 << (g.b1 - 1) : 0;
+  return (size_t)(F * g.d / 32 + g.m / 32) * 2 * 2 * 32;
+}
+
 size_t decode_ws_bytes(const Geom& g, int Hq, int splits) {
-  const size_t bq = (size_t)g.B * Hq;
+  const size_t bq = (size_t)g.B * Hq, units = (size_t)g.B * g.Hkv;
   size_t o = 0;
-  o += align256(bq * g.d * sizeof(float));           // qf
-  o += align256(bq * g.d * sizeof(float));           // qr
-  o += align256(bq * g.m * sizeof(float));           // qs
-  o += align256(bq * splits * 2 * sizeof(float));    // part_ml
-  o += align256(bq * splits * g.d * sizeof(float));  // part_o
+  o += align256(bq * g.d * sizeof(float));                // qf
+  o += align256(bq * g.d * sizeof(float));                // qr
+  o += align256(bq * g.m * sizeof(float));                // qs
+  o += align256(units * frag_words(g) * sizeof(uint32_t)); // frag
+  o += align256(units * 8 * 4 * sizeof(float));           // qconst
+  o += 256;                                               // err
+  o += align256(bq * splits * 2 * sizeof(float));         // part_ml
+  o += align256(bq * splits * g.d * sizeof(float));       // part_o
   return o;
 }
 
 DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits) {
-  const size_t bq = (size_t)g.B * Hq;
+  const size_t bq = (size_t)g.B * Hq, units = (size_t)g.B * g.Hkv;
   char* p = static_cast<char*>(base);
   DecodeWs w;
   w.qf = reinterpret_cast<float*>(p);
@@ -311,16 +320,28 @@ DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits) {
   p += align256(bq * g.d * sizeof(float));
   w.qs = reinterpret_cast<float*>(p);
   p += align256(bq * g.m * sizeof(float));
+  w.frag = reinterpret_cast<uint32_t*>(p);
+  p += align256(units * frag_words(g) * sizeof(uint32_t));
+  w.qconst = reinterpret_cast<float*>(p);
+  p += align256(units * 8 * 4 * sizeof(float));
+  w.err = reinterpret_cast<int*>(p);
+  p += 256;
   w.part_ml = reinterpret_cast<float*>(p);
   p += align256(bq * splits * 2 * sizeof(float));
   w.part_o = reinterpret_cast<float*>(p);
   return w;
 }
 
-int decode_auto_splits(const Geom& g, int64_t n_comp) {
+int decode_auto_splits(const Geom& g, int G, int64_t n_comp) {
   const int64_t nblk = (n_comp + kBlockTokens - 1) / kBlockTokens;
   const int units = g.B * g.Hkv;
-  int64_t s = (kTargetCtas + units - 1) / units;
+  int64_t s;
+  if (decode_mma_supported(g, G)) {
+    // one wave of the tensor-core kernel (148 SMs x 3 resident CTAs), never more
+    s = (int64_t)(148 * 3) / units;
+  } else {
+    s = (kTargetCtas + units - 1) / units;
+  }
   if (s > nblk) s = nblk;
   if (s < 1) s = 1;
   return (int)s;

@@ -1,0 +1,659 @@
+// Tensor-core decode attention on the packed cache ([TQ] 四-六; [AQJL] QJL).
+//
+// Why tensor cores: per cached token a GQA group of G = 4 query heads needs
+// 4 x (256 + 128) sign/plane products plus 4 x 128 P V products; on CUDA cores
+// that is several times the instruction budget of streaming 120 bytes per
+// token at HBM speed.  Both contractions are dense (tokens x features x heads),
+// so they run on warp-level MMA:
+//
+//   logits  int8 mma.sync m16n8k32: A = key feature bits of 16 tokens as u8
+//           (0 or 128; one IMAD shift + one LOP3 per 4 bits), B = the query
+//           weights as three signed int8 slices of a 21-bit fixed-point value,
+//           so the integer accumulation is exact.  For a symmetric Lloyd-Max
+//           codebook c[idx] = sum over odd bit-subsets S of w_S (-1)^{xor of
+//           the bits in S} (a Walsh expansion whose even terms vanish), so the
+//           MSE term is linear in the stored bit-planes:
+//             <Pi q, c[idx]> = (sum_S w_S)(sum_j qr_j) - 2 sum_S w_S sum_j qr_j x_Sj.
+//           The QJL term uses <qs, 2 s - 1> = 2 <qs, s> - sum qs.
+//   P V     f16 mma.sync m16n8k16: A = value codes (channels x tokens) as f16
+//           subnormals code * 2^(2k-24) (one PRMT + one AND per 2 codes; the
+//           per-channel power of two is undone once per split), B = p * s split
+//           into f16 hi + lo (the value scale s is per token and group).
+//
+// One CTA = one (batch, KV head, split) with 4 warps; each warp owns 16 of the
+// 64 tokens of every block and keeps its own online-softmax state; blocks are
+// staged in shared memory by cp.async.bulk with mbarrier completion (4 stages,
+// bounded waits that raise an error flag instead of hanging).  The last split
+// also folds in the exact ring tokens.  Warps merge at the end; the split's
+// (m, l, o) goes to the same workspace the combine kernel reads.
+//
+// Specialisation: head dim 128, G = 4, 2-bit values in groups of 32, b1 in
+// {0, 1, 2}, m in {64, 128, 256}.  Other shapes use decode_kernels.cu.
+#include <cfloat>
+
+#include "common.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int MD = 128;          // head dim of this path
+constexpr int MG = 4;            // query heads per KV head
+constexpr int NST = 4;           // pipeline stages (blocks in flight per CTA)
+constexpr int MT = 128;          // threads per CTA
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+struct MParams {
+  Geom g;
+  const uint8_t* base;
+  int64_t n_comp, n_total;
+  int n_ring, Hq;
+  float scale_log2;
+  float* logits;
+  int64_t n_log;
+  int splits, bps;
+  DecodeWs ws;
+  int* err;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void hmma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Bounded wait on phase `parity` of an mbarrier; false after kWaitLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// Exact int -> float for |x| <= 2^22 (mantissa add, no conversion unit).
+__device__ __forceinline__ float i2f_exact(int x) {
+  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+}
+
+// Workspace views used here: per (batch, KV head) unit, fragment words
+// [kstep][ntile][reg][lane] (uint32) and per head {kM, CM, kQ, CQ} (float).
+
+// ---------------------------------------------------------------- prep
+// One CTA per (batch, KV head): the G queries in fp32 (for the ring), Pi q and
+// sqrt(pi/2)/m S q, the Walsh weights, their 21-bit fixed-point quantisation
+// and three int8 slices laid out as the lanes' B fragments, and the per-head
+// affine constants of the logit (already in log2 units of the softmax).
+__global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, int Hq,
+                                                         const float* Pi, const float* S,
+                                                         const float* cent, float scale_log2,
+                                                         DecodeWs ws, uint32_t* frag,
+                                                         float* qconst) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int unit = blockIdx.x;
+  const int b = unit / g.Hkv, h = unit % g.Hkv;
+  const int d = g.d, m = g.m, b1 = g.b1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* sq = reinterpret_cast<float*>(smem_raw);   // [G][d]
+  float* sqr = sq + MG * d;                          // [G][d]
+  float* sqs = sqr + MG * d;                         // [G][m]
+  __shared__ float s_w[4];                           // Walsh weights of the odd subsets
+  __shared__ unsigned s_maxM[MG], s_maxQ[MG];
+  __shared__ float s_sumqr[MG], s_sumqs[MG];
+  const int bq0 = b * Hq + h * MG;
+  if (unit == 0 && tid == 0) *ws.err = 0;
+  for (int i = tid; i < MG * d; i += blockDim.x) {
+    const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
+    sq[i] = v;
+    ws.qf[(int64_t)bq0 * d + i] = v;
+  }
+  if (tid < MG) {
+    s_maxM[tid] = 0u;
+    s_maxQ[tid] = 0u;
+    s_sumqr[tid] = 0.f;
+    s_sumqs[tid] = 0.f;
+  }
+  if (tid == 0) {
+    // w_S = (1/L) sum_idx c[idx] (-1)^{popc(idx & S)} for the odd subsets S, in the
+    // order of the feature planes: {0}, {1}, {2}, {0,1,2}.
+    const int L = b1 > 0 ? 1 << b1 : 0;
+    const int subsets[4] = {1, 2, 4, 7};
+    for (int k = 0; k < 4; ++k) {
+      double acc = 0.0;
+      for (int idx = 0; idx < L; ++idx)
+        acc += (double)cent[idx] * ((__popc(idx & subsets[k]) & 1) ? -1.0 : 1.0);
+      s_w[k] = L ? (float)(acc / L) : 0.f;
+    }
+  }
+  __syncthreads();
+  const float qscale = 1.2533141373155003f / (float)m;
+  const int rows_pi = b1 > 0 ? d : 0;
+  for (int r = warp; r < MG * (rows_pi + m); r += blockDim.x / 32) {
+    const int hh = r / (rows_pi + m), rr = r % (rows_pi + m);
+    const float* row = rr < rows_pi ? Pi + (int64_t)rr * d : S + (int64_t)(rr - rows_pi) * d;
+    float a = 0.f;
+    for (int i = lane; i < d; i += 32) a = fmaf(row[i], sq[hh * d + i], a);
+    a = warp_sum(a);
+    if (lane == 0) {
+      if (rr < rows_pi) sqr[hh * d + rr] = a;
+      else sqs[hh * m + (rr - rows_pi)] = a * qscale;
+    }
+  }
+  __syncthreads();
+  const int F = b1 > 0 ? 1 << (b1 - 1) : 0;     // feature planes per coordinate
+  // maxima of |W| and the plain sums, per head
+  for (int i = tid; i < MG * d; i += blockDim.x) {
+    const int hh = i / d;
+    const float qr = sqr[i];
+    float wmax = 0.f;
+    for (int k = 0; k < F; ++k) wmax = fmaxf(wmax, fabsf(2.f * s_w[k] * qr));
+    if (F) {
+      atomicMax(&s_maxM[hh], __float_as_uint(wmax));
+      atomicAdd(&s_sumqr[hh], qr);
+    }
+  }
+  for (int i = tid; i < MG * m; i += blockDim.x) {
+    const int hh = i / m;
+    atomicMax(&s_maxQ[hh], __float_as_uint(fabsf(2.f * sqs[i])));
+    atomicAdd(&s_sumqs[hh], sqs[i]);
+  }
+  __syncthreads();
+  const float two21 = 2097152.f;
+  if (tid < MG) {
+    const float mM = __uint_as_float(s_maxM[tid]), mQ = __uint_as_float(s_maxQ[tid]);
+    const float dM = mM > 0.f ? mM / two21 : 1.f, dQ = mQ > 0.f ? mQ / two21 : 1.f;
+    float wsum = 0.f;
+    for (int k = 0; k < F; ++k) wsum += s_w[k];
+    float* c = qconst + ((int64_t)unit * MG + tid) * 4;
+    c[0] = dM / 128.f * scale_log2;
+    c[1] = wsum * s_sumqr[tid] * scale_log2;
+    c[2] = dQ / 128.f * scale_log2;
+    c[3] = -s_sumqs[tid] * scale_log2;
+  }
+  // fragment words
+  const int ksM = F * d / 32, ksQ = m / 32;
+  const int words = (ksM + ksQ) * 2 * 2 * 32;
+  uint32_t* fr = frag + (int64_t)unit * words;
+  for (int wi = tid; wi < words; wi += blockDim.x) {
+    const int ln = wi & 31, r = (wi >> 5) & 1, nt = (wi >> 6) & 1, ks = wi >> 7;
+    const int col = ln >> 2, tg = ln & 3;
+    const int hh = col >> 1;
+    const int slice = nt == 0 ? (col & 1) : ((col & 1) ? -1 : 2);
+    uint32_t word = 0;
+    if (slice >= 0) {
+      const bool mse = ks < ksM;
+      const float mx = __uint_as_float(mse ? s_maxM[hh] : s_maxQ[hh]);
+      const float delta = mx > 0.f ? mx / two21 : 1.f;
+      for (int i = 0; i < 4; ++i) {
+        const int bit = tg + 8 * i + (r ? 4 : 0);
+        float w;
+        if (mse) {
+          const int plane = ks / (d / 32), j = (ks % (d / 32)) * 32 + bit;
+          w = -2.f * s_w[plane] * sqr[hh * d + j];
+        } else {
+          w = 2.f * sqs[hh * m + (ks - ksM) * 32 + bit];
+        }
+        const int wint = __float2int_rn(w / delta);
+        const int s0 = ((wint + 128) & 255) - 128;
+        const int t1 = (wint - s0) >> 8;
+        const int s1 = ((t1 + 128) & 255) - 128;
+        const int s2 = (t1 - s1) >> 8;
+        const int sv = slice == 0 ? s0 : slice == 1 ? s1 : s2;
+        word |= ((uint32_t)(sv & 255)) << (8 * i);
+      }
+    }
+    fr[wi] = word;
+  }
+}
+
+// ---------------------------------------------------------------- partial
+template <int B1, int KSQ>
+__global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
+  constexpr int F = B1 > 0 ? 1 << (B1 - 1) : 0;
+  constexpr int KSM = F * MD / 32;
+  constexpr int KS = KSM + KSQ;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[NST];
+  __shared__ int s_abort;
+  __shared__ float s_m[4][MG], s_l[4][MG];
+  __shared__ float s_mn[4][MG][4];
+
+  const Geom& g = p.g;
+  const int split = blockIdx.x, unit = blockIdx.y;
+  const int b = unit / g.Hkv, h = unit % g.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int bq0 = b * p.Hq + h * MG;
+  const int bb = (int)g.block_bytes;
+  unsigned char* stage = smem_raw;                       // [NST][bb]
+  float* s_out = reinterpret_cast<float*>(smem_raw + (size_t)NST * bb);   // [4][MG][MD]
+
+  const int64_t nblk = (p.n_comp + kBlockTokens - 1) / kBlockTokens;
+  const int64_t blk0 = (int64_t)split * p.bps;
+  const int64_t blk1 = min(nblk, blk0 + p.bps);
+  const int nb = blk1 > blk0 ? (int)(blk1 - blk0) : 0;
+  const uint8_t* region = p.base + (int64_t)unit * g.region_bytes;
+
+  if (tid == 0) {
+    s_abort = 0;
+    for (int s = 0; s < NST; ++s) mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int s = 0; s < NST && s < nb; ++s) {
+      mbar_expect_tx(&full[s], (uint32_t)bb);
+      bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
+    }
+  }
+
+  // B fragments of the score (query slices) in registers
+  uint32_t bf[KS][2][2];
+  {
+    const uint32_t* fr = p.ws.frag + (int64_t)unit * (KS * 128);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) bf[ks][nt][r] = fr[((ks * 2 + nt) * 2 + r) * 32 + lane];
+  }
+  const float* qc = p.ws.qconst + ((int64_t)unit * MG + tig) * 4;
+  const float kM = qc[0], CM = qc[1], kQ = qc[2], CQ = qc[3];
+  __syncthreads();
+
+  const uint32_t mulA = 1u << (7 - tig), mulB = 1u << (3 - tig);
+  const uint32_t codeMask = 0x00030003u << (2 * (gid & 3));
+  // PRMT selectors: result byte 0 <- byte bsel of token A's word, byte 2 <- byte
+  // bsel of token B's word (bytes 1, 3 are masked off); bsel + 2 for channel + 8.
+  const uint32_t bsel = (uint32_t)(gid >> 2);
+  const uint32_t pLo = bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12);
+  const uint32_t pHi = (2 + bsel) | ((2 + bsel) << 4) | ((6 + bsel) << 8) | ((6 + bsel) << 12);
+
+  float m_run = -INFINITY, l_run = 0.f;
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+  float mnacc[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool odd = (gid & 1) != 0;
+  const int hP = gid >> 1;
+
+  // One 16-token step of this warp: logits l0 (token row gid) / l1 (row gid+8) for
+  // head tig are given; update the softmax state and return p0, p1.
+  auto softmax_step = [&](float l0, float l1, float& p0, float& p1) {
+    float mx = fmaxf(l0, l1);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float m_new = fmaxf(m_run, mx);
+    float alpha = 1.f;
+    p0 = 0.f;
+    p1 = 0.f;
+    if (m_new != -INFINITY) {
+      alpha = exp2f(m_run - m_new);
+      p0 = exp2f(l0 - m_new);
+      p1 = exp2f(l1 - m_new);
+    }
+    float s = p0 + p1;
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    l_run = l_run * alpha + s;
+    m_run = m_new;
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] *= alpha;
+      const float aP = __shfl_sync(0xffffffffu, alpha, hP);     // lane hP has tig == hP
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) mnacc[gi] *= aP;
+    }
+  };
+
+  int issued = nb < NST ? nb : NST;     // loads issued by thread 0
+  int it = 0;
+  for (; it < nb; ++it) {
+    const int st = it % NST;
+    const uint32_t phase = (uint32_t)((it / NST) & 1);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], phase));
+    if (!ok) {
+      if (lane == 0) {
+        atomicExch(p.err, 1);
+        s_abort = 1;
+      }
+    }
+    if (ok) {
+    const unsigned char* blk = stage + (size_t)st * bb;
+    const int64_t tok0 = (blk0 + it) * kBlockTokens;
+    const int nt_valid = (int)min((int64_t)kBlockTokens, p.n_comp - tok0);
+    const int t0 = 16 * warp + gid, t1 = t0 + 8;
+
+    // ---------------- logits
+    float vM0 = 0.f, vM1 = 0.f, vQ0 = 0.f, vQ1 = 0.f;
+    if (KSM > 0) {
+      int a[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+      const uint32_t* w0p = reinterpret_cast<const uint32_t*>(blk + g.o_idx + t0 * (B1 * MD / 8));
+      const uint32_t* w1p = reinterpret_cast<const uint32_t*>(blk + g.o_idx + t1 * (B1 * MD / 8));
+#pragma unroll
+      for (int ks = 0; ks < KSM; ++ks) {
+        const uint32_t w0 = w0p[ks], w1 = w1p[ks];
+        const uint32_t a0 = (w0 * mulA) & 0x80808080u, a1 = (w1 * mulA) & 0x80808080u;
+        const uint32_t a2 = (w0 * mulB) & 0x80808080u, a3 = (w1 * mulB) & 0x80808080u;
+        imma16832(a[0], a0, a1, a2, a3, bf[ks][0][0], bf[ks][0][1]);
+        imma16832(a[1], a0, a1, a2, a3, bf[ks][1][0], bf[ks][1][1]);
+      }
+      vM0 = i2f_exact(a[0][0]) + 256.f * i2f_exact(a[0][1]) + 65536.f * i2f_exact(a[1][0]);
+      vM1 = i2f_exact(a[0][2]) + 256.f * i2f_exact(a[0][3]) + 65536.f * i2f_exact(a[1][2]);
+    }
+    {
+      int a[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+      const uint32_t* w0p = reinterpret_cast<const uint32_t*>(blk + g.o_sign + t0 * (KSQ * 4));
+      const uint32_t* w1p = reinterpret_cast<const uint32_t*>(blk + g.o_sign + t1 * (KSQ * 4));
+#pragma unroll
+      for (int ks = 0; ks < KSQ; ++ks) {
+        const uint32_t w0 = w0p[ks], w1 = w1p[ks];
+        const uint32_t a0 = (w0 * mulA) & 0x80808080u, a1 = (w1 * mulA) & 0x80808080u;
+        const uint32_t a2 = (w0 * mulB) & 0x80808080u, a3 = (w1 * mulB) & 0x80808080u;
+        imma16832(a[0], a0, a1, a2, a3, bf[KSM + ks][0][0], bf[KSM + ks][0][1]);
+        imma16832(a[1], a0, a1, a2, a3, bf[KSM + ks][1][0], bf[KSM + ks][1][1]);
+      }
+      vQ0 = i2f_exact(a[0][0]) + 256.f * i2f_exact(a[0][1]) + 65536.f * i2f_exact(a[1][0]);
+      vQ1 = i2f_exact(a[0][2]) + 256.f * i2f_exact(a[0][3]) + 65536.f * i2f_exact(a[1][2]);
+    }
+    const float* rho = reinterpret_cast<const float*>(blk + g.o_rho);
+    float l0, l1;
+    if (B1 > 0) {
+      const float* rn = reinterpret_cast<const float*>(blk + g.o_rnorm);
+      l0 = rho[t0] * fmaf(kM, vM0, CM) + rn[t0] * fmaf(kQ, vQ0, CQ);
+      l1 = rho[t1] * fmaf(kM, vM1, CM) + rn[t1] * fmaf(kQ, vQ1, CQ);
+    } else {
+      l0 = rho[t0] * fmaf(kQ, vQ0, CQ);
+      l1 = rho[t1] * fmaf(kQ, vQ1, CQ);
+    }
+    if (t0 >= nt_valid) l0 = -INFINITY;
+    if (t1 >= nt_valid) l1 = -INFINITY;
+    if (p.logits) {
+      const float inv = 1.f / p.scale_log2;
+      float* lg = p.logits + (int64_t)(bq0 + tig) * p.n_log + tok0;
+      if (t0 < nt_valid) lg[t0] = l0 * inv;
+      if (t1 < nt_valid) lg[t1] = l1 * inv;
+    }
+
+    // ---------------- softmax
+    float p0, p1;
+    softmax_step(l0, l1, p0, p1);
+
+    // ---------------- P V
+    // tokens of this lane's B fragment (head hP): TA, TB = 2tig, 2tig+1; TC, TD = +8
+    const float pA = __shfl_sync(0xffffffffu, p0, 4 * (2 * tig) + hP);
+    const float pB = __shfl_sync(0xffffffffu, p0, 4 * (2 * tig + 1) + hP);
+    const float pC = __shfl_sync(0xffffffffu, p1, 4 * (2 * tig) + hP);
+    const float pD = __shfl_sync(0xffffffffu, p1, 4 * (2 * tig + 1) + hP);
+    const int TA = 16 * warp + 2 * tig, TB = TA + 1, TC = TA + 8, TD = TA + 9;
+    const float4* vs4 = reinterpret_cast<const float4*>(blk + g.o_vscale);
+    const float4* vm4 = reinterpret_cast<const float4*>(blk + g.o_vmin);
+    const float4 sA = vs4[TA], sB = vs4[TB], sC = vs4[TC], sD = vs4[TD];
+    const float4 mA = vm4[TA], mB = vm4[TB], mC = vm4[TC], mD = vm4[TD];
+    uint32_t bpv[4][2];
+    {
+      const float sa[4] = {sA.x, sA.y, sA.z, sA.w}, sb[4] = {sB.x, sB.y, sB.z, sB.w};
+      const float sc[4] = {sC.x, sC.y, sC.z, sC.w}, sd[4] = {sD.x, sD.y, sD.z, sD.w};
+      const float ma[4] = {mA.x, mA.y, mA.z, mA.w}, mb[4] = {mB.x, mB.y, mB.z, mB.w};
+      const float mc[4] = {mC.x, mC.y, mC.z, mC.w}, mdd[4] = {mD.x, mD.y, mD.z, mD.w};
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        const float xA = pA != 0.f ? pA * sa[gi] : 0.f, xB = pB != 0.f ? pB * sb[gi] : 0.f;
+        const float xC = pC != 0.f ? pC * sc[gi] : 0.f, xD = pD != 0.f ? pD * sd[gi] : 0.f;
+        __half2 h0 = __floats2half2_rn(xA, xB), h1 = __floats2half2_rn(xC, xD);
+        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+        const __half2 l0h = __floats2half2_rn(xA - f0.x, xB - f0.y);
+        const __half2 l1h = __floats2half2_rn(xC - f1.x, xD - f1.y);
+        h0 = odd ? l0h : h0;
+        h1 = odd ? l1h : h1;
+        bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
+        bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
+        float mnv = 0.f;
+        if (pA != 0.f) mnv = fmaf(pA, ma[gi], mnv);
+        if (pB != 0.f) mnv = fmaf(pB, mb[gi], mnv);
+        if (pC != 0.f) mnv = fmaf(pC, mc[gi], mnv);
+        if (pD != 0.f) mnv = fmaf(pD, mdd[gi], mnv);
+        mnacc[gi] += mnv;
+      }
+    }
+    {
+      const uint4* vc = reinterpret_cast<const uint4*>(blk + g.o_vcode);   // 2 x uint4 per token
+      const uint4 cA0 = vc[2 * TA], cA1 = vc[2 * TA + 1], cB0 = vc[2 * TB], cB1 = vc[2 * TB + 1];
+      const uint4 cC0 = vc[2 * TC], cC1 = vc[2 * TC + 1], cD0 = vc[2 * TD], cD1 = vc[2 * TD + 1];
+      const uint32_t wa[8] = {cA0.x, cA0.y, cA0.z, cA0.w, cA1.x, cA1.y, cA1.z, cA1.w};
+      const uint32_t wb[8] = {cB0.x, cB0.y, cB0.z, cB0.w, cB1.x, cB1.y, cB1.z, cB1.w};
+      const uint32_t wc[8] = {cC0.x, cC0.y, cC0.z, cC0.w, cC1.x, cC1.y, cC1.z, cC1.w};
+      const uint32_t wd[8] = {cD0.x, cD0.y, cD0.z, cD0.w, cD1.x, cD1.y, cD1.z, cD1.w};
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t a0 = prmt(wa[mt], wb[mt], pLo) & codeMask;
+        const uint32_t a1 = prmt(wa[mt], wb[mt], pHi) & codeMask;
+        const uint32_t a2 = prmt(wc[mt], wd[mt], pLo) & codeMask;
+        const uint32_t a3 = prmt(wc[mt], wd[mt], pHi) & codeMask;
+        hmma16816(acc[mt], a0, a1, a2, a3, bpv[mt >> 1][0], bpv[mt >> 1][1]);
+      }
+    }
+    }  // ok
+    __syncthreads();
+    if (s_abort) break;
+    if (tid == 0 && it + NST < nb) {
+      mbar_expect_tx(&full[st], (uint32_t)bb);
+      bulk_load(stage + (size_t)st * bb, region + (blk0 + it + NST) * bb, (uint32_t)bb, &full[st]);
+      ++issued;
+    }
+  }
+
+  if (s_abort) {
+    // a wait gave up: wait (bounded) for this CTA's copies still in flight, then leave
+    if (tid == 0)
+      for (int j = it; j < issued; ++j) (void)mbar_wait(&full[j % NST], (uint32_t)((j / NST) & 1));
+    return;
+  }
+
+  // ---------------- exact ring tokens (last split, warp 0)
+  // The value part of acc counts codes in units of 2^(2k-24) (k = gid & 3, the
+  // bit offset of this lane's channels in their byte): o = acc / code_unit.
+  const float code_unit = __int_as_float((127 - 24 + 2 * (gid & 3)) << 23);       // 2^(2k-24)
+  const float inv_unit = __int_as_float((127 + 24 - 2 * (gid & 3)) << 23);        // 2^(24-2k)
+  if (split == p.splits - 1 && p.n_ring > 0 && warp == 0) {
+    const int64_t first = p.n_total - p.n_ring;
+    const float* qf = p.ws.qf + (int64_t)(bq0 + tig) * MD;
+    for (int r0 = 0; r0 < p.n_ring; r0 += 16) {
+      float lr[2];
+      for (int k = 0; k < 2; ++k) {
+        const int rt = r0 + gid + 8 * k;
+        float dot = -INFINITY;
+        if (rt < p.n_ring) {
+          const int64_t slot = (first + rt) % g.W;
+          const int64_t e = ((int64_t)unit * g.W + slot) * MD;
+          dot = 0.f;
+          for (int j = 0; j < MD; ++j) dot = fmaf(qf[j], load_f(p.base + g.ring_k_off, e + j, g.dtype), dot);
+          if (p.logits) p.logits[(int64_t)(bq0 + tig) * p.n_log + p.n_comp + rt] = dot;
+          dot *= p.scale_log2;
+        }
+        lr[k] = dot;
+      }
+      float p0, p1;
+      softmax_step(lr[0], lr[1], p0, p1);
+      // acc[mt][c]: channel 16 mt + gid (+8 for c >= 2), column 2 tig + (c & 1) = head tig;
+      // add p * v into the hi column (c even) in code units
+      for (int T = 0; T < 16; ++T) {
+        const float pt = __shfl_sync(0xffffffffu, T < 8 ? p0 : p1, 4 * (T & 7) + tig);
+        const int rt = r0 + T;
+        if (rt >= p.n_ring) continue;
+        const int64_t slot = (first + rt) % g.W;
+        const int64_t e = ((int64_t)unit * g.W + slot) * MD;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const float v0 = load_f(p.base + g.ring_v_off, e + 16 * mt + gid, g.dtype);
+          const float v1 = load_f(p.base + g.ring_v_off, e + 16 * mt + gid + 8, g.dtype);
+          acc[mt][0] = fmaf(pt * v0, code_unit, acc[mt][0]);
+          acc[mt][2] = fmaf(pt * v1, code_unit, acc[mt][2]);
+        }
+      }
+    }
+  }
+
+  // ---------------- merge the 4 warps
+  if (gid == 0) {
+    s_m[warp][tig] = m_run;
+    s_l[warp][tig] = l_run;
+  }
+  // mn sums: lanes of the hi column (gid even) of head hP, reduce over tig
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    float v = odd ? 0.f : mnacc[gi];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    if (tig == 0 && !odd) s_mn[warp][hP][gi] = v;
+  }
+  __syncthreads();
+  // this lane's channels, head tig: o = code part (hi + lo) + mn part, scaled to the CTA max
+  float Mh = -INFINITY;
+  for (int w = 0; w < 4; ++w) Mh = fmaxf(Mh, s_m[w][tig]);
+  const float sc = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mh);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int ch0 = 16 * mt + gid, ch1 = ch0 + 8;
+    const int gi = mt >> 1;
+    const float mnv = s_mn[warp][tig][gi];
+    const float o0 = ((acc[mt][0] + acc[mt][1]) * inv_unit + mnv) * sc;
+    const float o1 = ((acc[mt][2] + acc[mt][3]) * inv_unit + mnv) * sc;
+    s_out[(warp * MG + tig) * MD + ch0] = o0;
+    s_out[(warp * MG + tig) * MD + ch1] = o1;
+  }
+  __syncthreads();
+  for (int i = tid; i < MG * MD; i += MT) {
+    const int hh = i / MD, ch = i % MD;
+    float o = 0.f;
+    for (int w = 0; w < 4; ++w) o += s_out[(w * MG + hh) * MD + ch];
+    p.ws.part_o[((int64_t)(bq0 + hh) * p.splits + split) * MD + ch] = o;
+  }
+  if (tid < MG) {
+    float M = -INFINITY, L = 0.f;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w][tid]);
+    if (M != -INFINITY)
+      for (int w = 0; w < 4; ++w)
+        if (s_m[w][tid] != -INFINITY) L += s_l[w][tid] * exp2f(s_m[w][tid] - M);
+    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 0] = M;
+    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 1] = L;
+  }
+}
+
+template <int B1, int KSQ>
+cudaError_t launch_partial_t(const MParams& p, cudaStream_t s) {
+  const size_t smem = (size_t)NST * p.g.block_bytes + sizeof(float) * 4 * MG * MD;
+  cudaError_t e = cudaFuncSetAttribute(k_decode_partial_mma<B1, KSQ>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)p.splits, (unsigned)(p.g.B * p.g.Hkv));
+  k_decode_partial_mma<B1, KSQ><<<grid, MT, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_mma_supported(const Geom& g, int G) {
+  return g.d == MD && G == MG && g.vbits == 2 && g.group == 32 && g.b1 <= 2 &&
+         (g.m == 64 || g.m == 128 || g.m == 256);
+}
+
+cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
+                                   const float* S, const float* cent, float scale,
+                                   const DecodeWs& ws, cudaStream_t s) {
+  const size_t smem = sizeof(float) * MG * (2 * g.d + g.m);
+  cudaError_t e = cudaFuncSetAttribute(k_decode_prep_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k_decode_prep_mma<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws,
+                                                   ws.frag, ws.qconst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
+                                      float scale, float* logits, int splits, const DecodeWs& ws,
+                                      cudaStream_t s) {
+  MParams p{};
+  p.g = g;
+  p.base = base;
+  p.n_total = n_total;
+  p.n_comp = n_total > g.W ? n_total - g.W : 0;
+  p.n_ring = (int)(n_total < g.W ? n_total : g.W);
+  p.Hq = Hq;
+  p.scale_log2 = scale * kLog2e;
+  p.logits = logits;
+  p.n_log = p.n_comp + p.n_ring;
+  const int64_t nblk = (p.n_comp + kBlockTokens - 1) / kBlockTokens;
+  p.splits = splits;
+  p.bps = (int)((nblk + splits - 1) / splits);
+  p.ws = ws;
+  p.err = ws.err;
+  const int ksq = g.m / 32;
+  switch (g.b1 * 16 + ksq) {
+    case 0 * 16 + 2: return launch_partial_t<0, 2>(p, s);
+    case 0 * 16 + 4: return launch_partial_t<0, 4>(p, s);
+    case 0 * 16 + 8: return launch_partial_t<0, 8>(p, s);
+    case 1 * 16 + 2: return launch_partial_t<1, 2>(p, s);
+    case 1 * 16 + 4: return launch_partial_t<1, 4>(p, s);
+    case 1 * 16 + 8: return launch_partial_t<1, 8>(p, s);
+    case 2 * 16 + 2: return launch_partial_t<2, 2>(p, s);
+    case 2 * 16 + 4: return launch_partial_t<2, 4>(p, s);
+    case 2 * 16 + 8: return launch_partial_t<2, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tq

@@ -63,15 +63,27 @@ cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const
 
 // ---- decode (decode_kernels.cu) ----
 struct DecodeWs {
-  float* qf;      // [B*Hq, d]   query in fp32
-  float* qr;      // [B*Hq, d]   Pi q
-  float* qs;      // [B*Hq, m]   sqrt(pi/2)/m * S q
-  float* part_o;  // [B*Hq, splits, d]
-  float* part_ml; // [B*Hq, splits, 2]
+  float* qf;        // [B*Hq, d]   query in fp32
+  float* qr;        // [B*Hq, d]   Pi q
+  float* qs;        // [B*Hq, m]   sqrt(pi/2)/m * S q
+  uint32_t* frag;   // [B*Hkv, ksteps, 2, 2, 32]  int8 query slices (tensor-core path)
+  float* qconst;    // [B*Hkv, 8, 4]  per-head logit constants (tensor-core path)
+  int* err;         // error flag set by a kernel whose bounded wait gave up
+  float* part_ml;   // [B*Hq, splits, 2]
+  float* part_o;    // [B*Hq, splits, d]
 };
 size_t decode_ws_bytes(const Geom& g, int Hq, int splits);
 DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits);
-int decode_auto_splits(const Geom& g, int64_t n_comp);
+int decode_auto_splits(const Geom& g, int G, int64_t n_comp);
+
+// tensor-core path (decode_mma.cu)
+bool decode_mma_supported(const Geom& g, int G);
+cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
+                                   const float* S, const float* cent, float scale,
+                                   const DecodeWs& ws, cudaStream_t s);
+cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
+                                      float scale, float* logits, int splits, const DecodeWs& ws,
+                                      cudaStream_t s);
 
 cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float* Pi,
                                const float* S, const DecodeWs& ws, cudaStream_t s);

@@ -80,7 +80,8 @@ def _load() -> ctypes.CDLL:
         "tq_decode_workspace_bytes": (SZ, [C, I, I]),
         "tq_decode_attention": (I, [C, P, I, F, P, P, P, P, P, I, P, SZ, P]),
         "tq_decode_attention_noalloc": (I, [C, P, I, F, P, P, P, P, P, I, P]),
-        "tq_decode_prep": (I, [C, P, I, P, P, I, P, SZ, P]),
+        "tq_decode_prep": (I, [C, P, I, F, P, P, P, I, P, SZ, P]),
+        "tq_decode_check": (I, [C, I, I, P, SZ, P]),
         "tq_decode_partial": (I, [C, I, F, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
@@ -210,10 +211,16 @@ def tq_decode_attention_noalloc(cache: tq_cache, Q, softmax_scale: float, Pi, S,
            "tq_decode_attention_noalloc")
 
 
-def tq_decode_prep(cache: tq_cache, Q, Pi, S, num_splits, workspace, stream=None):
-    _check(lib.tq_decode_prep(ctypes.byref(cache), _ptr(Q), Q.shape[1], _ptr(Pi), _ptr(S),
-                              num_splits, _ptr(workspace), _ws(workspace), _stream(stream)),
-           "tq_decode_prep")
+def tq_decode_prep(cache: tq_cache, Q, softmax_scale, Pi, S, centroids, num_splits, workspace,
+                   stream=None):
+    _check(lib.tq_decode_prep(ctypes.byref(cache), _ptr(Q), Q.shape[1], softmax_scale, _ptr(Pi),
+                              _ptr(S), _ptr(centroids), num_splits, _ptr(workspace),
+                              _ws(workspace), _stream(stream)), "tq_decode_prep")
+
+
+def tq_decode_check(cache: tq_cache, Hq, num_splits, workspace, stream=None):
+    _check(lib.tq_decode_check(ctypes.byref(cache), Hq, num_splits, _ptr(workspace),
+                               _ws(workspace), _stream(stream)), "tq_decode_check")
 
 
 def tq_decode_partial(cache: tq_cache, Hq, softmax_scale, centroids, logits, num_splits,

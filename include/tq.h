@@ -264,14 +264,28 @@ int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_
                         void* stream);
 
 /* The three stages of tq_decode_attention, for callers that time or overlap
- * them separately.  Same arguments and workspace as tq_decode_attention. */
-int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, const float* Pi, const float* S,
-                   int num_splits, void* workspace, size_t ws_bytes, void* stream);
+ * them separately.  Same arguments and workspace as tq_decode_attention; the
+ * preparation stage also takes the softmax scale and the centroids (the
+ * tensor-core path folds them into the query-side constants). */
+int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                   const float* Pi, const float* S, const float* centroids, int num_splits,
+                   void* workspace, size_t ws_bytes, void* stream);
 int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const float* centroids,
                       float* logits, int num_splits, void* workspace, size_t ws_bytes,
                       void* stream);
 int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void* workspace,
                       size_t ws_bytes, void* stream);
+
+/*
+ * tq_decode_check -- SYNCHRONOUS: waits for `stream`, then reports whether the
+ * last decode that used `workspace` completed its staged loads.  A decode
+ * kernel whose bounded wait on a shared-memory load gives up (it never should)
+ * skips its work and raises a flag instead of hanging; this call returns
+ * TQ_ERR_CUDA when the flag is set, TQ_OK otherwise.  Arguments as for
+ * tq_decode_attention.
+ */
+int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* workspace,
+                    size_t ws_bytes, void* stream);
 
 /*
  * tq_decode_attention_noalloc -- the same decode as tq_decode_attention, for

@@ -130,9 +130,10 @@ def _decode_identical_codes(w, n_tokens, capacity, num_splits=0, Hq=None):
 
 
 @pytest.mark.parametrize("n_tokens,splits", [(300, 0), (300, 1), (300, 3), (17, 0), (64 + 16, 2),
-                                             (1000, 7), (16, 0), (5, 0), (1, 0)])
+                                             (1000, 7), (16, 0), (5, 0), (1, 0), (2000, 0),
+                                             (4096 + 16 + 63, 5), (3000, 40)])
 def test_decode_identical_codes_lengths_and_splits(n_tokens, splits):
-    _decode_identical_codes(_workload(), n_tokens, 1024, splits)
+    _decode_identical_codes(_workload(), n_tokens, max(1024, n_tokens + 64), splits)
 
 
 @pytest.mark.parametrize("kw", [
@@ -143,6 +144,9 @@ def test_decode_identical_codes_lengths_and_splits(n_tokens, splits):
     dict(b1=1, m=96, vbits=4, dtype="f32"),
     dict(W=0, dtype="f32", B=1, Hq=4, Hkv=1, k_outlier_count=4, outlier_scale=10.0,
          k_outlier_frac=0.0, v_outlier_frac=0.0),                  # the tiny workload's shape
+    # shapes of the tensor-core path (d=128, G=4, 2-bit values g=32)
+    dict(m=256), dict(b1=1, m=64), dict(b1=0, m=128, dtype="f16"), dict(b1=0, m=256, W=3),
+    dict(B=3, Hkv=5, Hq=20, W=1),
 ])
 def test_decode_identical_codes_shapes(kw):
     w = _workload(**kw)
