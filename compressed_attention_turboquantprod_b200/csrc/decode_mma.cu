@@ -59,7 +59,7 @@ struct MParams {
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -68,7 +68,7 @@ __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1,
 
 __device__ __forceinline__ void hmma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -79,6 +79,39 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
+}
+
+// Integer multiply kept as a multiply (the FMA-pipe IMAD), used for shifts by a
+// per-lane amount so that they do not occupy the integer ALU pipe.
+__device__ __forceinline__ uint32_t mul_lo(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// n consecutive 32-bit words from 16-byte-aligned shared memory, widest loads.
+template <int N>
+__device__ __forceinline__ void lds_words(const unsigned char* p, uint32_t (&w)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (N % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const uint2 v = reinterpret_cast<const uint2*>(p)[i];
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  }
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -129,39 +162,73 @@ __device__ __forceinline__ float i2f_exact(int x) {
 // [kstep][ntile][reg][lane] (uint32) and per head {kM, CM, kQ, CQ} (float).
 
 // ---------------------------------------------------------------- prep
-// One CTA per (batch, KV head): the G queries in fp32 (for the ring), Pi q and
-// sqrt(pi/2)/m S q, the Walsh weights, their 21-bit fixed-point quantisation
-// and three int8 slices laid out as the lanes' B fragments, and the per-head
-// affine constants of the logit (already in log2 units of the softmax).
-__global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, int Hq,
-                                                         const float* Pi, const float* S,
-                                                         const float* cent, float scale_log2,
-                                                         DecodeWs ws, uint32_t* frag,
-                                                         float* qconst) {
+// (1) Projections of the queries, all (b, query head) at once: CTA (unit, chunk)
+// computes 32 output rows r of [Pi; S] (d + m rows) for the G = 4 queries of
+// one (b, KV head); each row is read once (one float4 per lane) and dotted with
+// the four queries.  qr = Pi q, qs = sqrt(pi/2)/m S q; chunk 0 also stores q.
+constexpr int PROJ_ROWS = 32;
+
+__global__ void __launch_bounds__(128) k_prep_proj(Geom g, const void* Q, int Hq, const float* Pi,
+                                                   const float* S, DecodeWs ws) {
+  __shared__ __align__(16) float sq[MG * 256];
+  const int unit = blockIdx.x, chunk = blockIdx.y;
+  const int b = unit / g.Hkv, h = unit % g.Hkv;
+  const int d = g.d, m = g.m;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bq0 = b * Hq + h * MG;
+  if (unit == 0 && chunk == 0 && tid == 0) *ws.err = 0;
+  for (int i = tid; i < MG * d; i += blockDim.x) {
+    const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
+    sq[i] = v;
+    if (chunk == 0) ws.qf[(int64_t)bq0 * d + i] = v;
+  }
+  __syncthreads();
+  const int rows_pi = g.b1 > 0 ? d : 0;
+  const float qscale = 1.2533141373155003f / (float)m;
+  for (int rr = warp; rr < PROJ_ROWS; rr += 4) {
+    const int r = chunk * PROJ_ROWS + rr;
+    if (r >= rows_pi + m) break;
+    const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
+    float acc[MG] = {0.f, 0.f, 0.f, 0.f};
+    for (int i0 = 4 * lane; i0 < d; i0 += 128) {
+      const float4 w = *reinterpret_cast<const float4*>(row + i0);
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh) {
+        const float4 q = *reinterpret_cast<const float4*>(sq + hh * d + i0);
+        acc[hh] = fmaf(w.x, q.x, fmaf(w.y, q.y, fmaf(w.z, q.z, fmaf(w.w, q.w, acc[hh]))));
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < MG; ++hh) acc[hh] = warp_sum(acc[hh]);
+    if (lane < MG) {
+      const float a = acc[0] * (lane == 0) + acc[1] * (lane == 1) + acc[2] * (lane == 2) + acc[3] * (lane == 3);
+      if (r < rows_pi) ws.qr[(int64_t)(bq0 + lane) * d + r] = a;
+      else ws.qs[(int64_t)(bq0 + lane) * m + (r - rows_pi)] = a * qscale;
+    }
+  }
+}
+
+// (2) One CTA per (b, KV head): the Walsh weights of the codebook, the 21-bit
+// fixed-point quantisation of the query weights, their three int8 slices laid
+// out as the lanes' B fragments, and the per-head affine constants of the
+// logit (in log2 units of the softmax).
+__global__ void __launch_bounds__(256) k_prep_frag(Geom g, int Hq, const float* cent,
+                                                   float scale_log2, DecodeWs ws) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int unit = blockIdx.x;
   const int b = unit / g.Hkv, h = unit % g.Hkv;
   const int d = g.d, m = g.m, b1 = g.b1;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* sq = reinterpret_cast<float*>(smem_raw);   // [G][d]
-  float* sqr = sq + MG * d;                          // [G][d]
-  float* sqs = sqr + MG * d;                         // [G][m]
-  __shared__ float s_w[4];                           // Walsh weights of the odd subsets
+  const int tid = threadIdx.x;
+  float* sqr = reinterpret_cast<float*>(smem_raw);   // [G][d]
+  float* sqs = sqr + MG * d;                          // [G][m]
+  __shared__ float s_w[4];                            // Walsh weights of the odd subsets
   __shared__ unsigned s_maxM[MG], s_maxQ[MG];
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
-  if (unit == 0 && tid == 0) *ws.err = 0;
-  for (int i = tid; i < MG * d; i += blockDim.x) {
-    const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
-    sq[i] = v;
-    ws.qf[(int64_t)bq0 * d + i] = v;
-  }
-  if (tid < MG) {
-    s_maxM[tid] = 0u;
-    s_maxQ[tid] = 0u;
-    s_sumqr[tid] = 0.f;
-    s_sumqs[tid] = 0.f;
-  }
+  const int F = b1 > 0 ? 1 << (b1 - 1) : 0;     // feature planes per coordinate
+  if (F)
+    for (int i = tid; i < MG * d; i += blockDim.x) sqr[i] = ws.qr[(int64_t)bq0 * d + i];
+  for (int i = tid; i < MG * m; i += blockDim.x) sqs[i] = ws.qs[(int64_t)bq0 * m + i];
   if (tid == 0) {
     // w_S = (1/L) sum_idx c[idx] (-1)^{popc(idx & S)} for the odd subsets S, in the
     // order of the feature planes: {0}, {1}, {2}, {0,1,2}.
@@ -175,36 +242,38 @@ __global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, 
     }
   }
   __syncthreads();
-  const float qscale = 1.2533141373155003f / (float)m;
-  const int rows_pi = b1 > 0 ? d : 0;
-  for (int r = warp; r < MG * (rows_pi + m); r += blockDim.x / 32) {
-    const int hh = r / (rows_pi + m), rr = r % (rows_pi + m);
-    const float* row = rr < rows_pi ? Pi + (int64_t)rr * d : S + (int64_t)(rr - rows_pi) * d;
-    float a = 0.f;
-    for (int i = lane; i < d; i += 32) a = fmaf(row[i], sq[hh * d + i], a);
-    a = warp_sum(a);
+  {
+    // warps 0-3: MSE weights of head w (max |W|, sum qr); warps 4-7: QJL of head w-4
+    const int warp = tid >> 5, lane = tid & 31;
+    const int hh = warp & 3;
+    float mx = 0.f, sm = 0.f;
+    if (warp < 4) {
+      float wk = 0.f;
+      for (int k = 0; k < F; ++k) wk = fmaxf(wk, fabsf(2.f * s_w[k]));
+      if (F)
+        for (int j = lane; j < d; j += 32) {
+          const float qr = sqr[hh * d + j];
+          mx = fmaxf(mx, wk * fabsf(qr));
+          sm += qr;
+        }
+    } else {
+      for (int i = lane; i < m; i += 32) {
+        const float qs = sqs[hh * m + i];
+        mx = fmaxf(mx, fabsf(2.f * qs));
+        sm += qs;
+      }
+    }
+    mx = warp_max(mx);
+    sm = warp_sum(sm);
     if (lane == 0) {
-      if (rr < rows_pi) sqr[hh * d + rr] = a;
-      else sqs[hh * m + (rr - rows_pi)] = a * qscale;
+      if (warp < 4) {
+        s_maxM[hh] = __float_as_uint(mx);
+        s_sumqr[hh] = sm;
+      } else {
+        s_maxQ[hh] = __float_as_uint(mx);
+        s_sumqs[hh] = sm;
+      }
     }
-  }
-  __syncthreads();
-  const int F = b1 > 0 ? 1 << (b1 - 1) : 0;     // feature planes per coordinate
-  // maxima of |W| and the plain sums, per head
-  for (int i = tid; i < MG * d; i += blockDim.x) {
-    const int hh = i / d;
-    const float qr = sqr[i];
-    float wmax = 0.f;
-    for (int k = 0; k < F; ++k) wmax = fmaxf(wmax, fabsf(2.f * s_w[k] * qr));
-    if (F) {
-      atomicMax(&s_maxM[hh], __float_as_uint(wmax));
-      atomicAdd(&s_sumqr[hh], qr);
-    }
-  }
-  for (int i = tid; i < MG * m; i += blockDim.x) {
-    const int hh = i / m;
-    atomicMax(&s_maxQ[hh], __float_as_uint(fabsf(2.f * sqs[i])));
-    atomicAdd(&s_sumqs[hh], sqs[i]);
   }
   __syncthreads();
   const float two21 = 2097152.f;
@@ -213,16 +282,15 @@ __global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, 
     const float dM = mM > 0.f ? mM / two21 : 1.f, dQ = mQ > 0.f ? mQ / two21 : 1.f;
     float wsum = 0.f;
     for (int k = 0; k < F; ++k) wsum += s_w[k];
-    float* c = qconst + ((int64_t)unit * MG + tid) * 4;
+    float* c = ws.qconst + ((int64_t)unit * MG + tid) * 4;
     c[0] = dM / 128.f * scale_log2;
     c[1] = wsum * s_sumqr[tid] * scale_log2;
     c[2] = dQ / 128.f * scale_log2;
     c[3] = -s_sumqs[tid] * scale_log2;
   }
-  // fragment words
   const int ksM = F * d / 32, ksQ = m / 32;
   const int words = (ksM + ksQ) * 2 * 2 * 32;
-  uint32_t* fr = frag + (int64_t)unit * words;
+  uint32_t* fr = ws.frag + (int64_t)unit * words;
   for (int wi = tid; wi < words; wi += blockDim.x) {
     const int ln = wi & 31, r = (wi >> 5) & 1, nt = (wi >> 6) & 1, ks = wi >> 7;
     const int col = ln >> 2, tg = ln & 3;
@@ -232,7 +300,7 @@ __global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, 
     if (slice >= 0) {
       const bool mse = ks < ksM;
       const float mx = __uint_as_float(mse ? s_maxM[hh] : s_maxQ[hh]);
-      const float delta = mx > 0.f ? mx / two21 : 1.f;
+      const float inv_delta = mx > 0.f ? two21 / mx : 1.f;
       for (int i = 0; i < 4; ++i) {
         const int bit = tg + 8 * i + (r ? 4 : 0);
         float w;
@@ -242,7 +310,7 @@ __global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, 
         } else {
           w = 2.f * sqs[hh * m + (ks - ksM) * 32 + bit];
         }
-        const int wint = __float2int_rn(w / delta);
+        const int wint = __float2int_rn(w * inv_delta);
         const int s0 = ((wint + 128) & 255) - 128;
         const int t1 = (wint - s0) >> 8;
         const int s1 = ((t1 + 128) & 255) - 128;
@@ -257,7 +325,7 @@ __global__ void __launch_bounds__(256) k_decode_prep_mma(Geom g, const void* Q, 
 
 // ---------------------------------------------------------------- partial
 template <int B1, int KSQ>
-__global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
+__global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   constexpr int F = B1 > 0 ? 1 << (B1 - 1) : 0;
   constexpr int KSM = F * MD / 32;
   constexpr int KS = KSM + KSQ;
@@ -266,6 +334,8 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
   __shared__ int s_abort;
   __shared__ float s_m[4][MG], s_l[4][MG];
   __shared__ float s_mn[4][MG][4];
+  __shared__ int s_cnt[NST];
+  __shared__ __align__(16) uint32_t s_frag[KS * 128];
 
   const Geom& g = p.g;
   const int split = blockIdx.x, unit = blockIdx.y;
@@ -293,20 +363,20 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
     }
   }
 
-  // B fragments of the score (query slices) in registers
-  uint32_t bf[KS][2][2];
+  // B fragments of the score (query slices), per k-step and lane four words
+  // {ntile0 r0, ntile0 r1, ntile1 r0, ntile1 r1}, staged in shared memory.
   {
     const uint32_t* fr = p.ws.frag + (int64_t)unit * (KS * 128);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) bf[ks][nt][r] = fr[((ks * 2 + nt) * 2 + r) * 32 + lane];
+    for (int i = tid; i < KS * 128; i += MT) {
+      const int ln = i & 31, r = (i >> 5) & 1, nt = (i >> 6) & 1, ks = i >> 7;
+      s_frag[(ks * 32 + ln) * 4 + nt * 2 + r] = fr[i];
+    }
   }
   const float* qc = p.ws.qconst + ((int64_t)unit * MG + tig) * 4;
   const float kM = qc[0], CM = qc[1], kQ = qc[2], CQ = qc[3];
+  if (tid < NST) s_cnt[tid] = 0;
   __syncthreads();
+  const uint4* bfr = reinterpret_cast<const uint4*>(s_frag) + lane;
 
   const uint32_t mulA = 1u << (7 - tig), mulB = 1u << (3 - tig);
   const uint32_t codeMask = 0x00030003u << (2 * (gid & 3));
@@ -324,31 +394,27 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
     for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
   float mnacc[4] = {0.f, 0.f, 0.f, 0.f};
   const bool odd = (gid & 1) != 0;
+  const float oddf = odd ? 1.f : 0.f;
   const int hP = gid >> 1;
 
   // One 16-token step of this warp: logits l0 (token row gid) / l1 (row gid+8) for
-  // head tig are given; update the softmax state and return p0, p1.
+  // head tig are given; returns p0, p1 relative to the running max of the head.
+  // The running max is raised (with a reduction over the warp and a rescale of
+  // the accumulators) only when a logit exceeds it by more than kLazy (log2
+  // units), so p <= 2^kLazy; the running sum is kept per lane and reduced once.
+  constexpr float kLazy = 4.f;
   auto softmax_step = [&](float l0, float l1, float& p0, float& p1) {
-    float mx = fmaxf(l0, l1);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    const float m_new = fmaxf(m_run, mx);
-    float alpha = 1.f;
-    p0 = 0.f;
-    p1 = 0.f;
-    if (m_new != -INFINITY) {
-      alpha = exp2f(m_run - m_new);
-      p0 = exp2f(l0 - m_new);
-      p1 = exp2f(l1 - m_new);
-    }
-    float s = p0 + p1;
-    s += __shfl_xor_sync(0xffffffffu, s, 4);
-    s += __shfl_xor_sync(0xffffffffu, s, 8);
-    s += __shfl_xor_sync(0xffffffffu, s, 16);
-    l_run = l_run * alpha + s;
-    m_run = m_new;
-    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+    const float lmax = fmaxf(l0, l1);
+    if (__any_sync(0xffffffffu, lmax > m_run + kLazy)) {
+      float mx = lmax;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_run, mx);
+      const float alpha = (m_run == -INFINITY) ? (m_new == -INFINITY ? 1.f : 0.f)
+                                               : exp2f(m_run - m_new);
+      m_run = m_new;
+      l_run *= alpha;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -357,9 +423,16 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) mnacc[gi] *= aP;
     }
+    if (m_run == -INFINITY) {
+      p0 = 0.f;
+      p1 = 0.f;
+    } else {
+      p0 = exp2f(l0 - m_run);
+      p1 = exp2f(l1 - m_run);
+    }
+    l_run += p0 + p1;
   };
 
-  int issued = nb < NST ? nb : NST;     // loads issued by thread 0
   int it = 0;
   for (; it < nb; ++it) {
     const int st = it % NST;
@@ -379,32 +452,36 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
 
     // ---------------- logits
     float vM0 = 0.f, vM1 = 0.f, vQ0 = 0.f, vQ1 = 0.f;
-    if (KSM > 0) {
-      int a[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-      const uint32_t* w0p = reinterpret_cast<const uint32_t*>(blk + g.o_idx + t0 * (B1 * MD / 8));
-      const uint32_t* w1p = reinterpret_cast<const uint32_t*>(blk + g.o_idx + t1 * (B1 * MD / 8));
+    if constexpr (KSM > 0) {
+      uint32_t w0[KSM], w1[KSM];
+      lds_words<KSM>(blk + g.o_idx + t0 * (KSM * 4), w0);
+      lds_words<KSM>(blk + g.o_idx + t1 * (KSM * 4), w1);
+      int a[2][2][4] = {};   // [parity][ntile][4]: two independent chains per ntile
 #pragma unroll
       for (int ks = 0; ks < KSM; ++ks) {
-        const uint32_t w0 = w0p[ks], w1 = w1p[ks];
-        const uint32_t a0 = (w0 * mulA) & 0x80808080u, a1 = (w1 * mulA) & 0x80808080u;
-        const uint32_t a2 = (w0 * mulB) & 0x80808080u, a3 = (w1 * mulB) & 0x80808080u;
-        imma16832(a[0], a0, a1, a2, a3, bf[ks][0][0], bf[ks][0][1]);
-        imma16832(a[1], a0, a1, a2, a3, bf[ks][1][0], bf[ks][1][1]);
+        const uint32_t a0 = mul_lo(w0[ks], mulA) & 0x80808080u, a1 = mul_lo(w1[ks], mulA) & 0x80808080u;
+        const uint32_t a2 = mul_lo(w0[ks], mulB) & 0x80808080u, a3 = mul_lo(w1[ks], mulB) & 0x80808080u;
+        const uint4 bq = bfr[ks * 32];
+        imma16832(a[ks & 1][0], a0, a1, a2, a3, bq.x, bq.y);
+        imma16832(a[ks & 1][1], a0, a1, a2, a3, bq.z, bq.w);
       }
-      vM0 = i2f_exact(a[0][0]) + 256.f * i2f_exact(a[0][1]) + 65536.f * i2f_exact(a[1][0]);
-      vM1 = i2f_exact(a[0][2]) + 256.f * i2f_exact(a[0][3]) + 65536.f * i2f_exact(a[1][2]);
+      int s00 = a[0][0][0] + a[1][0][0], s01 = a[0][0][1] + a[1][0][1], s10 = a[0][1][0] + a[1][1][0];
+      int s02 = a[0][0][2] + a[1][0][2], s03 = a[0][0][3] + a[1][0][3], s12 = a[0][1][2] + a[1][1][2];
+      vM0 = i2f_exact(s00) + 256.f * i2f_exact(s01) + 65536.f * i2f_exact(s10);
+      vM1 = i2f_exact(s02) + 256.f * i2f_exact(s03) + 65536.f * i2f_exact(s12);
     }
     {
-      int a[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-      const uint32_t* w0p = reinterpret_cast<const uint32_t*>(blk + g.o_sign + t0 * (KSQ * 4));
-      const uint32_t* w1p = reinterpret_cast<const uint32_t*>(blk + g.o_sign + t1 * (KSQ * 4));
+      uint32_t w0[KSQ], w1[KSQ];
+      lds_words<KSQ>(blk + g.o_sign + t0 * (KSQ * 4), w0);
+      lds_words<KSQ>(blk + g.o_sign + t1 * (KSQ * 4), w1);
+      int a[2][4] = {};
 #pragma unroll
       for (int ks = 0; ks < KSQ; ++ks) {
-        const uint32_t w0 = w0p[ks], w1 = w1p[ks];
-        const uint32_t a0 = (w0 * mulA) & 0x80808080u, a1 = (w1 * mulA) & 0x80808080u;
-        const uint32_t a2 = (w0 * mulB) & 0x80808080u, a3 = (w1 * mulB) & 0x80808080u;
-        imma16832(a[0], a0, a1, a2, a3, bf[KSM + ks][0][0], bf[KSM + ks][0][1]);
-        imma16832(a[1], a0, a1, a2, a3, bf[KSM + ks][1][0], bf[KSM + ks][1][1]);
+        const uint32_t a0 = mul_lo(w0[ks], mulA) & 0x80808080u, a1 = mul_lo(w1[ks], mulA) & 0x80808080u;
+        const uint32_t a2 = mul_lo(w0[ks], mulB) & 0x80808080u, a3 = mul_lo(w1[ks], mulB) & 0x80808080u;
+        const uint4 bq = bfr[(KSM + ks) * 32];
+        imma16832(a[0], a0, a1, a2, a3, bq.x, bq.y);
+        imma16832(a[1], a0, a1, a2, a3, bq.z, bq.w);
       }
       vQ0 = i2f_exact(a[0][0]) + 256.f * i2f_exact(a[0][1]) + 65536.f * i2f_exact(a[1][0]);
       vQ1 = i2f_exact(a[0][2]) + 256.f * i2f_exact(a[0][3]) + 65536.f * i2f_exact(a[1][2]);
@@ -451,22 +528,16 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
       const float mc[4] = {mC.x, mC.y, mC.z, mC.w}, mdd[4] = {mD.x, mD.y, mD.z, mD.w};
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
-        const float xA = pA != 0.f ? pA * sa[gi] : 0.f, xB = pB != 0.f ? pB * sb[gi] : 0.f;
-        const float xC = pC != 0.f ? pC * sc[gi] : 0.f, xD = pD != 0.f ? pD * sd[gi] : 0.f;
-        __half2 h0 = __floats2half2_rn(xA, xB), h1 = __floats2half2_rn(xC, xD);
-        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-        const __half2 l0h = __floats2half2_rn(xA - f0.x, xB - f0.y);
-        const __half2 l1h = __floats2half2_rn(xC - f1.x, xD - f1.y);
-        h0 = odd ? l0h : h0;
-        h1 = odd ? l1h : h1;
+        // tokens past the end have p = 0 and finite (zeroed or earlier) metadata
+        const float xA = pA * sa[gi], xB = pB * sb[gi], xC = pC * sc[gi], xD = pD * sd[gi];
+        // column gid even carries fp16(x), odd carries fp16(x - fp16(x))
+        const float2 f0 = __half22float2(__floats2half2_rn(xA, xB));
+        const float2 f1 = __half22float2(__floats2half2_rn(xC, xD));
+        __half2 h0 = __floats2half2_rn(fmaf(-oddf, f0.x, xA), fmaf(-oddf, f0.y, xB));
+        __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
         bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
         bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
-        float mnv = 0.f;
-        if (pA != 0.f) mnv = fmaf(pA, ma[gi], mnv);
-        if (pB != 0.f) mnv = fmaf(pB, mb[gi], mnv);
-        if (pC != 0.f) mnv = fmaf(pC, mc[gi], mnv);
-        if (pD != 0.f) mnv = fmaf(pD, mdd[gi], mnv);
-        mnacc[gi] += mnv;
+        mnacc[gi] = fmaf(pA, ma[gi], fmaf(pB, mb[gi], fmaf(pC, mc[gi], fmaf(pD, mdd[gi], mnacc[gi]))));
       }
     }
     {
@@ -487,19 +558,32 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
       }
     }
     }  // ok
-    __syncthreads();
-    if (s_abort) break;
-    if (tid == 0 && it + NST < nb) {
-      mbar_expect_tx(&full[st], (uint32_t)bb);
-      bulk_load(stage + (size_t)st * bb, region + (blk0 + it + NST) * bb, (uint32_t)bb, &full[st]);
-      ++issued;
+    // Release the stage: the last of the four warps to finish it refills it.
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      const int done = atomicAdd(&s_cnt[st], 1);
+      if (done == 3) {
+        __threadfence_block();
+        s_cnt[st] = 0;
+        if (it + NST < nb && !s_abort) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_expect_tx(&full[st], (uint32_t)bb);
+          bulk_load(stage + (size_t)st * bb, region + (blk0 + it + NST) * bb, (uint32_t)bb,
+                    &full[st]);
+        }
+      }
     }
+    if (*((volatile int*)&s_abort)) break;
   }
+  __syncthreads();
 
   if (s_abort) {
-    // a wait gave up: wait (bounded) for this CTA's copies still in flight, then leave
+    // a wait gave up: wait (bounded) for every copy this CTA may still have in
+    // flight (at most the last NST blocks), then leave
     if (tid == 0)
-      for (int j = it; j < issued; ++j) (void)mbar_wait(&full[j % NST], (uint32_t)((j / NST) & 1));
+      for (int j = (nb > NST ? nb - NST : 0); j < nb; ++j)
+        (void)mbar_wait(&full[j % NST], (uint32_t)((j / NST) & 1));
     return;
   }
 
@@ -548,6 +632,9 @@ __global__ void __launch_bounds__(MT) k_decode_partial_mma(MParams p) {
   }
 
   // ---------------- merge the 4 warps
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
   if (gid == 0) {
     s_m[warp][tig] = m_run;
     s_l[warp][tig] = l_run;
@@ -614,12 +701,15 @@ bool decode_mma_supported(const Geom& g, int G) {
 cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
                                    const float* S, const float* cent, float scale,
                                    const DecodeWs& ws, cudaStream_t s) {
-  const size_t smem = sizeof(float) * MG * (2 * g.d + g.m);
-  cudaError_t e = cudaFuncSetAttribute(k_decode_prep_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const int rows = (g.b1 > 0 ? g.d : 0) + g.m;
+  dim3 grid((unsigned)(g.B * g.Hkv), (unsigned)((rows + PROJ_ROWS - 1) / PROJ_ROWS));
+  k_prep_proj<<<grid, 128, 0, s>>>(g, Q, Hq, Pi, S, ws);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_decode_prep_mma<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws,
-                                                   ws.frag, ws.qconst);
+  const size_t smem = sizeof(float) * MG * (g.d + g.m);
+  e = cudaFuncSetAttribute(k_prep_frag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_prep_frag<<<g.B * g.Hkv, 256, smem, s>>>(g, Hq, cent, scale * kLog2e, ws);
   return cudaGetLastError();
 }
 

@@ -353,10 +353,161 @@ __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V
   }
 }
 
+// One CTA per token, for launches with only a few tokens per (b, kv head) (the
+// decode step appends one): the same arithmetic as the 64-token tile, with the
+// matrix-vector products done warp-per-row (lanes over the inner dimension).
+constexpr int SMALL_THREADS = 128;
+
+__global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int d = p.d, m = p.m, b1 = p.b1;
+  float* sx = reinterpret_cast<float*>(smem_raw);       // [d]
+  float* sy = sx + d;                                    // [d]  e = y - c[idx]
+  float* sz = sy + d;                                    // [max(m, 32)]
+  __shared__ double s_red[SMALL_THREADS / 32];
+  __shared__ double s_rho;
+  __shared__ float s_cb[32];
+  const int bh = blockIdx.y;
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = SMALL_THREADS / 32;
+  if (tid < 16) {
+    const int L = b1 > 0 ? (1 << b1) : 0;
+    s_cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
+    s_cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
+  }
+  if (p.do_keys) {
+    int64_t e0;
+    const void* src = src_row(p, false, bh, row, e0);
+    double ss = 0.0;
+    for (int c = tid; c < d; c += SMALL_THREADS) {
+      const float v = load_f(src, e0 + c, p.dtype);
+      sx[c] = v;
+      ss += (double)v * (double)v;
+    }
+    ss = warp_sum_d(ss);
+    if (lane == 0) s_red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < NW; ++w) t += s_red[w];
+      s_rho = sqrt(t);
+    }
+    __syncthreads();
+    const double rho64 = s_rho;
+    const float rho = (float)rho64;
+    const float inv = rho64 > 0.0 ? (float)(1.0 / rho64) : 0.f;
+    const float* E = sx;
+    // thread-per-row matrix-vector products: each thread streams its own row as
+    // float4 (independent loads, the vector is a shared-memory broadcast)
+    if (b1 > 0) {
+      const int L = 1 << b1;
+      uint8_t* idx_dst = dst_field(p, bh, row, 0);
+      double se = 0.0;
+      for (int j = tid; j < d; j += SMALL_THREADS) {
+        const float4* rp = reinterpret_cast<const float4*>(p.Pi + (int64_t)j * d);
+        float a = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < d / 4; ++i) {
+          const float4 w = rp[i];
+          a = fmaf(w.x, sx[4 * i], a);
+          a = fmaf(w.y, sx[4 * i + 1], a);
+          a = fmaf(w.z, sx[4 * i + 2], a);
+          a = fmaf(w.w, sx[4 * i + 3], a);
+        }
+        const float y = a * inv;
+        int idx = 0;
+        for (int k = 0; k + 1 < L; ++k) idx += (s_cb[16 + k] < y) ? 1 : 0;
+        const float e = y - s_cb[idx];
+        sy[j] = e;
+        se += (double)e * (double)e;
+        for (int pl = 0; pl < b1; ++pl) {
+          const unsigned word = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
+          if (lane == 0) *reinterpret_cast<uint32_t*>(idx_dst + pl * (d / 8) + (j - lane) / 8) = word;
+        }
+      }
+      se = warp_sum_d(se);
+      if (lane == 0) s_red[warp] = se;
+      __syncthreads();
+      if (tid == 0) {
+        double t = 0.0;
+        for (int w = 0; w < NW; ++w) t += s_red[w];
+        *reinterpret_cast<float*>(dst_field(p, bh, row, 3)) = (float)(rho64 * sqrt(t));
+      }
+      E = sy;
+    }
+    uint8_t* sdst = dst_field(p, bh, row, 1);
+    for (int a = tid; a < m; a += SMALL_THREADS) {
+      const float4* rp = reinterpret_cast<const float4*>(p.T + (int64_t)a * d);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < d / 4; ++i) {
+        const float4 w = rp[i];
+        acc = fmaf(w.x, E[4 * i], acc);
+        acc = fmaf(w.y, E[4 * i + 1], acc);
+        acc = fmaf(w.z, E[4 * i + 2], acc);
+        acc = fmaf(w.w, E[4 * i + 3], acc);
+      }
+      const float z = (b1 > 0) ? acc * rho : acc;
+      const unsigned word = __ballot_sync(0xffffffffu, z >= 0.f);
+      if (lane == 0) *reinterpret_cast<uint32_t*>(sdst + (a - lane) / 8) = word;
+    }
+    if (tid == 0) *reinterpret_cast<float*>(dst_field(p, bh, row, 2)) = rho;
+    __syncthreads();
+  }
+  if (p.do_values) {
+    const int g = p.group, ng = d / g, vb = p.vbits;
+    const float levels = (float)((1 << vb) - 1);
+    int64_t e0;
+    const void* src = src_row(p, true, bh, row, e0);
+    for (int c = tid; c < d; c += SMALL_THREADS) sx[c] = load_f(src, e0 + c, p.dtype);
+    __syncthreads();
+    float* vs = sz;            // [ng] scales, [ng] minima (reuses the sketch buffer)
+    float* vm = sz + 16;
+    for (int gi = tid; gi < ng; gi += SMALL_THREADS) {
+      float mn = FLT_MAX, mx = -FLT_MAX;
+      for (int k = 0; k < g; ++k) {
+        const float v = sx[gi * g + k];
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+      }
+      const float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
+      vs[gi] = sc;
+      vm[gi] = mn;
+      reinterpret_cast<float*>(dst_field(p, bh, row, 5))[gi] = sc;
+      reinterpret_cast<float*>(dst_field(p, bh, row, 6))[gi] = mn;
+    }
+    __syncthreads();
+    const int per_word = 32 / vb, wpr = d / per_word;
+    for (int w = tid; w < wpr; w += SMALL_THREADS) {
+      uint32_t word = 0;
+      for (int k = 0; k < per_word; ++k) {
+        const int ch = w * per_word + k;
+        const float sc = vs[ch / g], mn = vm[ch / g];
+        uint32_t code = 0;
+        if (sc != 0.f) {
+          float q = rintf(__fdiv_rn(__fsub_rn(sx[ch], mn), sc));
+          q = fminf(fmaxf(q, 0.f), levels);
+          code = (uint32_t)q;
+        }
+        word |= code << (k * vb);
+      }
+      reinterpret_cast<uint32_t*>(dst_field(p, bh, row, 4))[w] = word;
+    }
+  }
+}
+
 }  // namespace
 
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
+  if (p.n <= 8) {
+    // a few tokens per (b, kv head): one CTA per token
+    const size_t smem = sizeof(float) * (2 * p.d + (p.m > 32 ? p.m : 32));
+    dim3 grid((unsigned)p.n, (unsigned)bh_count);
+    k_quantize_small<<<grid, SMALL_THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+  }
   const size_t smem = smem_bytes(p.d);
   cudaError_t e = cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
