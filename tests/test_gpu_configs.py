@@ -1,0 +1,164 @@
+"""Full-size parity for the five workloads, on sampled (batch, KV head) units.
+
+The library runs every workload at its full size, in the launch configuration
+of the bench (automatic split count); the oracle recomputes sampled units one
+by one from the same input tensors:
+  * packed fields of the unit's region: codes/signs bit-exact outside the
+    boundary band, value fields bit-exact, norms within tolerance;
+  * decode outputs of the unit's query heads within 2e-3 (+ storage rounding);
+  * logits given identical codes: the unit's region is overwritten with the
+    oracle's bytes and decoded with the oracle's projections.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_common import (TORCH_DT, check_logits, check_out, compare_keys, host, oracle_setup,
+                        to_dev)
+from oracle import cache as ocache
+from oracle import layout as olayout
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+class _Proj:
+    def __init__(self, po):
+        self.Pi, self.S, self.T = to_dev(po["Pi"]), to_dev(po["S"]), to_dev(po["T"])
+
+
+class _Cb:
+    def __init__(self, cb):
+        self.centroids, self.boundaries = to_dev(cb[0]), to_dev(cb[1])
+
+
+def _unit_oracle(w, K1, V1, po, cb, chunk=32768):
+    """Oracle cache of one (batch, KV head) unit fed the same tokens (in chunks,
+    which the append semantics make identical to one shot)."""
+    oc = ocache.OracleCache(1, 1, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T, w.dtype, po,
+                            cb if w.b1 else None)
+    for t in range(0, K1.shape[0], chunk):
+        oc.append(K1[None, None, t:t + chunk], V1[None, None, t:t + chunk])
+    return oc
+
+
+def _region(cache, b, h):
+    st = cache.state
+    off = (b * cache.desc.Hkv + h) * st.region_bytes
+    return cache.buffer[off:off + st.region_bytes].cpu().numpy()
+
+
+def _check_region(cache, b, h, oc):
+    """GPU region (b, h) vs the oracle unit's region, field by field."""
+    lay = oc.lay
+    gpu = _region(cache, b, h)
+    ref = oc.to_bytes()[:lay.region_bytes]
+    if np.array_equal(gpu, ref):
+        return 0
+    r = oc.rec[0][0]
+    n = r["rho"].shape[0]
+    buf = np.zeros(lay.total_bytes, np.uint8)
+    buf[:lay.region_bytes] = gpu
+    fg = olayout.read_region(buf, lay, 0, 0, n)
+    fr = olayout.read_region(oc.to_bytes(), lay, 0, 0, n)
+    for name in ("vcode", "vscale", "vmin"):
+        assert np.array_equal(fg[name], fr[name]), name
+    got = {"idx": fg["idx"], "signs": fg["sign"],
+           "rho": np.ascontiguousarray(fg["rho"]).view("<f4").ravel(),
+           "rnorm": np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel() if oc.b1 else None}
+    st = compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None)
+    return st["skipped_tokens"]
+
+
+def _run_workload(w, layer, units, check_identical=True):
+    from compressed_attention_turboquantprod_b200 import Codebook, CompressedKVCache, Projections
+    m = w.m_for_layer(layer)
+    w = w.scaled(m=m)
+    K, V = synth.keys_values(w, layer=layer, device="cuda")
+    Q = synth.queries(w, layer=layer, device="cuda")
+    pj = Projections(w.d, m, layer, rotation=w.b1 > 0)
+    cbg = Codebook(w.d, w.b1) if w.b1 else None
+    cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, m, w.vbits, w.group, w.W, w.T,
+                              dtype=TORCH_DT[w.dtype])
+    cache.append(K, V, pj, cbg)
+    out = cache.decode(Q, pj, cbg)
+    torch.cuda.synchronize()
+    po, cb = oracle_setup(w.d, w.b1, m, layer)
+    G = w.Hq // w.Hkv
+    units_data = {}
+    for (b, h) in units:
+        K1, V1 = host(K[b, h]), host(V[b, h])
+        oc = _unit_oracle(w, K1, V1, po, cb)
+        skipped = _check_region(cache, b, h, oc)
+        assert skipped <= max(2, w.T // 1000)
+        ro, _ = oc.decode(host(Q[b:b + 1, h * G:(h + 1) * G]))
+        check_out(host(out[b:b + 1, h * G:(h + 1) * G]), ro, w.dtype)
+        units_data[(b, h)] = oc
+    del K, V
+    gc.collect()
+    torch.cuda.empty_cache()
+    if check_identical:
+        # logits given identical codes: oracle bytes into the unit's region and ring
+        proj_o = _Proj(po)
+        cb_o = _Cb(cb) if w.b1 else None
+        for (b, h), oc in units_data.items():
+            ref = oc.to_bytes()
+            lay = oc.lay
+            st = cache.state
+            off = (b * cache.desc.Hkv + h) * st.region_bytes
+            cache.buffer[off:off + st.region_bytes].copy_(torch.from_numpy(ref[:lay.region_bytes]))
+            rs = w.W * w.d * (4 if w.dtype == "f32" else 2)
+            if rs:
+                u = b * w.Hkv + h
+                cache.buffer[st.ring_k_off + u * rs: st.ring_k_off + (u + 1) * rs].copy_(
+                    torch.from_numpy(ref[lay.ring_k_off:lay.ring_k_off + rs]))
+                cache.buffer[st.ring_v_off + u * rs: st.ring_v_off + (u + 1) * rs].copy_(
+                    torch.from_numpy(ref[lay.ring_v_off:lay.ring_v_off + rs]))
+        out2, logits = cache.decode(Q, proj_o, cb_o, want_logits=True)
+        torch.cuda.synchronize()
+        for (b, h), oc in units_data.items():
+            ro, rl = oc.decode(host(Q[b:b + 1, h * G:(h + 1) * G]))
+            check_logits(logits[b, h * G:(h + 1) * G].cpu().numpy().astype(np.float64), rl[(0, 0)])
+            check_out(host(out2[b:b + 1, h * G:(h + 1) * G]), ro, w.dtype)
+    del cache
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_tiny_full():
+    _run_workload(synth.WORKLOADS["tiny"], 0, [(0, 0)])
+
+
+def test_gqa32k_full_size_sampled_units():
+    _run_workload(synth.WORKLOADS["gqa32k"], 0, [(0, 0), (7, 7)])
+
+
+def test_quant_workload_bit_exact_cache_across_chunks():
+    """131072 tokens x 8 KV heads appended in chunks of 4096: the packed cache of
+    sampled heads equals the oracle's one-shot quantisation."""
+    from compressed_attention_turboquantprod_b200 import Codebook, CompressedKVCache, Projections
+    w = synth.WORKLOADS["quant"]
+    K, V = synth.keys_values(w, device="cuda")
+    pj, cbg = Projections(w.d, w.m, 0), Codebook(w.d, w.b1)
+    cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
+                              dtype=TORCH_DT[w.dtype])
+    for t in range(0, w.T, w.chunk):
+        cache.append(K[:, :, t:t + w.chunk].contiguous(), V[:, :, t:t + w.chunk].contiguous(),
+                     pj, cbg)
+    torch.cuda.synchronize()
+    assert cache.n_comp == w.T
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    for h in (0, 5):
+        oc = _unit_oracle(w, host(K[0, h]), host(V[0, h]), po, cb)
+        assert _check_region(cache, 0, h, oc) <= max(2, w.T // 1000)
+
+
+@pytest.mark.parametrize("layer", [0, 8, 16, 24, 31])
+def test_aqjl_layer_groups_full_size(layer):
+    _run_workload(synth.WORKLOADS["aqjl"], layer, [(3, 2)])
+
+
+def test_wide_full_size_sampled_unit():
+    _run_workload(synth.WORKLOADS["wide"], 0, [(1, 3)])
