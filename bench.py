@@ -6,7 +6,8 @@ workload (batch 8, 32 query heads over 8 KV heads, d=128, context 32768, bf16,
 16-token ring, 3-bit keys b1=2 + m=128, 2-bit values g=32):
     tq_append (1 new token per sequence: the oldest ring token is quantised
                into the packed cache, the new one enters the ring)
-    tq_decode_prep -> tq_decode_partial (split-K) -> tq_decode_combine.
+    tq_decode_prep -> tq_decode_partial (split-K; the last split of each
+               (batch, KV head) merges the splits into the output).
 Inputs are resident in HBM before timing; L2 is flushed (256 MB write) between
 steps, outside the timed events.  `value` is algorithmic bytes (packed cache +
 ring + append traffic) per second.  Also reported: the dominant kernel's
@@ -83,54 +84,92 @@ def profiled_traffic(kernel_file: str, src_hash: str):
 
 
 class ClockSampler:
+    """SM clocks and clock-event reasons sampled every 50 ms during the timed region,
+    through NVML (read-only queries), else through one nvidia-smi query per sample."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    def __init__(self, device_index: int, uuid: str | None = None, period_s: float = 0.05):
+        self.index, self.uuid, self.period = device_index, uuid, period_s
+        self.samples, self.reasons, self.smax = [], set(), None
+        self._stop = None
+        self._thread = None
+        self.source = None
+
+    def _nvml_reader(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = None
+        if self.uuid:
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except Exception:
+                h = None
+        if h is None:
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+        def read():
+            return (float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)), int(get_reasons(h)))
+        self.source = "nvml"
+        return read
+
+    def _smi_reader(self):
+        def read():
+            r = subprocess.run(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                "-i", str(self.index)], capture_output=True, text=True, timeout=5)
+            parts = [p.strip() for p in r.stdout.strip().split(",")]
+            self.smax = float(parts[2])
+            bits = 0
+            for nm, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                "sw_power_cap"), parts[5:9]):
+                if val.lower() == "active":
+                    bits |= self.REASONS[nm]
+            return float(parts[1]), bits
+        self.source = "nvidia-smi"
+        return read
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
-            self.t0 = time.time()
+            read = self._nvml_reader()
+            read()
         except Exception:
-            self.proc = None
+            try:
+                read = self._smi_reader()
+                read()
+            except Exception:
+                return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    mhz, bits = read()
+                    self.samples.append(mhz)
+                    for nm, bit in self.REASONS.items():
+                        if bits & bit:
+                            self.reasons.add(nm)
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, smax, reasons = [], None, set()
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
-                except ValueError:
-                    continue
-                for nm, val in zip(names[1:], parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self._stop.set()
+        self._thread.join(timeout=10)
+        sm = self.samples
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "reasons": sorted(self.reasons), "samples": len(sm), "source": self.source}
 
 
 def dist_setup(args):
@@ -294,6 +333,7 @@ def run_ours(args):
     K, V = synth.keys_values(w, device=dev)
     cache.append(K, V, pj, cb)
     del K, V
+    torch.cuda.empty_cache()
     Qs, Kn, Vn = synth.decode_stream(w, n_steps, device=dev)
     ws = cache.workspace(w.Hq, args.splits)
     out = torch.empty(w.B, w.Hq, w.d, dtype=w.torch_dtype, device=dev)
@@ -318,15 +358,18 @@ def run_ours(args):
         native.tq_decode_prep(cache.state, Qs[i], scale, pj.Pi, pj.S, cent, args.splits, ws)
         if evs:
             evs[1].record(stream)
-        native.tq_decode_partial(cache.state, w.Hq, scale, cent, None, args.splits, ws)
+        native.tq_decode_partial(cache.state, w.Hq, scale, cent, None, args.splits, ws, out=out)
         if evs:
             evs[2].record(stream)
-        native.tq_decode_combine(cache.state, w.Hq, out, args.splits, ws)
-        if evs:
-            evs[3].record(stream)
 
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    try:
+        nvml_index = int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    except (KeyError, ValueError, IndexError):
+        nvml_index = local
+    clocks = ClockSampler(nvml_index, uuid=f"GPU-{uuid}" if uuid is not None else None,
+                          period_s=0.01)
     clocks.start()
     for i in range(args.warmup):
         flush.zero_()
@@ -334,7 +377,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     dec_bytes, all_bytes = [], []
     for k in range(args.steps):
         flush.zero_()
@@ -346,7 +389,7 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    t_step = [e[0].elapsed_time(e[3]) for e in events]             # ms
+    t_step = [e[0].elapsed_time(e[2]) for e in events]             # ms
     t_part = [e[1].elapsed_time(e[2]) for e in events]
     tot_ms = sum(t_step)
     tot_ms_max = reduce_max(tot_ms, world)
@@ -356,7 +399,7 @@ def run_ours(args):
     part_avg_ms = sum(t_part) / len(t_part)
     part_bytes = sum(dec_bytes) / len(dec_bytes)
     peak, peak_kind = measured_peak()
-    src_hash = source_hash("decode_kernels.cu")
+    src_hash = source_hash("decode_mma.cu")
     traffic = profiled_traffic("decode_partial_gqa32k.json", src_hash)
     achieved = part_bytes / (part_avg_ms * 1e-3) / 1e9
 
@@ -407,7 +450,8 @@ def run_ours(args):
                          "(append one token + decode its query heads), NumPy float64; GB/s of "
                          "that unit's packed bytes"}
 
-    launches = 5 * args.steps
+    # per step: quantise of the token leaving the ring, ring write, prep, partial
+    launches = 4 * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_ms_max / args.steps, "higher_is_better": True,
@@ -415,7 +459,7 @@ def run_ours(args):
         "config": _config(w, args),
         "pct_of_8TBps": 100.0 * value / NOMINAL_HBM,
         "tokens_per_s": tokens_s,
-        "roofline": {"bound": "hbm", "kernel": "k_decode_partial", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "k_decode_partial_mma", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes_per_launch": part_bytes,
                      "avg_launch_ms": part_avg_ms, "source_hash": src_hash},

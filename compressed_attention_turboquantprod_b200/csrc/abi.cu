@@ -442,11 +442,14 @@ static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_
     if (e != cudaSuccess) return cuda_fail(e, name);
   }
   if (partial) {
+    // the tensor-core partial kernel merges the splits itself when given `out`
+    void* fused_out = (mma && combine) ? out : nullptr;
     e = mma ? tq::launch_decode_partial_mma(g, static_cast<const uint8_t*>(c->base), c->n_total,
-                                            Hq, softmax_scale, logits, splits, ws, s)
+                                            Hq, softmax_scale, logits, splits, ws, fused_out, s)
             : tq::launch_decode_partial(g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
                                         softmax_scale, centroids, logits, splits, ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
+    if (fused_out) combine = false;
   }
   if (combine) {
     e = tq::launch_decode_combine(g, Hq, out, splits, ws, s);
@@ -473,11 +476,11 @@ int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale
 }
 
 int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const float* centroids,
-                      float* logits, int num_splits, void* workspace, size_t ws_bytes,
+                      float* logits, void* out, int num_splits, void* workspace, size_t ws_bytes,
                       void* stream) {
   TQ_FAULT_POINT("tq_decode_partial");
-  return decode_stage(c, nullptr, Hq, softmax_scale, nullptr, nullptr, centroids, nullptr, logits,
-                      num_splits, workspace, ws_bytes, stream, false, true, false,
+  return decode_stage(c, nullptr, Hq, softmax_scale, nullptr, nullptr, centroids, out, logits,
+                      num_splits, workspace, ws_bytes, stream, false, true, out != nullptr,
                       "tq_decode_partial");
 }
 

@@ -305,6 +305,7 @@ size_t decode_ws_bytes(const Geom& g, int Hq, int splits) {
   o += align256(units * frag_words(g) * sizeof(uint32_t)); // frag
   o += align256(units * 8 * 4 * sizeof(float));           // qconst
   o += 256;                                               // err
+  o += align256(units * sizeof(int));                     // counter
   o += align256(bq * splits * 2 * sizeof(float));         // part_ml
   o += align256(bq * splits * g.d * sizeof(float));       // part_o
   return o;
@@ -326,6 +327,8 @@ DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits) {
   p += align256(units * 8 * 4 * sizeof(float));
   w.err = reinterpret_cast<int*>(p);
   p += 256;
+  w.counter = reinterpret_cast<int*>(p);
+  p += align256(units * sizeof(int));
   w.part_ml = reinterpret_cast<float*>(p);
   p += align256(bq * splits * 2 * sizeof(float));
   w.part_o = reinterpret_cast<float*>(p);

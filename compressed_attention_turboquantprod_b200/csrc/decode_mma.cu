@@ -54,6 +54,7 @@ struct MParams {
   int splits, bps;
   DecodeWs ws;
   int* err;
+  void* out;        // when non-null, the last split of a unit also writes the output
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -162,73 +163,37 @@ __device__ __forceinline__ float i2f_exact(int x) {
 // [kstep][ntile][reg][lane] (uint32) and per head {kM, CM, kQ, CQ} (float).
 
 // ---------------------------------------------------------------- prep
-// (1) Projections of the queries, all (b, query head) at once: CTA (unit, chunk)
-// computes 32 output rows r of [Pi; S] (d + m rows) for the G = 4 queries of
-// one (b, KV head); each row is read once (one float4 per lane) and dotted with
-// the four queries.  qr = Pi q, qs = sqrt(pi/2)/m S q; chunk 0 also stores q.
-constexpr int PROJ_ROWS = 32;
-
-__global__ void __launch_bounds__(128) k_prep_proj(Geom g, const void* Q, int Hq, const float* Pi,
-                                                   const float* S, DecodeWs ws) {
-  __shared__ __align__(16) float sq[MG * 256];
-  const int unit = blockIdx.x, chunk = blockIdx.y;
-  const int b = unit / g.Hkv, h = unit % g.Hkv;
-  const int d = g.d, m = g.m;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bq0 = b * Hq + h * MG;
-  if (unit == 0 && chunk == 0 && tid == 0) *ws.err = 0;
-  for (int i = tid; i < MG * d; i += blockDim.x) {
-    const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
-    sq[i] = v;
-    if (chunk == 0) ws.qf[(int64_t)bq0 * d + i] = v;
-  }
-  __syncthreads();
-  const int rows_pi = g.b1 > 0 ? d : 0;
-  const float qscale = 1.2533141373155003f / (float)m;
-  for (int rr = warp; rr < PROJ_ROWS; rr += 4) {
-    const int r = chunk * PROJ_ROWS + rr;
-    if (r >= rows_pi + m) break;
-    const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
-    float acc[MG] = {0.f, 0.f, 0.f, 0.f};
-    for (int i0 = 4 * lane; i0 < d; i0 += 128) {
-      const float4 w = *reinterpret_cast<const float4*>(row + i0);
-#pragma unroll
-      for (int hh = 0; hh < MG; ++hh) {
-        const float4 q = *reinterpret_cast<const float4*>(sq + hh * d + i0);
-        acc[hh] = fmaf(w.x, q.x, fmaf(w.y, q.y, fmaf(w.z, q.z, fmaf(w.w, q.w, acc[hh]))));
-      }
-    }
-#pragma unroll
-    for (int hh = 0; hh < MG; ++hh) acc[hh] = warp_sum(acc[hh]);
-    if (lane < MG) {
-      const float a = acc[0] * (lane == 0) + acc[1] * (lane == 1) + acc[2] * (lane == 2) + acc[3] * (lane == 3);
-      if (r < rows_pi) ws.qr[(int64_t)(bq0 + lane) * d + r] = a;
-      else ws.qs[(int64_t)(bq0 + lane) * m + (r - rows_pi)] = a * qscale;
-    }
-  }
-}
-
-// (2) One CTA per (b, KV head): the Walsh weights of the codebook, the 21-bit
-// fixed-point quantisation of the query weights, their three int8 slices laid
-// out as the lanes' B fragments, and the per-head affine constants of the
-// logit (in log2 units of the softmax).
-__global__ void __launch_bounds__(256) k_prep_frag(Geom g, int Hq, const float* cent,
-                                                   float scale_log2, DecodeWs ws) {
+// One CTA per (b, KV head), for its G = 4 queries:
+//  * qf = q in fp32 (for the ring), qr = Pi q, qs = sqrt(pi/2)/m S q, each row of
+//    [Pi; S] read once (a float4 per lane) and dotted with the four queries;
+//  * the Walsh weights of the codebook, the 21-bit fixed-point quantisation of
+//    the query weights and their three int8 slices laid out as the lanes' B
+//    fragments, and the per-head affine constants of the logit (log2 units);
+//  * zeroes the unit's split counter and, in CTA 0, the error flag.
+__global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq, const float* Pi,
+                                                  const float* S, const float* cent,
+                                                  float scale_log2, DecodeWs ws) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int unit = blockIdx.x;
   const int b = unit / g.Hkv, h = unit % g.Hkv;
   const int d = g.d, m = g.m, b1 = g.b1;
-  const int tid = threadIdx.x;
-  float* sqr = reinterpret_cast<float*>(smem_raw);   // [G][d]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* sq = reinterpret_cast<float*>(smem_raw);     // [G][d]
+  float* sqr = sq + MG * d;                           // [G][d]
   float* sqs = sqr + MG * d;                          // [G][m]
   __shared__ float s_w[4];                            // Walsh weights of the odd subsets
   __shared__ unsigned s_maxM[MG], s_maxQ[MG];
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
-  const int F = b1 > 0 ? 1 << (b1 - 1) : 0;     // feature planes per coordinate
-  if (F)
-    for (int i = tid; i < MG * d; i += blockDim.x) sqr[i] = ws.qr[(int64_t)bq0 * d + i];
-  for (int i = tid; i < MG * m; i += blockDim.x) sqs[i] = ws.qs[(int64_t)bq0 * m + i];
+  if (tid == 0) {
+    ws.counter[unit] = 0;
+    if (unit == 0) *ws.err = 0;
+  }
+  for (int i = tid; i < MG * d; i += blockDim.x) {
+    const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
+    sq[i] = v;
+    ws.qf[(int64_t)bq0 * d + i] = v;
+  }
   if (tid == 0) {
     // w_S = (1/L) sum_idx c[idx] (-1)^{popc(idx & S)} for the odd subsets S, in the
     // order of the feature planes: {0}, {1}, {2}, {0,1,2}.
@@ -242,9 +207,36 @@ __global__ void __launch_bounds__(256) k_prep_frag(Geom g, int Hq, const float* 
     }
   }
   __syncthreads();
+  const int rows_pi = b1 > 0 ? d : 0;
+  const float qscale = 1.2533141373155003f / (float)m;
+  for (int r = warp; r < rows_pi + m; r += blockDim.x / 32) {
+    const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
+    float acc[MG] = {0.f, 0.f, 0.f, 0.f};
+    for (int i0 = 4 * lane; i0 < d; i0 += 128) {
+      const float4 w = *reinterpret_cast<const float4*>(row + i0);
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh) {
+        const float4 q = *reinterpret_cast<const float4*>(sq + hh * d + i0);
+        acc[hh] = fmaf(w.x, q.x, fmaf(w.y, q.y, fmaf(w.z, q.z, fmaf(w.w, q.w, acc[hh]))));
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < MG; ++hh) acc[hh] = warp_sum(acc[hh]);
+    if (lane < MG) {
+      const float a = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
+      if (r < rows_pi) {
+        sqr[lane * d + r] = a;
+        ws.qr[(int64_t)(bq0 + lane) * d + r] = a;
+      } else {
+        sqs[lane * m + (r - rows_pi)] = a * qscale;
+        ws.qs[(int64_t)(bq0 + lane) * m + (r - rows_pi)] = a * qscale;
+      }
+    }
+  }
+  __syncthreads();
+  const int F = b1 > 0 ? 1 << (b1 - 1) : 0;     // feature planes per coordinate
   {
     // warps 0-3: MSE weights of head w (max |W|, sum qr); warps 4-7: QJL of head w-4
-    const int warp = tid >> 5, lane = tid & 31;
     const int hh = warp & 3;
     float mx = 0.f, sm = 0.f;
     if (warp < 4) {
@@ -678,6 +670,39 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 0] = M;
     p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 1] = L;
   }
+  if (!p.out) return;
+  // The last split of this unit to finish merges all splits' (m, l, o).
+  __shared__ int s_last;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const int done = atomicAdd(&p.ws.counter[unit], 1);
+    s_last = (done == p.splits - 1);
+    if (s_last) p.ws.counter[unit] = 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = tid; i < MG * MD; i += MT) {
+    const int hh = i / MD, ch = i % MD;
+    const int bq = bq0 + hh;
+    const volatile float* ml = p.ws.part_ml + (int64_t)bq * p.splits * 2;
+    const volatile float* po = p.ws.part_o + (int64_t)bq * p.splits * MD;
+    float M = -INFINITY;
+    for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, ml[2 * sp]);
+    float o = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+      for (int sp = 0; sp < p.splits; ++sp) {
+        const float ms = ml[2 * sp];
+        if (ms == -INFINITY) continue;
+        const float wgt = exp2f(ms - M);
+        L = fmaf(ml[2 * sp + 1], wgt, L);
+        o = fmaf(po[sp * MD + ch], wgt, o);
+      }
+      o = o / L;
+    }
+    store_f(p.out, (int64_t)bq * MD + ch, g.dtype, o);
+  }
 }
 
 template <int B1, int KSQ>
@@ -701,22 +726,18 @@ bool decode_mma_supported(const Geom& g, int G) {
 cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
                                    const float* S, const float* cent, float scale,
                                    const DecodeWs& ws, cudaStream_t s) {
-  const int rows = (g.b1 > 0 ? g.d : 0) + g.m;
-  dim3 grid((unsigned)(g.B * g.Hkv), (unsigned)((rows + PROJ_ROWS - 1) / PROJ_ROWS));
-  k_prep_proj<<<grid, 128, 0, s>>>(g, Q, Hq, Pi, S, ws);
-  cudaError_t e = cudaGetLastError();
+  const size_t smem = sizeof(float) * MG * (2 * g.d + g.m);
+  cudaError_t e = cudaFuncSetAttribute(k_prep_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(float) * MG * (g.d + g.m);
-  e = cudaFuncSetAttribute(k_prep_frag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  k_prep_frag<<<g.B * g.Hkv, 256, smem, s>>>(g, Hq, cent, scale * kLog2e, ws);
+  k_prep_mma<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
                                       float scale, float* logits, int splits, const DecodeWs& ws,
-                                      cudaStream_t s) {
+                                      void* out, cudaStream_t s) {
   MParams p{};
+  p.out = out;
   p.g = g;
   p.base = base;
   p.n_total = n_total;

@@ -138,18 +138,56 @@ __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t 
   }
 }
 
-// Load rows [row0, row0+NT) of the key or value source into X (fp32, zero past n).
+// code = clamp(rint(fl((v - mn) / s)), 0, levels) with fl the IEEE fp32 quotient.
+// a * (1/s) is within 3 ulp of fl(a / s) (|quotient| <= 15), so their rints agree
+// unless the quotient lies within 1e-5 of a half-integer; only then is the exact
+// division taken.  Bit-identical to the plain definition.
+__device__ __forceinline__ uint32_t value_code(float v, float mn, float sc, float inv, float levels) {
+  if (sc == 0.f) return 0u;
+  const float a = __fsub_rn(v, mn);
+  const float x = a * inv;
+  float r = rintf(x);
+  if (fabsf(fabsf(x - r) - 0.5f) < 1e-5f) r = rintf(__fdiv_rn(a, sc));
+  r = fminf(fmaxf(r, 0.f), levels);
+  return (uint32_t)r;
+}
+
+// Four consecutive elements of a row (16-bit types as one 8-byte load).
+__device__ __forceinline__ void load4(const void* base, int64_t e, int dtype, float (&o)[4]) {
+  if (dtype == TQ_F32) {
+    const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + e);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + e);
+    const uint32_t w[2] = {u.x, u.y};
+    for (int k = 0; k < 2; ++k) {
+      if (dtype == TQ_F16) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&w[k]);
+        const float2 f = __half22float2(h);
+        o[2 * k] = f.x; o[2 * k + 1] = f.y;
+      } else {
+        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+        const float2 f = __bfloat1622float2(h);
+        o[2 * k] = f.x; o[2 * k + 1] = f.y;
+      }
+    }
+  }
+}
+
+// Load rows [row0, row0+NT) of the key or value source into X (fp32, zero past n):
+// a warp per row, the source address computed once per row, 4 elements per lane.
 __device__ void load_tile(const QParams& p, bool values, int bh, int64_t row0, float* X) {
   const int d = p.d, sx = d + 4;
-  for (int idx = threadIdx.x; idx < NT * d; idx += THREADS) {
-    const int r = idx / d, c = idx % d;
-    float v = 0.f;
-    if (row0 + r < p.n) {
-      int64_t e;
-      const void* src = src_row(p, values, bh, row0 + r, e);
-      v = load_f(src, e + c, p.dtype);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = warp; r < NT; r += blockDim.x / 32) {
+    const bool valid = row0 + r < p.n;
+    int64_t e = 0;
+    const void* src = valid ? src_row(p, values, bh, row0 + r, e) : nullptr;
+    for (int c = 4 * lane; c < d; c += 128) {
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) load4(src, e + c, p.dtype, v);
+      *reinterpret_cast<float4*>(X + r * sx + c) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    X[r * sx + c] = v;
   }
 }
 
@@ -276,7 +314,7 @@ __device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, in
   const int tid = threadIdx.x;
   load_tile(p, true, bh, row0, s.X);
   __syncthreads();
-  for (int pr = tid; pr < NT * ng; pr += THREADS) {
+  for (int pr = tid; pr < NT * ng; pr += blockDim.x) {
     const int r = pr / ng, gi = pr % ng;
     float mn = FLT_MAX, mx = -FLT_MAX;
     for (int k = 0; k < g; ++k) {
@@ -295,21 +333,16 @@ __device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, in
   __syncthreads();
   const int per_word = 32 / vb;
   const int wpr = d / per_word;
-  for (int pw = tid; pw < NT * wpr; pw += THREADS) {
+  for (int pw = tid; pw < NT * wpr; pw += blockDim.x) {
     const int r = pw / wpr, w = pw % wpr;
     if (row0 + r >= p.n) continue;
     uint32_t word = 0;
+    const int gi = (w * per_word) / g;      // a word never straddles two groups (g >= 16)
+    const float sc = s.vs[r * ng + gi], mn = s.vm[r * ng + gi];
+    const float inv = sc != 0.f ? __frcp_rn(sc) : 0.f;
     for (int k = 0; k < per_word; ++k) {
       const int ch = w * per_word + k;
-      const int gi = ch / g;
-      const float sc = s.vs[r * ng + gi], mn = s.vm[r * ng + gi];
-      uint32_t code = 0;
-      if (sc != 0.f) {
-        float q = rintf(__fdiv_rn(__fsub_rn(s.X[r * sx + ch], mn), sc));
-        q = fminf(fmaxf(q, 0.f), levels);
-        code = (uint32_t)q;
-      }
-      word |= code << (k * vb);
+      word |= value_code(s.X[r * sx + ch], mn, sc, inv, levels) << (k * vb);
     }
     reinterpret_cast<uint32_t*>(dst_field(p, bh, row0 + r, 4))[w] = word;
   }
@@ -353,30 +386,47 @@ __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V
   }
 }
 
-// One CTA per token, for launches with only a few tokens per (b, kv head) (the
-// decode step appends one): the same arithmetic as the 64-token tile, with the
-// matrix-vector products done warp-per-row (lanes over the inner dimension).
-constexpr int SMALL_THREADS = 128;
+// One CTA per token and per half (blockIdx.z = 0: key, 1: value), for launches
+// with only a few tokens per (b, kv head) (the decode step appends one): the
+// same arithmetic as the 64-token tile.  The key CTA runs its matrix-vector
+// products two threads per row (each streams half the row as float4, the vector
+// is a shared-memory broadcast) and reduces rho while Pi x is being formed.
+constexpr int SMALL_THREADS = 256;
+
+__device__ __forceinline__ float half_row_dot(const float* rowp, const float* v, int d, int half) {
+  const float4* rp = reinterpret_cast<const float4*>(rowp) + half * (d / 8);
+  const float* vp = v + half * (d / 2);
+  float a = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < d / 8; ++i) {
+    const float4 w = rp[i];
+    a = fmaf(w.x, vp[4 * i], a);
+    a = fmaf(w.y, vp[4 * i + 1], a);
+    a = fmaf(w.z, vp[4 * i + 2], a);
+    a = fmaf(w.w, vp[4 * i + 3], a);
+  }
+  return a + __shfl_xor_sync(0xffffffffu, a, 1);
+}
 
 __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int d = p.d, m = p.m, b1 = p.b1;
   float* sx = reinterpret_cast<float*>(smem_raw);       // [d]
-  float* sy = sx + d;                                    // [d]  e = y - c[idx]
+  float* sy = sx + d;                                    // [d]  Pi x, then e = y - c[idx]
   float* sz = sy + d;                                    // [max(m, 32)]
   __shared__ double s_red[SMALL_THREADS / 32];
-  __shared__ double s_rho;
   __shared__ float s_cb[32];
   const int bh = blockIdx.y;
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = SMALL_THREADS / 32;
-  if (tid < 16) {
-    const int L = b1 > 0 ? (1 << b1) : 0;
-    s_cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
-    s_cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
-  }
-  if (p.do_keys) {
+  if (blockIdx.z == 0) {
+    if (!p.do_keys) return;
+    if (tid < 16) {
+      const int L = b1 > 0 ? (1 << b1) : 0;
+      s_cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
+      s_cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
+    }
     int64_t e0;
     const void* src = src_row(p, false, bh, row, e0);
     double ss = 0.0;
@@ -388,81 +438,70 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
     ss = warp_sum_d(ss);
     if (lane == 0) s_red[warp] = ss;
     __syncthreads();
-    if (tid == 0) {
-      double t = 0.0;
-      for (int w = 0; w < NW; ++w) t += s_red[w];
-      s_rho = sqrt(t);
-    }
-    __syncthreads();
-    const double rho64 = s_rho;
+    double t = 0.0;
+    for (int w = 0; w < NW; ++w) t += s_red[w];
+    const double rho64 = sqrt(t);
     const float rho = (float)rho64;
     const float inv = rho64 > 0.0 ? (float)(1.0 / rho64) : 0.f;
     const float* E = sx;
-    // thread-per-row matrix-vector products: each thread streams its own row as
-    // float4 (independent loads, the vector is a shared-memory broadcast)
+    const int half = tid & 1;
     if (b1 > 0) {
+      for (int j = tid >> 1; j < d; j += SMALL_THREADS / 2) {
+        const float a = half_row_dot(p.Pi + (int64_t)j * d, sx, d, half);
+        if (half == 0) sy[j] = a * inv;
+      }
+      __syncthreads();
       const int L = 1 << b1;
       uint8_t* idx_dst = dst_field(p, bh, row, 0);
       double se = 0.0;
       for (int j = tid; j < d; j += SMALL_THREADS) {
-        const float4* rp = reinterpret_cast<const float4*>(p.Pi + (int64_t)j * d);
-        float a = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < d / 4; ++i) {
-          const float4 w = rp[i];
-          a = fmaf(w.x, sx[4 * i], a);
-          a = fmaf(w.y, sx[4 * i + 1], a);
-          a = fmaf(w.z, sx[4 * i + 2], a);
-          a = fmaf(w.w, sx[4 * i + 3], a);
-        }
-        const float y = a * inv;
+        const float y = sy[j];
         int idx = 0;
         for (int k = 0; k + 1 < L; ++k) idx += (s_cb[16 + k] < y) ? 1 : 0;
         const float e = y - s_cb[idx];
-        sy[j] = e;
         se += (double)e * (double)e;
         for (int pl = 0; pl < b1; ++pl) {
           const unsigned word = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
           if (lane == 0) *reinterpret_cast<uint32_t*>(idx_dst + pl * (d / 8) + (j - lane) / 8) = word;
         }
+        sz[j] = e;                          // staged: sy is still being read by other warps
       }
       se = warp_sum_d(se);
+      __syncthreads();
+      for (int j = tid; j < d; j += SMALL_THREADS) sy[j] = sz[j];
       if (lane == 0) s_red[warp] = se;
       __syncthreads();
       if (tid == 0) {
-        double t = 0.0;
-        for (int w = 0; w < NW; ++w) t += s_red[w];
-        *reinterpret_cast<float*>(dst_field(p, bh, row, 3)) = (float)(rho64 * sqrt(t));
+        double u = 0.0;
+        for (int w = 0; w < NW; ++w) u += s_red[w];
+        *reinterpret_cast<float*>(dst_field(p, bh, row, 3)) = (float)(rho64 * sqrt(u));
       }
       E = sy;
     }
+    // z = rho T e (or S x), two threads per row; a warp covers 16 rows, so the
+    // 32 sign bits of a word come from two warps and are staged in shared memory.
+    for (int a = tid >> 1; a < m; a += SMALL_THREADS / 2) {
+      const float acc = half_row_dot(p.T + (int64_t)a * d, E, d, half);
+      if (half == 0) sz[a] = (b1 > 0) ? acc * rho : acc;
+    }
+    __syncthreads();
     uint8_t* sdst = dst_field(p, bh, row, 1);
-    for (int a = tid; a < m; a += SMALL_THREADS) {
-      const float4* rp = reinterpret_cast<const float4*>(p.T + (int64_t)a * d);
-      float acc = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < d / 4; ++i) {
-        const float4 w = rp[i];
-        acc = fmaf(w.x, E[4 * i], acc);
-        acc = fmaf(w.y, E[4 * i + 1], acc);
-        acc = fmaf(w.z, E[4 * i + 2], acc);
-        acc = fmaf(w.w, E[4 * i + 3], acc);
-      }
-      const float z = (b1 > 0) ? acc * rho : acc;
-      const unsigned word = __ballot_sync(0xffffffffu, z >= 0.f);
-      if (lane == 0) *reinterpret_cast<uint32_t*>(sdst + (a - lane) / 8) = word;
+    for (int ab = warp * 32; ab < m; ab += SMALL_THREADS) {
+      const unsigned word = __ballot_sync(0xffffffffu, sz[ab + lane] >= 0.f);
+      if (lane == 0) *reinterpret_cast<uint32_t*>(sdst + ab / 8) = word;
     }
     if (tid == 0) *reinterpret_cast<float*>(dst_field(p, bh, row, 2)) = rho;
-    __syncthreads();
+    return;
   }
-  if (p.do_values) {
+  if (!p.do_values) return;
+  {
     const int g = p.group, ng = d / g, vb = p.vbits;
     const float levels = (float)((1 << vb) - 1);
     int64_t e0;
     const void* src = src_row(p, true, bh, row, e0);
     for (int c = tid; c < d; c += SMALL_THREADS) sx[c] = load_f(src, e0 + c, p.dtype);
     __syncthreads();
-    float* vs = sz;            // [ng] scales, [ng] minima (reuses the sketch buffer)
+    float* vs = sz;            // [ng] scales, [ng] minima
     float* vm = sz + 16;
     for (int gi = tid; gi < ng; gi += SMALL_THREADS) {
       float mn = FLT_MAX, mx = -FLT_MAX;
@@ -481,19 +520,238 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
     const int per_word = 32 / vb, wpr = d / per_word;
     for (int w = tid; w < wpr; w += SMALL_THREADS) {
       uint32_t word = 0;
+      const float sc = vs[(w * per_word) / g], mn = vm[(w * per_word) / g];
+      const float inv = sc != 0.f ? __frcp_rn(sc) : 0.f;
       for (int k = 0; k < per_word; ++k) {
         const int ch = w * per_word + k;
-        const float sc = vs[ch / g], mn = vm[ch / g];
-        uint32_t code = 0;
-        if (sc != 0.f) {
-          float q = rintf(__fdiv_rn(__fsub_rn(sx[ch], mn), sc));
-          q = fminf(fmaxf(q, 0.f), levels);
-          code = (uint32_t)q;
-        }
-        word |= code << (k * vb);
+        word |= value_code(sx[ch], mn, sc, inv, levels) << (k * vb);
       }
       reinterpret_cast<uint32_t*>(dst_field(p, bh, row, 4))[w] = word;
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core tile path (head dim 128, b1 > 0, m = 128): a persistent CTA per SM
+// keeps Pi and T = S Pi^T resident in shared memory as fp16 hi/lo pairs
+// (v * 2^10 = hi + lo, |lo| <= 2^-11 |hi|), and loops over 64-token tiles:
+//   U = X / rho -> fp16 hi/lo;  Y = U Pi^T  and  Z = E T^T (E = Y - c[idx])
+// each as three mma.sync m16n8k16 products (hi*hi + hi*lo + lo*hi, fp32
+// accumulate), i.e. about 22 significant bits: well inside the 1e-5 band that
+// separates a code or a sign from its decision boundary.
+// ---------------------------------------------------------------------------
+constexpr int QD = 128;             // head dim of this path
+constexpr int QM = 128;             // sketch rows of this path
+constexpr int HS = QD + 8;          // fp16 row stride (272 B: conflict-free ldmatrix)
+constexpr int YS = QD + 4;          // fp32 row stride of the Y / Z / V tile
+constexpr float kSplit = 1024.f;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void split_store(__half* hi, __half* lo, float v) {
+  const float x = v * kSplit;
+  const __half h = __float2half_rn(x);
+  *hi = h;
+  *lo = __float2half_rn(x - __half2float(h));
+}
+
+struct MmaSmem {
+  __half *PH, *PL, *TH, *TL, *AH, *AL;
+  float* YZ;
+  double* rho64;
+  float *rho, *inv, *cb, *vs, *vm;
+};
+
+__host__ __device__ inline size_t mma_smem_bytes() {
+  return sizeof(__half) * (4 * 128 * HS + 2 * NT * HS) + sizeof(float) * NT * YS +
+         sizeof(double) * NT + sizeof(float) * (2 * NT + 32 + 2 * NT * 16);
+}
+
+__device__ MmaSmem mma_carve(unsigned char* raw) {
+  MmaSmem s;
+  s.PH = reinterpret_cast<__half*>(raw);
+  s.PL = s.PH + 128 * HS;
+  s.TH = s.PL + 128 * HS;
+  s.TL = s.TH + 128 * HS;
+  s.AH = s.TL + 128 * HS;
+  s.AL = s.AH + NT * HS;
+  s.YZ = reinterpret_cast<float*>(s.AL + NT * HS);
+  s.rho64 = reinterpret_cast<double*>(s.YZ + NT * YS);
+  s.rho = reinterpret_cast<float*>(s.rho64 + NT);
+  s.inv = s.rho + NT;
+  s.cb = s.inv + NT;
+  s.vs = s.cb + 32;
+  s.vm = s.vs + NT * 16;
+  return s;
+}
+
+constexpr int QTHREADS = 512;       // 16 warps per CTA on the tensor-core tile path
+
+// C[64 x 128] = A[64 x 128] * B^T, A and B as fp16 hi/lo pairs (rows of 128,
+// stride HS); warp w (of 16) owns rows 32 (w & 1) .. +32 and columns 16 (w >> 1)
+// .. +16.  The result (scaled back by 2^-20) goes to C (fp32, stride YS).
+__device__ void mma_gemm_64x128(const __half* AH, const __half* AL, const __half* BH,
+                                const __half* BL, float* C) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r0 = 32 * (warp & 1), c0 = 16 * (warp >> 1);
+  float acc[2][2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+  const int ar = lane & 15, ac = 8 * (lane >> 4);                    // A: rows, k offset
+  const int bn = (lane & 7) + 8 * (lane >> 4), bk = 8 * ((lane >> 3) & 1);   // B: n, k offset
+#pragma unroll 2
+  for (int ks = 0; ks < QD / 16; ++ks) {
+    uint32_t ah[2][4], al[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ldsm_x4(ah[i], AH + (r0 + 16 * i + ar) * HS + 16 * ks + ac);
+      ldsm_x4(al[i], AL + (r0 + 16 * i + ar) * HS + 16 * ks + ac);
+    }
+    {
+      uint32_t bh[4], bl[4];
+      ldsm_x4(bh, BH + (c0 + bn) * HS + 16 * ks + bk);
+      ldsm_x4(bl, BL + (c0 + bn) * HS + 16 * ks + bk);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mma16816(acc[i][0], ah[i], bh[0], bh[1]);
+        mma16816(acc[i][0], ah[i], bl[0], bl[1]);
+        mma16816(acc[i][0], al[i], bh[0], bh[1]);
+        mma16816(acc[i][1], ah[i], bh[2], bh[3]);
+        mma16816(acc[i][1], ah[i], bl[2], bl[3]);
+        mma16816(acc[i][1], al[i], bh[2], bh[3]);
+      }
+    }
+  }
+  const int gid = lane >> 2, tig = lane & 3;
+  const float sc = 1.f / (kSplit * kSplit);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int row = r0 + 16 * i + gid, col = c0 + 8 * j + 2 * tig;
+      C[row * YS + col] = acc[i][j][0] * sc;
+      C[row * YS + col + 1] = acc[i][j][1] * sc;
+      C[(row + 8) * YS + col] = acc[i][j][2] * sc;
+      C[(row + 8) * YS + col + 1] = acc[i][j][3] * sc;
+    }
+}
+
+__global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t tiles_per_bh,
+                                                             int64_t total_tiles) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  MmaSmem s = mma_carve(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b1 = p.b1;
+  // resident operands: Pi and T as fp16 hi/lo, rows of 128 (four elements a thread)
+  for (int i = 4 * tid; i < QD * QD; i += 4 * QTHREADS) {
+    const int r = i / QD, c = i % QD;
+    const float4 a = *reinterpret_cast<const float4*>(p.Pi + i);
+    const float4 b = *reinterpret_cast<const float4*>(p.T + i);
+    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      split_store(s.PH + r * HS + c + k, s.PL + r * HS + c + k, av[k]);
+      split_store(s.TH + r * HS + c + k, s.TL + r * HS + c + k, bv[k]);
+    }
+  }
+  if (tid < 16) {
+    const int L = 1 << b1;
+    s.cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
+    s.cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
+  }
+  __syncthreads();
+  Smem vs{};            // view for the shared value-tile code
+  vs.X = s.YZ;
+  vs.vs = s.vs;
+  vs.vm = s.vm;
+  for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    const int bh = (int)(tile / tiles_per_bh);
+    const int64_t row0 = (tile % tiles_per_bh) * NT;
+    // ---- keys: rho (float64), U = X / rho as fp16 hi/lo
+    for (int r = warp; r < NT; r += QTHREADS / 32) {
+      const bool valid = row0 + r < p.n;
+      int64_t e0 = 0;
+      const void* src = valid ? src_row(p, false, bh, row0 + r, e0) : nullptr;
+      float x[QD / 32];
+      double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < QD / 32; ++k) {
+        x[k] = valid ? load_f(src, e0 + lane + 32 * k, p.dtype) : 0.f;
+        ss += (double)x[k] * (double)x[k];
+      }
+      ss = warp_sum_d(ss);
+      const double rho = sqrt(ss);
+      const float inv = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
+      if (lane == 0) {
+        s.rho64[r] = rho;
+        s.rho[r] = (float)rho;
+      }
+#pragma unroll
+      for (int k = 0; k < QD / 32; ++k)
+        split_store(s.AH + r * HS + lane + 32 * k, s.AL + r * HS + lane + 32 * k, x[k] * inv);
+    }
+    __syncthreads();
+    mma_gemm_64x128(s.AH, s.AL, s.PH, s.PL, s.YZ);           // Y = U Pi^T
+    __syncthreads();
+    // ---- codes, residual E (fp16 hi/lo into A), ||r||
+    const int L = 1 << b1;
+    for (int r = warp; r < NT; r += QTHREADS / 32) {
+      const bool valid = row0 + r < p.n;
+      uint8_t* idx_dst = valid ? dst_field(p, bh, row0 + r, 0) : nullptr;
+      double se = 0.0;
+#pragma unroll
+      for (int jb = 0; jb < QD; jb += 32) {
+        const float y = s.YZ[r * YS + jb + lane];
+        int idx = 0;
+        for (int k = 0; k + 1 < L; ++k) idx += (s.cb[16 + k] < y) ? 1 : 0;
+        const float e = y - s.cb[idx];
+        se += (double)e * (double)e;
+        split_store(s.AH + r * HS + jb + lane, s.AL + r * HS + jb + lane, e);
+        for (int pl = 0; pl < b1; ++pl) {
+          const unsigned word = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
+          if (lane == 0 && valid)
+            *reinterpret_cast<uint32_t*>(idx_dst + pl * (QD / 8) + jb / 8) = word;
+        }
+      }
+      se = warp_sum_d(se);
+      if (lane == 0 && valid) {
+        *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 3)) = (float)(s.rho64[r] * sqrt(se));
+        *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = s.rho[r];
+      }
+    }
+    __syncthreads();
+    mma_gemm_64x128(s.AH, s.AL, s.TH, s.TL, s.YZ);           // Z = E T^T
+    __syncthreads();
+    for (int r = warp; r < NT; r += QTHREADS / 32) {
+      if (row0 + r >= p.n) continue;
+      uint8_t* sdst = dst_field(p, bh, row0 + r, 1);
+      const float rho = s.rho[r];
+#pragma unroll
+      for (int cb = 0; cb < QM; cb += 32) {
+        const unsigned word = __ballot_sync(0xffffffffu, s.YZ[r * YS + cb + lane] * rho >= 0.f);
+        if (lane == 0) *reinterpret_cast<uint32_t*>(sdst + cb / 8) = word;
+      }
+    }
+    __syncthreads();
+    // ---- values (the shared tile code, on the Y/Z buffer)
+    if (p.do_values) quantize_values_tile(p, vs, bh, row0);
+    __syncthreads();
   }
 }
 
@@ -501,10 +759,25 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
 
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
+  if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0) {
+    // tensor-core tiles: one persistent CTA per SM over all 64-token tiles
+    const int64_t tiles_per_bh = (p.n + NT - 1) / NT;
+    const int64_t total = tiles_per_bh * bh_count;
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = mma_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(k_quantize_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = total < sms ? total : sms;
+    k_quantize_mma<<<(unsigned)grid, QTHREADS, smem, s>>>(p, tiles_per_bh, total);
+    return cudaGetLastError();
+  }
   if (p.n <= 8) {
     // a few tokens per (b, kv head): one CTA per token
-    const size_t smem = sizeof(float) * (2 * p.d + (p.m > 32 ? p.m : 32));
-    dim3 grid((unsigned)p.n, (unsigned)bh_count);
+    const size_t smem = sizeof(float) * (2 * p.d + (p.m > p.d ? p.m : p.d) + 32);
+    dim3 grid((unsigned)p.n, (unsigned)bh_count, 2);
     k_quantize_small<<<grid, SMALL_THREADS, smem, s>>>(p);
     return cudaGetLastError();
   }

@@ -69,6 +69,7 @@ struct DecodeWs {
   uint32_t* frag;   // [B*Hkv, ksteps, 2, 2, 32]  int8 query slices (tensor-core path)
   float* qconst;    // [B*Hkv, 8, 4]  per-head logit constants (tensor-core path)
   int* err;         // error flag set by a kernel whose bounded wait gave up
+  int* counter;     // [B*Hkv] finished splits of each unit (fused combine)
   float* part_ml;   // [B*Hq, splits, 2]
   float* part_o;    // [B*Hq, splits, d]
 };
@@ -83,7 +84,7 @@ cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const f
                                    const DecodeWs& ws, cudaStream_t s);
 cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
                                       float scale, float* logits, int splits, const DecodeWs& ws,
-                                      cudaStream_t s);
+                                      void* out, cudaStream_t s);
 
 cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float* Pi,
                                const float* S, const DecodeWs& ws, cudaStream_t s);

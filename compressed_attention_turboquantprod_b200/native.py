@@ -82,7 +82,7 @@ def _load() -> ctypes.CDLL:
         "tq_decode_attention_noalloc": (I, [C, P, I, F, P, P, P, P, P, I, P]),
         "tq_decode_prep": (I, [C, P, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_check": (I, [C, I, I, P, SZ, P]),
-        "tq_decode_partial": (I, [C, I, F, P, P, I, P, SZ, P]),
+        "tq_decode_partial": (I, [C, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
         "tq_m_for_layer": (I, [ctypes.POINTER(tq_layer_groups), I]),
@@ -224,10 +224,10 @@ def tq_decode_check(cache: tq_cache, Hq, num_splits, workspace, stream=None):
 
 
 def tq_decode_partial(cache: tq_cache, Hq, softmax_scale, centroids, logits, num_splits,
-                      workspace, stream=None):
+                      workspace, out=None, stream=None):
     _check(lib.tq_decode_partial(ctypes.byref(cache), Hq, softmax_scale, _ptr(centroids),
-                                 _ptr(logits), num_splits, _ptr(workspace), _ws(workspace),
-                                 _stream(stream)), "tq_decode_partial")
+                                 _ptr(logits), _ptr(out), num_splits, _ptr(workspace),
+                                 _ws(workspace), _stream(stream)), "tq_decode_partial")
 
 
 def tq_decode_combine(cache: tq_cache, Hq, out, num_splits, workspace, stream=None):

@@ -266,12 +266,15 @@ int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_
 /* The three stages of tq_decode_attention, for callers that time or overlap
  * them separately.  Same arguments and workspace as tq_decode_attention; the
  * preparation stage also takes the softmax scale and the centroids (the
- * tensor-core path folds them into the query-side constants). */
+ * tensor-core path folds them into the query-side constants).  When `out` is
+ * non-NULL, tq_decode_partial also merges the splits into `out` (on the
+ * tensor-core path inside the same kernel), and tq_decode_combine is not
+ * needed. */
 int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
                    const float* Pi, const float* S, const float* centroids, int num_splits,
                    void* workspace, size_t ws_bytes, void* stream);
 int tq_decode_partial(const tq_cache* c, int Hq, float softmax_scale, const float* centroids,
-                      float* logits, int num_splits, void* workspace, size_t ws_bytes,
+                      float* logits, void* out, int num_splits, void* workspace, size_t ws_bytes,
                       void* stream);
 int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void* workspace,
                       size_t ws_bytes, void* stream);
