@@ -55,4 +55,9 @@ __device__ __forceinline__ uint8_t* field_ptr(uint8_t* base, const Geom& g, int 
          (t % kBlockTokens) * size;
 }
 
+// Hint: bring the 128-byte line holding p into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 }  // namespace tq

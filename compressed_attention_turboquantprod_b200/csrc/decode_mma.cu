@@ -185,6 +185,12 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
   __shared__ unsigned s_maxM[MG], s_maxQ[MG];
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
+  {
+    // the rows of [Pi; S] are read after the queries: start them towards L2 now
+    const int lines_pi = b1 > 0 ? d * d / 32 : 0, lines = lines_pi + m * d / 32;
+    for (int i = tid; i < lines; i += blockDim.x)
+      prefetch_l2(i < lines_pi ? Pi + 32 * (int64_t)i : S + 32 * (int64_t)(i - lines_pi));
+  }
   if (tid == 0) {
     ws.counter[unit] = 0;
     if (unit == 0) *ws.err = 0;
@@ -209,28 +215,49 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
   __syncthreads();
   const int rows_pi = b1 > 0 ? d : 0;
   const float qscale = 1.2533141373155003f / (float)m;
-  for (int r = warp; r < rows_pi + m; r += blockDim.x / 32) {
-    const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
-    float acc[MG] = {0.f, 0.f, 0.f, 0.f};
-    for (int i0 = 4 * lane; i0 < d; i0 += 128) {
-      const float4 w = *reinterpret_cast<const float4*>(row + i0);
+  // Rows of [Pi; S] in passes of 8 per warp: lane l dots float4 l of each row
+  // (coalesced) with columns 4l..4l+3 of the four queries (held in registers);
+  // a reduce-scatter over the warp then leaves the sum of (row l/4, head l%4) in
+  // lane l.  (d = 128: one float4 per lane per row.)
+  float4 qv[MG];
 #pragma unroll
-      for (int hh = 0; hh < MG; ++hh) {
-        const float4 q = *reinterpret_cast<const float4*>(sq + hh * d + i0);
-        acc[hh] = fmaf(w.x, q.x, fmaf(w.y, q.y, fmaf(w.z, q.z, fmaf(w.w, q.w, acc[hh]))));
+  for (int hh = 0; hh < MG; ++hh) qv[hh] = *reinterpret_cast<const float4*>(sq + hh * d + 4 * lane);
+  const int R = rows_pi + m;
+  for (int r0 = 8 * warp; r0 < R; r0 += 8 * (blockDim.x / 32)) {
+    float4 wv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = r0 + k;
+      const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
+      wv[k] = *reinterpret_cast<const float4*>(row + 4 * lane);
+    }
+    float v[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh)
+        v[4 * k + hh] = fmaf(wv[k].x, qv[hh].x, fmaf(wv[k].y, qv[hh].y,
+                        fmaf(wv[k].z, qv[hh].z, wv[k].w * qv[hh].w)));
+    // reduce-scatter: after the round with offset o, a lane keeps the half of its
+    // values selected by (lane & o) and adds its partner's copy of that half
+#pragma unroll
+    for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int k = 0; k < n; ++k) {
+        const float send = upper ? v[k] : v[k + n];
+        const float keep = upper ? v[k + n] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
-#pragma unroll
-    for (int hh = 0; hh < MG; ++hh) acc[hh] = warp_sum(acc[hh]);
-    if (lane < MG) {
-      const float a = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
-      if (r < rows_pi) {
-        sqr[lane * d + r] = a;
-        ws.qr[(int64_t)(bq0 + lane) * d + r] = a;
-      } else {
-        sqs[lane * m + (r - rows_pi)] = a * qscale;
-        ws.qs[(int64_t)(bq0 + lane) * m + (r - rows_pi)] = a * qscale;
-      }
+    const int r = r0 + (lane >> 2), hh = lane & 3;
+    const float a = v[0];
+    if (r < rows_pi) {
+      sqr[hh * d + r] = a;
+      ws.qr[(int64_t)(bq0 + hh) * d + r] = a;
+    } else {
+      sqs[hh * m + (r - rows_pi)] = a * qscale;
+      ws.qs[(int64_t)(bq0 + hh) * m + (r - rows_pi)] = a * qscale;
     }
   }
   __syncthreads();
@@ -328,6 +355,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __shared__ float s_mn[4][MG][4];
   __shared__ int s_cnt[NST];
   __shared__ __align__(16) uint32_t s_frag[KS * 128];
+  __shared__ __align__(8) uint64_t ringbar;
+  __shared__ __align__(16) float s_qf[MG * MD];
 
   const Geom& g = p.g;
   const int split = blockIdx.x, unit = blockIdx.y;
@@ -345,15 +374,34 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   const int nb = blk1 > blk0 ? (int)(blk1 - blk0) : 0;
   const uint8_t* region = p.base + (int64_t)unit * g.region_bytes;
 
+  // The exact ring tokens are folded in by the last split, a chunk of RC of them at
+  // a time staged in the (until the final merge unused) s_out area; the first chunk
+  // is requested here, before the cache blocks.
+  const bool ring_split = split == p.splits - 1 && p.n_ring > 0;
+  const int es = g.dtype == TQ_F32 ? 4 : 2;
+  const int RC = (4 * MG * MD * (int)sizeof(float)) / (2 * MD * es);
+  const unsigned char* ring_k = p.base + g.ring_k_off + (int64_t)unit * g.W * MD * es;
+  const unsigned char* ring_v = p.base + g.ring_v_off + (int64_t)unit * g.W * MD * es;
+  unsigned char* s_rk = reinterpret_cast<unsigned char*>(s_out);
+  unsigned char* s_rv = s_rk + (size_t)RC * MD * es;
   if (tid == 0) {
     s_abort = 0;
     for (int s = 0; s < NST; ++s) mbar_init(&full[s], 1);
+    mbar_init(&ringbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (ring_split) {
+      const uint32_t nbytes = (uint32_t)(min(RC, p.n_ring) * MD * es);
+      mbar_expect_tx(&ringbar, 2 * nbytes);
+      bulk_load(s_rk, ring_k, nbytes, &ringbar);
+      bulk_load(s_rv, ring_v, nbytes, &ringbar);
+    }
     for (int s = 0; s < NST && s < nb; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
       bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
     }
   }
+  if (ring_split)
+    for (int i = tid; i < MG * MD; i += MT) s_qf[i] = p.ws.qf[(int64_t)bq0 * MD + i];
 
   // B fragments of the score (query slices), per k-step and lane four words
   // {ntile0 r0, ntile0 r1, ntile1 r0, ntile1 r1}, staged in shared memory.
@@ -573,53 +621,72 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   if (s_abort) {
     // a wait gave up: wait (bounded) for every copy this CTA may still have in
     // flight (at most the last NST blocks), then leave
-    if (tid == 0)
+    if (tid == 0) {
       for (int j = (nb > NST ? nb - NST : 0); j < nb; ++j)
         (void)mbar_wait(&full[j % NST], (uint32_t)((j / NST) & 1));
+      if (ring_split) (void)mbar_wait(&ringbar, 0);
+    }
     return;
   }
 
-  // ---------------- exact ring tokens (last split, warp 0)
+  // ---------------- exact ring tokens (last split)
   // The value part of acc counts codes in units of 2^(2k-24) (k = gid & 3, the
   // bit offset of this lane's channels in their byte): o = acc / code_unit.
   const float code_unit = __int_as_float((127 - 24 + 2 * (gid & 3)) << 23);       // 2^(2k-24)
   const float inv_unit = __int_as_float((127 + 24 - 2 * (gid & 3)) << 23);        // 2^(24-2k)
-  if (split == p.splits - 1 && p.n_ring > 0 && warp == 0) {
+  if (ring_split) {
+    // Ring slots in slot order (softmax and P V do not depend on the order); slot s
+    // holds the token at ring position ((s - first) mod W).  Warp w takes the slots
+    // per_warp * w + (0 .. per_warp-1) of each chunk as its rows gid < per_warp.
     const int64_t first = p.n_total - p.n_ring;
-    const float* qf = p.ws.qf + (int64_t)(bq0 + tig) * MD;
-    for (int r0 = 0; r0 < p.n_ring; r0 += 16) {
-      float lr[2];
-      for (int k = 0; k < 2; ++k) {
-        const int rt = r0 + gid + 8 * k;
-        float dot = -INFINITY;
-        if (rt < p.n_ring) {
-          const int64_t slot = (first + rt) % g.W;
-          const int64_t e = ((int64_t)unit * g.W + slot) * MD;
-          dot = 0.f;
-          for (int j = 0; j < MD; ++j) dot = fmaf(qf[j], load_f(p.base + g.ring_k_off, e + j, g.dtype), dot);
-          if (p.logits) p.logits[(int64_t)(bq0 + tig) * p.n_log + p.n_comp + rt] = dot;
-          dot *= p.scale_log2;
-        }
-        lr[k] = dot;
+    const int per_warp = RC / 4;
+    for (int c0 = 0, ci = 0; c0 < p.n_ring; c0 += RC, ++ci) {
+      const int nc = min(RC, p.n_ring - c0);
+      if (ci > 0 && tid == 0) {
+        const uint32_t nbytes = (uint32_t)(nc * MD * es);
+        mbar_expect_tx(&ringbar, 2 * nbytes);
+        bulk_load(s_rk, ring_k + (int64_t)c0 * MD * es, nbytes, &ringbar);
+        bulk_load(s_rv, ring_v + (int64_t)c0 * MD * es, nbytes, &ringbar);
+      }
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&ringbar, (uint32_t)(ci & 1)));
+      if (!ok && lane == 0) {
+        atomicExch(p.err, 1);
+        s_abort = 1;
+      }
+      __syncthreads();
+      if (s_abort) {
+        if (tid == 0) (void)mbar_wait(&ringbar, (uint32_t)(ci & 1));
+        return;
+      }
+      const int sl = per_warp * warp + gid;
+      float l = -INFINITY;
+      if (gid < per_warp && sl < nc) {
+        const float* q = s_qf + tig * MD;
+        float dot = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < MD; ++j) dot = fmaf(q[j], load_f(s_rk, (int64_t)sl * MD + j, g.dtype), dot);
+        const int64_t rt = ((int64_t)(c0 + sl) - first % g.W + g.W) % g.W;
+        if (p.logits) p.logits[(int64_t)(bq0 + tig) * p.n_log + p.n_comp + rt] = dot;
+        l = dot * p.scale_log2;
       }
       float p0, p1;
-      softmax_step(lr[0], lr[1], p0, p1);
+      softmax_step(l, -INFINITY, p0, p1);
       // acc[mt][c]: channel 16 mt + gid (+8 for c >= 2), column 2 tig + (c & 1) = head tig;
       // add p * v into the hi column (c even) in code units
-      for (int T = 0; T < 16; ++T) {
-        const float pt = __shfl_sync(0xffffffffu, T < 8 ? p0 : p1, 4 * (T & 7) + tig);
-        const int rt = r0 + T;
-        if (rt >= p.n_ring) continue;
-        const int64_t slot = (first + rt) % g.W;
-        const int64_t e = ((int64_t)unit * g.W + slot) * MD;
+      for (int T = 0; T < per_warp; ++T) {
+        const float pt = __shfl_sync(0xffffffffu, p0, 4 * T + tig);
+        const int sl2 = per_warp * warp + T;
+        if (sl2 >= nc) break;
+        const int64_t e = (int64_t)sl2 * MD;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const float v0 = load_f(p.base + g.ring_v_off, e + 16 * mt + gid, g.dtype);
-          const float v1 = load_f(p.base + g.ring_v_off, e + 16 * mt + gid + 8, g.dtype);
+          const float v0 = load_f(s_rv, e + 16 * mt + gid, g.dtype);
+          const float v1 = load_f(s_rv, e + 16 * mt + gid + 8, g.dtype);
           acc[mt][0] = fmaf(pt * v0, code_unit, acc[mt][0]);
           acc[mt][2] = fmaf(pt * v1, code_unit, acc[mt][2]);
         }
       }
+      __syncthreads();     // the chunk is consumed before the next one is requested
     }
   }
 

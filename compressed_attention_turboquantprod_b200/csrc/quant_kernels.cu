@@ -427,6 +427,15 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
       s_cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
       s_cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
     }
+    {
+      // this thread's halves of its rows of Pi and T are read after the norm
+      const int half = tid & 1;
+      for (int j = tid >> 1; j < d; j += SMALL_THREADS / 2)
+        if (b1 > 0)
+          for (int c = half * (d / 2); c < (half + 1) * (d / 2); c += 32) prefetch_l2(p.Pi + (int64_t)j * d + c);
+      for (int a = tid >> 1; a < m; a += SMALL_THREADS / 2)
+        for (int c = half * (d / 2); c < (half + 1) * (d / 2); c += 32) prefetch_l2(p.T + (int64_t)a * d + c);
+    }
     int64_t e0;
     const void* src = src_row(p, false, bh, row, e0);
     double ss = 0.0;

@@ -147,6 +147,7 @@ def test_decode_identical_codes_lengths_and_splits(n_tokens, splits):
     # shapes of the tensor-core path (d=128, G=4, 2-bit values g=32)
     dict(m=256), dict(b1=1, m=64), dict(b1=0, m=128, dtype="f16"), dict(b1=0, m=256, W=3),
     dict(B=3, Hkv=5, Hq=20, W=1),
+    dict(W=40), dict(dtype="f32", W=20), dict(dtype="f16", W=33, b1=1),   # several ring chunks
 ])
 def test_decode_identical_codes_shapes(kw):
     w = _workload(**kw)
