@@ -195,24 +195,33 @@ def barrier(world):
         dist.barrier()
 
 
-def reduce_max(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op: str) -> float:
+    """All-reduce of one float over the ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = (torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl"
+           else torch.device("cpu"))
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def reduce_max(x: float, world: int) -> float:
+    return _reduce(x, world, "max")
 
 
 def reduce_sum(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, world, "sum")
+
+
+def aggregate(local_bytes: float, local_ms: float, world: int):
+    """Whole-job throughput: every rank's bytes over the slowest rank's device time.
+    Returns (GB/s, max ms)."""
+    ms = reduce_max(local_ms, world)
+    total = reduce_sum(local_bytes, world)
+    return total / (ms * 1e-3) / 1e9, ms
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -341,7 +350,7 @@ def run_ours(args):
     ws = cache.workspace(w.Hq, args.splits)
     out = torch.empty(w.B, w.Hq, w.d, dtype=w.torch_dtype, device=dev)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flush_r = torch.ones(64 << 20, dtype=torch.int32, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
     def flush_l2():
         flush_w.zero_()
@@ -359,16 +368,19 @@ def run_ours(args):
         app = w.B * w.Hkv * (2 * w.d * es + tb + 2 * w.d * es)   # read ring token + new token, write record + ring
         return dec, dec + app
 
-    def step(i, evs=None):
-        if evs:
+    def step(i, evs=None, around_partial=False):
+        """One step; evs = (start, end) events at the step's boundaries, or around
+        the partial kernel alone when around_partial (an event between two kernels
+        also ends the programmatic overlap of their launches)."""
+        if evs and not around_partial:
             evs[0].record(stream)
         native.tq_append(cache.state, Kn[i], Vn[i], pj.Pi, pj.T, cent, bnd)
         native.tq_decode_prep(cache.state, Qs[i], scale, pj.Pi, pj.S, cent, args.splits, ws)
-        if evs:
-            evs[1].record(stream)
+        if evs and around_partial:
+            evs[0].record(stream)
         native.tq_decode_partial(cache.state, w.Hq, scale, cent, None, args.splits, ws, out=out)
         if evs:
-            evs[2].record(stream)
+            evs[1].record(stream)
 
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
@@ -385,7 +397,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     dec_bytes, all_bytes = [], []
     for k in range(args.steps):
         flush_l2()
@@ -396,16 +408,24 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    # the same steps again, timing the partial kernel alone (roofline)
+    pevents = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    part_bytes_list = []
+    for k in range(args.steps):
+        flush_l2()
+        step(args.warmup + k, pevents[k], around_partial=True)
+        part_bytes_list.append(step_bytes()[0])
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
     clk = clocks.stop()
-    t_step = [e[0].elapsed_time(e[2]) for e in events]             # ms
-    t_part = [e[1].elapsed_time(e[2]) for e in events]
+    t_step = [e[0].elapsed_time(e[1]) for e in events]             # ms
+    t_part = [e[0].elapsed_time(e[1]) for e in pevents]
     tot_ms = sum(t_step)
-    tot_ms_max = reduce_max(tot_ms, world)
-    bytes_all = reduce_sum(float(sum(all_bytes)), world)
-    value = bytes_all / (tot_ms_max * 1e-3) / 1e9
+    value, tot_ms_max = aggregate(float(sum(all_bytes)), tot_ms, world)
     tokens_s = reduce_sum(float(w.B * args.steps), world) / (tot_ms_max * 1e-3)
     part_avg_ms = sum(t_part) / len(t_part)
-    part_bytes = sum(dec_bytes) / len(dec_bytes)
+    part_bytes = sum(part_bytes_list) / len(part_bytes_list)
     peak, peak_kind = measured_peak()
     src_hash = source_hash("decode_mma.cu")
     traffic = profiled_traffic("decode_partial_gqa32k.json", src_hash)

@@ -6,10 +6,14 @@
 // token at HBM speed.  Both contractions are dense (tokens x features x heads),
 // so they run on warp-level MMA:
 //
-//   logits  int8 mma.sync m16n8k32: A = key feature bits of 16 tokens as u8
-//           (0 or 128; one IMAD shift + one LOP3 per 4 bits), B = the query
-//           weights as three signed int8 slices of a 21-bit fixed-point value,
-//           so the integer accumulation is exact.  For a symmetric Lloyd-Max
+//   logits  int8 mma.sync m16n8k32: A = key feature bits of 16 tokens as u8,
+//           one AND per 4 bits: the stored bit of MMA index k sits at bit t of
+//           its byte (t = (k mod 16) / 4, + 4 for k >= 16), so the masked byte
+//           is 2^t or 2^(4+t); B = the query weights in 21-bit fixed point,
+//           times 2^(7-t) (resp. 2^(3-t)) so that every product carries the
+//           same 2^7, as four signed int8 slices (the two n-tiles hold the four
+//           slices of the four heads); the integer accumulation is exact.
+//           For a symmetric Lloyd-Max
 //           codebook c[idx] = sum over odd bit-subsets S of w_S (-1)^{xor of
 //           the bits in S} (a Walsh expansion whose even terms vanish), so the
 //           MSE term is linear in the stored bit-planes:
@@ -20,8 +24,9 @@
 //           per-channel power of two is undone once per split), B = p * s split
 //           into f16 hi + lo (the value scale s is per token and group).
 //
-// One CTA = one (batch, KV head, split) with 4 warps; each warp owns 16 of the
-// 64 tokens of every block and keeps its own online-softmax state; blocks are
+// One CTA = one (batch, KV head, split) with 4 warps; the two warp pairs take
+// alternate blocks and each warp owns 32 of the 64 tokens of its pair's blocks
+// (two m-tiles) and keeps its own online-softmax state; blocks are
 // staged in shared memory by cp.async.bulk with mbarrier completion (4 stages,
 // bounded waits that raise an error flag instead of hanging).  The last split
 // also folds in the exact ring tokens.  Warps merge at the end; the split's
@@ -82,13 +87,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-// Integer multiply kept as a multiply (the FMA-pipe IMAD), used for shifts by a
-// per-lane amount so that they do not occupy the integer ALU pipe.
-__device__ __forceinline__ uint32_t mul_lo(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
 
 // n consecutive 32-bit words from 16-byte-aligned shared memory, widest loads.
 template <int N>
@@ -154,9 +152,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
-// Exact int -> float for |x| <= 2^22 (mantissa add, no conversion unit).
-__device__ __forceinline__ float i2f_exact(int x) {
-  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+// s0 + 2^8 s1 + 2^16 s2 + 2^24 s3 for the four slice sums of a score (each below
+// 2^23 in magnitude): the pairs are joined exactly in 32-bit integers (< 2^31),
+// then converted once each; the result carries fp32 rounding only.
+__device__ __forceinline__ float slices_to_float(int s0, int s1, int s2, int s3) {
+  const int lo = s0 + 256 * s1, hi = s2 + 256 * s3;
+  return fmaf(65536.f, __int2float_rn(hi), __int2float_rn(lo));
 }
 
 // Workspace views used here: per (batch, KV head) unit, fragment words
@@ -167,7 +168,7 @@ __device__ __forceinline__ float i2f_exact(int x) {
 //  * qf = q in fp32 (for the ring), qr = Pi q, qs = sqrt(pi/2)/m S q, each row of
 //    [Pi; S] read once (a float4 per lane) and dotted with the four queries;
 //  * the Walsh weights of the codebook, the 21-bit fixed-point quantisation of
-//    the query weights and their three int8 slices laid out as the lanes' B
+//    the query weights and their four int8 slices laid out as the lanes' B
 //    fragments, and the per-head affine constants of the logit (log2 units);
 //  * zeroes the unit's split counter and, in CTA 0, the error flag.
 __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq, const float* Pi,
@@ -185,6 +186,7 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
   __shared__ unsigned s_maxM[MG], s_maxQ[MG];
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
+  pdl_launch_dependents();   // the partial kernel may launch; it waits for this grid
   {
     // the rows of [Pi; S] are read after the queries: start them towards L2 now
     const int lines_pi = b1 > 0 ? d * d / 32 : 0, lines = lines_pi + m * d / 32;
@@ -314,9 +316,11 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
     const int ln = wi & 31, r = (wi >> 5) & 1, nt = (wi >> 6) & 1, ks = wi >> 7;
     const int col = ln >> 2, tg = ln & 3;
     const int hh = col >> 1;
-    const int slice = nt == 0 ? (col & 1) : ((col & 1) ? -1 : 2);
+    const int slice = 2 * nt + (col & 1);
+    // the A byte of MMA index k carries 2^t (k < 16) or 2^(4+t) (k >= 16), t = tg
+    const int shift = r ? 3 - tg : 7 - tg;
     uint32_t word = 0;
-    if (slice >= 0) {
+    {
       const bool mse = ks < ksM;
       const float mx = __uint_as_float(mse ? s_maxM[hh] : s_maxQ[hh]);
       const float inv_delta = mx > 0.f ? two21 / mx : 1.f;
@@ -329,12 +333,14 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
         } else {
           w = 2.f * sqs[hh * m + (ks - ksM) * 32 + bit];
         }
-        const int wint = __float2int_rn(w * inv_delta);
+        const int wint = __float2int_rn(w * inv_delta) * (1 << shift);   // |wint| <= 2^28
         const int s0 = ((wint + 128) & 255) - 128;
         const int t1 = (wint - s0) >> 8;
         const int s1 = ((t1 + 128) & 255) - 128;
-        const int s2 = (t1 - s1) >> 8;
-        const int sv = slice == 0 ? s0 : slice == 1 ? s1 : s2;
+        const int t2 = (t1 - s1) >> 8;
+        const int s2 = ((t2 + 128) & 255) - 128;
+        const int s3 = (t2 - s2) >> 8;
+        const int sv = slice == 0 ? s0 : slice == 1 ? s1 : slice == 2 ? s2 : s3;
         word |= ((uint32_t)(sv & 255)) << (8 * i);
       }
     }
@@ -354,6 +360,7 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __shared__ float s_m[4][MG], s_l[4][MG];
   __shared__ float s_mn[4][MG][4];
   __shared__ int s_cnt[NST];
+  __shared__ int s_iss[NST];       // copies issued into each stage (for the error-path drain)
   __shared__ __align__(16) uint32_t s_frag[KS * 128];
   __shared__ __align__(8) uint64_t ringbar;
   __shared__ __align__(16) float s_qf[MG * MD];
@@ -389,15 +396,22 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     for (int s = 0; s < NST; ++s) mbar_init(&full[s], 1);
     mbar_init(&ringbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Launched programmatically after the preparation kernel: nothing that kernel or
+  // an earlier one writes is touched before this wait.
+  pdl_wait();
+  if (tid == 0) {
     if (ring_split) {
       const uint32_t nbytes = (uint32_t)(min(RC, p.n_ring) * MD * es);
       mbar_expect_tx(&ringbar, 2 * nbytes);
       bulk_load(s_rk, ring_k, nbytes, &ringbar);
       bulk_load(s_rv, ring_v, nbytes, &ringbar);
     }
+    for (int s = 0; s < NST; ++s) s_iss[s] = 0;
     for (int s = 0; s < NST && s < nb; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
       bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
+      s_iss[s] = 1;
     }
   }
   if (ring_split)
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __syncthreads();
   const uint4* bfr = reinterpret_cast<const uint4*>(s_frag) + lane;
 
-  const uint32_t mulA = 1u << (7 - tig), mulB = 1u << (3 - tig);
+  const uint32_t maskA = 0x01010101u << tig, maskB = 0x10101010u << tig;
   const uint32_t codeMask = 0x00030003u << (2 * (gid & 3));
   // PRMT selectors: result byte 0 <- byte bsel of token A's word, byte 2 <- byte
   // bsel of token B's word (bytes 1, 3 are masked off); bsel + 2 for channel + 8.
@@ -443,9 +457,10 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   // the accumulators) only when a logit exceeds it by more than kLazy (log2
   // units), so p <= 2^kLazy; the running sum is kept per lane and reduced once.
   constexpr float kLazy = 4.f;
-  auto softmax_step = [&](float l0, float l1, float& p0, float& p1) {
-    const float lmax = fmaxf(l0, l1);
-    if (__any_sync(0xffffffffu, lmax > m_run + kLazy)) {
+  // Raise the running max of head tig to at least the warp's max of lmax over gid,
+  // rescaling the running sum and the accumulators.
+  auto raise_max = [&](float lmax) {
+    {
       float mx = lmax;
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -463,6 +478,10 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) mnacc[gi] *= aP;
     }
+  };
+  auto softmax_step = [&](float l0, float l1, float& p0, float& p1) {
+    const float lmax = fmaxf(l0, l1);
+    if (__any_sync(0xffffffffu, lmax > m_run + kLazy)) raise_max(lmax);
     if (m_run == -INFINITY) {
       p0 = 0.f;
       p1 = 0.f;
@@ -473,10 +492,13 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     l_run += p0 + p1;
   };
 
-  int it = 0;
-  for (; it < nb; ++it) {
-    const int st = it % NST;
-    const uint32_t phase = (uint32_t)((it / NST) & 1);
+  // Warp w takes the blocks j = (w >> 1) (mod 2) of this split (stages alternate
+  // between the two warp pairs, NST even) and, in each, the 32 tokens
+  // 32 (w & 1) .. +31 as two 16-token m-tiles.
+  const int pair = warp >> 1, tb = 32 * (warp & 1);
+  for (int j = pair; j < nb; j += 2) {
+    const int st = j % NST;
+    const uint32_t phase = (uint32_t)((j / NST) & 1);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], phase));
     if (!ok) {
       if (lane == 0) {
@@ -486,101 +508,146 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     }
     if (ok) {
     const unsigned char* blk = stage + (size_t)st * bb;
-    const int64_t tok0 = (blk0 + it) * kBlockTokens;
+    const int64_t tok0 = (blk0 + j) * kBlockTokens;
     const int nt_valid = (int)min((int64_t)kBlockTokens, p.n_comp - tok0);
-    const int t0 = 16 * warp + gid, t1 = t0 + 8;
 
-    // ---------------- logits
-    float vM0 = 0.f, vM1 = 0.f, vQ0 = 0.f, vQ1 = 0.f;
+    // ---------------- logits of tokens tb + 16 r + gid + 8 e (r, e in {0, 1})
+    float vM[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, vQ[2][2];
     if constexpr (KSM > 0) {
-      uint32_t w0[KSM], w1[KSM];
-      lds_words<KSM>(blk + g.o_idx + t0 * (KSM * 4), w0);
-      lds_words<KSM>(blk + g.o_idx + t1 * (KSM * 4), w1);
-      int a[2][2][4] = {};   // [parity][ntile][4]: two independent chains per ntile
+      int a[2][2][4] = {};   // [m-tile][ntile][4]
 #pragma unroll
-      for (int ks = 0; ks < KSM; ++ks) {
-        const uint32_t a0 = mul_lo(w0[ks], mulA) & 0x80808080u, a1 = mul_lo(w1[ks], mulA) & 0x80808080u;
-        const uint32_t a2 = mul_lo(w0[ks], mulB) & 0x80808080u, a3 = mul_lo(w1[ks], mulB) & 0x80808080u;
-        const uint4 bq = bfr[ks * 32];
-        imma16832(a[ks & 1][0], a0, a1, a2, a3, bq.x, bq.y);
-        imma16832(a[ks & 1][1], a0, a1, a2, a3, bq.z, bq.w);
+      for (int c = 0; c < KSM; c += 4) {
+        uint32_t w[2][2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            lds_words<4>(blk + g.o_idx + (tb + 16 * r + gid + 8 * e) * (KSM * 4) + 4 * c, w[r][e]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint4 bq = bfr[(c + kk) * 32];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const uint32_t a0 = w[r][0][kk] & maskA, a1 = w[r][1][kk] & maskA;
+            const uint32_t a2 = w[r][0][kk] & maskB, a3 = w[r][1][kk] & maskB;
+            imma16832(a[r][0], a0, a1, a2, a3, bq.x, bq.y);
+            imma16832(a[r][1], a0, a1, a2, a3, bq.z, bq.w);
+          }
+        }
       }
-      int s00 = a[0][0][0] + a[1][0][0], s01 = a[0][0][1] + a[1][0][1], s10 = a[0][1][0] + a[1][1][0];
-      int s02 = a[0][0][2] + a[1][0][2], s03 = a[0][0][3] + a[1][0][3], s12 = a[0][1][2] + a[1][1][2];
-      vM0 = i2f_exact(s00) + 256.f * i2f_exact(s01) + 65536.f * i2f_exact(s10);
-      vM1 = i2f_exact(s02) + 256.f * i2f_exact(s03) + 65536.f * i2f_exact(s12);
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) vM[r][e] = slices_to_float(a[r][0][2 * e], a[r][0][2 * e + 1],
+                                                               a[r][1][2 * e], a[r][1][2 * e + 1]);
     }
     {
-      uint32_t w0[KSQ], w1[KSQ];
-      lds_words<KSQ>(blk + g.o_sign + t0 * (KSQ * 4), w0);
-      lds_words<KSQ>(blk + g.o_sign + t1 * (KSQ * 4), w1);
-      int a[2][4] = {};
+      constexpr int CQ4 = KSQ < 4 ? KSQ : 4;
+      int a[2][2][4] = {};
 #pragma unroll
-      for (int ks = 0; ks < KSQ; ++ks) {
-        const uint32_t a0 = mul_lo(w0[ks], mulA) & 0x80808080u, a1 = mul_lo(w1[ks], mulA) & 0x80808080u;
-        const uint32_t a2 = mul_lo(w0[ks], mulB) & 0x80808080u, a3 = mul_lo(w1[ks], mulB) & 0x80808080u;
-        const uint4 bq = bfr[(KSM + ks) * 32];
-        imma16832(a[0], a0, a1, a2, a3, bq.x, bq.y);
-        imma16832(a[1], a0, a1, a2, a3, bq.z, bq.w);
+      for (int c = 0; c < KSQ; c += CQ4) {
+        uint32_t w[2][2][CQ4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            lds_words<CQ4>(blk + g.o_sign + (tb + 16 * r + gid + 8 * e) * (KSQ * 4) + 4 * c, w[r][e]);
+#pragma unroll
+        for (int kk = 0; kk < CQ4; ++kk) {
+          const uint4 bq = bfr[(KSM + c + kk) * 32];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const uint32_t a0 = w[r][0][kk] & maskA, a1 = w[r][1][kk] & maskA;
+            const uint32_t a2 = w[r][0][kk] & maskB, a3 = w[r][1][kk] & maskB;
+            imma16832(a[r][0], a0, a1, a2, a3, bq.x, bq.y);
+            imma16832(a[r][1], a0, a1, a2, a3, bq.z, bq.w);
+          }
+        }
       }
-      vQ0 = i2f_exact(a[0][0]) + 256.f * i2f_exact(a[0][1]) + 65536.f * i2f_exact(a[1][0]);
-      vQ1 = i2f_exact(a[0][2]) + 256.f * i2f_exact(a[0][3]) + 65536.f * i2f_exact(a[1][2]);
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) vQ[r][e] = slices_to_float(a[r][0][2 * e], a[r][0][2 * e + 1],
+                                                               a[r][1][2 * e], a[r][1][2 * e + 1]);
     }
     const float* rho = reinterpret_cast<const float*>(blk + g.o_rho);
-    float l0, l1;
-    if (B1 > 0) {
-      const float* rn = reinterpret_cast<const float*>(blk + g.o_rnorm);
-      l0 = rho[t0] * fmaf(kM, vM0, CM) + rn[t0] * fmaf(kQ, vQ0, CQ);
-      l1 = rho[t1] * fmaf(kM, vM1, CM) + rn[t1] * fmaf(kQ, vQ1, CQ);
-    } else {
-      l0 = rho[t0] * fmaf(kQ, vQ0, CQ);
-      l1 = rho[t1] * fmaf(kQ, vQ1, CQ);
-    }
-    if (t0 >= nt_valid) l0 = -INFINITY;
-    if (t1 >= nt_valid) l1 = -INFINITY;
+    const float* rn = reinterpret_cast<const float*>(blk + g.o_rnorm);
+    float l[2][2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = tb + 16 * r + gid + 8 * e;
+        float v = B1 > 0 ? rho[t] * fmaf(kM, vM[r][e], CM) + rn[t] * fmaf(kQ, vQ[r][e], CQ)
+                         : rho[t] * fmaf(kQ, vQ[r][e], CQ);
+        if (t >= nt_valid) v = -INFINITY;
+        l[r][e] = v;
+      }
     if (p.logits) {
       const float inv = 1.f / p.scale_log2;
       float* lg = p.logits + (int64_t)(bq0 + tig) * p.n_log + tok0;
-      if (t0 < nt_valid) lg[t0] = l0 * inv;
-      if (t1 < nt_valid) lg[t1] = l1 * inv;
-    }
-
-    // ---------------- softmax
-    float p0, p1;
-    softmax_step(l0, l1, p0, p1);
-
-    // ---------------- P V
-    // tokens of this lane's B fragment (head hP): TA, TB = 2tig, 2tig+1; TC, TD = +8
-    const float pA = __shfl_sync(0xffffffffu, p0, 4 * (2 * tig) + hP);
-    const float pB = __shfl_sync(0xffffffffu, p0, 4 * (2 * tig + 1) + hP);
-    const float pC = __shfl_sync(0xffffffffu, p1, 4 * (2 * tig) + hP);
-    const float pD = __shfl_sync(0xffffffffu, p1, 4 * (2 * tig + 1) + hP);
-    const int TA = 16 * warp + 2 * tig, TB = TA + 1, TC = TA + 8, TD = TA + 9;
-    const float4* vs4 = reinterpret_cast<const float4*>(blk + g.o_vscale);
-    const float4* vm4 = reinterpret_cast<const float4*>(blk + g.o_vmin);
-    const float4 sA = vs4[TA], sB = vs4[TB], sC = vs4[TC], sD = vs4[TD];
-    const float4 mA = vm4[TA], mB = vm4[TB], mC = vm4[TC], mD = vm4[TD];
-    uint32_t bpv[4][2];
-    {
-      const float sa[4] = {sA.x, sA.y, sA.z, sA.w}, sb[4] = {sB.x, sB.y, sB.z, sB.w};
-      const float sc[4] = {sC.x, sC.y, sC.z, sC.w}, sd[4] = {sD.x, sD.y, sD.z, sD.w};
-      const float ma[4] = {mA.x, mA.y, mA.z, mA.w}, mb[4] = {mB.x, mB.y, mB.z, mB.w};
-      const float mc[4] = {mC.x, mC.y, mC.z, mC.w}, mdd[4] = {mD.x, mD.y, mD.z, mD.w};
 #pragma unroll
-      for (int gi = 0; gi < 4; ++gi) {
-        // tokens past the end have p = 0 and finite (zeroed or earlier) metadata
-        const float xA = pA * sa[gi], xB = pB * sb[gi], xC = pC * sc[gi], xD = pD * sd[gi];
-        // column gid even carries fp16(x), odd carries fp16(x - fp16(x))
-        const float2 f0 = __half22float2(__floats2half2_rn(xA, xB));
-        const float2 f1 = __half22float2(__floats2half2_rn(xC, xD));
-        __half2 h0 = __floats2half2_rn(fmaf(-oddf, f0.x, xA), fmaf(-oddf, f0.y, xB));
-        __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
-        bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
-        bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
-        mnacc[gi] = fmaf(pA, ma[gi], fmaf(pB, mb[gi], fmaf(pC, mc[gi], fmaf(pD, mdd[gi], mnacc[gi]))));
-      }
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = tb + 16 * r + gid + 8 * e;
+          if (t < nt_valid) lg[t] = l[r][e] * inv;
+        }
     }
+
+    // ---------------- softmax (lazy running max, see softmax_step)
+    float pr[2][2];
     {
+      const float lmax = fmaxf(fmaxf(l[0][0], l[0][1]), fmaxf(l[1][0], l[1][1]));
+      if (__any_sync(0xffffffffu, lmax > m_run + kLazy)) raise_max(lmax);
+      if (m_run == -INFINITY) {
+        pr[0][0] = pr[0][1] = pr[1][0] = pr[1][1] = 0.f;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) pr[r][e] = exp2f(l[r][e] - m_run);
+      }
+      l_run += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+    }
+
+    // ---------------- P V, one 16-token m-tile at a time
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      // MMA indices k = 2tig, 2tig+1, 2tig+8, 2tig+9 of this lane stand for the
+      // m-tile's tokens TA..TD = tig, tig+4, tig+8, tig+12 (a permutation of the 16
+      // tokens, the same for A and B) so that the four tig lanes read distinct
+      // shared-memory banks; their p (head hP) come from the score lanes gid = tig,
+      // tig + 4 (rows e = 0, 1).
+      const float pA = __shfl_sync(0xffffffffu, pr[r][0], 4 * tig + hP);
+      const float pB = __shfl_sync(0xffffffffu, pr[r][0], 4 * (tig + 4) + hP);
+      const float pC = __shfl_sync(0xffffffffu, pr[r][1], 4 * tig + hP);
+      const float pD = __shfl_sync(0xffffffffu, pr[r][1], 4 * (tig + 4) + hP);
+      const int TA = tb + 16 * r + tig, TB = TA + 4, TC = TA + 8, TD = TA + 12;
+      const float4* vs4 = reinterpret_cast<const float4*>(blk + g.o_vscale);
+      const float4* vm4 = reinterpret_cast<const float4*>(blk + g.o_vmin);
+      const float4 sA = vs4[TA], sB = vs4[TB], sC = vs4[TC], sD = vs4[TD];
+      const float4 mA = vm4[TA], mB = vm4[TB], mC = vm4[TC], mD = vm4[TD];
+      uint32_t bpv[4][2];
+      {
+        const float sa[4] = {sA.x, sA.y, sA.z, sA.w}, sb[4] = {sB.x, sB.y, sB.z, sB.w};
+        const float sc[4] = {sC.x, sC.y, sC.z, sC.w}, sd[4] = {sD.x, sD.y, sD.z, sD.w};
+        const float ma[4] = {mA.x, mA.y, mA.z, mA.w}, mb[4] = {mB.x, mB.y, mB.z, mB.w};
+        const float mc[4] = {mC.x, mC.y, mC.z, mC.w}, mdd[4] = {mD.x, mD.y, mD.z, mD.w};
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          // tokens past the end have p = 0 and finite (zeroed or earlier) metadata
+          const float xA = pA * sa[gi], xB = pB * sb[gi], xC = pC * sc[gi], xD = pD * sd[gi];
+          // column gid even carries fp16(x), odd carries fp16(x - fp16(x))
+          const float2 f0 = __half22float2(__floats2half2_rn(xA, xB));
+          const float2 f1 = __half22float2(__floats2half2_rn(xC, xD));
+          __half2 h0 = __floats2half2_rn(fmaf(-oddf, f0.x, xA), fmaf(-oddf, f0.y, xB));
+          __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
+          bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
+          bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
+          mnacc[gi] = fmaf(pA, ma[gi], fmaf(pB, mb[gi], fmaf(pC, mc[gi], fmaf(pD, mdd[gi], mnacc[gi]))));
+        }
+      }
       const uint4* vc = reinterpret_cast<const uint4*>(blk + g.o_vcode);   // 2 x uint4 per token
       const uint4 cA0 = vc[2 * TA], cA1 = vc[2 * TA + 1], cB0 = vc[2 * TB], cB1 = vc[2 * TB + 1];
       const uint4 cC0 = vc[2 * TC], cC1 = vc[2 * TC + 1], cD0 = vc[2 * TD], cD1 = vc[2 * TD + 1];
@@ -598,19 +665,21 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       }
     }
     }  // ok
-    // Release the stage: the last of the four warps to finish it refills it.
+    // Release the stage: the second warp of the pair to finish it refills it
+    // with block j + NST (same parity, so the same pair consumes it).
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
       const int done = atomicAdd(&s_cnt[st], 1);
-      if (done == 3) {
+      if (done == 1) {
         __threadfence_block();
         s_cnt[st] = 0;
-        if (it + NST < nb && !s_abort) {
+        if (j + NST < nb && !s_abort) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[st], (uint32_t)bb);
-          bulk_load(stage + (size_t)st * bb, region + (blk0 + it + NST) * bb, (uint32_t)bb,
+          bulk_load(stage + (size_t)st * bb, region + (blk0 + j + NST) * bb, (uint32_t)bb,
                     &full[st]);
+          s_iss[st] += 1;
         }
       }
     }
@@ -619,11 +688,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __syncthreads();
 
   if (s_abort) {
-    // a wait gave up: wait (bounded) for every copy this CTA may still have in
-    // flight (at most the last NST blocks), then leave
+    // a wait gave up: wait (bounded) for the last copy issued into every stage,
+    // then leave
     if (tid == 0) {
-      for (int j = (nb > NST ? nb - NST : 0); j < nb; ++j)
-        (void)mbar_wait(&full[j % NST], (uint32_t)((j / NST) & 1));
+      for (int s = 0; s < NST; ++s)
+        if (s_iss[s] > 0) (void)mbar_wait(&full[s], (uint32_t)((s_iss[s] - 1) & 1));
       if (ring_split) (void)mbar_wait(&ringbar, 0);
     }
     return;
@@ -779,8 +848,7 @@ cudaError_t launch_partial_t(const MParams& p, cudaStream_t s) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)p.splits, (unsigned)(p.g.B * p.g.Hkv));
-  k_decode_partial_mma<B1, KSQ><<<grid, MT, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k_decode_partial_mma<B1, KSQ>, grid, dim3(MT), smem, s, p);
 }
 
 }  // namespace

@@ -367,6 +367,10 @@ __global__ void __launch_bounds__(THREADS) k_quantize(QParams p) {
 
 __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V, int64_t n_old,
                              int64_t n_new) {
+  // launched programmatically: let the next kernel start, then wait for the
+  // previous one (which may still read the ring slots overwritten here)
+  pdl_launch_dependents();
+  pdl_wait();
   const int bh = blockIdx.x;
   const int es = (g.dtype == TQ_F32) ? 4 : 2;
   const int64_t n_tot = n_old + n_new;
@@ -410,6 +414,7 @@ __device__ __forceinline__ float half_row_dot(const float* rowp, const float* v,
 
 __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_launch_dependents();    // the ring write that follows waits for this kernel itself
   const int d = p.d, m = p.m, b1 = p.b1;
   float* sx = reinterpret_cast<float*>(smem_raw);       // [d]
   float* sy = sx + d;                                    // [d]  Pi x, then e = y - c[idx]
@@ -858,8 +863,7 @@ cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* b
 cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,
                               int64_t n_old, int64_t n_new, cudaStream_t s) {
   if (g.W == 0 || n_new == 0) return cudaSuccess;
-  k_ring_write<<<g.B * g.Hkv, 256, 0, s>>>(g, base, K, V, n_old, n_new);
-  return cudaGetLastError();
+  return launch_pdl(k_ring_write, dim3(g.B * g.Hkv), dim3(256), 0, s, g, base, K, V, n_old, n_new);
 }
 
 }  // namespace tq

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "tq.h"
@@ -93,5 +94,27 @@ cudaError_t launch_decode_partial(const Geom& g, const uint8_t* base, int64_t n_
                                   int splits, const DecodeWs& ws, cudaStream_t s);
 cudaError_t launch_decode_combine(const Geom& g, int Hq, void* out, int splits,
                                   const DecodeWs& ws, cudaStream_t s);
+
+// Launch with programmatic stream serialisation (programmatic dependent launch):
+// the kernel may begin once the previous kernel of the stream has let its
+// dependents launch (griddepcontrol.launch_dependents) instead of after that
+// kernel completes.  Every kernel launched this way executes
+// griddepcontrol.wait before it touches memory the previous kernel writes or
+// reads, so stream order is kept for data, and completion still chains.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace tq
