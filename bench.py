@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantize", action="store_true")
+    ap.add_argument("--no-other-decodes", action="store_true")
     ap.add_argument("--workload", default="gqa32k")
     return ap.parse_args()
 
@@ -436,20 +437,31 @@ def run_ours(args):
     e2e = None
     if args.steps > 0:
         n_e2e = min(args.steps, 100)
-        Qh = Qs[:n_e2e].cpu().pin_memory()
-        Kh = Kn[:n_e2e].cpu().pin_memory()
-        Vh = Vn[:n_e2e].cpu().pin_memory()
+        # one pinned host record per step holding that step's Q, new K and new V
+        # (bytes), copied with one H2D copy into a device record of the same shape
+        parts = [Qs[0], Kn[0], Vn[0]]
+        sizes = [t.numel() * t.element_size() for t in parts]
+        rec = sum(sizes)
+        host = torch.empty(n_e2e, rec, dtype=torch.uint8).pin_memory()
+        for k in range(n_e2e):
+            o = 0
+            for t, nbytes in zip((Qs[k], Kn[k], Vn[k]), sizes):
+                host[k, o:o + nbytes].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+                o += nbytes
+        dev_rec = torch.empty(rec, dtype=torch.uint8, device=dev)
+        views, o = [], 0
+        for t, nbytes in zip(parts, sizes):
+            views.append(dev_rec[o:o + nbytes].view(t.dtype).view(t.shape))
+            o += nbytes
+        qd, kd, vd = views
         outh = torch.empty(n_e2e, *out.shape, dtype=out.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(Qs[0]), torch.empty_like(Kn[0]), torch.empty_like(Vn[0])
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
         e2e_bytes = 0
         torch.cuda.synchronize()
         for k in range(n_e2e):
             flush_l2()
             ev[k][0].record(stream)
-            qd.copy_(Qh[k], non_blocking=True)
-            kd.copy_(Kh[k], non_blocking=True)
-            vd.copy_(Vh[k], non_blocking=True)
+            dev_rec.copy_(host[k], non_blocking=True)
             native.tq_append(cache.state, kd, vd, pj.Pi, pj.T, cent, bnd)
             native.tq_decode_attention(cache.state, qd, scale, pj.Pi, pj.S, cent, out, None,
                                        args.splits, ws)
@@ -459,8 +471,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ev), world)
         e2e_val = reduce_sum(float(e2e_bytes), world) / (e2e_ms * 1e-3) / 1e9
-        e2e = {"value": e2e_val, "unit": "GB/s",
-               "h2d_bytes_per_step": int(Qh[0].numel() * Qh.element_size() + 2 * Kh[0].numel() * Kh.element_size()),
+        e2e = {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": int(rec),
                "d2h_bytes_per_step": int(out.numel() * out.element_size()),
                "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e}
 
@@ -468,6 +479,11 @@ def run_ours(args):
     quant = None
     if not args.no_quantize:
         quant = bench_quantize(dev, world)
+    others = None
+    if not args.no_other_decodes:
+        del cache, Qs, Kn, Vn
+        torch.cuda.empty_cache()
+        others = bench_other_decodes(dev, world, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -493,6 +509,7 @@ def run_ours(args):
                      "avg_launch_ms": part_avg_ms, "source_hash": src_hash},
         "e2e": e2e,
         "quantize": quant,
+        "other_decodes": others,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": launches,
@@ -504,6 +521,89 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _time_decode(w, layer, dev, reps=10, warm=3):
+    """Full-size cache of workload w (layer `layer`), then prep + partial (merged
+    output) with L2 flushed before each decode; CUDA events around the partial.
+    Returns (mean partial ms, mean prep+partial ms, algorithmic bytes per decode)."""
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import (Codebook, CompressedKVCache, Projections,
+                                                           native)
+    m = w.m_for_layer(layer)
+    wl = w.scaled(m=m)
+    pj = Projections(wl.d, m, layer, rotation=wl.b1 > 0, device=dev)
+    cb = Codebook(wl.d, wl.b1, device=dev) if wl.b1 else None
+    cache = CompressedKVCache(wl.B, wl.Hkv, wl.d, wl.b1, m, wl.vbits, wl.group, wl.W, wl.T,
+                              dtype=wl.torch_dtype, device=dev)
+    K, V = synth.keys_values(wl, layer=layer, device=dev)
+    cache.append(K, V, pj, cb)
+    del K, V
+    torch.cuda.empty_cache()
+    Q = synth.queries(wl, layer=layer, device=dev)
+    ws = cache.workspace(wl.Hq, 0)
+    out = torch.empty(wl.B, wl.Hq, wl.d, dtype=wl.torch_dtype, device=dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(wl.d)
+    cent = cb.centroids if cb else None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for i in range(warm + reps):
+        flush_w.zero_()
+        flush_r.sum()
+        e = ev[i - warm] if i >= warm else None
+        if e:
+            e[0].record(stream)
+        native.tq_decode_prep(cache.state, Q, scale, pj.Pi, pj.S, cent, 0, ws)
+        if e:
+            e[1].record(stream)
+        native.tq_decode_partial(cache.state, wl.Hq, scale, cent, None, 0, ws, out=out)
+        if e:
+            e[2].record(stream)
+    torch.cuda.synchronize()
+    part = sum(a[1].elapsed_time(a[2]) for a in ev) / reps
+    whole = sum(a[0].elapsed_time(a[2]) for a in ev) / reps
+    es = 4 if wl.dtype == "f32" else 2
+    nbytes = wl.B * wl.Hkv * (cache.n_comp * cache.state.token_bytes + 2 * cache.n_ring * wl.d * es)
+    del cache, ws, out, flush_w, flush_r
+    torch.cuda.empty_cache()
+    return part, whole, nbytes
+
+
+def bench_other_decodes(dev, world, peak):
+    """The A-QJL (32 layers; one layer per sketch-size group timed, x8) and the
+    wide-head 262K decodes at full size."""
+    import synth
+    res = {}
+    w = synth.WORKLOADS["aqjl"]
+    groups, tot_ms, tot_bytes = [], 0.0, 0.0
+    for layer in (0, 8, 16, 24):
+        part, whole, nb = _time_decode(w, layer, dev)
+        part, whole = reduce_max(part, world), reduce_max(whole, world)
+        nb_all = reduce_sum(float(nb), world)
+        groups.append({"layers": f"{layer}-{layer + 7}", "m": w.m_for_layer(layer),
+                       "partial_ms": part, "decode_ms": whole, "GB_per_s": nb_all / (part * 1e-3) / 1e9,
+                       "frac_of_peak": nb / (part * 1e-3) / 1e9 / peak})
+        tot_ms += 8 * whole
+        tot_bytes += 8 * nb_all
+    res["aqjl"] = {"workload": "A-QJL: 32 layers, batch 16, 32 query heads over 8 KV heads, d=128, "
+                               "context 65536, pure QJL fp16 keys, m 512/384/256/192 by layer group, "
+                               "2-bit values g=32; one layer per group timed, times 8",
+                   "groups": groups, "GB_per_s": tot_bytes / (tot_ms * 1e-3) / 1e9,
+                   "tokens_per_s": reduce_sum(16.0, world) / (tot_ms * 1e-3),
+                   "ms_per_token_step": tot_ms}
+    w = synth.WORKLOADS["wide"]
+    part, whole, nb = _time_decode(w, 0, dev)
+    part, whole = reduce_max(part, world), reduce_max(whole, world)
+    nb_all = reduce_sum(float(nb), world)
+    res["wide"] = {"workload": "wide: batch 4, 16 query heads over 4 KV heads, d=256, context 262144, "
+                               "keys b1=3 + m=256, 4-bit values g=64",
+                   "partial_ms": part, "decode_ms": whole, "GB_per_s": nb_all / (part * 1e-3) / 1e9,
+                   "frac_of_peak": nb / (part * 1e-3) / 1e9 / peak,
+                   "tokens_per_s": reduce_sum(4.0, world) / (whole * 1e-3)}
+    return res
 
 
 def bench_quantize(dev, world, reps=3):

@@ -340,8 +340,8 @@ int decode_auto_splits(const Geom& g, int G, int64_t n_comp) {
   const int units = g.B * g.Hkv;
   int64_t s;
   if (decode_mma_supported(g, G)) {
-    // one wave of the tensor-core kernel (148 SMs x 4 resident CTAs), never more
-    s = (int64_t)(148 * 4) / units;
+    // one wave of the tensor-core kernel (148 SMs x its resident CTAs), never more
+    s = (int64_t)(148 * decode_mma_ctas_per_sm(g)) / units;
   } else {
     s = (kTargetCtas + units - 1) / units;
   }

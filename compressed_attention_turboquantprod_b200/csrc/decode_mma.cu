@@ -9,7 +9,7 @@
 //   logits  int8 mma.sync m16n8k32: A = key feature bits of 16 tokens as u8,
 //           one AND per 4 bits: the stored bit of MMA index k sits at bit t of
 //           its byte (t = (k mod 16) / 4, + 4 for k >= 16), so the masked byte
-//           is 2^t or 2^(4+t); B = the query weights in 21-bit fixed point,
+//           is 2^t or 2^(4+t); B = the query weights in 24-bit fixed point,
 //           times 2^(7-t) (resp. 2^(3-t)) so that every product carries the
 //           same 2^7, as four signed int8 slices (the two n-tiles hold the four
 //           slices of the four heads); the integer accumulation is exact.
@@ -33,144 +33,31 @@
 // (m, l, o) goes to the same workspace the combine kernel reads.
 //
 // Specialisation: head dim 128, G = 4, 2-bit values in groups of 32, b1 in
-// {0, 1, 2}, m in {64, 128, 256}.  Other shapes use decode_kernels.cu.
+// {0, 1, 2}, m in {64, 128, 192, 256, 384, 512}.  Other shapes use
+// decode_kernels.cu.
 #include <cfloat>
 
-#include "common.cuh"
+#include "mma_common.cuh"
 
 namespace tq {
 namespace {
+using namespace mmadec;
 
 constexpr int MD = 128;          // head dim of this path
-constexpr int MG = 4;            // query heads per KV head
 constexpr int NST = 4;           // pipeline stages (blocks in flight per CTA)
 constexpr int MT = 128;          // threads per CTA
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kWaitLimit = 1u << 22;
-
-struct MParams {
-  Geom g;
-  const uint8_t* base;
-  int64_t n_comp, n_total;
-  int n_ring, Hq;
-  float scale_log2;
-  float* logits;
-  int64_t n_log;
-  int splits, bps;
-  DecodeWs ws;
-  int* err;
-  void* out;        // when non-null, the last split of a unit also writes the output
-};
-
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void hmma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-
-// n consecutive 32-bit words from 16-byte-aligned shared memory, widest loads.
-template <int N>
-__device__ __forceinline__ void lds_words(const unsigned char* p, uint32_t (&w)[N]) {
-  if constexpr (N % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i) {
-      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
-      w[4 * i] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-  } else if constexpr (N % 2 == 0) {
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-      const uint2 v = reinterpret_cast<const uint2*>(p)[i];
-      w[2 * i] = v.x;
-      w[2 * i + 1] = v.y;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < N; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
-  }
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Bounded wait on phase `parity` of an mbarrier; false after kWaitLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
-}
-
-// s0 + 2^8 s1 + 2^16 s2 + 2^24 s3 for the four slice sums of a score (each below
-// 2^23 in magnitude): the pairs are joined exactly in 32-bit integers (< 2^31),
-// then converted once each; the result carries fp32 rounding only.
-__device__ __forceinline__ float slices_to_float(int s0, int s1, int s2, int s3) {
-  const int lo = s0 + 256 * s1, hi = s2 + 256 * s3;
-  return fmaf(65536.f, __int2float_rn(hi), __int2float_rn(lo));
-}
-
 // Workspace views used here: per (batch, KV head) unit, fragment words
-// [kstep][ntile][reg][lane] (uint32) and per head {kM, CM, kQ, CQ} (float).
+// [kstep][lane][ntile][reg] (uint32) and per head {kM, CM, kQ, CQ} (float).
 
 // ---------------------------------------------------------------- prep
 // One CTA per (b, KV head), for its G = 4 queries:
 //  * qf = q in fp32 (for the ring), qr = Pi q, qs = sqrt(pi/2)/m S q, each row of
 //    [Pi; S] read once (a float4 per lane) and dotted with the four queries;
-//  * the Walsh weights of the codebook, the 21-bit fixed-point quantisation of
+//  * the Walsh weights of the codebook, the 24-bit fixed-point quantisation of
 //    the query weights and their four int8 slices laid out as the lanes' B
 //    fragments, and the per-head affine constants of the logit (log2 units);
 //  * zeroes the unit's split counter and, in CTA 0, the error flag.
+template <int NV>     // float4s of a row per lane: head dim 128 * NV
 __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq, const float* Pi,
                                                   const float* S, const float* cent,
                                                   float scale_log2, DecodeWs ws) {
@@ -220,26 +107,35 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
   // Rows of [Pi; S] in passes of 8 per warp: lane l dots float4 l of each row
   // (coalesced) with columns 4l..4l+3 of the four queries (held in registers);
   // a reduce-scatter over the warp then leaves the sum of (row l/4, head l%4) in
-  // lane l.  (d = 128: one float4 per lane per row.)
-  float4 qv[MG];
+  // lane l.  (NV float4s per lane per row: columns 128 c + 4 lane.)
+  float4 qv[MG][NV];
 #pragma unroll
-  for (int hh = 0; hh < MG; ++hh) qv[hh] = *reinterpret_cast<const float4*>(sq + hh * d + 4 * lane);
+  for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+    for (int c = 0; c < NV; ++c)
+      qv[hh][c] = *reinterpret_cast<const float4*>(sq + hh * d + 128 * c + 4 * lane);
   const int R = rows_pi + m;
   for (int r0 = 8 * warp; r0 < R; r0 += 8 * (blockDim.x / 32)) {
-    float4 wv[8];
+    float4 wv[8][NV];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int r = r0 + k;
       const float* row = r < rows_pi ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
-      wv[k] = *reinterpret_cast<const float4*>(row + 4 * lane);
+#pragma unroll
+      for (int c = 0; c < NV; ++c) wv[k][c] = *reinterpret_cast<const float4*>(row + 128 * c + 4 * lane);
     }
     float v[32];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
 #pragma unroll
-      for (int hh = 0; hh < MG; ++hh)
-        v[4 * k + hh] = fmaf(wv[k].x, qv[hh].x, fmaf(wv[k].y, qv[hh].y,
-                        fmaf(wv[k].z, qv[hh].z, wv[k].w * qv[hh].w)));
+      for (int hh = 0; hh < MG; ++hh) {
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < NV; ++c)
+          a = fmaf(wv[k][c].x, qv[hh][c].x, fmaf(wv[k][c].y, qv[hh][c].y,
+              fmaf(wv[k][c].z, qv[hh][c].z, fmaf(wv[k][c].w, qv[hh][c].w, a))));
+        v[4 * k + hh] = a;
+      }
     // reduce-scatter: after the round with offset o, a lane keeps the half of its
     // values selected by (lane & o) and adds its partner's copy of that half
 #pragma unroll
@@ -297,10 +193,13 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
     }
   }
   __syncthreads();
-  const float two21 = 2097152.f;
+  // query weights in fixed point with |W| <= kFix = 2^24 - 2^17, so that W * 2^7
+  // (the largest A-byte compensation) stays below 2^31 and splits into four
+  // signed int8 slices
+  const float kFix = 16646144.f;
   if (tid < MG) {
     const float mM = __uint_as_float(s_maxM[tid]), mQ = __uint_as_float(s_maxQ[tid]);
-    const float dM = mM > 0.f ? mM / two21 : 1.f, dQ = mQ > 0.f ? mQ / two21 : 1.f;
+    const float dM = mM > 0.f ? mM / kFix : 1.f, dQ = mQ > 0.f ? mQ / kFix : 1.f;
     float wsum = 0.f;
     for (int k = 0; k < F; ++k) wsum += s_w[k];
     float* c = ws.qconst + ((int64_t)unit * MG + tid) * 4;
@@ -313,7 +212,8 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
   const int words = (ksM + ksQ) * 2 * 2 * 32;
   uint32_t* fr = ws.frag + (int64_t)unit * words;
   for (int wi = tid; wi < words; wi += blockDim.x) {
-    const int ln = wi & 31, r = (wi >> 5) & 1, nt = (wi >> 6) & 1, ks = wi >> 7;
+    // word order [ks][lane][ntile][reg]: a lane's four words of a k-step are one uint4
+    const int r = wi & 1, nt = (wi >> 1) & 1, ln = (wi >> 2) & 31, ks = wi >> 7;
     const int col = ln >> 2, tg = ln & 3;
     const int hh = col >> 1;
     const int slice = 2 * nt + (col & 1);
@@ -323,7 +223,7 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
     {
       const bool mse = ks < ksM;
       const float mx = __uint_as_float(mse ? s_maxM[hh] : s_maxQ[hh]);
-      const float inv_delta = mx > 0.f ? two21 / mx : 1.f;
+      const float inv_delta = mx > 0.f ? kFix / mx : 1.f;
       for (int i = 0; i < 4; ++i) {
         const int bit = tg + 8 * i + (r ? 4 : 0);
         float w;
@@ -333,7 +233,7 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
         } else {
           w = 2.f * sqs[hh * m + (ks - ksM) * 32 + bit];
         }
-        const int wint = __float2int_rn(w * inv_delta) * (1 << shift);   // |wint| <= 2^28
+        const int wint = __float2int_rn(w * inv_delta) * (1 << shift);   // |wint| < 2^31
         const int s0 = ((wint + 128) & 255) - 128;
         const int t1 = (wint - s0) >> 8;
         const int s1 = ((t1 + 128) & 255) - 128;
@@ -420,11 +320,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   // B fragments of the score (query slices), per k-step and lane four words
   // {ntile0 r0, ntile0 r1, ntile1 r0, ntile1 r1}, staged in shared memory.
   {
-    const uint32_t* fr = p.ws.frag + (int64_t)unit * (KS * 128);
-    for (int i = tid; i < KS * 128; i += MT) {
-      const int ln = i & 31, r = (i >> 5) & 1, nt = (i >> 6) & 1, ks = i >> 7;
-      s_frag[(ks * 32 + ln) * 4 + nt * 2 + r] = fr[i];
-    }
+    const uint4* fr = reinterpret_cast<const uint4*>(p.ws.frag + (int64_t)unit * (KS * 128));
+    for (int i = tid; i < KS * 32; i += MT) reinterpret_cast<uint4*>(s_frag)[i] = fr[i];
   }
   const float* qc = p.ws.qconst + ((int64_t)unit * MG + tig) * 4;
   const float kM = qc[0], CM = qc[1], kQ = qc[2], CQ = qc[3];
@@ -474,9 +371,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[i][c] *= alpha;
-      const float aP = __shfl_sync(0xffffffffu, alpha, hP);     // lane hP has tig == hP
 #pragma unroll
-      for (int gi = 0; gi < 4; ++gi) mnacc[gi] *= aP;
+      for (int gi = 0; gi < 4; ++gi) mnacc[gi] *= alpha;       // head tig, like m_run
     }
   };
   auto softmax_step = [&](float l0, float l1, float& p0, float& p1) {
@@ -542,7 +438,7 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
                                                                a[r][1][2 * e], a[r][1][2 * e + 1]);
     }
     {
-      constexpr int CQ4 = KSQ < 4 ? KSQ : 4;
+      constexpr int CQ4 = KSQ % 4 == 0 ? 4 : 2;       // words per shared-memory load
       int a[2][2][4] = {};
 #pragma unroll
       for (int c = 0; c < KSQ; c += CQ4) {
@@ -609,6 +505,18 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
           for (int e = 0; e < 2; ++e) pr[r][e] = exp2f(l[r][e] - m_run);
       }
       l_run += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+      // the value minima enter as sum_t p_t mn_{t,g} per head (tig) and group
+      const float4* vm4 = reinterpret_cast<const float4*>(blk + g.o_vmin);
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float4 mv = vm4[tb + 16 * r + gid + 8 * e];
+          mnacc[0] = fmaf(pr[r][e], mv.x, mnacc[0]);
+          mnacc[1] = fmaf(pr[r][e], mv.y, mnacc[1]);
+          mnacc[2] = fmaf(pr[r][e], mv.z, mnacc[2]);
+          mnacc[3] = fmaf(pr[r][e], mv.w, mnacc[3]);
+        }
     }
 
     // ---------------- P V, one 16-token m-tile at a time
@@ -625,15 +533,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       const float pD = __shfl_sync(0xffffffffu, pr[r][1], 4 * (tig + 4) + hP);
       const int TA = tb + 16 * r + tig, TB = TA + 4, TC = TA + 8, TD = TA + 12;
       const float4* vs4 = reinterpret_cast<const float4*>(blk + g.o_vscale);
-      const float4* vm4 = reinterpret_cast<const float4*>(blk + g.o_vmin);
       const float4 sA = vs4[TA], sB = vs4[TB], sC = vs4[TC], sD = vs4[TD];
-      const float4 mA = vm4[TA], mB = vm4[TB], mC = vm4[TC], mD = vm4[TD];
       uint32_t bpv[4][2];
       {
         const float sa[4] = {sA.x, sA.y, sA.z, sA.w}, sb[4] = {sB.x, sB.y, sB.z, sB.w};
         const float sc[4] = {sC.x, sC.y, sC.z, sC.w}, sd[4] = {sD.x, sD.y, sD.z, sD.w};
-        const float ma[4] = {mA.x, mA.y, mA.z, mA.w}, mb[4] = {mB.x, mB.y, mB.z, mB.w};
-        const float mc[4] = {mC.x, mC.y, mC.z, mC.w}, mdd[4] = {mD.x, mD.y, mD.z, mD.w};
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
           // tokens past the end have p = 0 and finite (zeroed or earlier) metadata
@@ -645,7 +549,6 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
           __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
           bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
           bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
-          mnacc[gi] = fmaf(pA, ma[gi], fmaf(pB, mb[gi], fmaf(pC, mc[gi], fmaf(pD, mdd[gi], mnacc[gi]))));
         }
       }
       const uint4* vc = reinterpret_cast<const uint4*>(blk + g.o_vcode);   // 2 x uint4 per token
@@ -767,13 +670,14 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     s_m[warp][tig] = m_run;
     s_l[warp][tig] = l_run;
   }
-  // mn sums: lanes of the hi column (gid even) of head hP, reduce over tig
+  // mn sums of head tig: reduce over gid
 #pragma unroll
   for (int gi = 0; gi < 4; ++gi) {
-    float v = odd ? 0.f : mnacc[gi];
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    if (tig == 0 && !odd) s_mn[warp][hP][gi] = v;
+    float v = mnacc[gi];
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    if (gid == 0) s_mn[warp][tig][gi] = v;
   }
   __syncthreads();
   // this lane's channels, head tig: o = code part (hi + lo) + mn part, scaled to the CTA max
@@ -854,17 +758,21 @@ cudaError_t launch_partial_t(const MParams& p, cudaStream_t s) {
 }  // namespace
 
 bool decode_mma_supported(const Geom& g, int G) {
+  if (decode_wide_supported(g, G)) return true;
   return g.d == MD && G == MG && g.vbits == 2 && g.group == 32 && g.b1 <= 2 &&
-         (g.m == 64 || g.m == 128 || g.m == 256);
+         (g.m == 64 || g.m == 128 || g.m == 192 || g.m == 256 || g.m == 384 || g.m == 512);
 }
+
+int decode_mma_ctas_per_sm(const Geom& g) { return g.d == 256 ? 2 : 4; }
 
 cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
                                    const float* S, const float* cent, float scale,
                                    const DecodeWs& ws, cudaStream_t s) {
   const size_t smem = sizeof(float) * MG * (2 * g.d + g.m);
-  cudaError_t e = cudaFuncSetAttribute(k_prep_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = g.d == 256 ? k_prep_mma<2> : k_prep_mma<1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_prep_mma<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws);
+  kern<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws);
   return cudaGetLastError();
 }
 
@@ -887,17 +795,27 @@ cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_
   p.bps = (int)((nblk + splits - 1) / splits);
   p.ws = ws;
   p.err = ws.err;
+  if (g.d == 256) return launch_partial_wide(p, s);
   const int ksq = g.m / 32;
-  switch (g.b1 * 16 + ksq) {
-    case 0 * 16 + 2: return launch_partial_t<0, 2>(p, s);
-    case 0 * 16 + 4: return launch_partial_t<0, 4>(p, s);
-    case 0 * 16 + 8: return launch_partial_t<0, 8>(p, s);
-    case 1 * 16 + 2: return launch_partial_t<1, 2>(p, s);
-    case 1 * 16 + 4: return launch_partial_t<1, 4>(p, s);
-    case 1 * 16 + 8: return launch_partial_t<1, 8>(p, s);
-    case 2 * 16 + 2: return launch_partial_t<2, 2>(p, s);
-    case 2 * 16 + 4: return launch_partial_t<2, 4>(p, s);
-    case 2 * 16 + 8: return launch_partial_t<2, 8>(p, s);
+  switch (g.b1 * 32 + ksq) {
+    case 0 * 32 + 2: return launch_partial_t<0, 2>(p, s);
+    case 0 * 32 + 4: return launch_partial_t<0, 4>(p, s);
+    case 0 * 32 + 6: return launch_partial_t<0, 6>(p, s);
+    case 0 * 32 + 8: return launch_partial_t<0, 8>(p, s);
+    case 0 * 32 + 12: return launch_partial_t<0, 12>(p, s);
+    case 0 * 32 + 16: return launch_partial_t<0, 16>(p, s);
+    case 1 * 32 + 2: return launch_partial_t<1, 2>(p, s);
+    case 1 * 32 + 4: return launch_partial_t<1, 4>(p, s);
+    case 1 * 32 + 6: return launch_partial_t<1, 6>(p, s);
+    case 1 * 32 + 8: return launch_partial_t<1, 8>(p, s);
+    case 1 * 32 + 12: return launch_partial_t<1, 12>(p, s);
+    case 1 * 32 + 16: return launch_partial_t<1, 16>(p, s);
+    case 2 * 32 + 2: return launch_partial_t<2, 2>(p, s);
+    case 2 * 32 + 4: return launch_partial_t<2, 4>(p, s);
+    case 2 * 32 + 6: return launch_partial_t<2, 6>(p, s);
+    case 2 * 32 + 8: return launch_partial_t<2, 8>(p, s);
+    case 2 * 32 + 12: return launch_partial_t<2, 12>(p, s);
+    case 2 * 32 + 16: return launch_partial_t<2, 16>(p, s);
     default: return cudaErrorInvalidValue;
   }
 }

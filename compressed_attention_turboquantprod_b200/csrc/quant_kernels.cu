@@ -694,31 +694,63 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
   vs.X = s.YZ;
   vs.vs = s.vs;
   vs.vm = s.vm;
+  // Bring the key and value rows of a tile towards L2 (one hint per 128-byte line).
+  const int es = p.dtype == TQ_F32 ? 4 : 2, lpr = QD * es / 128;
+  auto prefetch_tile = [&](int64_t t) {
+    if (t >= total_tiles) return;
+    const int pbh = (int)(t / tiles_per_bh);
+    const int64_t prow0 = (t % tiles_per_bh) * NT;
+    for (int i = tid; i < NT * 2 * lpr; i += QTHREADS) {
+      const int r = i / (2 * lpr), which = (i / lpr) & 1, ln = i % lpr;
+      if (prow0 + r >= p.n || (which && !p.do_values)) continue;
+      int64_t e0;
+      const void* src = src_row(p, which != 0, pbh, prow0 + r, e0);
+      prefetch_l2(reinterpret_cast<const char*>(src) + e0 * es + 128 * ln);
+    }
+  };
+  prefetch_tile(blockIdx.x);
+  constexpr int RPW = NT / (QTHREADS / 32);      // key rows per warp
   for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
     const int bh = (int)(tile / tiles_per_bh);
     const int64_t row0 = (tile % tiles_per_bh) * NT;
-    // ---- keys: rho (float64), U = X / rho as fp16 hi/lo
-    for (int r = warp; r < NT; r += QTHREADS / 32) {
-      const bool valid = row0 + r < p.n;
-      int64_t e0 = 0;
-      const void* src = valid ? src_row(p, false, bh, row0 + r, e0) : nullptr;
-      float x[QD / 32];
-      double ss = 0.0;
+    prefetch_tile(tile + gridDim.x);
+    // ---- keys: rho (float64), U = X / rho as fp16 hi/lo; a warp's rows are all
+    // loaded (4 consecutive elements a lane) before their reductions
+    {
+      float x[RPW][4];
 #pragma unroll
-      for (int k = 0; k < QD / 32; ++k) {
-        x[k] = valid ? load_f(src, e0 + lane + 32 * k, p.dtype) : 0.f;
-        ss += (double)x[k] * (double)x[k];
+      for (int i = 0; i < RPW; ++i) {
+        const int r = warp + i * (QTHREADS / 32);
+        if (row0 + r < p.n) {
+          int64_t e0;
+          const void* src = src_row(p, false, bh, row0 + r, e0);
+          load4(src, e0 + 4 * lane, p.dtype, x[i]);
+        } else {
+          x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+        }
       }
-      ss = warp_sum_d(ss);
-      const double rho = sqrt(ss);
-      const float inv = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
-      if (lane == 0) {
-        s.rho64[r] = rho;
-        s.rho[r] = (float)rho;
+      double ss[RPW];
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        ss[i] = 0.0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ss[i] += (double)x[i][k] * (double)x[i][k];
       }
 #pragma unroll
-      for (int k = 0; k < QD / 32; ++k)
-        split_store(s.AH + r * HS + lane + 32 * k, s.AL + r * HS + lane + 32 * k, x[k] * inv);
+      for (int i = 0; i < RPW; ++i) ss[i] = warp_sum_d(ss[i]);
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        const int r = warp + i * (QTHREADS / 32);
+        const double rho = sqrt(ss[i]);
+        const float inv = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
+        if (lane == 0) {
+          s.rho64[r] = rho;
+          s.rho[r] = (float)rho;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          split_store(s.AH + r * HS + 4 * lane + k, s.AL + r * HS + 4 * lane + k, x[i][k] * inv);
+      }
     }
     __syncthreads();
     mma_gemm_64x128(s.AH, s.AL, s.PH, s.PL, s.YZ);           // Y = U Pi^T

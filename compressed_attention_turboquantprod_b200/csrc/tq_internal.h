@@ -80,6 +80,7 @@ int decode_auto_splits(const Geom& g, int G, int64_t n_comp);
 
 // tensor-core path (decode_mma.cu)
 bool decode_mma_supported(const Geom& g, int G);
+int decode_mma_ctas_per_sm(const Geom& g);      // resident CTAs per SM of the partial kernel
 cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
                                    const float* S, const float* cent, float scale,
                                    const DecodeWs& ws, cudaStream_t s);

@@ -148,6 +148,13 @@ def test_decode_identical_codes_lengths_and_splits(n_tokens, splits):
     dict(m=256), dict(b1=1, m=64), dict(b1=0, m=128, dtype="f16"), dict(b1=0, m=256, W=3),
     dict(B=3, Hkv=5, Hq=20, W=1),
     dict(W=40), dict(dtype="f32", W=20), dict(dtype="f16", W=33, b1=1),   # several ring chunks
+    dict(m=384), dict(b1=1, m=512, W=7), dict(b1=0, m=192, dtype="f16"),  # larger sketches
+    # shapes of the head-dim-256 tensor-core path (G=4, 4-bit values g=64)
+    dict(d=256, b1=3, m=256, vbits=4, group=64, Hq=16, Hkv=4),
+    dict(d=256, b1=3, m=128, vbits=4, group=64, dtype="f32", W=5),
+    dict(d=256, b1=2, m=256, vbits=4, group=64, W=20),
+    dict(d=256, b1=0, m=128, vbits=4, group=64, Hq=4, Hkv=1, dtype="f16", W=0),
+    dict(d=256, b1=1, m=256, vbits=4, group=64, dtype="f16", W=9),
 ])
 def test_decode_identical_codes_shapes(kw):
     w = _workload(**kw)
@@ -189,6 +196,12 @@ def test_staged_decode_fused_and_separate_merge(n_tokens, splits):
         check_out(host(sep), ro, w.dtype)
         diff = (fused.float() - sep.float()).abs().max().item()
         assert diff <= 2 * float(torch.finfo(TORCH_DT[w.dtype]).eps)
+
+
+@pytest.mark.parametrize("n_tokens,splits", [(1, 0), (80, 2), (333, 3), (2000, 0), (3000, 40)])
+def test_decode_identical_codes_wide_lengths_and_splits(n_tokens, splits):
+    w = _workload(d=256, b1=3, m=256, vbits=4, group=64, Hq=8, Hkv=2)
+    _decode_identical_codes(w, n_tokens, max(1024, n_tokens + 64), splits)
 
 
 def test_decode_empty_cache_is_zero():
