@@ -106,6 +106,24 @@ class CompressedKVCache:
             self._ws = torch.empty(need, dtype=torch.uint8, device=self.buffer.device)
         return self._ws
 
+    def decode_step(self, K: torch.Tensor, V: torch.Tensor, Q: torch.Tensor, proj: Projections,
+                    cb: Optional[Codebook], softmax_scale: Optional[float] = None,
+                    want_logits: bool = False, num_splits: int = 0,
+                    out: Optional[torch.Tensor] = None):
+        """append(K, V) then decode(Q) as one call (fused when the shapes allow)."""
+        B, Hq, d = Q.shape
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+        out = torch.empty_like(Q) if out is None else out
+        logits = None
+        if want_logits:        # compressed + ring tokens after the append
+            logits = torch.empty(B, Hq, self.n_total + K.shape[2], dtype=torch.float32,
+                                 device=Q.device)
+        ws = self.workspace(Hq, num_splits)
+        native.tq_decode_step(self.state, K, V, Q, scale, proj.Pi, proj.S, proj.T,
+                              cb.centroids if cb is not None else None,
+                              cb.boundaries if cb is not None else None, out, logits, num_splits, ws)
+        return (out, logits) if want_logits else out
+
     def decode(self, Q: torch.Tensor, proj: Projections, cb: Optional[Codebook],
                softmax_scale: Optional[float] = None, want_logits: bool = False,
                num_splits: int = 0, out: Optional[torch.Tensor] = None):

@@ -360,13 +360,11 @@ int64_t tq_cache_ring_tokens(const tq_cache* c) {
   return c->n_total < c->desc.W ? c->n_total : c->desc.W;
 }
 
-int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const float* Pi,
-              const float* T, const float* centroids, const float* boundaries, void* stream) {
-  TQ_FAULT_POINT("tq_append");
-  int st = check_cache(c);
-  if (st != TQ_OK) return st;
-  if (n_new < 0) return fail(TQ_ERR_INVALID_ARG, "n_new=%lld", (long long)n_new);
-  if (n_new == 0) return ok();
+// Arguments of an append of n_new >= 1 tokens; the compressed-token counts before
+// and after go to *c_old / *c_new.
+static int append_checks(const tq_cache* c, const void* K, const void* V, int64_t n_new,
+                         const float* Pi, const float* T, const float* centroids,
+                         const float* boundaries, int64_t* c_old_out, int64_t* c_new_out) {
   if (!K || !V || !aligned16(K) || !aligned16(V))
     return fail(TQ_ERR_INVALID_ARG, "K and V must be non-null and 16-byte aligned");
   const tq_cache_desc& dsc = c->desc;
@@ -380,6 +378,24 @@ int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const fl
     if (!T || !aligned16(T) || (dsc.b1 > 0 && (!Pi || !centroids || !boundaries || !aligned16(Pi))))
       return fail(TQ_ERR_INVALID_ARG, "projections / codebook pointers missing");
   }
+  *c_old_out = c_old;
+  *c_new_out = c_new;
+  return TQ_OK;
+}
+
+int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const float* Pi,
+              const float* T, const float* centroids, const float* boundaries, void* stream) {
+  TQ_FAULT_POINT("tq_append");
+  int st = check_cache(c);
+  if (st != TQ_OK) return st;
+  if (n_new < 0) return fail(TQ_ERR_INVALID_ARG, "n_new=%lld", (long long)n_new);
+  if (n_new == 0) return ok();
+  const tq_cache_desc& dsc = c->desc;
+  const int64_t n_old = c->n_total, n_tot = n_old + n_new;
+  int64_t c_old = 0, c_new = 0;
+  st = append_checks(c, K, V, n_new, Pi, T, centroids, boundaries, &c_old, &c_new);
+  if (st != TQ_OK) return st;
+  (void)dsc;
   st = check_pending("tq_append");
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -407,19 +423,27 @@ size_t tq_decode_workspace_bytes(const tq_cache* c, int Hq, int num_splits) {
   return tq::decode_ws_bytes(tq::geom_of(c), Hq, max_splits(c, Hq, num_splits));
 }
 
-static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
-                        const float* Pi, const float* S, const float* centroids, void* out,
-                        float* logits, int num_splits, void* workspace, size_t ws_bytes,
-                        void* stream, bool prep, bool partial, bool combine, const char* name) {
+struct DecodePlan {
+  tq::Geom g;
+  int splits = 1;
+  bool mma = false;
+  tq::DecodeWs ws{};
+};
+
+// Every check of a decode (or of its stages) on cache state c, before any launch.
+static int decode_plan(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                       const float* Pi, const float* S, const float* centroids, void* out,
+                       int num_splits, void* workspace, size_t ws_bytes, bool prep, bool partial,
+                       bool combine, const char* name, DecodePlan& P) {
   int st = check_decode_common(c, Hq, num_splits);
   if (st != TQ_OK) return st;
   const tq_cache_desc& dsc = c->desc;
-  tq::Geom g = tq::geom_of(c);
+  P.g = tq::geom_of(c);
   const int64_t n_comp = n_comp_of(c);
   const int G = Hq / dsc.Hkv;
-  const int splits = eff_splits(g, G, n_comp, num_splits);
-  const bool mma = tq::decode_mma_supported(g, G);
-  const size_t need = tq::decode_ws_bytes(g, Hq, splits);
+  P.splits = eff_splits(P.g, G, n_comp, num_splits);
+  P.mma = tq::decode_mma_supported(P.g, G);
+  const size_t need = tq::decode_ws_bytes(P.g, Hq, P.splits);
   if (!workspace || !aligned16(workspace) || ws_bytes < need)
     return fail(TQ_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed", name, need);
   if (prep) {
@@ -431,31 +455,49 @@ static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_
     if (dsc.b1 > 0 && !centroids) return fail(TQ_ERR_INVALID_ARG, "%s: centroids needed", name);
   }
   if (combine && !out) return fail(TQ_ERR_INVALID_ARG, "%s: out needed", name);
-  st = check_pending(name);
-  if (st != TQ_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  tq::DecodeWs ws = tq::decode_ws_carve(workspace, g, Hq, splits);
+  P.ws = tq::decode_ws_carve(workspace, P.g, Hq, P.splits);
+  return TQ_OK;
+}
+
+static int decode_launch(const tq_cache* c, const DecodePlan& P, const void* Q, int Hq,
+                         float softmax_scale, const float* Pi, const float* S,
+                         const float* centroids, void* out, float* logits, cudaStream_t s,
+                         bool prep, bool partial, bool combine, const char* name) {
   cudaError_t e = cudaSuccess;
   if (prep) {
-    e = mma ? tq::launch_decode_prep_mma(g, Q, Hq, Pi, S, centroids, softmax_scale, ws, s)
-            : tq::launch_decode_prep(g, Q, Hq, Pi, S, ws, s);
+    e = P.mma ? tq::launch_decode_prep_mma(P.g, Q, Hq, Pi, S, centroids, softmax_scale, P.ws, s)
+              : tq::launch_decode_prep(P.g, Q, Hq, Pi, S, P.ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
   }
   if (partial) {
     // the tensor-core partial kernel merges the splits itself when given `out`
-    void* fused_out = (mma && combine) ? out : nullptr;
-    e = mma ? tq::launch_decode_partial_mma(g, static_cast<const uint8_t*>(c->base), c->n_total,
-                                            Hq, softmax_scale, logits, splits, ws, fused_out, s)
-            : tq::launch_decode_partial(g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
-                                        softmax_scale, centroids, logits, splits, ws, s);
+    void* fused_out = (P.mma && combine) ? out : nullptr;
+    e = P.mma ? tq::launch_decode_partial_mma(P.g, static_cast<const uint8_t*>(c->base), c->n_total,
+                                              Hq, softmax_scale, logits, P.splits, P.ws, fused_out, s)
+              : tq::launch_decode_partial(P.g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
+                                          softmax_scale, centroids, logits, P.splits, P.ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
     if (fused_out) combine = false;
   }
   if (combine) {
-    e = tq::launch_decode_combine(g, Hq, out, splits, ws, s);
+    e = tq::launch_decode_combine(P.g, Hq, out, P.splits, P.ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
   }
   return ok();
+}
+
+static int decode_stage(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
+                        const float* Pi, const float* S, const float* centroids, void* out,
+                        float* logits, int num_splits, void* workspace, size_t ws_bytes,
+                        void* stream, bool prep, bool partial, bool combine, const char* name) {
+  DecodePlan P;
+  int st = decode_plan(c, Q, Hq, softmax_scale, Pi, S, centroids, out, num_splits, workspace,
+                       ws_bytes, prep, partial, combine, name, P);
+  if (st != TQ_OK) return st;
+  st = check_pending(name);
+  if (st != TQ_OK) return st;
+  return decode_launch(c, P, Q, Hq, softmax_scale, Pi, S, centroids, out, logits,
+                       static_cast<cudaStream_t>(stream), prep, partial, combine, name);
 }
 
 int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_scale,
@@ -465,6 +507,47 @@ int tq_decode_attention(const tq_cache* c, const void* Q, int Hq, float softmax_
   TQ_FAULT_POINT("tq_decode_attention");
   return decode_stage(c, Q, Hq, softmax_scale, Pi, S, centroids, out, logits, num_splits,
                       workspace, ws_bytes, stream, true, true, true, "tq_decode_attention");
+}
+
+int tq_decode_step(tq_cache* c, const void* K, const void* V, int64_t n_new, const void* Q, int Hq,
+                   float softmax_scale, const float* Pi, const float* S, const float* T,
+                   const float* centroids, const float* boundaries, void* out, float* logits,
+                   int num_splits, void* workspace, size_t ws_bytes, void* stream) {
+  TQ_FAULT_POINT("tq_decode_step");
+  int st = check_cache(c);
+  if (st != TQ_OK) return st;
+  if (n_new < 0) return fail(TQ_ERR_INVALID_ARG, "n_new=%lld", (long long)n_new);
+  const tq_cache_desc& dsc = c->desc;
+  const tq::Geom g = tq::geom_of(c);
+  const bool fusable = n_new >= 1 && n_new <= 8 && n_new <= dsc.W && dsc.Hkv > 0 &&
+                       Hq % dsc.Hkv == 0 && tq::decode_mma_supported(g, Hq / dsc.Hkv);
+  if (!fusable) {
+    st = tq_append(c, K, V, n_new, Pi, T, centroids, boundaries, stream);
+    if (st != TQ_OK) return st;
+    return tq_decode_attention(c, Q, Hq, softmax_scale, Pi, S, centroids, out, logits, num_splits,
+                               workspace, ws_bytes, stream);
+  }
+  int64_t c_old = 0, c_new = 0;
+  st = append_checks(c, K, V, n_new, Pi, T, centroids, boundaries, &c_old, &c_new);
+  if (st != TQ_OK) return st;
+  const int64_t n_old = c->n_total, n_tot = n_old + n_new;
+  tq_cache after = *c;            // the decode reads the cache as the append leaves it
+  after.n_total = n_tot;
+  DecodePlan P;
+  st = decode_plan(&after, Q, Hq, softmax_scale, Pi, S, centroids, out, num_splits, workspace,
+                   ws_bytes, true, true, true, "tq_decode_step", P);
+  if (st != TQ_OK) return st;
+  st = check_pending("tq_decode_step");
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nq = c_new - c_old;
+  tq::QuantSrc src{K, V, nq, c_old, n_old, n_new};
+  cudaError_t e = tq::launch_decode_step_pre(src, n_new - nq, g, static_cast<uint8_t*>(c->base), Pi, T,
+                                             centroids, boundaries, Q, Hq, S, softmax_scale, P.ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step: quantise + prepare");
+  c->n_total = n_tot;
+  return decode_launch(c, P, Q, Hq, softmax_scale, Pi, S, centroids, out, logits, s, false, true,
+                       true, "tq_decode_step");
 }
 
 int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale,

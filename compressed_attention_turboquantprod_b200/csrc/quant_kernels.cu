@@ -15,6 +15,7 @@
 #include <cfloat>
 
 #include "common.cuh"
+#include "prep_mma.cuh"
 
 namespace tq {
 namespace {
@@ -412,20 +413,27 @@ __device__ __forceinline__ float half_row_dot(const float* rowp, const float* v,
   return a + __shfl_xor_sync(0xffffffffu, a, 1);
 }
 
-__global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  pdl_launch_dependents();    // the ring write that follows waits for this kernel itself
+// d elements of `dtype` (a multiple of 16 bytes) from src to dst, 16 bytes a thread.
+__device__ __forceinline__ void copy_row16(void* dst, const void* src, int bytes, int tid, int nthreads) {
+  for (int i = tid; i < bytes / 16; i += nthreads)
+    reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+}
+
+// One token (row) of one (b, kv head): role 0 = key, 1 = value.  When ring_new is
+// non-null the token is read from its ring slot and, once it is in shared memory,
+// the slot is overwritten with ring_new (the incoming token that takes the slot).
+__device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t row, int bh, int role,
+                                                    unsigned char* smem_raw, const void* ring_new) {
   const int d = p.d, m = p.m, b1 = p.b1;
+  const int es = p.dtype == TQ_F32 ? 4 : 2;
   float* sx = reinterpret_cast<float*>(smem_raw);       // [d]
   float* sy = sx + d;                                    // [d]  Pi x, then e = y - c[idx]
   float* sz = sy + d;                                    // [max(m, 32)]
   __shared__ double s_red[SMALL_THREADS / 32];
   __shared__ float s_cb[32];
-  const int bh = blockIdx.y;
-  const int64_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = SMALL_THREADS / 32;
-  if (blockIdx.z == 0) {
+  if (role == 0) {
     if (!p.do_keys) return;
     if (tid < 16) {
       const int L = b1 > 0 ? (1 << b1) : 0;
@@ -452,6 +460,9 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
     ss = warp_sum_d(ss);
     if (lane == 0) s_red[warp] = ss;
     __syncthreads();
+    if (ring_new)    // the token is in shared memory: its ring slot takes the new one
+      copy_row16(reinterpret_cast<char*>(const_cast<void*>(src)) + e0 * es, ring_new, d * es, tid,
+                 SMALL_THREADS);
     double t = 0.0;
     for (int w = 0; w < NW; ++w) t += s_red[w];
     const double rho64 = sqrt(t);
@@ -515,6 +526,9 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
     const void* src = src_row(p, true, bh, row, e0);
     for (int c = tid; c < d; c += SMALL_THREADS) sx[c] = load_f(src, e0 + c, p.dtype);
     __syncthreads();
+    if (ring_new)
+      copy_row16(reinterpret_cast<char*>(const_cast<void*>(src)) + e0 * es, ring_new, d * es, tid,
+                 SMALL_THREADS);
     float* vs = sz;            // [ng] scales, [ng] minima
     float* vm = sz + 16;
     for (int gi = tid; gi < ng; gi += SMALL_THREADS) {
@@ -543,6 +557,61 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
       reinterpret_cast<uint32_t*>(dst_field(p, bh, row, 4))[w] = word;
     }
   }
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS) k_quantize_small(QParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_launch_dependents();    // the ring write that follows waits for this kernel itself
+  quantize_small_body(p, blockIdx.x, blockIdx.y, blockIdx.z, smem_raw, nullptr);
+}
+
+// Decode step, first launch: the single-token quantise of the tokens that leave
+// the ring (each CTA also writes the incoming token into the ring slot it just
+// read), the ring write of incoming tokens whose slot held no token, and the
+// query preparation of the tensor-core decode, as one grid of independent CTAs.
+struct StepPrep {
+  Geom g;
+  const void* Q;
+  int Hq;
+  const float* Pi;
+  const float* S;
+  const float* cent;
+  float scale_log2;
+  DecodeWs ws;
+};
+
+template <int NV>
+__global__ void __launch_bounds__(SMALL_THREADS) k_step_pre(QParams p, int nq_ctas, int nr_ctas,
+                                                            StepPrep sp) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_launch_dependents();       // the partial kernel that follows waits for this grid
+  const int units = p.g.B * p.g.Hkv;
+  const int es = p.dtype == TQ_F32 ? 4 : 2;
+  int bid = blockIdx.x;
+  if (bid < nq_ctas) {
+    const int role = bid & 1, rest = bid >> 1, bh = rest % units;
+    const int64_t row = rest / units;                       // token t_first + row leaves the ring
+    const int64_t t_new = p.t_first + row + p.g.W;          // the incoming token taking its slot
+    const char* chunk = reinterpret_cast<const char*>(role ? p.V : p.K);
+    const char* nsrc = chunk + ((int64_t)bh * p.n_new + (t_new - p.n_old)) * p.d * es;
+    quantize_small_body(p, row, bh, role, smem_raw, nsrc);
+    return;
+  }
+  bid -= nq_ctas;
+  if (bid < nr_ctas) {
+    const int bh = bid % units;
+    const int64_t j = bid / units;                          // incoming token n_old + j
+    const int64_t off = ((int64_t)bh * p.g.W + (p.n_old + j) % p.g.W) * p.d * es;
+    const int64_t soff = ((int64_t)bh * p.n_new + j) * p.d * es;
+    copy_row16(p.base + p.g.ring_k_off + off, reinterpret_cast<const char*>(p.K) + soff, p.d * es,
+               threadIdx.x, SMALL_THREADS);
+    copy_row16(p.base + p.g.ring_v_off + off, reinterpret_cast<const char*>(p.V) + soff, p.d * es,
+               threadIdx.x, SMALL_THREADS);
+    return;
+  }
+  bid -= nr_ctas;
+  mmadec::prep_mma_body<NV>(sp.g, sp.Q, sp.Hq, sp.Pi, sp.S, sp.cent, sp.scale_log2, sp.ws, bid,
+                            smem_raw);
 }
 
 // ---------------------------------------------------------------------------
@@ -581,16 +650,28 @@ __device__ __forceinline__ void split_store(__half* hi, __half* lo, float v) {
   *lo = __float2half_rn(x - __half2float(h));
 }
 
-struct MmaSmem {
-  __half *PH, *PL, *TH, *TL, *AH, *AL;
-  float* YZ;
-  double* rho64;
-  float *rho, *inv, *cb, *vs, *vm;
+constexpr int QG = 2;              // independent warp groups per CTA
+constexpr int QNT = 32;            // rows of a group's tile
+
+struct MmaGroupSmem {
+  __half *AH, *AL;                 // [QNT][HS]
+  float* YZ;                       // [QNT][YS]
+  double* rho64;                   // [QNT]
+  float* rho;                      // [QNT]
 };
 
+struct MmaSmem {
+  __half *PH, *PL, *TH, *TL;       // [128][HS] each
+  float* cb;                       // [32]
+};
+
+__host__ __device__ inline size_t mma_group_bytes() {
+  return sizeof(__half) * 2 * QNT * HS + sizeof(float) * QNT * YS + sizeof(double) * QNT +
+         sizeof(float) * QNT;
+}
+
 __host__ __device__ inline size_t mma_smem_bytes() {
-  return sizeof(__half) * (4 * 128 * HS + 2 * NT * HS) + sizeof(float) * NT * YS +
-         sizeof(double) * NT + sizeof(float) * (2 * NT + 32 + 2 * NT * 16);
+  return sizeof(__half) * 4 * 128 * HS + QG * mma_group_bytes() + sizeof(float) * 32;
 }
 
 __device__ MmaSmem mma_carve(unsigned char* raw) {
@@ -599,27 +680,30 @@ __device__ MmaSmem mma_carve(unsigned char* raw) {
   s.PL = s.PH + 128 * HS;
   s.TH = s.PL + 128 * HS;
   s.TL = s.TH + 128 * HS;
-  s.AH = s.TL + 128 * HS;
-  s.AL = s.AH + NT * HS;
-  s.YZ = reinterpret_cast<float*>(s.AL + NT * HS);
-  s.rho64 = reinterpret_cast<double*>(s.YZ + NT * YS);
-  s.rho = reinterpret_cast<float*>(s.rho64 + NT);
-  s.inv = s.rho + NT;
-  s.cb = s.inv + NT;
-  s.vs = s.cb + 32;
-  s.vm = s.vs + NT * 16;
+  s.cb = reinterpret_cast<float*>(raw + sizeof(__half) * 4 * 128 * HS + QG * mma_group_bytes());
   return s;
+}
+
+__device__ MmaGroupSmem mma_group_carve(unsigned char* raw, int grp) {
+  MmaGroupSmem m;
+  unsigned char* q = raw + sizeof(__half) * 4 * 128 * HS + (size_t)grp * mma_group_bytes();
+  m.AH = reinterpret_cast<__half*>(q);
+  m.AL = m.AH + QNT * HS;
+  m.YZ = reinterpret_cast<float*>(m.AL + QNT * HS);
+  m.rho64 = reinterpret_cast<double*>(m.YZ + QNT * YS);
+  m.rho = reinterpret_cast<float*>(m.rho64 + QNT);
+  return m;
 }
 
 constexpr int QTHREADS = 512;       // 16 warps per CTA on the tensor-core tile path
 
-// C[64 x 128] = A[64 x 128] * B^T, A and B as fp16 hi/lo pairs (rows of 128,
-// stride HS); warp w (of 16) owns rows 32 (w & 1) .. +32 and columns 16 (w >> 1)
-// .. +16.  The result (scaled back by 2^-20) goes to C (fp32, stride YS).
-__device__ void mma_gemm_64x128(const __half* AH, const __half* AL, const __half* BH,
-                                const __half* BL, float* C) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r0 = 32 * (warp & 1), c0 = 16 * (warp >> 1);
+// C[32 x 128] = A[32 x 128] * B^T for one warp group, A and B as fp16 hi/lo pairs
+// (rows of 128, stride HS); warp gw (of 8) owns the 32 rows and columns
+// 16 gw .. +16.  The result (scaled back by 2^-20) goes to C (fp32, stride YS).
+__device__ void mma_gemm_32x128(const __half* AH, const __half* AL, const __half* BH,
+                                const __half* BL, float* C, int gw) {
+  const int lane = threadIdx.x & 31;
+  const int r0 = 0, c0 = 16 * gw;
   float acc[2][2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -666,12 +750,51 @@ __device__ void mma_gemm_64x128(const __half* AH, const __half* AL, const __half
     }
 }
 
+// Values of a warp's rows straight from the source: lane l holds channels
+// 4l..4l+3; the group min / max come from xor-shuffles over the g/4 lanes of the
+// group; codes leave as one byte (2-bit) or two bytes (4-bit) per lane.
+__device__ __forceinline__ void quantize_values_rows(const QParams& p, int bh, int64_t row0, int nrows,
+                                                     int warp, int lane, int nwarps) {
+  const int d = p.d, g = p.group, vb = p.vbits, lanes_g = g / 4;
+  const float levels = (float)((1 << vb) - 1);
+  for (int r = warp; r < nrows; r += nwarps) {
+    if (row0 + r >= p.n) break;
+    int64_t e0;
+    const void* src = src_row(p, true, bh, row0 + r, e0);
+    float x[4];
+    load4(src, e0 + 4 * lane, p.dtype, x);
+    float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    for (int o = 1; o < lanes_g; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
+    const float inv = sc != 0.f ? __frcp_rn(sc) : 0.f;
+    uint32_t bits = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) bits |= value_code(x[k], mn, sc, inv, levels) << (k * vb);
+    uint8_t* vc = dst_field(p, bh, row0 + r, 4);
+    if (vb == 2) vc[lane] = (uint8_t)bits;
+    else reinterpret_cast<uint16_t*>(vc)[lane] = (uint16_t)bits;
+    if ((lane % lanes_g) == 0) {
+      const int gi = (4 * lane) / g;
+      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 5))[gi] = sc;
+      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 6))[gi] = mn;
+    }
+    (void)d;
+  }
+}
+
+template <int B1>
 __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t tiles_per_bh,
                                                              int64_t total_tiles) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   MmaSmem s = mma_carve(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b1 = p.b1;
+  constexpr int L = 1 << B1;
+  constexpr int GW = QTHREADS / 32 / QG;         // warps per group
+  constexpr int RPW = QNT / GW;                  // rows per warp of a group tile
   // resident operands: Pi and T as fp16 hi/lo, rows of 128 (four elements a thread)
   for (int i = 4 * tid; i < QD * QD; i += 4 * QTHREADS) {
     const int r = i / QD, c = i % QD;
@@ -685,22 +808,27 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
     }
   }
   if (tid < 16) {
-    const int L = 1 << b1;
     s.cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
     s.cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
   }
   __syncthreads();
-  Smem vs{};            // view for the shared value-tile code
-  vs.X = s.YZ;
-  vs.vs = s.vs;
-  vs.vm = s.vm;
+  float bnd[L - 1];
+#pragma unroll
+  for (int k = 0; k + 1 < L; ++k) bnd[k] = s.cb[16 + k];
+
+  // From here the two warp groups run independently on alternate 32-row tiles,
+  // each with its own operand / result buffers and its own named barrier, so one
+  // group's tensor-core products overlap the other's per-row work.
+  const int grp = warp / GW, gw = warp % GW, gtid = tid % (GW * 32);
+  const MmaGroupSmem m = mma_group_carve(smem_raw, grp);
+  auto group_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GW * 32) : "memory"); };
   // Bring the key and value rows of a tile towards L2 (one hint per 128-byte line).
   const int es = p.dtype == TQ_F32 ? 4 : 2, lpr = QD * es / 128;
   auto prefetch_tile = [&](int64_t t) {
     if (t >= total_tiles) return;
     const int pbh = (int)(t / tiles_per_bh);
-    const int64_t prow0 = (t % tiles_per_bh) * NT;
-    for (int i = tid; i < NT * 2 * lpr; i += QTHREADS) {
+    const int64_t prow0 = (t % tiles_per_bh) * QNT;
+    for (int i = gtid; i < QNT * 2 * lpr; i += GW * 32) {
       const int r = i / (2 * lpr), which = (i / lpr) & 1, ln = i % lpr;
       if (prow0 + r >= p.n || (which && !p.do_values)) continue;
       int64_t e0;
@@ -708,19 +836,19 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
       prefetch_l2(reinterpret_cast<const char*>(src) + e0 * es + 128 * ln);
     }
   };
-  prefetch_tile(blockIdx.x);
-  constexpr int RPW = NT / (QTHREADS / 32);      // key rows per warp
-  for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+  const int64_t t_step = (int64_t)QG * gridDim.x;
+  prefetch_tile((int64_t)QG * blockIdx.x + grp);
+  for (int64_t tile = (int64_t)QG * blockIdx.x + grp; tile < total_tiles; tile += t_step) {
     const int bh = (int)(tile / tiles_per_bh);
-    const int64_t row0 = (tile % tiles_per_bh) * NT;
-    prefetch_tile(tile + gridDim.x);
+    const int64_t row0 = (tile % tiles_per_bh) * QNT;
+    prefetch_tile(tile + t_step);
     // ---- keys: rho (float64), U = X / rho as fp16 hi/lo; a warp's rows are all
     // loaded (4 consecutive elements a lane) before their reductions
     {
       float x[RPW][4];
 #pragma unroll
       for (int i = 0; i < RPW; ++i) {
-        const int r = warp + i * (QTHREADS / 32);
+        const int r = gw + i * GW;
         if (row0 + r < p.n) {
           int64_t e0;
           const void* src = src_row(p, false, bh, row0 + r, e0);
@@ -740,64 +868,82 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
       for (int i = 0; i < RPW; ++i) ss[i] = warp_sum_d(ss[i]);
 #pragma unroll
       for (int i = 0; i < RPW; ++i) {
-        const int r = warp + i * (QTHREADS / 32);
+        const int r = gw + i * GW;
         const double rho = sqrt(ss[i]);
         const float inv = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
         if (lane == 0) {
-          s.rho64[r] = rho;
-          s.rho[r] = (float)rho;
+          m.rho64[r] = rho;
+          m.rho[r] = (float)rho;
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          split_store(s.AH + r * HS + 4 * lane + k, s.AL + r * HS + 4 * lane + k, x[i][k] * inv);
+          split_store(m.AH + r * HS + 4 * lane + k, m.AL + r * HS + 4 * lane + k, x[i][k] * inv);
       }
     }
-    __syncthreads();
-    mma_gemm_64x128(s.AH, s.AL, s.PH, s.PL, s.YZ);           // Y = U Pi^T
-    __syncthreads();
-    // ---- codes, residual E (fp16 hi/lo into A), ||r||
-    const int L = 1 << b1;
-    for (int r = warp; r < NT; r += QTHREADS / 32) {
-      const bool valid = row0 + r < p.n;
-      uint8_t* idx_dst = valid ? dst_field(p, bh, row0 + r, 0) : nullptr;
-      double se = 0.0;
+    group_sync();
+    mma_gemm_32x128(m.AH, m.AL, s.PH, s.PL, m.YZ, gw);           // Y = U Pi^T
+    group_sync();
+    // ---- codes, residual E (fp16 hi/lo into A), ||r||: a warp's rows, lane =
+    // coordinate within each 32-coordinate chunk; the plane words of a row are
+    // collected by ballot and stored as one 16-byte write per plane
+    {
+      double se[RPW];
 #pragma unroll
-      for (int jb = 0; jb < QD; jb += 32) {
-        const float y = s.YZ[r * YS + jb + lane];
-        int idx = 0;
-        for (int k = 0; k + 1 < L; ++k) idx += (s.cb[16 + k] < y) ? 1 : 0;
-        const float e = y - s.cb[idx];
-        se += (double)e * (double)e;
-        split_store(s.AH + r * HS + jb + lane, s.AL + r * HS + jb + lane, e);
-        for (int pl = 0; pl < b1; ++pl) {
-          const unsigned word = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
-          if (lane == 0 && valid)
-            *reinterpret_cast<uint32_t*>(idx_dst + pl * (QD / 8) + jb / 8) = word;
+      for (int i = 0; i < RPW; ++i) {
+        const int r = gw + i * GW;
+        se[i] = 0.0;
+        uint32_t pw[B1][QD / 32];
+#pragma unroll
+        for (int c = 0; c < QD / 32; ++c) {
+          const float y = m.YZ[r * YS + 32 * c + lane];
+          int idx = 0;
+#pragma unroll
+          for (int k = 0; k + 1 < L; ++k) idx += (bnd[k] < y) ? 1 : 0;
+          const float e = y - s.cb[idx];
+          se[i] += (double)e * (double)e;
+          split_store(m.AH + r * HS + 32 * c + lane, m.AL + r * HS + 32 * c + lane, e);
+#pragma unroll
+          for (int pl = 0; pl < B1; ++pl) pw[pl][c] = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
+        }
+        if (lane < B1 && row0 + r < p.n) {
+          uint4 v = make_uint4(pw[0][0], pw[0][1], pw[0][2], pw[0][3]);
+#pragma unroll
+          for (int pl = 1; pl < B1; ++pl)
+            if (lane == pl) v = make_uint4(pw[pl][0], pw[pl][1], pw[pl][2], pw[pl][3]);
+          *reinterpret_cast<uint4*>(dst_field(p, bh, row0 + r, 0) + lane * (QD / 8)) = v;
         }
       }
-      se = warp_sum_d(se);
-      if (lane == 0 && valid) {
-        *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 3)) = (float)(s.rho64[r] * sqrt(se));
-        *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = s.rho[r];
-      }
-    }
-    __syncthreads();
-    mma_gemm_64x128(s.AH, s.AL, s.TH, s.TL, s.YZ);           // Z = E T^T
-    __syncthreads();
-    for (int r = warp; r < NT; r += QTHREADS / 32) {
-      if (row0 + r >= p.n) continue;
-      uint8_t* sdst = dst_field(p, bh, row0 + r, 1);
-      const float rho = s.rho[r];
 #pragma unroll
-      for (int cb = 0; cb < QM; cb += 32) {
-        const unsigned word = __ballot_sync(0xffffffffu, s.YZ[r * YS + cb + lane] * rho >= 0.f);
-        if (lane == 0) *reinterpret_cast<uint32_t*>(sdst + cb / 8) = word;
+      for (int i = 0; i < RPW; ++i) se[i] = warp_sum_d(se[i]);
+      if (lane < RPW) {
+        // lane i writes row gw + GW i (a constant-index select, no dynamic register index)
+        double sv = se[0];
+#pragma unroll
+        for (int i = 1; i < RPW; ++i)
+          if (lane == i) sv = se[i];
+        const int r = gw + lane * GW;
+        if (row0 + r < p.n) {
+          *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 3)) = (float)(m.rho64[r] * sqrt(sv));
+          *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = m.rho[r];
+        }
       }
     }
-    __syncthreads();
-    // ---- values (the shared tile code, on the Y/Z buffer)
-    if (p.do_values) quantize_values_tile(p, vs, bh, row0);
-    __syncthreads();
+    group_sync();
+    mma_gemm_32x128(m.AH, m.AL, s.TH, s.TL, m.YZ, gw);           // Z = E T^T
+    group_sync();
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+      const int r = gw + i * GW;
+      const float rho = m.rho[r];
+      uint32_t sw[QM / 32];
+#pragma unroll
+      for (int c = 0; c < QM / 32; ++c) sw[c] = __ballot_sync(0xffffffffu, m.YZ[r * YS + 32 * c + lane] * rho >= 0.f);
+      if (lane == 0 && row0 + r < p.n)
+        *reinterpret_cast<uint4*>(dst_field(p, bh, row0 + r, 1)) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+    }
+    // ---- values, straight from the source rows
+    if (p.do_values) quantize_values_rows(p, bh, row0, QNT, gw, lane, GW);
+    group_sync();
   }
 }
 
@@ -806,18 +952,20 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
   if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0) {
-    // tensor-core tiles: one persistent CTA per SM over all 64-token tiles
-    const int64_t tiles_per_bh = (p.n + NT - 1) / NT;
+    // tensor-core tiles: one persistent CTA per SM, two warp groups over all
+    // 32-token tiles
+    const int64_t tiles_per_bh = (p.n + QNT - 1) / QNT;
     const int64_t total = tiles_per_bh * bh_count;
     int sms = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = mma_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(k_quantize_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    auto kern = p.b1 == 1 ? k_quantize_mma<1> : p.b1 == 2 ? k_quantize_mma<2> : k_quantize_mma<3>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = total < sms ? total : sms;
-    k_quantize_mma<<<(unsigned)grid, QTHREADS, smem, s>>>(p, tiles_per_bh, total);
+    const int64_t want = (total + QG - 1) / QG;
+    const int64_t grid = want < sms ? want : sms;
+    kern<<<(unsigned)grid, QTHREADS, smem, s>>>(p, tiles_per_bh, total);
     return cudaGetLastError();
   }
   if (p.n <= 8) {
@@ -896,6 +1044,48 @@ cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const
                               int64_t n_old, int64_t n_new, cudaStream_t s) {
   if (g.W == 0 || n_new == 0) return cudaSuccess;
   return launch_pdl(k_ring_write, dim3(g.B * g.Hkv), dim3(256), 0, s, g, base, K, V, n_old, n_new);
+}
+
+cudaError_t launch_decode_step_pre(const QuantSrc& src, int64_t n_ring_only, const Geom& g,
+                                   uint8_t* base, const float* Pi, const float* T,
+                                   const float* cent, const float* bnd, const void* Q, int Hq,
+                                   const float* S, float softmax_scale, const DecodeWs& ws,
+                                   cudaStream_t s) {
+  QParams p{};
+  p.K = src.K;
+  p.V = src.V;
+  p.dtype = g.dtype;
+  p.n = src.n;
+  p.t_first = src.t_first;
+  p.n_old = src.n_old;
+  p.n_new = src.n_new;
+  p.cache_mode = true;
+  p.ringK = base + g.ring_k_off;
+  p.ringV = base + g.ring_v_off;
+  p.d = g.d;
+  p.b1 = g.b1;
+  p.m = g.m;
+  p.vbits = g.vbits;
+  p.group = g.group;
+  p.do_keys = true;
+  p.do_values = true;
+  p.Pi = Pi;
+  p.T = T;
+  p.cent = cent;
+  p.bnd = bnd;
+  p.base = base;
+  p.g = g;
+  const int units = g.B * g.Hkv;
+  const int nq = (int)(src.n * units * 2), nr = (int)(n_ring_only * units);
+  StepPrep sp{g, Q, Hq, Pi, S, cent, softmax_scale * mmadec::kLog2e, ws};
+  const size_t qsm = sizeof(float) * (2 * g.d + (g.m > g.d ? g.m : g.d) + 32);
+  const size_t psm = mmadec::prep_smem_bytes(g.d, g.m);
+  const size_t smem = qsm > psm ? qsm : psm;
+  auto kern = g.d == 256 ? k_step_pre<2> : k_step_pre<1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<nq + nr + units, SMALL_THREADS, smem, s>>>(p, nq, nr, sp);
+  return cudaGetLastError();
 }
 
 }  // namespace tq

@@ -61,6 +61,15 @@ cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* b
                                   const float* bnd, cudaStream_t s);
 cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,
                               int64_t n_old, int64_t n_new, cudaStream_t s);
+// Decode step (tq_decode_step): quantise of the tokens leaving the ring with the
+// ring write fused in, ring writes of incoming tokens into empty slots, and the
+// tensor-core query preparation, in one launch.
+struct DecodeWs;
+cudaError_t launch_decode_step_pre(const QuantSrc& src, int64_t n_ring_only, const Geom& g,
+                                   uint8_t* base, const float* Pi, const float* T,
+                                   const float* cent, const float* bnd, const void* Q, int Hq,
+                                   const float* S, float softmax_scale, const DecodeWs& ws,
+                                   cudaStream_t s);
 
 // ---- decode (decode_kernels.cu) ----
 struct DecodeWs {

@@ -84,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "tq_decode_check": (I, [C, I, I, P, SZ, P]),
         "tq_decode_partial": (I, [C, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
+        "tq_decode_step": (I, [C, P, P, I64, P, I, F, P, P, P, P, P, P, P, I, P, SZ, P]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
         "tq_m_for_layer": (I, [ctypes.POINTER(tq_layer_groups), I]),
     }
@@ -228,6 +229,14 @@ def tq_decode_partial(cache: tq_cache, Hq, softmax_scale, centroids, logits, num
     _check(lib.tq_decode_partial(ctypes.byref(cache), Hq, softmax_scale, _ptr(centroids),
                                  _ptr(logits), _ptr(out), num_splits, _ptr(workspace),
                                  _ws(workspace), _stream(stream)), "tq_decode_partial")
+
+
+def tq_decode_step(cache: tq_cache, K, V, Q, softmax_scale, Pi, S, T, centroids, boundaries, out,
+                   logits, num_splits, workspace, stream=None):
+    _check(lib.tq_decode_step(ctypes.byref(cache), _ptr(K), _ptr(V), K.shape[2], _ptr(Q), Q.shape[1],
+                              softmax_scale, _ptr(Pi), _ptr(S), _ptr(T), _ptr(centroids),
+                              _ptr(boundaries), _ptr(out), _ptr(logits), num_splits, _ptr(workspace),
+                              _ws(workspace), _stream(stream)), "tq_decode_step")
 
 
 def tq_decode_combine(cache: tq_cache, Hq, out, num_splits, workspace, stream=None):

@@ -280,6 +280,29 @@ int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void
                       size_t ws_bytes, void* stream);
 
 /*
+ * tq_decode_step -- one decode step with its append: the same result (cache
+ * bytes, n_total, out, logits) as tq_append(c, K, V, n_new, Pi, T, centroids,
+ * boundaries, stream) followed by tq_decode_attention(c, Q, Hq, softmax_scale,
+ * Pi, S, centroids, out, logits, num_splits, workspace, ws_bytes, stream).  The
+ * pages keep these as two steps ([TQ] 六: capture the new token, then score);
+ * this call is the fused form of a decode loop.  When 1 <= n_new <= min(8, W)
+ * and the decode runs on the tensor-core path, it takes two launches: one grid
+ * quantises the tokens that leave the ring (each such CTA also writes the
+ * incoming token into the ring slot it has just read), writes incoming tokens
+ * into empty ring slots, and prepares the queries; then the split-K partial
+ * attention merges its splits into `out`.  Otherwise it makes the two calls.
+ * Arguments as for tq_append and tq_decode_attention; the workspace is sized for
+ * the cache after the append (tq_decode_workspace_bytes of a cache with
+ * n_total + n_new tokens; the workspace size does not depend on n_total).
+ * All checks of both parts are made before anything is launched.
+ * Errors: INVALID_ARG, CAPACITY, UNSUPPORTED, CUDA.
+ */
+int tq_decode_step(tq_cache* c, const void* K, const void* V, int64_t n_new, const void* Q, int Hq,
+                   float softmax_scale, const float* Pi, const float* S, const float* T,
+                   const float* centroids, const float* boundaries, void* out, float* logits,
+                   int num_splits, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * tq_decode_check -- SYNCHRONOUS: waits for `stream`, then reports whether the
  * last decode that used `workspace` completed its staged loads.  A decode
  * kernel whose bounded wait on a shared-memory load gives up (it never should)

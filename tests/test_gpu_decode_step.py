@@ -1,0 +1,66 @@
+"""tq_decode_step (append + decode as one call) against tq_append followed by
+tq_decode_attention on a twin cache: the packed cache, the ring, the outputs and
+the logits must be identical after every step, whichever path the call takes
+(the fused two-launch path, or the two calls)."""
+import math
+
+import pytest
+import torch
+
+import synth
+from gpu_common import TORCH_DT, oracle_setup, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+class _Proj:
+    def __init__(self, po):
+        self.Pi, self.S, self.T = to_dev(po["Pi"]), to_dev(po["S"]), to_dev(po["T"])
+
+
+class _Cb:
+    def __init__(self, cb):
+        self.centroids, self.boundaries = to_dev(cb[0]), to_dev(cb[1])
+
+
+def _workload(**kw):
+    base = dict(name="t", B=2, Hq=8, Hkv=2, d=128, T=400, W=16, b1=2, m=128, vbits=2, group=32,
+                dtype="bf16", seed=5, k_outlier_frac=0.02, v_outlier_frac=0.02, outlier_scale=8.0)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+@pytest.mark.parametrize("kw,n0,steps", [
+    (dict(), 300, [1, 1, 1, 1, 1]),                                     # full ring, one token a step
+    (dict(), 5, [3, 8, 8, 1]),                                          # ring filling up
+    (dict(dtype="f32", W=20, b1=1, m=64), 40, [2, 5, 1]),
+    (dict(b1=0, m=256, dtype="f16"), 100, [1, 4]),                      # pure QJL
+    (dict(d=256, b1=3, m=256, vbits=4, group=64, Hq=16, Hkv=4), 200, [1, 2, 1]),   # head dim 256
+    (dict(Hq=2, Hkv=2), 150, [1, 1]),                                   # G = 1: the two calls
+    (dict(W=3), 50, [5, 1]),                                            # n_new > W: the two calls
+])
+def test_decode_step_matches_append_then_decode(kw, n0, steps):
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache
+    w = _workload(**kw)
+    total = n0 + sum(steps)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    pj, cbd = _Proj(po), (_Cb(cb) if w.b1 else None)
+    K, V = synth.keys_values(w, device="cuda", T=total)
+    caches = [CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
+                                dtype=TORCH_DT[w.dtype]) for _ in range(2)]
+    for c in caches:
+        c.append(K[:, :, :n0].contiguous(), V[:, :, :n0].contiguous(), pj, cbd)
+    t = n0
+    for i, n in enumerate(steps):
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        Q = synth.queries(w.scaled(seed=50 + i), device="cuda")
+        o1, l1 = caches[0].decode_step(k, v, Q, pj, cbd, want_logits=True)
+        caches[1].append(k, v, pj, cbd)
+        o2, l2 = caches[1].decode(Q, pj, cbd, want_logits=True)
+        torch.cuda.synchronize()
+        t += n
+        assert caches[0].n_total == caches[1].n_total == t
+        assert torch.equal(caches[0].buffer, caches[1].buffer), f"cache bytes differ after step {i}"
+        assert torch.equal(o1, o2), f"outputs differ after step {i}"
+        assert torch.equal(l1, l2), f"logits differ after step {i}"
+        assert torch.isfinite(o1.float()).all()
