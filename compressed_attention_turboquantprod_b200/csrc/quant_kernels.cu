@@ -650,8 +650,8 @@ __device__ __forceinline__ void split_store(__half* hi, __half* lo, float v) {
   *lo = __float2half_rn(x - __half2float(h));
 }
 
-constexpr int QG = 2;              // independent warp groups per CTA
-constexpr int QNT = 32;            // rows of a group's tile
+constexpr int QG = 4;              // independent warp groups per CTA
+constexpr int QNT = 16;            // rows of a group's tile
 
 struct MmaGroupSmem {
   __half *AH, *AL;                 // [QNT][HS]
@@ -697,52 +697,55 @@ __device__ MmaGroupSmem mma_group_carve(unsigned char* raw, int grp) {
 
 constexpr int QTHREADS = 512;       // 16 warps per CTA on the tensor-core tile path
 
-// C[32 x 128] = A[32 x 128] * B^T for one warp group, A and B as fp16 hi/lo pairs
-// (rows of 128, stride HS); warp gw (of 8) owns the 32 rows and columns
-// 16 gw .. +16.  The result (scaled back by 2^-20) goes to C (fp32, stride YS).
-__device__ void mma_gemm_32x128(const __half* AH, const __half* AL, const __half* BH,
-                                const __half* BL, float* C, int gw) {
+// C[QNT x 128] = A[QNT x 128] * B^T for one warp group, A and B as fp16 hi/lo
+// pairs (rows of 128, stride HS); warp gw (of the group's GW) owns the QNT rows
+// and columns (128 / GW) gw .. +128 / GW.  The result (scaled back by 2^-20) goes
+// to C (fp32, stride YS).
+template <int MTI, int NTI>     // 16-row m-tiles, 16-column B loads per warp
+__device__ __forceinline__ void mma_gemm_group(const __half* AH, const __half* AL, const __half* BH,
+                                               const __half* BL, float* C, int gw) {
   const int lane = threadIdx.x & 31;
-  const int r0 = 0, c0 = 16 * gw;
-  float acc[2][2][4];
+  const int c0 = 16 * NTI * gw;
+  float acc[MTI][2 * NTI][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < MTI; ++i)
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < 2 * NTI; ++j)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
   const int ar = lane & 15, ac = 8 * (lane >> 4);                    // A: rows, k offset
   const int bn = (lane & 7) + 8 * (lane >> 4), bk = 8 * ((lane >> 3) & 1);   // B: n, k offset
 #pragma unroll 2
   for (int ks = 0; ks < QD / 16; ++ks) {
-    uint32_t ah[2][4], al[2][4];
+    uint32_t ah[MTI][4], al[MTI][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      ldsm_x4(ah[i], AH + (r0 + 16 * i + ar) * HS + 16 * ks + ac);
-      ldsm_x4(al[i], AL + (r0 + 16 * i + ar) * HS + 16 * ks + ac);
+    for (int i = 0; i < MTI; ++i) {
+      ldsm_x4(ah[i], AH + (16 * i + ar) * HS + 16 * ks + ac);
+      ldsm_x4(al[i], AL + (16 * i + ar) * HS + 16 * ks + ac);
     }
-    {
-      uint32_t bh[4], bl[4];
-      ldsm_x4(bh, BH + (c0 + bn) * HS + 16 * ks + bk);
-      ldsm_x4(bl, BL + (c0 + bn) * HS + 16 * ks + bk);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        mma16816(acc[i][0], ah[i], bh[0], bh[1]);
-        mma16816(acc[i][0], ah[i], bl[0], bl[1]);
-        mma16816(acc[i][0], al[i], bh[0], bh[1]);
-        mma16816(acc[i][1], ah[i], bh[2], bh[3]);
-        mma16816(acc[i][1], ah[i], bl[2], bl[3]);
-        mma16816(acc[i][1], al[i], bh[2], bh[3]);
+    for (int jb = 0; jb < NTI; ++jb) {
+      uint32_t bh[4], bl[4];
+      ldsm_x4(bh, BH + (c0 + 16 * jb + bn) * HS + 16 * ks + bk);
+      ldsm_x4(bl, BL + (c0 + 16 * jb + bn) * HS + 16 * ks + bk);
+#pragma unroll
+      for (int i = 0; i < MTI; ++i) {
+        mma16816(acc[i][2 * jb], ah[i], bh[0], bh[1]);
+        mma16816(acc[i][2 * jb], ah[i], bl[0], bl[1]);
+        mma16816(acc[i][2 * jb], al[i], bh[0], bh[1]);
+        mma16816(acc[i][2 * jb + 1], ah[i], bh[2], bh[3]);
+        mma16816(acc[i][2 * jb + 1], ah[i], bl[2], bl[3]);
+        mma16816(acc[i][2 * jb + 1], al[i], bh[2], bh[3]);
       }
     }
   }
   const int gid = lane >> 2, tig = lane & 3;
   const float sc = 1.f / (kSplit * kSplit);
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < MTI; ++i)
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int row = r0 + 16 * i + gid, col = c0 + 8 * j + 2 * tig;
+    for (int j = 0; j < 2 * NTI; ++j) {
+      const int row = 16 * i + gid, col = c0 + 8 * j + 2 * tig;
       C[row * YS + col] = acc[i][j][0] * sc;
       C[row * YS + col + 1] = acc[i][j][1] * sc;
       C[(row + 8) * YS + col] = acc[i][j][2] * sc;
@@ -816,7 +819,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
 #pragma unroll
   for (int k = 0; k + 1 < L; ++k) bnd[k] = s.cb[16 + k];
 
-  // From here the two warp groups run independently on alternate 32-row tiles,
+  // From here the QG warp groups run independently on interleaved QNT-row tiles,
   // each with its own operand / result buffers and its own named barrier, so one
   // group's tensor-core products overlap the other's per-row work.
   const int grp = warp / GW, gw = warp % GW, gtid = tid % (GW * 32);
@@ -869,19 +872,34 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
 #pragma unroll
       for (int i = 0; i < RPW; ++i) {
         const int r = gw + i * GW;
-        const double rho = sqrt(ss[i]);
-        const float inv = rho > 0.0 ? (float)(1.0 / rho) : 0.f;
+        // rho = ss * rsqrt(ss) and 1/rho = rsqrt(ss): one float64 reciprocal square
+        // root instead of a square root and a division
+        const double rs = ss[i] > 0.0 ? rsqrt(ss[i]) : 0.0;
+        const double rho = ss[i] * rs;
+        const float inv = (float)rs;
         if (lane == 0) {
           m.rho64[r] = rho;
           m.rho[r] = (float)rho;
         }
+        // this lane's 4 consecutive elements: hi / lo as two f16x2 pairs each
+        float a[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          split_store(m.AH + r * HS + 4 * lane + k, m.AL + r * HS + 4 * lane + k, x[i][k] * inv);
+        for (int k = 0; k < 4; ++k) a[k] = x[i][k] * inv * kSplit;
+        const __half2 h01 = __floats2half2_rn(a[0], a[1]), h23 = __floats2half2_rn(a[2], a[3]);
+        const float2 b01 = __half22float2(h01), b23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(a[0] - b01.x, a[1] - b01.y);
+        const __half2 l23 = __floats2half2_rn(a[2] - b23.x, a[3] - b23.y);
+        uint2 hv, lv;
+        hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+        hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+        lv.x = *reinterpret_cast<const uint32_t*>(&l01);
+        lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+        *reinterpret_cast<uint2*>(m.AH + r * HS + 4 * lane) = hv;
+        *reinterpret_cast<uint2*>(m.AL + r * HS + 4 * lane) = lv;
       }
     }
     group_sync();
-    mma_gemm_32x128(m.AH, m.AL, s.PH, s.PL, m.YZ, gw);           // Y = U Pi^T
+    mma_gemm_group<QNT / 16, 128 / 16 / GW>(m.AH, m.AL, s.PH, s.PL, m.YZ, gw);   // Y = U Pi^T
     group_sync();
     // ---- codes, residual E (fp16 hi/lo into A), ||r||: a warp's rows, lane =
     // coordinate within each 32-coordinate chunk; the plane words of a row are
@@ -929,7 +947,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
       }
     }
     group_sync();
-    mma_gemm_32x128(m.AH, m.AL, s.TH, s.TL, m.YZ, gw);           // Z = E T^T
+    mma_gemm_group<QNT / 16, 128 / 16 / GW>(m.AH, m.AL, s.TH, s.TL, m.YZ, gw);   // Z = E T^T
     group_sync();
 #pragma unroll
     for (int i = 0; i < RPW; ++i) {
@@ -952,8 +970,8 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
   if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0) {
-    // tensor-core tiles: one persistent CTA per SM, two warp groups over all
-    // 32-token tiles
+    // tensor-core tiles: one persistent CTA per SM, QG warp groups over all
+    // QNT-token tiles
     const int64_t tiles_per_bh = (p.n + QNT - 1) / QNT;
     const int64_t total = tiles_per_bh * bh_count;
     int sms = 0, dev = 0;
