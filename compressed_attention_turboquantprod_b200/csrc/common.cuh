@@ -55,6 +55,16 @@ __device__ __forceinline__ uint8_t* field_ptr(uint8_t* base, const Geom& g, int 
          (t % kBlockTokens) * size;
 }
 
+// Byte offset, inside a block's value-code field, of 16-bit half x (the codes of
+// channels (16/vbits) x ...) of block token tk: the field is 32 token-pair records
+// of d*vbits/16 words; half x = gi*H + s (H = g*vbits/16 halves per group) of the
+// pair's even token is the low half of word s*(d/g) + gi, the odd token's the high.
+__device__ __forceinline__ int vcode_half_off(const Geom& g, int tk, int x) {
+  const int H = (g.group * g.vbits) >> 4, NG = g.d / g.group;
+  const int word = (x % H) * NG + x / H;
+  return (tk >> 1) * 2 * g.f_vcode + 4 * word + 2 * (tk & 1);
+}
+
 // Hint: bring the 128-byte line holding p into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

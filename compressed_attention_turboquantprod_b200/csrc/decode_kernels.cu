@@ -158,13 +158,15 @@ __global__ void __launch_bounds__(DT) k_decode_partial(DParams p) {
       const float* vm = reinterpret_cast<const float*>(sBuf + g.o_vmin);
       const int gi = ch / g.group;
       const int bit = ch * g.vbits;
+      const int hoff = g.o_vcode + vcode_half_off(g, 0, bit >> 4);   // token-pair records
 #pragma unroll
       for (int k = 0; k < kMaxG; ++k) {
         const int hh = hs + k * nhs;
         if (hh < G) acc[k] *= sAl[hh];
       }
       for (int tk = 0; tk < nt; ++tk) {
-        const int code = (sBuf[g.o_vcode + tk * g.f_vcode + (bit >> 3)] >> (bit & 7)) & vmask;
+        const int code = (*reinterpret_cast<const uint16_t*>(sBuf + hoff + (tk >> 1) * 2 * g.f_vcode +
+                                                              2 * (tk & 1)) >> (bit & 15)) & vmask;
         const float v = fmaf((float)code, vs[tk * ng + gi], vm[tk * ng + gi]);
 #pragma unroll
         for (int k = 0; k < kMaxG; ++k) {

@@ -20,9 +20,12 @@
 //             <Pi q, c[idx]> = (sum_S w_S)(sum_j qr_j) - 2 sum_S w_S sum_j qr_j x_Sj.
 //           The QJL term uses <qs, 2 s - 1> = 2 <qs, s> - sum qs.
 //   P V     f16 mma.sync m16n8k16: A = value codes (channels x tokens) as f16
-//           subnormals code * 2^(2k-24) (one PRMT + one AND per 2 codes; the
-//           per-channel power of two is undone once per split), B = p * s split
-//           into f16 hi + lo (the value scale s is per token and group).
+//           code * 2^(2k-24), k the code's place in its byte: the cache keeps
+//           the codes of a token pair interleaved by 16-bit halves, so one AND
+//           of a stored word (shifted by a byte for half of the lanes) is the
+//           operand of two tokens (the per-channel power of two is undone once
+//           per split); B = p * s split into f16 hi + lo (the value scale s is
+//           per token and group).
 //
 // One CTA = one (batch, KV head, split) with 4 warps; the two warp pairs take
 // alternate blocks and each warp owns 32 of the 64 tokens of its pair's blocks
@@ -47,6 +50,7 @@ using namespace mmadec;
 constexpr int MD = 128;          // head dim of this path
 constexpr int NST = 4;           // pipeline stages (blocks in flight per CTA)
 constexpr int MT = 128;          // threads per CTA
+constexpr int kPairBytes = 2 * MD * 2 / 8;   // value codes of a token pair (2-bit)
 // Workspace views used here: per (batch, KV head) unit, fragment words
 // [kstep][lane][ntile][reg] (uint32) and per head {kM, CM, kQ, CQ} (float).
 
@@ -142,12 +146,14 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   const uint4* bfr = reinterpret_cast<const uint4*>(s_frag) + lane;
 
   const uint32_t maskA = 0x01010101u << tig, maskB = 0x10101010u << tig;
-  const uint32_t codeMask = 0x00030003u << (2 * (gid & 3));
-  // PRMT selectors: result byte 0 <- byte bsel of token A's word, byte 2 <- byte
-  // bsel of token B's word (bytes 1, 3 are masked off); bsel + 2 for channel + 8.
-  const uint32_t bsel = (uint32_t)(gid >> 2);
-  const uint32_t pLo = bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12);
-  const uint32_t pHi = (2 + bsel) | ((2 + bsel) << 4) | ((6 + bsel) << 8) | ((6 + bsel) << 12);
+  // P V rows: row gid (h = 0) and gid + 8 (h = 1) of m-tile mt = 2 gi + e are the
+  // channels 32 gi + 4 gid + 2 e + h: byte gid & 1, code 2 e + h of that byte, of
+  // the 16-bit half s = gid >> 1 of value group gi.  A word of a token-pair record
+  // (even token low, odd token high) shifted right by 8 (gid & 1) and masked with
+  // 0x00030003 << 2k (k = 2 e + h) is the f16x2 operand code * 2^(2k - 24) of both
+  // tokens (raw values below 2^10: exact subnormals).
+  const uint32_t vshift = 8u * (uint32_t)(gid & 1);
+  const int vc_lane = 16 * (gid >> 1);        // byte of this lane's four words in a pair record
 
   float m_run = -INFINITY, l_run = 0.f;
   float acc[8][4];
@@ -334,16 +340,15 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     // ---------------- P V, one 16-token m-tile at a time
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      // MMA indices k = 2tig, 2tig+1, 2tig+8, 2tig+9 of this lane stand for the
-      // m-tile's tokens TA..TD = tig, tig+4, tig+8, tig+12 (a permutation of the 16
-      // tokens, the same for A and B) so that the four tig lanes read distinct
-      // shared-memory banks; their p (head hP) come from the score lanes gid = tig,
-      // tig + 4 (rows e = 0, 1).
-      const float pA = __shfl_sync(0xffffffffu, pr[r][0], 4 * tig + hP);
-      const float pB = __shfl_sync(0xffffffffu, pr[r][0], 4 * (tig + 4) + hP);
-      const float pC = __shfl_sync(0xffffffffu, pr[r][1], 4 * tig + hP);
-      const float pD = __shfl_sync(0xffffffffu, pr[r][1], 4 * (tig + 4) + hP);
-      const int TA = tb + 16 * r + tig, TB = TA + 4, TC = TA + 8, TD = TA + 12;
+      // MMA indices k = 2tig, 2tig+1 of this lane are the m-tile's tokens TA = 2tig,
+      // TB = 2tig+1 (token pair tig), k = 2tig+8, 2tig+9 are TC = TA+8, TD = TA+9
+      // (pair tig+4); their p (head hP) come from the score lanes gid = 2tig, 2tig+1
+      // (rows e = 0 for TA, TB and e = 1 for TC, TD).
+      const float pA = __shfl_sync(0xffffffffu, pr[r][0], 8 * tig + hP);
+      const float pB = __shfl_sync(0xffffffffu, pr[r][0], 8 * tig + 4 + hP);
+      const float pC = __shfl_sync(0xffffffffu, pr[r][1], 8 * tig + hP);
+      const float pD = __shfl_sync(0xffffffffu, pr[r][1], 8 * tig + 4 + hP);
+      const int TA = tb + 16 * r + 2 * tig, TB = TA + 1, TC = TA + 8, TD = TA + 9;
       const float4* vs4 = reinterpret_cast<const float4*>(blk + g.o_vscale);
       const float4 sA = vs4[TA], sB = vs4[TB], sC = vs4[TC], sD = vs4[TD];
       uint32_t bpv[4][2];
@@ -363,20 +368,18 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
           bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
         }
       }
-      const uint4* vc = reinterpret_cast<const uint4*>(blk + g.o_vcode);   // 2 x uint4 per token
-      const uint4 cA0 = vc[2 * TA], cA1 = vc[2 * TA + 1], cB0 = vc[2 * TB], cB1 = vc[2 * TB + 1];
-      const uint4 cC0 = vc[2 * TC], cC1 = vc[2 * TC + 1], cD0 = vc[2 * TD], cD1 = vc[2 * TD + 1];
-      const uint32_t wa[8] = {cA0.x, cA0.y, cA0.z, cA0.w, cA1.x, cA1.y, cA1.z, cA1.w};
-      const uint32_t wb[8] = {cB0.x, cB0.y, cB0.z, cB0.w, cB1.x, cB1.y, cB1.z, cB1.w};
-      const uint32_t wc[8] = {cC0.x, cC0.y, cC0.z, cC0.w, cC1.x, cC1.y, cC1.z, cC1.w};
-      const uint32_t wd[8] = {cD0.x, cD0.y, cD0.z, cD0.w, cD1.x, cD1.y, cD1.z, cD1.w};
+      // this lane's words (s = gid >> 1, groups 0..3) of the pairs tig and tig + 4
+      const unsigned char* vc = blk + g.o_vcode + vc_lane;
+      const uint4 wAB = *reinterpret_cast<const uint4*>(vc + (TA >> 1) * kPairBytes);
+      const uint4 wCD = *reinterpret_cast<const uint4*>(vc + (TC >> 1) * kPairBytes);
+      const uint32_t ab[4] = {wAB.x >> vshift, wAB.y >> vshift, wAB.z >> vshift, wAB.w >> vshift};
+      const uint32_t cd[4] = {wCD.x >> vshift, wCD.y >> vshift, wCD.z >> vshift, wCD.w >> vshift};
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        const uint32_t a0 = prmt(wa[mt], wb[mt], pLo) & codeMask;
-        const uint32_t a1 = prmt(wa[mt], wb[mt], pHi) & codeMask;
-        const uint32_t a2 = prmt(wc[mt], wd[mt], pLo) & codeMask;
-        const uint32_t a3 = prmt(wc[mt], wd[mt], pHi) & codeMask;
-        hmma16816(acc[mt], a0, a1, a2, a3, bpv[mt >> 1][0], bpv[mt >> 1][1]);
+        const int gi = mt >> 1;
+        const uint32_t m0 = 0x00030003u << (4 * (mt & 1)), m1 = m0 << 2;
+        hmma16816(acc[mt], ab[gi] & m0, ab[gi] & m1, cd[gi] & m0, cd[gi] & m1, bpv[gi][0],
+                  bpv[gi][1]);
       }
     }
     }  // ok
@@ -414,10 +417,12 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   }
 
   // ---------------- exact ring tokens (last split)
-  // The value part of acc counts codes in units of 2^(2k-24) (k = gid & 3, the
-  // bit offset of this lane's channels in their byte): o = acc / code_unit.
-  const float code_unit = __int_as_float((127 - 24 + 2 * (gid & 3)) << 23);       // 2^(2k-24)
-  const float inv_unit = __int_as_float((127 + 24 - 2 * (gid & 3)) << 23);        // 2^(24-2k)
+  // acc[mt][c] is channel 32 (mt >> 1) + 4 gid + 2 (mt & 1) (+1 for c >= 2) of head
+  // tig in units of 2^(2k - 24), k = 2 (mt & 1) (+1 for c >= 2).
+  auto code_unit = [&](int mt) {      // 2^(2k - 24) of row gid; row gid + 8: times 4
+    return __int_as_float((127 - 24 + 4 * (mt & 1)) << 23);
+  };
+  auto chan = [&](int mt) { return 32 * (mt >> 1) + 4 * gid + 2 * (mt & 1); };
   if (ring_split) {
     // Ring slots in slot order (softmax and P V do not depend on the order); slot s
     // holds the token at ring position ((s - first) mod W).  Warp w takes the slots
@@ -455,8 +460,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       }
       float p0, p1;
       softmax_step(l, -INFINITY, p0, p1);
-      // acc[mt][c]: channel 16 mt + gid (+8 for c >= 2), column 2 tig + (c & 1) = head tig;
-      // add p * v into the hi column (c even) in code units
+      // column 2 tig + (c & 1) of acc is head tig: add p * v into the hi column (c
+      // even) in code units
       for (int T = 0; T < per_warp; ++T) {
         const float pt = __shfl_sync(0xffffffffu, p0, 4 * T + tig);
         const int sl2 = per_warp * warp + T;
@@ -464,10 +469,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
         const int64_t e = (int64_t)sl2 * MD;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const float v0 = load_f(s_rv, e + 16 * mt + gid, g.dtype);
-          const float v1 = load_f(s_rv, e + 16 * mt + gid + 8, g.dtype);
-          acc[mt][0] = fmaf(pt * v0, code_unit, acc[mt][0]);
-          acc[mt][2] = fmaf(pt * v1, code_unit, acc[mt][2]);
+          const float v0 = load_f(s_rv, e + chan(mt), g.dtype);
+          const float v1 = load_f(s_rv, e + chan(mt) + 1, g.dtype);
+          const float u = code_unit(mt);
+          acc[mt][0] = fmaf(pt * v0, u, acc[mt][0]);
+          acc[mt][2] = fmaf(pt * v1, 4.f * u, acc[mt][2]);
         }
       }
       __syncthreads();     // the chunk is consumed before the next one is requested
@@ -498,13 +504,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   const float sc = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mh);
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    const int ch0 = 16 * mt + gid, ch1 = ch0 + 8;
-    const int gi = mt >> 1;
-    const float mnv = s_mn[warp][tig][gi];
-    const float o0 = ((acc[mt][0] + acc[mt][1]) * inv_unit + mnv) * sc;
-    const float o1 = ((acc[mt][2] + acc[mt][3]) * inv_unit + mnv) * sc;
-    s_out[(warp * MG + tig) * MD + ch0] = o0;
-    s_out[(warp * MG + tig) * MD + ch1] = o1;
+    const float mnv = s_mn[warp][tig][mt >> 1];
+    const float inv = __int_as_float((127 + 24 - 4 * (mt & 1)) << 23);   // 1 / code_unit(mt)
+    const float o0 = ((acc[mt][0] + acc[mt][1]) * inv + mnv) * sc;
+    const float o1 = ((acc[mt][2] + acc[mt][3]) * (0.25f * inv) + mnv) * sc;
+    *reinterpret_cast<float2*>(&s_out[(warp * MG + tig) * MD + chan(mt)]) = make_float2(o0, o1);
   }
   __syncthreads();
   for (int i = tid; i < MG * MD; i += MT) {

@@ -8,9 +8,10 @@
 //  * b1 = 3: a symmetric 8-level codebook has four odd Walsh subsets {0}, {1},
 //    {2}, {0,1,2}; the fourth feature plane is the XOR of the three stored
 //    planes, formed on the fly (one LOP3 per 32 coordinates).
-//  * 4-bit codes: code of channel c sits in nibble c mod 8 of word c / 8; a PRMT
-//    brings its byte to both halves and an AND keeps the nibble, so the half is
-//    code * 16^(c mod 2) * 2^-24 (the power of sixteen is undone at the end).
+//  * 4-bit codes: a 16-bit half of a token-pair record holds 4 codes of each of
+//    the two tokens; an AND of the word (shifted by a byte for the upper two)
+//    keeps code k in {0, 1} of a byte of both, code * 16^k * 2^-24 as an f16
+//    subnormal (the power of sixteen is undone at the end).
 //  * 256 output channels need 64 accumulator registers per lane, so the two
 //    warps of a pair work on the same block: each scores 32 of its 64 tokens,
 //    the pair exchanges block maxima and probabilities through shared memory
@@ -30,6 +31,7 @@ constexpr int WD = 256;          // head dim
 constexpr int WNST = 4;          // stages: two per warp pair
 constexpr int WT = 128;          // threads per CTA (2 pairs of 2 warps)
 constexpr int WCTAS = 2;         // resident CTAs per SM (shared memory)
+constexpr int kWPairBytes = 2 * WD * 4 / 8;   // value codes of a token pair (4-bit)
 
 // s0 + 2^8 s1 + 2^16 s2 + 2^24 s3 with every slice sum below 2^24: each converts
 // exactly; the result carries fp32 rounding only.
@@ -52,9 +54,6 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   __shared__ __align__(8) uint64_t full[WNST];
   __shared__ __align__(8) uint64_t ringbar;
   __shared__ int s_abort, s_abort_pair[2][2];       // [pair][buf]
-  // the block's value codes of each pair at a 144-byte token stride (four
-  // consecutive tokens fall in four different bank groups)
-  __shared__ __align__(16) uint32_t s_vc[2][64][36];
   __shared__ int s_cnt[WNST], s_iss[WNST];
   __shared__ float s_bmax[2][2][2][MG];              // [pair][buf][half][head]
   __shared__ float s_p[2][2][64][MG];                // [pair][buf][token][head]
@@ -122,13 +121,11 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   __syncthreads();
 
   const uint32_t maskA = 0x01010101u << tig, maskB = 0x10101010u << tig;
-  // 4-bit codes: row gid of a channel m-tile is nibble gid of its word: byte
-  // gid >> 1 to bytes 0 and 2 (tokens A and B), then keep nibble gid & 1
-  const uint32_t bsel = (uint32_t)(gid >> 1);
-  const uint32_t psel = bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12);
-  const uint32_t codeMask = 0x000F000Fu << (4 * (gid & 1));
-  const float code_unit = __int_as_float((127 - 24 + 4 * (gid & 1)) << 23);   // 2^(4k-24)
-  const float inv_unit = __int_as_float((127 + 24 - 4 * (gid & 1)) << 23);    // 2^(24-4k)
+  // P V rows: row gid (h = 0) and gid + 8 (h = 1) of channel m-tile mt (0..7) of
+  // this warp's half are channel 64 G + 4 gid + 32 ((mt >> 1) & 1) + 2 (mt & 1) + h
+  // of value group G = 2 half + (mt >> 2): code 2 (mt & 1) + h of the 16-bit half
+  // s = gid + 8 ((mt >> 1) & 1) of group G, i.e. word s * 4 + G of a token-pair
+  // record, shifted right by 8 (mt & 1) and masked with 0x000F000F << 4h.
 
   float m_run = -INFINITY, l_run = 0.f;
   float acc[8][4];
@@ -278,16 +275,6 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
       if (gid == 0) s_bmax[pair][buf][half][tig] = lm;
     }
     pair_sync(pair);
-    // this warp's 32 tokens of codes into the padded copy (the previous block's
-    // P V of both warps ended before the barrier above)
-    if (ok) {
-      const uint4* src = reinterpret_cast<const uint4*>(blk + g.o_vcode) + 8 * tb;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int k = lane + 32 * i, t = k >> 3, c = k & 7;
-        *reinterpret_cast<uint4*>(&s_vc[pair][tb + t][4 * c]) = src[k];
-      }
-    }
     const float bm = fmaxf(s_bmax[pair][buf][0][tig], s_bmax[pair][buf][1][tig]);
     if (__any_sync(0xffffffffu, bm > m_run + kLazy)) raise_to(bm);
     {
@@ -320,9 +307,9 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
     if (pair_ok) {
 #pragma unroll 1
       for (int tm = 0; tm < 4; ++tm) {
-        // MMA indices k = 2tig, 2tig+1, 2tig+8, 2tig+9 stand for the m-tile's tokens
-        // TA..TD = tig, tig+4, tig+8, tig+12 (the same permutation for A and B)
-        const int TA = 16 * tm + tig, TB = TA + 4, TC = TA + 8, TD = TA + 12;
+        // MMA indices k = 2tig, 2tig+1 are the m-tile's tokens TA = 2tig, TB = TA+1
+        // (token pair tig), k = 2tig+8, 2tig+9 are TC = TA+8, TD = TA+9 (pair tig+4)
+        const int TA = 16 * tm + 2 * tig, TB = TA + 1, TC = TA + 8, TD = TA + 9;
         const float pA = s_p[pair][buf][TA][hP], pB = s_p[pair][buf][TB][hP];
         const float pC = s_p[pair][buf][TC][hP], pD = s_p[pair][buf][TD][hP];
         const float* vs = reinterpret_cast<const float*>(blk + g.o_vscale);
@@ -346,27 +333,20 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
             bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
           }
         }
-        // this half's 16 code words of a token: 4 x uint4 from word 16 half
+        // words (s, G) = (gid + 8 u, 2 half + v) of the pairs tig and tig + 4
+        const unsigned char* vc = blk + g.o_vcode + 16 * gid + 8 * half;
+        uint2 wAB[2], wCD[2];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          // words 4 q4 .. 4 q4 + 3 = channel m-tiles 2 q4 and 2 q4 + 1 of this half
-          const int wo = 16 * half + 4 * q4;
-          const uint4 cA = *reinterpret_cast<const uint4*>(&s_vc[pair][TA][wo]);
-          const uint4 cB = *reinterpret_cast<const uint4*>(&s_vc[pair][TB][wo]);
-          const uint4 cC = *reinterpret_cast<const uint4*>(&s_vc[pair][TC][wo]);
-          const uint4 cD = *reinterpret_cast<const uint4*>(&s_vc[pair][TD][wo]);
-          const uint32_t wa[4] = {cA.x, cA.y, cA.z, cA.w}, wb[4] = {cB.x, cB.y, cB.z, cB.w};
-          const uint32_t wc[4] = {cC.x, cC.y, cC.z, cC.w}, wd[4] = {cD.x, cD.y, cD.z, cD.w};
+        for (int u = 0; u < 2; ++u) {
+          wAB[u] = *reinterpret_cast<const uint2*>(vc + (TA >> 1) * kWPairBytes + 128 * u);
+          wCD[u] = *reinterpret_cast<const uint2*>(vc + (TC >> 1) * kWPairBytes + 128 * u);
+        }
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int mt = 2 * q4 + u;          // channels 128 half + 16 mt + gid (+8)
-            const uint32_t a0 = prmt(wa[2 * u], wb[2 * u], psel) & codeMask;
-            const uint32_t a1 = prmt(wa[2 * u + 1], wb[2 * u + 1], psel) & codeMask;
-            const uint32_t a2 = prmt(wc[2 * u], wd[2 * u], psel) & codeMask;
-            const uint32_t a3 = prmt(wc[2 * u + 1], wd[2 * u + 1], psel) & codeMask;
-            const int gi = mt >> 2;             // group within this half (64 channels)
-            hmma16816(acc[mt], a0, a1, a2, a3, bpv[gi][0], bpv[gi][1]);
-          }
+        for (int mt = 0; mt < 8; ++mt) {
+          const int u = (mt >> 1) & 1, v = mt >> 2, sh = 8 * (mt & 1);
+          const uint32_t ab = (v ? wAB[u].y : wAB[u].x) >> sh, cd = (v ? wCD[u].y : wCD[u].x) >> sh;
+          hmma16816(acc[mt], ab & 0x000F000Fu, ab & 0x00F000F0u, cd & 0x000F000Fu, cd & 0x00F000F0u,
+                    bpv[v][0], bpv[v][1]);
         }
       }
     }
@@ -401,6 +381,12 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
     return;
   }
 
+  // acc[mt][c] is channel chan(mt) (+1 for c >= 2) of head tig in units of
+  // 2^-24 (row gid + 8: 2^-20)
+  auto chan = [&](int mt) {
+    return 64 * (2 * half + (mt >> 2)) + 4 * gid + 32 * ((mt >> 1) & 1) + 2 * (mt & 1);
+  };
+  auto code_unit = [&](int mt) { return (void)mt, 5.9604644775390625e-8f; };   // 2^-24
   // ---------------- exact ring tokens (last split): pair q takes slots
   // per_pair q .. +per_pair-1 of each chunk; both warps of the pair score them
   // (identical logits, identical running-max decisions), each adds p v on its
@@ -445,13 +431,14 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
         const float pt = __shfl_sync(0xffffffffu, p0, 4 * T + tig);
         const int sl2 = per_pair * pair + T;
         if (sl2 >= nc) break;
-        const int64_t e = (int64_t)sl2 * WD + 128 * half;
+        const int64_t e = (int64_t)sl2 * WD;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const float v0 = load_f(s_rv, e + 16 * mt + gid, g.dtype);
-          const float v1 = load_f(s_rv, e + 16 * mt + gid + 8, g.dtype);
-          acc[mt][0] = fmaf(pt * v0, code_unit, acc[mt][0]);
-          acc[mt][2] = fmaf(pt * v1, code_unit, acc[mt][2]);
+          const float v0 = load_f(s_rv, e + chan(mt), g.dtype);
+          const float v1 = load_f(s_rv, e + chan(mt) + 1, g.dtype);
+          const float u = code_unit(mt);
+          acc[mt][0] = fmaf(pt * v0, u, acc[mt][0]);
+          acc[mt][2] = fmaf(pt * v1, 16.f * u, acc[mt][2]);
         }
       }
       __syncthreads();     // the chunk is consumed before the next one is requested
@@ -479,11 +466,12 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   const float sc = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mh);
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    const int ch0 = 128 * half + 16 * mt + gid, ch1 = ch0 + 8;
     const int grp = 2 * half + (mt >> 2);
     const float mnv = s_mn[pair][0][tig][grp] + s_mn[pair][1][tig][grp];
-    s_out[(pair * MG + tig) * WD + ch0] = ((acc[mt][0] + acc[mt][1]) * inv_unit + mnv) * sc;
-    s_out[(pair * MG + tig) * WD + ch1] = ((acc[mt][2] + acc[mt][3]) * inv_unit + mnv) * sc;
+    const float inv = 16777216.f;      // 2^24 = 1 / code_unit(mt)
+    *reinterpret_cast<float2*>(&s_out[(pair * MG + tig) * WD + chan(mt)]) =
+        make_float2(((acc[mt][0] + acc[mt][1]) * inv + mnv) * sc,
+                    ((acc[mt][2] + acc[mt][3]) * (0.0625f * inv) + mnv) * sc);
   }
   __syncthreads();
   for (int i = tid; i < MG * WD; i += WT) {

@@ -111,8 +111,20 @@ __device__ __forceinline__ const void* src_row(const QParams& p, bool values, in
   return chunk;
 }
 
+// 16-bit half x (codes of channels (16/vbits) x ...) of the value codes of row i:
+// token-major in the standalone arrays, token-pair records in the cache.
+__device__ __forceinline__ uint16_t* code_half_ptr(const QParams& p, int bh, int64_t i, int x) {
+  if (p.cache_mode) {
+    const Geom& g = p.g;
+    const int64_t t = p.t_first + i;
+    uint8_t* blk = p.base + (int64_t)bh * g.region_bytes + (t / kBlockTokens) * g.block_bytes;
+    return reinterpret_cast<uint16_t*>(blk + g.o_vcode + vcode_half_off(g, (int)(t % kBlockTokens), x));
+  }
+  return reinterpret_cast<uint16_t*>(p.arr.codes + (p.t_first + i) * (p.d * p.vbits / 8)) + x;
+}
+
 __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t i, int which) {
-  // which: 0 idx, 1 sign, 2 rho, 3 rnorm, 4 vcode, 5 vscale, 6 vmin
+  // which: 0 idx, 1 sign, 2 rho, 3 rnorm, 5 vscale, 6 vmin (value codes: code_half_ptr)
   if (p.cache_mode) {
     const Geom& g = p.g;
     const int64_t t = p.t_first + i;
@@ -121,7 +133,6 @@ __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t 
       case 1: return field_ptr(p.base, g, bh, t, g.o_sign, g.f_sign);
       case 2: return field_ptr(p.base, g, bh, t, g.o_rho, 4);
       case 3: return field_ptr(p.base, g, bh, t, g.o_rnorm, 4);
-      case 4: return field_ptr(p.base, g, bh, t, g.o_vcode, g.f_vcode);
       case 5: return field_ptr(p.base, g, bh, t, g.o_vscale, g.f_vmeta);
       default: return field_ptr(p.base, g, bh, t, g.o_vmin, g.f_vmeta);
     }
@@ -133,7 +144,6 @@ __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t 
     case 1: return p.arr.signs + ti * (p.m / 8);
     case 2: return reinterpret_cast<uint8_t*>(p.arr.rho + ti);
     case 3: return reinterpret_cast<uint8_t*>(p.arr.rnorm + ti);
-    case 4: return p.arr.codes + ti * (d * p.vbits / 8);
     case 5: return reinterpret_cast<uint8_t*>(p.arr.vscale + ti * (d / p.group));
     default: return reinterpret_cast<uint8_t*>(p.arr.vmin + ti * (d / p.group));
   }
@@ -345,7 +355,8 @@ __device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, in
       const int ch = w * per_word + k;
       word |= value_code(s.X[r * sx + ch], mn, sc, inv, levels) << (k * vb);
     }
-    reinterpret_cast<uint32_t*>(dst_field(p, bh, row0 + r, 4))[w] = word;
+    *code_half_ptr(p, bh, row0 + r, 2 * w) = (uint16_t)word;
+    *code_half_ptr(p, bh, row0 + r, 2 * w + 1) = (uint16_t)(word >> 16);
   }
   __syncthreads();
 }
@@ -554,7 +565,8 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
         const int ch = w * per_word + k;
         word |= value_code(sx[ch], mn, sc, inv, levels) << (k * vb);
       }
-      reinterpret_cast<uint32_t*>(dst_field(p, bh, row, 4))[w] = word;
+      *code_half_ptr(p, bh, row, 2 * w) = (uint16_t)word;
+      *code_half_ptr(p, bh, row, 2 * w + 1) = (uint16_t)(word >> 16);
     }
   }
 }
@@ -777,9 +789,13 @@ __device__ __forceinline__ void quantize_values_rows(const QParams& p, int bh, i
     uint32_t bits = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) bits |= value_code(x[k], mn, sc, inv, levels) << (k * vb);
-    uint8_t* vc = dst_field(p, bh, row0 + r, 4);
-    if (vb == 2) vc[lane] = (uint8_t)bits;
-    else reinterpret_cast<uint16_t*>(vc)[lane] = (uint16_t)bits;
+    if (vb == 2) {
+      // a 16-bit half holds the 8 codes of lanes 2x and 2x + 1
+      const uint32_t hi = __shfl_down_sync(0xffffffffu, bits, 1);
+      if ((lane & 1) == 0) *code_half_ptr(p, bh, row0 + r, lane >> 1) = (uint16_t)(bits | (hi << 8));
+    } else {
+      *code_half_ptr(p, bh, row0 + r, lane) = (uint16_t)bits;
+    }
     if ((lane % lanes_g) == 0) {
       const int gi = (4 * lane) / g;
       reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 5))[gi] = sc;

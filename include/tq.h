@@ -173,7 +173,13 @@ typedef struct tq_cache_desc {
  * for each (b, h) a region of ceil(capacity/64) blocks of 64 tokens; a block
  * stores, field after field, the 64 tokens' idx planes (b1*d/8 B each), sign
  * bits (m/8 B), rho (fp32), ||r|| (fp32, absent if b1 == 0), value codes
- * (d*vbits/8 B), value scales (d/g fp32) and value minima (d/g fp32).  After the
+ * (d*vbits/8 B), value scales (d/g fp32) and value minima (d/g fp32).  The
+ * value codes alone are stored by token pairs (tokens 2i, 2i+1 of the block):
+ * cut a token's codes (code j at bit (j*vbits) mod 16 of 16-bit half
+ * (j*vbits)/16) into halves; with H = g*vbits/16 halves per group and NG = d/g,
+ * half gi*H + s of token 2i is the low and that of token 2i+1 the high 16 bits
+ * of 32-bit word s*NG + gi of the pair's record (d*vbits/16 words), so that one
+ * masked word is a tensor-core operand of two tokens.  After the
  * regions, 256-byte aligned: ring keys [B, Hkv, W, d] then ring values, in dtype.
  * Token t (counting every token ever appended) sits in ring slot t mod W.
  * After each append the ring holds the last min(W, n_total) tokens and every

@@ -16,7 +16,13 @@ Token record (little-endian, LSB-first bit order):
 
 Block: TB = 64 consecutive tokens, stored field by field (all 64 idx records,
 then all 64 sign records, ...); every field is a multiple of 16 bytes long, so
-a block is one contiguous, 16-byte aligned chunk.
+a block is one contiguous, 16-byte aligned chunk.  The value codes of a block
+are the one field not stored token by token: they form 32 token-pair records
+(tokens 2i and 2i+1 of the block), each of d*vb/16 little-endian 32-bit words.
+Cut a token's vcodes (above) into 16-bit halves, half x holding the 16/vb
+channels starting at (16/vb)*x; with H = g*vb/16 halves per value group and
+NG = d/g groups, half x = gi*H + s of token 2i goes to the low 16 bits and that
+of token 2i+1 to the high 16 bits of word s*NG + gi of the pair record.
 
 Cache buffer: for each (batch b, kv head h) a region of ceil(capacity/TB)
 blocks, regions in (b, h) order; then, at the next 256-byte boundary, the ring
@@ -135,8 +141,18 @@ def _dest(lay: Layout, b: int, h: int, t, name: str):
     """Byte addresses [n, size] of field ``name`` of tokens t (array) in region (b, h)."""
     off, size = _field_geom(lay)[name]
     t = np.asarray(t, dtype=np.int64)
-    start = lay.region_off(b, h) + (t // TB) * lay.block_bytes + off + (t % TB) * size
-    return start[:, None] + np.arange(size, dtype=np.int64)[None, :]
+    blk = lay.region_off(b, h) + (t // TB) * lay.block_bytes + off
+    k = np.arange(size, dtype=np.int64)[None, :]
+    if name != "vcode":
+        return (blk + (t % TB) * size)[:, None] + k
+    # byte k of the token's vcodes: half x = k // 2, byte k % 2 of that half
+    H = lay.group * lay.vbits // 16
+    NG = lay.d // lay.group
+    x = k // 2
+    word = (x % H) * NG + x // H
+    tt = t % TB
+    pair = blk + (tt // 2) * (2 * size) + 2 * (tt % 2)
+    return pair[:, None] + 4 * word + k % 2
 
 
 def write_region(buf: np.ndarray, lay: Layout, b: int, h: int, t0: int, fields: dict):

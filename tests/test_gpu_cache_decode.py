@@ -88,6 +88,54 @@ def test_append_packed_bytes_match_oracle_across_chunks():
         _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
 
 
+def test_append_degenerate_tokens_every_quantise_path():
+    """Zero keys, constant value rows (s = 0), exact half-step value ties and zero
+    value rows through the tensor-core tile kernel (a 300-token chunk), the
+    single-token kernel (chunks of 1 and 5) and the fused decode step: packed
+    bytes equal the oracle's (codes outside the boundary band)."""
+    w = _workload(B=1, Hkv=2, Hq=8, T=420)
+    cap = 512
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda")
+    # A token is quantised when it leaves the 16-token ring: positions < 284 in the
+    # 300-token chunk (tile kernel), 284..290 in the appends of 1, 5, 1 (single-token
+    # kernel), 291..403 in the decode steps (fused pre-grid), 404.. stay in the ring.
+    ties = (torch.arange(32, device="cuda") % 7).to(V.dtype) * 0.5   # range 3 -> s = 1
+    for t in (3, 150, 284, 286, 301, 307, 411):
+        K[0, 1, t].zero_()                                   # zero-norm keys
+        V[0, 0, t] = 0.75                                    # constant rows: s = 0
+        V[0, 1, t, :32] = ties                               # exact half-step ties
+    for t in (151, 287, 304):
+        V[0, 0, t].zero_()
+    gc = _gpu_cache(w, cap)
+    oc = _oracle_cache(w, cap, po, cb)
+    pj, cbd = _Proj(po), _Cb(cb)
+    t = 0
+    for n in (300, 1, 5, 1):                                 # tile kernel, then single-token
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        gc.append(k, v, pj, cbd)
+        oc.append(host(k), host(v))
+        t += n
+    while t < w.T:                                           # fused decode steps
+        n = min(2, w.T - t)
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        Q = synth.queries(w.scaled(seed=t), device="cuda")
+        gc.decode_step(k, v, Q, pj, cbd)
+        oc.append(host(k), host(v))
+        t += n
+    torch.cuda.synchronize()
+    assert gc.n_total == oc.n_total == w.T
+    buf = gc.buffer.cpu().numpy()
+    _compare_cache_bytes(buf, oc)
+    fg = olayout.read_region(buf, oc.lay, 0, 1, oc.rec[0][1]["rho"].shape[0])
+    zero = [3, 150, 284, 286, 301, 307]                      # compressed zero keys
+    rho = np.ascontiguousarray(fg["rho"]).view("<f4").ravel()
+    rn = np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel()
+    assert np.all(rho[zero] == 0) and np.all(rn[zero] == 0)
+    bits = olayout.unpack_bits(fg["sign"], w.m)
+    assert np.array_equal(bits[zero], oc.rec[0][1]["bits"][zero])   # sign(0) convention
+
+
 @pytest.mark.parametrize("b1,m,vb,g,dt", [(2, 128, 2, 32, "f32"), (0, 256, 2, 32, "f16"),
                                           (3, 256, 4, 64, "bf16"), (1, 64, 4, 16, "bf16")])
 def test_append_quantize_variants(b1, m, vb, g, dt):

@@ -70,6 +70,34 @@ def test_region_write_read_round_trip():
     assert not buf[:lay.region_off(1, 0)].any()            # other regions untouched
 
 
+@pytest.mark.parametrize("d,vb,g,tok,ch,byte,bit", [
+    # d 128, 2-bit, g 32: token 5 = high half of pair 2 (64-byte records); channel
+    # 37 = group 1, half s 0 (8 channels a half), 6th code -> word 0*4 + 1, bits 10-11
+    (128, 2, 32, 5, 37, 2 * 64 + 4 * 1 + 2 + 1, 2),
+    # d 256, 4-bit, g 64: token 10 = low half of pair 5 (256-byte records); channel
+    # 200 = group 3, half s 2 (4 channels a half), 1st code -> word 2*4 + 3, bits 0-3
+    (256, 4, 64, 10, 200, 5 * 256 + 4 * 11, 0),
+    # second block, g 16: token 64 + 3 = high half of pair 1; channel 127 = group 7,
+    # half s 1 (2 halves a group), 8th code -> word 1*8 + 7, bits 14-15
+    (128, 2, 16, 67, 127, 1 * 64 + 4 * 15 + 2 + 1, 6)])
+def test_value_code_pair_records_by_hand(d, vb, g, tok, ch, byte, bit):
+    lay = layout.Layout(1, 1, d, 0, 64, vb, g, 0, 128, "f32")
+    n = tok + 1
+    codes = np.zeros((n, d), np.uint8)
+    codes[tok, ch] = (1 << vb) - 1
+    f = {"idx": np.zeros((n, 0), np.uint8), "sign": np.zeros((n, 8), np.uint8),
+         "rho": np.zeros((n, 4), np.uint8), "rnorm": np.zeros((n, 0), np.uint8),
+         "vcode": layout.pack_codes(codes, vb),
+         "vscale": np.zeros((n, 4 * d // g), np.uint8), "vmin": np.zeros((n, 4 * d // g), np.uint8)}
+    buf = np.zeros(lay.total_bytes, np.uint8)
+    layout.write_region(buf, lay, 0, 0, 0, f)
+    at = (tok // layout.TB) * lay.block_bytes + lay.o_vcode + byte
+    assert buf[at] == ((1 << vb) - 1) << bit
+    assert np.count_nonzero(buf) == 1
+    back = layout.decode_fields(layout.read_region(buf, lay, 0, 0, n), lay)
+    assert np.array_equal(back["codes"], codes)
+
+
 def test_all_exact_decode_equals_dense_attention():
     rng = np.random.default_rng(2)
     G, d, n = 4, 64, 40
