@@ -592,6 +592,14 @@ int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* works
   return ok();
 }
 
+int tq_quantize_check(void* stream) {
+  int flag = 0;
+  cudaError_t e = tq::quantize_error_flag(&flag, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_quantize_check");
+  if (flag) return fail(TQ_ERR_CUDA, "quantise: a tensor-core product did not complete within its wait limit");
+  return ok();
+}
+
 static int parse_list(const char* s, int* out, int max_n) {
   int n = 0;
   const char* p = s;

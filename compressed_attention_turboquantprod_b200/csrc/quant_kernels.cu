@@ -1,21 +1,24 @@
 // Key/value quantisation and append ([TQ] 二 three-stage pipeline, 五
 // ProdQuantized, 六 store + ring, 七 value group quantisation).
 //
-// One CTA quantises a tile of 64 tokens of one (b, kv head):
-//   keys   rho = ||x|| (float64 sum of exact fp32 squares)
-//          Y = X Pi^T (fp32 FMA), y = Y / rho, idx_j = #{k : beta_k < y_j},
+//   keys   rho = ||x||, y = Pi x / rho, idx_j = #{k : beta_k < y_j},
 //          e = y - c[idx], ||r|| = rho ||e||, z = rho (T e) with T = S Pi^T,
-//          sign bit = [z >= 0]; bit-planes and signs packed with warp ballots
-//          (lane i -> bit i, so words are LSB-first / little-endian).
+//          sign bit = [z >= 0]; words LSB-first / little-endian.
 //          Pure QJL (b1 = 0): z = S x.
 //   values per (token, group): mn, mx, s = (mx - mn)/(2^vb - 1),
 //          code = clamp(rint((v - mn)/s)) in IEEE fp32 (__fsub_rn/__fdiv_rn/rintf).
-// The contractions run as a register-tiled fp32 SGEMM (64 tokens x 128 columns
-// per pass, 4x8 outputs per thread).
+// Three kernels:
+//   * head dim 128, m = 128, b1 >= 1, more than 8 tokens: 128-token tiles on the
+//     fifth-generation tensor cores (tcgen05 MMAs into tensor memory, one token
+//     row per thread in the epilogue; k_quantize_tc);
+//   * at most 8 tokens (a decode step's append): a CTA per token (k_quantize_small);
+//   * every other shape: 64-token tiles with the contractions as a register-tiled
+//     fp32 SGEMM (k_quantize).
 #include <cfloat>
 
 #include "common.cuh"
 #include "prep_mma.cuh"
+#include "tc_common.cuh"
 
 namespace tq {
 namespace {
@@ -626,380 +629,434 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_step_pre(QParams p, int nq_ct
                             smem_raw);
 }
 
-// ---------------------------------------------------------------------------
-// Tensor-core tile path (head dim 128, b1 > 0, m = 128): a persistent CTA per SM
-// keeps Pi and T = S Pi^T resident in shared memory as fp16 hi/lo pairs
-// (v * 2^10 = hi + lo, |lo| <= 2^-11 |hi|), and loops over 64-token tiles:
-//   U = X / rho -> fp16 hi/lo;  Y = U Pi^T  and  Z = E T^T (E = Y - c[idx])
-// each as three mma.sync m16n8k16 products (hi*hi + hi*lo + lo*hi, fp32
-// accumulate), i.e. about 22 significant bits: well inside the 1e-5 band that
-// separates a code or a sign from its decision boundary.
-// ---------------------------------------------------------------------------
+// Operands of the tensor-core tile path (head dim 128, b1 > 0, m = 128) are held
+// as fp16 hi/lo pairs of v * 2^10 (|lo| <= 2^-11 |hi|); three products hi*hi +
+// hi*lo + lo*hi with fp32 accumulation keep about 22 significant bits, well
+// inside the 1e-5 band that separates a code or a sign from its decision boundary.
 constexpr int QD = 128;             // head dim of this path
 constexpr int QM = 128;             // sketch rows of this path
-constexpr int HS = QD + 8;          // fp16 row stride (272 B: conflict-free ldmatrix)
-constexpr int YS = QD + 4;          // fp32 row stride of the Y / Z / V tile
 constexpr float kSplit = 1024.f;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+// ---------------------------------------------------------------- tcgen05 tiles
+// Batched key quantisation on the fifth-generation tensor cores: a persistent
+// CTA per SM takes 128-token tiles of one (b, kv head).  Its 16 warps own one
+// token row per thread: warp w takes row 32 (w mod 4) + lane (the tensor-memory
+// lanes that warp may read) and coordinates 32 (w / 4) .. +31 of it; thread 0
+// also issues the MMAs after the barrier that completes their operand.
+//   1. rho = ||x|| (fp32 partial sums of 4 squares, float64 total), u = x / rho
+//      as f16 hi + lo (x 2^10) into A
+//   2. Y = U Pi^T: hi*hi + hi*lo + lo*hi per 16-wide k-step, fp32 in tensor memory;
+//      meanwhile the tile's values: per (token, group) mn, s, codes (fp32, IEEE order)
+//   3. y, idx_j = #{k : beta_k < y_j}, e = y - c[idx] as hi + lo into A,
+//      ||r|| = rho ||e||
+//   4. Z = E T^T the same way (T = S Pi^T, so z = rho Z); sign bit [rho Z >= 0]
+// Pi and T stay resident as f16 hi + lo in the canonical operand layout.
+constexpr int TCM = 128;                   // rows of a tile (MMA M)
+constexpr int TC_PARTS = 4;                // 32-coordinate parts of a row
+constexpr int TC_THREADS = TCM * TC_PARTS; // 16 warps
+constexpr uint32_t TC_COLS = 128;          // tensor-memory columns: one 128 x 128 fp32 tile
+constexpr int TC_OPB = TCM * QD * 2;       // bytes of one f16 operand (32 KB)
+constexpr float kRound = 12582912.f;       // 1.5 * 2^23: x + kRound rounds x (|x| < 2^22) to an integer
+
+__device__ int g_quant_tc_err;             // sticky: a bounded wait gave up
+
+__host__ __device__ inline size_t tc_smem_bytes() {
+  return (size_t)6 * TC_OPB + (sizeof(double) * 2 + sizeof(float2)) * TC_PARTS * TCM;
 }
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void split_store(__half* hi, __half* lo, float v) {
-  const float x = v * kSplit;
-  const __half h = __float2half_rn(x);
-  *hi = h;
-  *lo = __float2half_rn(x - __half2float(h));
-}
-
-constexpr int QG = 4;              // independent warp groups per CTA
-constexpr int QNT = 16;            // rows of a group's tile
-
-struct MmaGroupSmem {
-  __half *AH, *AL;                 // [QNT][HS]
-  float* YZ;                       // [QNT][YS]
-  double* rho64;                   // [QNT]
-  float* rho;                      // [QNT]
-};
-
-struct MmaSmem {
-  __half *PH, *PL, *TH, *TL;       // [128][HS] each
-  float* cb;                       // [32]
-};
-
-__host__ __device__ inline size_t mma_group_bytes() {
-  return sizeof(__half) * 2 * QNT * HS + sizeof(float) * QNT * YS + sizeof(double) * QNT +
-         sizeof(float) * QNT;
-}
-
-__host__ __device__ inline size_t mma_smem_bytes() {
-  return sizeof(__half) * 4 * 128 * HS + QG * mma_group_bytes() + sizeof(float) * 32;
-}
-
-__device__ MmaSmem mma_carve(unsigned char* raw) {
-  MmaSmem s;
-  s.PH = reinterpret_cast<__half*>(raw);
-  s.PL = s.PH + 128 * HS;
-  s.TH = s.PL + 128 * HS;
-  s.TL = s.TH + 128 * HS;
-  s.cb = reinterpret_cast<float*>(raw + sizeof(__half) * 4 * 128 * HS + QG * mma_group_bytes());
-  return s;
-}
-
-__device__ MmaGroupSmem mma_group_carve(unsigned char* raw, int grp) {
-  MmaGroupSmem m;
-  unsigned char* q = raw + sizeof(__half) * 4 * 128 * HS + (size_t)grp * mma_group_bytes();
-  m.AH = reinterpret_cast<__half*>(q);
-  m.AL = m.AH + QNT * HS;
-  m.YZ = reinterpret_cast<float*>(m.AL + QNT * HS);
-  m.rho64 = reinterpret_cast<double*>(m.YZ + QNT * YS);
-  m.rho = reinterpret_cast<float*>(m.rho64 + QNT);
-  return m;
-}
-
-constexpr int QTHREADS = 512;       // 16 warps per CTA on the tensor-core tile path
-
-// C[QNT x 128] = A[QNT x 128] * B^T for one warp group, A and B as fp16 hi/lo
-// pairs (rows of 128, stride HS); warp gw (of the group's GW) owns the QNT rows
-// and columns (128 / GW) gw .. +128 / GW.  The result (scaled back by 2^-20) goes
-// to C (fp32, stride YS).
-template <int MTI, int NTI>     // 16-row m-tiles, 16-column B loads per warp
-__device__ __forceinline__ void mma_gemm_group(const __half* AH, const __half* AL, const __half* BH,
-                                               const __half* BL, float* C, int gw) {
-  const int lane = threadIdx.x & 31;
-  const int c0 = 16 * NTI * gw;
-  float acc[MTI][2 * NTI][4];
+// Eight consecutive values (times 2^10) as f16 hi and lo parts, one 16-byte chunk each.
+__device__ __forceinline__ void split8(const float (&v)[8], float scale, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
 #pragma unroll
-  for (int i = 0; i < MTI; ++i)
+  for (int j = 0; j < 4; ++j) {
+    const float a0 = v[2 * j] * scale, a1 = v[2 * j + 1] * scale;
+    const __half2 hh = __floats2half2_rn(a0, a1);
+    const float2 f = __half22float2(hh);
+    const __half2 ll = __floats2half2_rn(a0 - f.x, a1 - f.y);
+    h[j] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[j] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 32 consecutive elements of a row as fp32 (16-byte loads); zeros when !valid.
+__device__ __forceinline__ void load32(const void* base, int64_t e, int dtype, bool valid, float (&o)[32]) {
+  if (!valid) {
 #pragma unroll
-    for (int j = 0; j < 2 * NTI; ++j)
+    for (int j = 0; j < 32; ++j) o[j] = 0.f;
+    return;
+  }
+  if (dtype == TQ_F32) {
+    const float4* p4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + e);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
-  const int ar = lane & 15, ac = 8 * (lane >> 4);                    // A: rows, k offset
-  const int bn = (lane & 7) + 8 * (lane >> 4), bk = 8 * ((lane >> 3) & 1);   // B: n, k offset
-#pragma unroll 2
-  for (int ks = 0; ks < QD / 16; ++ks) {
-    uint32_t ah[MTI][4], al[MTI][4];
-#pragma unroll
-    for (int i = 0; i < MTI; ++i) {
-      ldsm_x4(ah[i], AH + (16 * i + ar) * HS + 16 * ks + ac);
-      ldsm_x4(al[i], AL + (16 * i + ar) * HS + 16 * ks + ac);
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = p4[j];
+      o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
     }
+    return;
+  }
+  const uint4* p4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + e);
 #pragma unroll
-    for (int jb = 0; jb < NTI; ++jb) {
-      uint32_t bh[4], bl[4];
-      ldsm_x4(bh, BH + (c0 + 16 * jb + bn) * HS + 16 * ks + bk);
-      ldsm_x4(bl, BL + (c0 + 16 * jb + bn) * HS + 16 * ks + bk);
+  for (int j = 0; j < 4; ++j) {
+    const uint4 u = p4[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int i = 0; i < MTI; ++i) {
-        mma16816(acc[i][2 * jb], ah[i], bh[0], bh[1]);
-        mma16816(acc[i][2 * jb], ah[i], bl[0], bl[1]);
-        mma16816(acc[i][2 * jb], al[i], bh[0], bh[1]);
-        mma16816(acc[i][2 * jb + 1], ah[i], bh[2], bh[3]);
-        mma16816(acc[i][2 * jb + 1], ah[i], bl[2], bl[3]);
-        mma16816(acc[i][2 * jb + 1], al[i], bh[2], bh[3]);
-      }
+    for (int k = 0; k < 4; ++k) {
+      float2 f;
+      if (dtype == TQ_F16) f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      else f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+      o[8 * j + 2 * k] = f.x;
+      o[8 * j + 2 * k + 1] = f.y;
     }
   }
-  const int gid = lane >> 2, tig = lane & 3;
-  const float sc = 1.f / (kSplit * kSplit);
-#pragma unroll
-  for (int i = 0; i < MTI; ++i)
-#pragma unroll
-    for (int j = 0; j < 2 * NTI; ++j) {
-      const int row = 16 * i + gid, col = c0 + 8 * j + 2 * tig;
-      C[row * YS + col] = acc[i][j][0] * sc;
-      C[row * YS + col + 1] = acc[i][j][1] * sc;
-      C[(row + 8) * YS + col] = acc[i][j][2] * sc;
-      C[(row + 8) * YS + col + 1] = acc[i][j][3] * sc;
-    }
 }
 
-// Values of a warp's rows straight from the source: lane l holds channels
-// 4l..4l+3; the group min / max come from xor-shuffles over the g/4 lanes of the
-// group; codes leave as one byte (2-bit) or two bytes (4-bit) per lane.
-__device__ __forceinline__ void quantize_values_rows(const QParams& p, int bh, int64_t row0, int nrows,
-                                                     int warp, int lane, int nwarps) {
-  const int d = p.d, g = p.group, vb = p.vbits, lanes_g = g / 4;
-  const float levels = (float)((1 << vb) - 1);
-  for (int r = warp; r < nrows; r += nwarps) {
-    if (row0 + r >= p.n) break;
-    int64_t e0;
-    const void* src = src_row(p, true, bh, row0 + r, e0);
-    float x[4];
-    load4(src, e0 + 4 * lane, p.dtype, x);
-    float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
-    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-    for (int o = 1; o < lanes_g; o <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    const float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
-    const float inv = sc != 0.f ? __frcp_rn(sc) : 0.f;
-    uint32_t bits = 0;
+// code = clamp(rint(fl((v - mn) / s)), 0, levels) as in value_code, with the
+// rounding done by adding kRound (exact for 0 <= x < 2^22, ties to even) and
+// the integer read from the sum's low mantissa bits.
+__device__ __forceinline__ uint32_t value_code_fast(float v, float mn, float sc, float inv, uint32_t levels) {
+  if (sc == 0.f) return 0u;
+  const float a = __fsub_rn(v, mn);
+  const float x = __fmul_rn(a, inv);
+  float t = __fadd_rn(x, kRound);
+  const float r = __fsub_rn(t, kRound);
+  if (fabsf(fabsf(__fsub_rn(x, r)) - 0.5f) < 1e-5f) t = __fadd_rn(rintf(__fdiv_rn(a, sc)), kRound);
+  const uint32_t c = __float_as_uint(t) - __float_as_uint(kRound);
+  return c < levels ? c : levels;
+}
+
+// The issuing thread: D = A B^T over K = 128 as three products per k-step.
+__device__ __forceinline__ void tc_gemm(uint32_t d_tmem, uint32_t ah, uint32_t al, uint32_t bh,
+                                        uint32_t bl) {
+  constexpr uint32_t idesc = tc::idesc_f16(TCM, QD);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) bits |= value_code(x[k], mn, sc, inv, levels) << (k * vb);
-    if (vb == 2) {
-      // a 16-bit half holds the 8 codes of lanes 2x and 2x + 1
-      const uint32_t hi = __shfl_down_sync(0xffffffffu, bits, 1);
-      if ((lane & 1) == 0) *code_half_ptr(p, bh, row0 + r, lane >> 1) = (uint16_t)(bits | (hi << 8));
-    } else {
-      *code_half_ptr(p, bh, row0 + r, lane) = (uint16_t)bits;
-    }
-    if ((lane % lanes_g) == 0) {
-      const int gi = (4 * lane) / g;
-      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 5))[gi] = sc;
-      reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 6))[gi] = mn;
-    }
-    (void)d;
+  for (int ks = 0; ks < QD / 16; ++ks) {
+    const uint32_t o = 256u * ks;
+    tc::mma_f16(d_tmem, tc::smem_desc(ah + o), tc::smem_desc(bh + o), idesc, ks > 0 ? 1u : 0u);
+    tc::mma_f16(d_tmem, tc::smem_desc(ah + o), tc::smem_desc(bl + o), idesc, 1u);
+    tc::mma_f16(d_tmem, tc::smem_desc(al + o), tc::smem_desc(bh + o), idesc, 1u);
   }
 }
 
 template <int B1>
-__global__ void __launch_bounds__(QTHREADS, 1) k_quantize_mma(QParams p, int64_t tiles_per_bh,
-                                                             int64_t total_tiles) {
+__global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_t tiles_per_bh,
+                                                              int64_t total_tiles) {
+  using mmadec::mbar_init;
+  using mmadec::mbar_wait;
+  using mmadec::smem_u32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  MmaSmem s = mma_carve(smem_raw);
+  __shared__ __align__(8) uint64_t s_mbar[2];      // Y done, Z done
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  unsigned char* PH = smem_raw;
+  unsigned char* PL = PH + TC_OPB;
+  unsigned char* TH = PL + TC_OPB;
+  unsigned char* TL = TH + TC_OPB;
+  unsigned char* AH = TL + TC_OPB;
+  unsigned char* AL = AH + TC_OPB;
+  double* ssp = reinterpret_cast<double*>(AL + TC_OPB);   // [part][row] partial sums of x^2
+  double* sep = ssp + TC_PARTS * TCM;                      // [part][row] partial sums of e^2
+  float2* vmm = reinterpret_cast<float2*>(sep + TC_PARTS * TCM);   // [part][row] value min / max
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int L = 1 << B1;
-  constexpr int GW = QTHREADS / 32 / QG;         // warps per group
-  constexpr int RPW = QNT / GW;                  // rows per warp of a group tile
-  // resident operands: Pi and T as fp16 hi/lo, rows of 128 (four elements a thread)
-  for (int i = 4 * tid; i < QD * QD; i += 4 * QTHREADS) {
-    const int r = i / QD, c = i % QD;
-    const float4 a = *reinterpret_cast<const float4*>(p.Pi + i);
-    const float4 b = *reinterpret_cast<const float4*>(p.T + i);
-    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      split_store(s.PH + r * HS + c + k, s.PL + r * HS + c + k, av[k]);
-      split_store(s.TH + r * HS + c + k, s.TL + r * HS + c + k, bv[k]);
-    }
-  }
-  if (tid < 16) {
-    s.cb[tid] = (tid < L) ? p.cent[tid] : 0.f;
-    s.cb[16 + tid] = (tid + 1 < L) ? p.bnd[tid] : 0.f;
-  }
-  __syncthreads();
-  float bnd[L - 1];
-#pragma unroll
-  for (int k = 0; k + 1 < L; ++k) bnd[k] = s.cb[16 + k];
 
-  // From here the QG warp groups run independently on interleaved QNT-row tiles,
-  // each with its own operand / result buffers and its own named barrier, so one
-  // group's tensor-core products overlap the other's per-row work.
-  const int grp = warp / GW, gw = warp % GW, gtid = tid % (GW * 32);
-  const MmaGroupSmem m = mma_group_carve(smem_raw, grp);
-  auto group_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GW * 32) : "memory"); };
-  // Bring the key and value rows of a tile towards L2 (one hint per 128-byte line).
-  const int es = p.dtype == TQ_F32 ? 4 : 2, lpr = QD * es / 128;
-  auto prefetch_tile = [&](int64_t t) {
-    if (t >= total_tiles) return;
-    const int pbh = (int)(t / tiles_per_bh);
-    const int64_t prow0 = (t % tiles_per_bh) * QNT;
-    for (int i = gtid; i < QNT * 2 * lpr; i += GW * 32) {
-      const int r = i / (2 * lpr), which = (i / lpr) & 1, ln = i % lpr;
-      if (prow0 + r >= p.n || (which && !p.do_values)) continue;
-      int64_t e0;
-      const void* src = src_row(p, which != 0, pbh, prow0 + r, e0);
-      prefetch_l2(reinterpret_cast<const char*>(src) + e0 * es + 128 * ln);
-    }
-  };
-  const int64_t t_step = (int64_t)QG * gridDim.x;
-  prefetch_tile((int64_t)QG * blockIdx.x + grp);
-  for (int64_t tile = (int64_t)QG * blockIdx.x + grp; tile < total_tiles; tile += t_step) {
+  // resident B operands: row n of Pi / T (output coordinate) over K = 128, a
+  // 16-byte chunk (8 consecutive k) per step, n fastest (conflict-free stores)
+  for (int c = tid; c < 2 * QD * (QD / 8); c += TC_THREADS) {
+    const int n = c % QD, kc = (c / QD) % (QD / 8), mat = c / (QD * (QD / 8));
+    const float* src = (mat ? p.T : p.Pi) + n * QD + 8 * kc;
+    const float4 f0 = *reinterpret_cast<const float4*>(src);
+    const float4 f1 = *reinterpret_cast<const float4*>(src + 4);
+    const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    uint4 hi, lo;
+    split8(v, kSplit, hi, lo);
+    const int off = tc::operand_off(n, 8 * kc);
+    *reinterpret_cast<uint4*>((mat ? TH : PH) + off) = hi;
+    *reinterpret_cast<uint4*>((mat ? TL : PL) + off) = lo;
+  }
+  float bnd[L - 1], cen[L];
+#pragma unroll
+  for (int k = 0; k < L; ++k) cen[k] = p.cent[k];
+#pragma unroll
+  for (int k = 0; k + 1 < L; ++k) bnd[k] = p.bnd[k];
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(&s_tmem), TC_COLS);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&s_mbar[0], 1);
+    mbar_init(&s_mbar[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_abort = 0;
+  }
+  tc::fence_async_shared();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  const uint32_t sAH = smem_u32(AH), sAL = smem_u32(AL);
+  const uint32_t sPH = smem_u32(PH), sPL = smem_u32(PL), sTH = smem_u32(TH), sTL = smem_u32(TL);
+
+  const int q = warp & 3, part = warp >> 2;
+  const int r = 32 * q + lane;                     // this thread's row of every tile
+  const int k0 = 32 * part;                        // and its first coordinate / channel
+  const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)k0;
+  const int es = p.dtype == TQ_F32 ? 4 : 2;
+  const int g = p.group, vb = p.vbits;
+  const uint32_t levels = (1u << vb) - 1u;
+  int issued = 0;                                  // thread 0: tiles whose products it issued
+  uint32_t it = 0;
+  for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
     const int bh = (int)(tile / tiles_per_bh);
-    const int64_t row0 = (tile % tiles_per_bh) * QNT;
-    prefetch_tile(tile + t_step);
-    // ---- keys: rho (float64), U = X / rho as fp16 hi/lo; a warp's rows are all
-    // loaded (4 consecutive elements a lane) before their reductions
+    const int64_t row0 = (tile % tiles_per_bh) * TCM;
+    const uint32_t ph = it & 1u;
+    const int64_t grow = row0 + r;
+    const bool valid = grow < p.n;
     {
-      float x[RPW][4];
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const int r = gw + i * GW;
-        if (row0 + r < p.n) {
+      // this thread's rows of the next tile towards L2
+      const int64_t nt = tile + gridDim.x;
+      if (nt < total_tiles) {
+        const int nbh = (int)(nt / tiles_per_bh);
+        const int64_t nrow = (nt % tiles_per_bh) * TCM + r;
+        if (nrow < p.n) {
           int64_t e0;
-          const void* src = src_row(p, false, bh, row0 + r, e0);
-          load4(src, e0 + 4 * lane, p.dtype, x[i]);
-        } else {
-          x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+          const void* src = src_row(p, false, nbh, nrow, e0);
+          prefetch_l2(reinterpret_cast<const char*>(src) + (e0 + k0) * es);
+          if (p.do_values) {
+            src = src_row(p, true, nbh, nrow, e0);
+            prefetch_l2(reinterpret_cast<const char*>(src) + (e0 + k0) * es);
+          }
         }
-      }
-      double ss[RPW];
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        ss[i] = 0.0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) ss[i] += (double)x[i][k] * (double)x[i][k];
-      }
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) ss[i] = warp_sum_d(ss[i]);
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const int r = gw + i * GW;
-        // rho = ss * rsqrt(ss) and 1/rho = rsqrt(ss): one float64 reciprocal square
-        // root instead of a square root and a division
-        const double rs = ss[i] > 0.0 ? rsqrt(ss[i]) : 0.0;
-        const double rho = ss[i] * rs;
-        const float inv = (float)rs;
-        if (lane == 0) {
-          m.rho64[r] = rho;
-          m.rho[r] = (float)rho;
-        }
-        // this lane's 4 consecutive elements: hi / lo as two f16x2 pairs each
-        float a[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) a[k] = x[i][k] * inv * kSplit;
-        const __half2 h01 = __floats2half2_rn(a[0], a[1]), h23 = __floats2half2_rn(a[2], a[3]);
-        const float2 b01 = __half22float2(h01), b23 = __half22float2(h23);
-        const __half2 l01 = __floats2half2_rn(a[0] - b01.x, a[1] - b01.y);
-        const __half2 l23 = __floats2half2_rn(a[2] - b23.x, a[3] - b23.y);
-        uint2 hv, lv;
-        hv.x = *reinterpret_cast<const uint32_t*>(&h01);
-        hv.y = *reinterpret_cast<const uint32_t*>(&h23);
-        lv.x = *reinterpret_cast<const uint32_t*>(&l01);
-        lv.y = *reinterpret_cast<const uint32_t*>(&l23);
-        *reinterpret_cast<uint2*>(m.AH + r * HS + 4 * lane) = hv;
-        *reinterpret_cast<uint2*>(m.AL + r * HS + 4 * lane) = lv;
       }
     }
-    group_sync();
-    mma_gemm_group<QNT / 16, 128 / 16 / GW>(m.AH, m.AL, s.PH, s.PL, m.YZ, gw);   // Y = U Pi^T
-    group_sync();
-    // ---- codes, residual E (fp16 hi/lo into A), ||r||: a warp's rows, lane =
-    // coordinate within each 32-coordinate chunk; the plane words of a row are
-    // collected by ballot and stored as one 16-byte write per plane
+    // ---- 1. rho and U = X / rho
+    float inv, rhof;
+    double rho64;
     {
-      double se[RPW];
+      float x[32];
+      int64_t e0 = 0;
+      const void* src = valid ? src_row(p, false, bh, grow, e0) : nullptr;
+      load32(src, e0 + k0, p.dtype, valid, x);
+      float s8[8];
 #pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const int r = gw + i * GW;
-        se[i] = 0.0;
-        uint32_t pw[B1][QD / 32];
+      for (int j = 0; j < 8; ++j) s8[j] = 0.f;
 #pragma unroll
-        for (int c = 0; c < QD / 32; ++c) {
-          const float y = m.YZ[r * YS + 32 * c + lane];
-          int idx = 0;
+      for (int j = 0; j < 32; ++j) s8[j & 7] = fmaf(x[j], x[j], s8[j & 7]);
+      double ss = 0.0;
 #pragma unroll
-          for (int k = 0; k + 1 < L; ++k) idx += (bnd[k] < y) ? 1 : 0;
-          const float e = y - s.cb[idx];
-          se[i] += (double)e * (double)e;
-          split_store(m.AH + r * HS + 32 * c + lane, m.AL + r * HS + 32 * c + lane, e);
+      for (int j = 0; j < 8; ++j) ss += (double)s8[j];
+      ssp[part * TCM + r] = ss;
+      tc::bar_sync(1, TC_THREADS);
+      ss = (ssp[r] + ssp[TCM + r]) + (ssp[2 * TCM + r] + ssp[3 * TCM + r]);
+      // rho = ss * rsqrt(ss) and 1/rho = rsqrt(ss) (float64)
+      const double rs = ss > 0.0 ? rsqrt(ss) : 0.0;
+      rho64 = ss * rs;
+      rhof = (float)rho64;
+      inv = (float)rs;
 #pragma unroll
-          for (int pl = 0; pl < B1; ++pl) pw[pl][c] = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
-        }
-        if (lane < B1 && row0 + r < p.n) {
-          uint4 v = make_uint4(pw[0][0], pw[0][1], pw[0][2], pw[0][3]);
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float v[8];
 #pragma unroll
-          for (int pl = 1; pl < B1; ++pl)
-            if (lane == pl) v = make_uint4(pw[pl][0], pw[pl][1], pw[pl][2], pw[pl][3]);
-          *reinterpret_cast<uint4*>(dst_field(p, bh, row0 + r, 0) + lane * (QD / 8)) = v;
+        for (int k = 0; k < 8; ++k) v[k] = x[8 * c8 + k] * inv;
+        uint4 hi, lo;
+        split8(v, kSplit, hi, lo);
+        const int off = tc::operand_off(r, k0 + 8 * c8);
+        *reinterpret_cast<uint4*>(AH + off) = hi;
+        *reinterpret_cast<uint4*>(AL + off) = lo;
+      }
+    }
+    tc::fence_async_shared();
+    tc::fence_before_sync();
+    tc::bar_sync(2, TC_THREADS);
+    if (tid == 0 && !*reinterpret_cast<volatile int*>(&s_abort)) {
+      tc::fence_after_sync();
+      tc_gemm(tmem, sAH, sAL, sPH, sPL);
+      tc::mma_commit(smem_u32(&s_mbar[0]));
+      ++issued;
+    }
+    // ---- 2. values of this thread's 32 channels, while Y = U Pi^T runs
+    if (p.do_values) {
+      float v[32];
+      int64_t e0 = 0;
+      const void* src = valid ? src_row(p, true, bh, grow, e0) : nullptr;
+      load32(src, e0 + k0, p.dtype, valid, v);
+      float mn[2], mx[2];                         // per 16-channel chunk
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        mn[c] = v[16 * c];
+        mx[c] = v[16 * c];
+#pragma unroll
+        for (int k = 1; k < 16; ++k) {
+          mn[c] = fminf(mn[c], v[16 * c + k]);
+          mx[c] = fmaxf(mx[c], v[16 * c + k]);
         }
       }
+      if (g >= 32) {                              // one group covers both chunks
+        mn[0] = mn[1] = fminf(mn[0], mn[1]);
+        mx[0] = mx[1] = fmaxf(mx[0], mx[1]);
+      }
+      if (g >= 64) {                              // and the parts of its group
+        vmm[part * TCM + r] = make_float2(mn[0], mx[0]);
+        tc::bar_sync(1, TC_THREADS);
+        const int np = g / 32, p0 = part & ~(np - 1);
+        float a = FLT_MAX, b = -FLT_MAX;
+        for (int j = 0; j < np; ++j) {
+          const float2 m2 = vmm[(p0 + j) * TCM + r];
+          a = fminf(a, m2.x);
+          b = fmaxf(b, m2.y);
+        }
+        mn[0] = mn[1] = a;
+        mx[0] = mx[1] = b;
+      }
+      if (valid) {
+        float sc[2], iv[2];
 #pragma unroll
-      for (int i = 0; i < RPW; ++i) se[i] = warp_sum_d(se[i]);
-      if (lane < RPW) {
-        // lane i writes row gw + GW i (a constant-index select, no dynamic register index)
-        double sv = se[0];
+        for (int c = 0; c < 2; ++c) {
+          sc[c] = __fdiv_rn(__fsub_rn(mx[c], mn[c]), (float)levels);
+          iv[c] = sc[c] != 0.f ? __frcp_rn(sc[c]) : 0.f;
+        }
+        // scales / minima: one store per group, by the thread holding its first channel
 #pragma unroll
-        for (int i = 1; i < RPW; ++i)
-          if (lane == i) sv = se[i];
-        const int r = gw + lane * GW;
-        if (row0 + r < p.n) {
-          *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 3)) = (float)(m.rho64[r] * sqrt(sv));
-          *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = m.rho[r];
+        for (int c = 0; c < 2; ++c) {
+          const int ch = k0 + 16 * c;
+          if (ch % g == 0) {
+            reinterpret_cast<float*>(dst_field(p, bh, grow, 5))[ch / g] = sc[c];
+            reinterpret_cast<float*>(dst_field(p, bh, grow, 6))[ch / g] = mn[c];
+          }
+        }
+        if (vb == 2) {
+          uint32_t hw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            hw[k >> 3] |= value_code_fast(v[k], mn[k >> 4], sc[k >> 4], iv[k >> 4], levels) << (2 * (k & 7));
+#pragma unroll
+          for (int x = 0; x < 4; ++x) *code_half_ptr(p, bh, grow, k0 / 8 + x) = (uint16_t)hw[x];
+        } else {
+          uint32_t hw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            hw[k >> 2] |= value_code_fast(v[k], mn[k >> 4], sc[k >> 4], iv[k >> 4], levels) << (4 * (k & 3));
+#pragma unroll
+          for (int x = 0; x < 8; ++x) *code_half_ptr(p, bh, grow, k0 / 4 + x) = (uint16_t)hw[x];
         }
       }
     }
-    group_sync();
-    mma_gemm_group<QNT / 16, 128 / 16 / GW>(m.AH, m.AL, s.TH, s.TL, m.YZ, gw);   // Z = E T^T
-    group_sync();
+    // ---- 3. codes, E, ||r||
+    bool ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait(&s_mbar[0], ph);
+    if (!ok) s_abort = 1;
+    tc::fence_after_sync();
+    uint32_t pw[B1];
+    {
+      uint32_t acc[32];
+      tc::tmem_ld32(trow, acc);
+      tc::tmem_wait_ld();
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-      const int r = gw + i * GW;
-      const float rho = m.rho[r];
-      uint32_t sw[QM / 32];
+      for (int pl = 0; pl < B1; ++pl) pw[pl] = 0u;
+      float e[32], s8[8];
 #pragma unroll
-      for (int c = 0; c < QM / 32; ++c) sw[c] = __ballot_sync(0xffffffffu, m.YZ[r * YS + 32 * c + lane] * rho >= 0.f);
-      if (lane == 0 && row0 + r < p.n)
-        *reinterpret_cast<uint4*>(dst_field(p, bh, row0 + r, 1)) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+      for (int j = 0; j < 8; ++j) s8[j] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float y = __uint_as_float(acc[c]) * (1.f / (kSplit * kSplit));
+        int idx = 0;
+        float cv = cen[0];
+#pragma unroll
+        for (int k = 0; k + 1 < L; ++k)
+          if (bnd[k] < y) {
+            idx = k + 1;
+            cv = cen[k + 1];
+          }
+#pragma unroll
+        for (int pl = 0; pl < B1; ++pl) pw[pl] |= (uint32_t)((idx >> pl) & 1) << c;
+        e[c] = y - cv;
+        s8[c & 7] = fmaf(e[c], e[c], s8[c & 7]);
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = e[8 * c8 + k];
+        uint4 hi, lo;
+        split8(v, kSplit, hi, lo);
+        const int off = tc::operand_off(r, k0 + 8 * c8);
+        *reinterpret_cast<uint4*>(AH + off) = hi;
+        *reinterpret_cast<uint4*>(AL + off) = lo;
+      }
+      double se = 0.0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) se += (double)s8[j];
+      sep[part * TCM + r] = se;
     }
-    // ---- values, straight from the source rows
-    if (p.do_values) quantize_values_rows(p, bh, row0, QNT, gw, lane, GW);
-    group_sync();
+    tc::fence_async_shared();
+    tc::fence_before_sync();
+    tc::bar_sync(3, TC_THREADS);
+    if (tid == 0 && !*reinterpret_cast<volatile int*>(&s_abort)) {
+      tc::fence_after_sync();
+      tc_gemm(tmem, sAH, sAL, sTH, sTL);
+      tc::mma_commit(smem_u32(&s_mbar[1]));
+    }
+    const bool write = valid && ok;
+    if (write) {
+      uint8_t* ip = dst_field(p, bh, grow, 0);
+#pragma unroll
+      for (int pl = 0; pl < B1; ++pl) *reinterpret_cast<uint32_t*>(ip + pl * (QD / 8) + 4 * part) = pw[pl];
+      if (part == 0) {
+        const double sev = (sep[r] + sep[TCM + r]) + (sep[2 * TCM + r] + sep[3 * TCM + r]);
+        *reinterpret_cast<float*>(dst_field(p, bh, grow, 3)) = (float)(rho64 * sqrt(sev));
+        *reinterpret_cast<float*>(dst_field(p, bh, grow, 2)) = rhof;
+      }
+    }
+    // ---- 4. sign bits of z = rho Z
+    ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait(&s_mbar[1], ph);
+    if (!ok) s_abort = 1;
+    tc::fence_after_sync();
+    {
+      uint32_t acc[32];
+      tc::tmem_ld32(trow, acc);
+      tc::tmem_wait_ld();
+      uint32_t w = 0u;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) w |= (uint32_t)(__uint_as_float(acc[c]) * rhof >= 0.f) << c;
+      if (valid && ok) *reinterpret_cast<uint32_t*>(dst_field(p, bh, grow, 1) + 4 * part) = w;
+    }
+    tc::fence_before_sync();
+    tc::bar_sync(4, TC_THREADS);
+    if (*reinterpret_cast<volatile int*>(&s_abort)) break;
+  }
+  if (warp == 0) {
+    if (*reinterpret_cast<volatile int*>(&s_abort)) {
+      // a wait gave up: let the last products finish (bounded) before freeing
+      if (lane == 0) {
+        atomicExch(&g_quant_tc_err, 1);
+        if (issued > 0) {
+          (void)mbar_wait(&s_mbar[0], (uint32_t)((issued - 1) & 1));
+          (void)mbar_wait(&s_mbar[1], (uint32_t)((issued - 1) & 1));
+        }
+      }
+      __syncwarp();
+    }
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, TC_COLS);
   }
 }
-
 }  // namespace
 
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
-  if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0) {
-    // tensor-core tiles: one persistent CTA per SM, QG warp groups over all
-    // QNT-token tiles
-    const int64_t tiles_per_bh = (p.n + QNT - 1) / QNT;
+  if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0 && p.b1 <= 3) {
+    // fifth-generation tensor cores: one persistent CTA per SM over 128-token tiles
+    const int64_t tiles_per_bh = (p.n + TCM - 1) / TCM;
     const int64_t total = tiles_per_bh * bh_count;
     int sms = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = mma_smem_bytes();
-    auto kern = p.b1 == 1 ? k_quantize_mma<1> : p.b1 == 2 ? k_quantize_mma<2> : k_quantize_mma<3>;
+    const size_t smem = tc_smem_bytes();
+    auto kern = p.b1 == 1 ? k_quantize_tc<1> : p.b1 == 2 ? k_quantize_tc<2> : k_quantize_tc<3>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t want = (total + QG - 1) / QG;
-    const int64_t grid = want < sms ? want : sms;
-    kern<<<(unsigned)grid, QTHREADS, smem, s>>>(p, tiles_per_bh, total);
+    const int64_t grid = total < sms ? total : sms;
+    kern<<<(unsigned)grid, TC_THREADS, smem, s>>>(p, tiles_per_bh, total);
     return cudaGetLastError();
   }
   if (p.n <= 8) {
@@ -1016,6 +1073,16 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   dim3 grid((unsigned)((p.n + NT - 1) / NT), (unsigned)bh_count);
   k_quantize<<<grid, THREADS, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t quantize_error_flag(int* flag, cudaStream_t s) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(flag, g_quant_tc_err, sizeof(int), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_quant_tc_err, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return e;
 }
 
 cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1, int m,

@@ -52,6 +52,9 @@ struct QuantDst {  // token-major arrays (standalone calls)
   float* vscale;
   float* vmin;
 };
+// Read and clear the sticky flag the tensor-core quantise kernel raises when a
+// bounded wait gives up (synchronises `s`).
+cudaError_t quantize_error_flag(int* flag, cudaStream_t s);
 cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1, int m,
                                    int vbits, int group, bool do_keys, bool do_values,
                                    const float* Pi, const float* T, const float* cent,

@@ -82,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "tq_decode_attention_noalloc": (I, [C, P, I, F, P, P, P, P, P, I, P]),
         "tq_decode_prep": (I, [C, P, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_check": (I, [C, I, I, P, SZ, P]),
+        "tq_quantize_check": (I, [P]),
         "tq_decode_partial": (I, [C, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
         "tq_decode_step": (I, [C, P, P, I64, P, I, F, P, P, P, P, P, P, P, I, P, SZ, P]),
@@ -217,6 +218,12 @@ def tq_decode_prep(cache: tq_cache, Q, softmax_scale, Pi, S, centroids, num_spli
     _check(lib.tq_decode_prep(ctypes.byref(cache), _ptr(Q), Q.shape[1], softmax_scale, _ptr(Pi),
                               _ptr(S), _ptr(centroids), num_splits, _ptr(workspace),
                               _ws(workspace), _stream(stream)), "tq_decode_prep")
+
+
+def tq_quantize_check(stream=None):
+    """Raise if the batched tensor-core key quantisation gave up a bounded wait
+    since the last check (waits for the stream; clears the flag)."""
+    _check(lib.tq_quantize_check(_stream(stream)), "tq_quantize_check")
 
 
 def tq_decode_check(cache: tq_cache, Hq, num_splits, workspace, stream=None):

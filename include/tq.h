@@ -320,6 +320,18 @@ int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* works
                     size_t ws_bytes, void* stream);
 
 /*
+ * tq_quantize_check -- SYNCHRONOUS: waits for `stream`, then reports (and
+ * clears) the sticky device flag of the batched tensor-core key quantisation
+ * (tq_quantize_keys and tq_append with more than 8 tokens, head dim 128,
+ * m = 128, b1 >= 1).  That kernel waits, with a bound, for its tensor-core
+ * products to complete; if a wait gives up (it never should) it stops and sets
+ * the flag instead of hanging.  Returns TQ_ERR_CUDA when the flag was set,
+ * TQ_OK otherwise.  The pages have no counterpart: this is a diagnostic of this
+ * library.
+ */
+int tq_quantize_check(void* stream);
+
+/*
  * tq_decode_attention_noalloc -- the same decode as tq_decode_attention, for
  * callers that cannot allocate device memory or pass a workspace (for example
  * an inference-engine plugin whose host framework owns all device memory and

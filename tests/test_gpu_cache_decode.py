@@ -124,6 +124,7 @@ def test_append_degenerate_tokens_every_quantise_path():
         oc.append(host(k), host(v))
         t += n
     torch.cuda.synchronize()
+    nat().tq_quantize_check()
     assert gc.n_total == oc.n_total == w.T
     buf = gc.buffer.cpu().numpy()
     _compare_cache_bytes(buf, oc)

@@ -89,6 +89,28 @@ def test_quantize_keys_given_oracle_projections(d, b1, m, dt, n):
     assert stats["skipped_tokens"] <= max(2, n // 200)
 
 
+@pytest.mark.parametrize("b1", [1, 2, 3])
+@pytest.mark.parametrize("n,dt", [(9, "bf16"), (127, "f32"), (128, "bf16"), (129, "f16"),
+                                  (1000, "bf16")])
+def test_quantize_keys_tensor_core_tiles(b1, n, dt):
+    """The batched tensor-core path (d = m = 128, more than 8 keys) at tile edges:
+    one partial 128-row tile, exactly one tile, one row into a second tile, many
+    tiles over the persistent grid; codes, signs and norms against the oracle, and
+    the kernel's wait flag clear."""
+    d, m = 128, 128
+    w = synth.Workload("t", B=1, Hq=1, Hkv=1, d=d, T=n, W=0, b1=b1, m=m, vbits=2, group=32,
+                       dtype=dt, seed=11 + b1, k_outlier_count=3, outlier_scale=8.0,
+                       lognormal_sigma=0.5)
+    K, _ = synth.keys_values(w, device="cuda")
+    K = K[0, 0].contiguous()
+    po, (c32, b32) = oracle_setup(d, b1, m)
+    got = _keys_gpu(K, b1, m, to_dev(po["Pi"]), to_dev(po["T"]), to_dev(c32), to_dev(b32))
+    nat().tq_quantize_check()
+    ref = oq.quantize_keys(host(K), po["Pi"], po["S"], c32, b32, b1)
+    stats = compare_keys(got, ref, d, b1, m, b32)
+    assert stats["skipped_tokens"] <= max(2, n // 200)
+
+
 def test_quantize_keys_end_to_end_projections_and_zero_key():
     """Library-made Pi/T/codebook; a zero key and a key equal to its codebook point."""
     from compressed_attention_turboquantprod_b200 import Codebook, Projections
