@@ -126,6 +126,21 @@ __device__ __forceinline__ uint16_t* code_half_ptr(const QParams& p, int bh, int
   return reinterpret_cast<uint16_t*>(p.arr.codes + (p.t_first + i) * (p.d * p.vbits / 8)) + x;
 }
 
+// Base of row i's value codes and the byte offset of its 16-bit half x from that
+// base (code_half_ptr(p, bh, i, x) == code_base(p, bh, i) + code_half_off(p, x)).
+__device__ __forceinline__ uint8_t* code_base(const QParams& p, int bh, int64_t i) {
+  if (p.cache_mode) {
+    const Geom& g = p.g;
+    const int64_t t = p.t_first + i;
+    uint8_t* blk = p.base + (int64_t)bh * g.region_bytes + (t / kBlockTokens) * g.block_bytes;
+    return blk + g.o_vcode + vcode_half_off(g, (int)(t % kBlockTokens), 0);
+  }
+  return p.arr.codes + (p.t_first + i) * (p.d * p.vbits / 8);
+}
+__device__ __forceinline__ int code_half_off(const QParams& p, int x) {
+  return p.cache_mode ? vcode_half_off(p.g, 0, x) : 2 * x;
+}
+
 __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t i, int which) {
   // which: 0 idx, 1 sign, 2 rho, 3 rnorm, 5 vscale, 6 vmin (value codes: code_half_ptr)
   if (p.cache_mode) {
@@ -680,34 +695,36 @@ __device__ __forceinline__ void split8(const float (&v)[8], float scale, uint4& 
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-// 32 consecutive elements of a row as fp32 (16-byte loads); zeros when !valid.
-__device__ __forceinline__ void load32(const void* base, int64_t e, int dtype, bool valid, float (&o)[32]) {
-  if (!valid) {
+// The 32 elements of a row segment as raw 16-byte words (issued early, converted
+// later): 4 words for 16-bit types, 8 for fp32.  Zeros when !valid.
+template <bool F32>
+struct RawSeg {
+  uint4 w[F32 ? 8 : 4];
+};
+template <bool F32>
+__device__ __forceinline__ void raw_load(RawSeg<F32>& r, const void* base, int64_t e, bool valid) {
+  const uint4* src = valid ? reinterpret_cast<const uint4*>(static_cast<const char*>(base) +
+                                                            e * (F32 ? 4 : 2))
+                           : nullptr;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) o[j] = 0.f;
-    return;
-  }
-  if (dtype == TQ_F32) {
-    const float4* p4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + e);
+  for (int i = 0; i < (F32 ? 8 : 4); ++i) r.w[i] = valid ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+}
+template <bool F32>
+__device__ __forceinline__ void raw_to_float(const RawSeg<F32>& r, int dtype, float (&o)[32]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 v = p4[j];
-      o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
-    }
-    return;
-  }
-  const uint4* p4 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + e);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 u = p4[j];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int i = 0; i < (F32 ? 8 : 4); ++i) {
+    const uint32_t w[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      float2 f;
-      if (dtype == TQ_F16) f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-      else f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
-      o[8 * j + 2 * k] = f.x;
-      o[8 * j + 2 * k + 1] = f.y;
+      if constexpr (F32) {
+        o[4 * i + k] = __uint_as_float(w[k]);
+      } else {
+        float2 f;
+        if (dtype == TQ_F16) f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        else f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+        o[8 * i + 2 * k] = f.x;
+        o[8 * i + 2 * k + 1] = f.y;
+      }
     }
   }
 }
@@ -726,6 +743,19 @@ __device__ __forceinline__ uint32_t value_code_fast(float v, float mn, float sc,
   return c < levels ? c : levels;
 }
 
+// The same code without the rare exact-division branch: `tie` is set when the
+// product lies within 1e-5 of a half-integer, and the caller recomputes those
+// elements with value_code_fast.
+__device__ __forceinline__ uint32_t value_code_nb(float v, float mn, float inv, uint32_t levels, bool& tie) {
+  const float a = __fsub_rn(v, mn);
+  const float x = __fmul_rn(a, inv);
+  const float t = __fadd_rn(x, kRound);
+  const float rr = __fsub_rn(t, kRound);
+  tie = fabsf(fabsf(__fsub_rn(x, rr)) - 0.5f) < 1e-5f;
+  const uint32_t c = __float_as_uint(t) - __float_as_uint(kRound);
+  return c < levels ? c : levels;
+}
+
 // The issuing thread: D = A B^T over K = 128 as three products per k-step.
 __device__ __forceinline__ void tc_gemm(uint32_t d_tmem, uint32_t ah, uint32_t al, uint32_t bh,
                                         uint32_t bl) {
@@ -739,16 +769,18 @@ __device__ __forceinline__ void tc_gemm(uint32_t d_tmem, uint32_t ah, uint32_t a
   }
 }
 
-template <int B1>
+template <int B1, bool F32>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_t tiles_per_bh,
                                                               int64_t total_tiles) {
   using mmadec::mbar_init;
   using mmadec::mbar_wait;
+  using mmadec::mbar_wait_sleep;
   using mmadec::smem_u32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t s_mbar[2];      // Y done, Z done
+  __shared__ __align__(8) uint64_t s_mbar[3];      // Y done, Z done, operand staged
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_hofs[TC_PARTS][8];               // value-code half offsets of each part
   unsigned char* PH = smem_raw;
   unsigned char* PL = PH + TC_OPB;
   unsigned char* TH = PL + TC_OPB;
@@ -761,19 +793,70 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int L = 1 << B1;
 
-  // resident B operands: row n of Pi / T (output coordinate) over K = 128, a
-  // 16-byte chunk (8 consecutive k) per step, n fastest (conflict-free stores)
-  for (int c = tid; c < 2 * QD * (QD / 8); c += TC_THREADS) {
-    const int n = c % QD, kc = (c / QD) % (QD / 8), mat = c / (QD * (QD / 8));
-    const float* src = (mat ? p.T : p.Pi) + n * QD + 8 * kc;
-    const float4 f0 = *reinterpret_cast<const float4*>(src);
-    const float4 f1 = *reinterpret_cast<const float4*>(src + 4);
-    const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    uint4 hi, lo;
-    split8(v, kSplit, hi, lo);
-    const int off = tc::operand_off(n, 8 * kc);
-    *reinterpret_cast<uint4*>((mat ? TH : PH) + off) = hi;
-    *reinterpret_cast<uint4*>((mat ? TL : PL) + off) = lo;
+  if (tid == 0) {
+    mbar_init(&s_mbar[0], 1);
+    mbar_init(&s_mbar[1], 1);
+    mbar_init(&s_mbar[2], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_abort = 0;
+  }
+  __syncthreads();
+  // resident B operands: Pi, then T, brought in fp32 by bulk copies into the (not
+  // yet used) A area at a 528-byte row stride (eight consecutive rows fall in
+  // distinct bank groups), then split there into f16 hi/lo in the operand layout:
+  // row n (output coordinate) over K = 128, a 16-byte chunk (8 consecutive k) per
+  // thread and step, eight consecutive rows per eight threads (conflict-free)
+  const int q = warp & 3, part = warp >> 2;
+  const int r = 32 * q + lane;                     // this thread's row of every tile
+  const int k0 = 32 * part;                        // and its first coordinate / channel
+  const int es = p.dtype == TQ_F32 ? 4 : 2;
+  const int g = p.group, vb = p.vbits;
+  const uint32_t levels = (1u << vb) - 1u;
+  // each part's value-code halves: byte offsets from a row's code base
+  if (tid < TC_PARTS * 8) s_hofs[tid >> 3][tid & 7] = code_half_off(p, (32 * (tid >> 3)) * vb / 16 + (tid & 7));
+  // this thread's key and value segments of a tile, requested one tile ahead (the
+  // first before the operand staging, so that its latency overlaps the staging)
+  RawSeg<F32> xr, vr;
+  auto request = [&](int64_t t) {
+    bool ok_row = false;
+    const void* ks = nullptr;
+    const void* vs = nullptr;
+    int64_t ek = 0, ev = 0;
+    if (t < total_tiles) {
+      const int tbh = (int)(t / tiles_per_bh);
+      const int64_t trow_i = (t % tiles_per_bh) * TCM + r;
+      ok_row = trow_i < p.n;
+      if (ok_row) {
+        ks = src_row(p, false, tbh, trow_i, ek);
+        if (p.do_values) vs = src_row(p, true, tbh, trow_i, ev);
+      }
+    }
+    raw_load(xr, ks, ek + k0, ok_row);
+    raw_load(vr, vs, ev + k0, ok_row && p.do_values);
+  };
+  request(blockIdx.x);
+
+  constexpr int kStage = QD * 4 + 16;
+  for (int mat = 0; mat < 2; ++mat) {
+    if (tid == 0) mmadec::mbar_expect_tx(&s_mbar[2], QD * QD * 4);
+    __syncthreads();
+    if (tid < QD) {                                  // one row copy per thread
+      tc::fence_async_shared();                      // the area's earlier reads come first
+      mmadec::bulk_load(AH + tid * kStage, (mat ? p.T : p.Pi) + tid * QD, QD * 4, &s_mbar[2]);
+    }
+    if (!mbar_wait_sleep(&s_mbar[2], (uint32_t)mat)) s_abort = 1;
+    for (int c = tid; c < QD * (QD / 8); c += TC_THREADS) {
+      const int n = (c & 7) + 8 * (c >> 7), kc = (c >> 3) & 15;
+      const float4 f0 = *reinterpret_cast<const float4*>(AH + n * kStage + 32 * kc);
+      const float4 f1 = *reinterpret_cast<const float4*>(AH + n * kStage + 32 * kc + 16);
+      const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+      uint4 hi, lo;
+      split8(v, kSplit, hi, lo);
+      const int off = tc::operand_off(n, 8 * kc);
+      *reinterpret_cast<uint4*>((mat ? TH : PH) + off) = hi;
+      *reinterpret_cast<uint4*>((mat ? TL : PL) + off) = lo;
+    }
+    __syncthreads();
   }
   float bnd[L - 1], cen[L];
 #pragma unroll
@@ -784,12 +867,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     tc::tmem_alloc(smem_u32(&s_tmem), TC_COLS);
     tc::tmem_relinquish();
   }
-  if (tid == 0) {
-    mbar_init(&s_mbar[0], 1);
-    mbar_init(&s_mbar[1], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_abort = 0;
-  }
   tc::fence_async_shared();
   tc::fence_before_sync();
   __syncthreads();
@@ -798,25 +875,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
   const uint32_t sAH = smem_u32(AH), sAL = smem_u32(AL);
   const uint32_t sPH = smem_u32(PH), sPL = smem_u32(PL), sTH = smem_u32(TH), sTL = smem_u32(TL);
 
-  const int q = warp & 3, part = warp >> 2;
-  const int r = 32 * q + lane;                     // this thread's row of every tile
-  const int k0 = 32 * part;                        // and its first coordinate / channel
   const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)k0;
-  const int es = p.dtype == TQ_F32 ? 4 : 2;
-  const int g = p.group, vb = p.vbits;
-  const uint32_t levels = (1u << vb) - 1u;
   int issued = 0;                                  // thread 0: tiles whose products it issued
   uint32_t it = 0;
-  for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+  const int64_t tiles_here = *reinterpret_cast<volatile int*>(&s_abort) ? 0 : total_tiles;
+  for (int64_t tile = blockIdx.x; tile < tiles_here; tile += gridDim.x, ++it) {
     const int bh = (int)(tile / tiles_per_bh);
     const int64_t row0 = (tile % tiles_per_bh) * TCM;
     const uint32_t ph = it & 1u;
     const int64_t grow = row0 + r;
     const bool valid = grow < p.n;
     {
-      // this thread's rows of the next tile towards L2
-      const int64_t nt = tile + gridDim.x;
-      if (nt < total_tiles) {
+      // the rows of the tile after next towards L2
+      const int64_t nt = tile + 2 * (int64_t)gridDim.x;
+      if (nt < tiles_here) {
         const int nbh = (int)(nt / tiles_per_bh);
         const int64_t nrow = (nt % tiles_per_bh) * TCM + r;
         if (nrow < p.n) {
@@ -835,9 +907,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     double rho64;
     {
       float x[32];
-      int64_t e0 = 0;
-      const void* src = valid ? src_row(p, false, bh, grow, e0) : nullptr;
-      load32(src, e0 + k0, p.dtype, valid, x);
+      raw_to_float(xr, p.dtype, x);
       float s8[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) s8[j] = 0.f;
@@ -878,9 +948,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     // ---- 2. values of this thread's 32 channels, while Y = U Pi^T runs
     if (p.do_values) {
       float v[32];
-      int64_t e0 = 0;
-      const void* src = valid ? src_row(p, true, bh, grow, e0) : nullptr;
-      load32(src, e0 + k0, p.dtype, valid, v);
+      raw_to_float(vr, p.dtype, v);
       float mn[2], mx[2];                         // per 16-channel chunk
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -911,39 +979,59 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       }
       if (valid) {
         float sc[2], iv[2];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          sc[c] = __fdiv_rn(__fsub_rn(mx[c], mn[c]), (float)levels);
-          iv[c] = sc[c] != 0.f ? __frcp_rn(sc[c]) : 0.f;
+        sc[0] = __fdiv_rn(__fsub_rn(mx[0], mn[0]), (float)levels);
+        iv[0] = sc[0] != 0.f ? __frcp_rn(sc[0]) : 0.f;
+        if (g >= 32) {
+          sc[1] = sc[0];
+          iv[1] = iv[0];
+        } else {
+          sc[1] = __fdiv_rn(__fsub_rn(mx[1], mn[1]), (float)levels);
+          iv[1] = sc[1] != 0.f ? __frcp_rn(sc[1]) : 0.f;
         }
         // scales / minima: one store per group, by the thread holding its first channel
+        float* vsp = reinterpret_cast<float*>(dst_field(p, bh, grow, 5));
+        float* vmp = reinterpret_cast<float*>(dst_field(p, bh, grow, 6));
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int ch = k0 + 16 * c;
           if (ch % g == 0) {
-            reinterpret_cast<float*>(dst_field(p, bh, grow, 5))[ch / g] = sc[c];
-            reinterpret_cast<float*>(dst_field(p, bh, grow, 6))[ch / g] = mn[c];
+            vsp[ch / g] = sc[c];
+            vmp[ch / g] = mn[c];
           }
         }
-        if (vb == 2) {
-          uint32_t hw[4] = {0u, 0u, 0u, 0u};
+        uint8_t* cb = code_base(p, bh, grow);
+        // codes of the 32 channels packed as they come (a zero scale has inv = 0, so
+        // x = 0 and code 0); near a half-integer (rare) all are redone with the
+        // exact division where needed
+        const int cpw = 16 / vb;                     // codes per 16-bit half
+        uint32_t hw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        bool any_tie = false;
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            hw[k >> 3] |= value_code_fast(v[k], mn[k >> 4], sc[k >> 4], iv[k >> 4], levels) << (2 * (k & 7));
-#pragma unroll
-          for (int x = 0; x < 4; ++x) *code_half_ptr(p, bh, grow, k0 / 8 + x) = (uint16_t)hw[x];
-        } else {
-          uint32_t hw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            hw[k >> 2] |= value_code_fast(v[k], mn[k >> 4], sc[k >> 4], iv[k >> 4], levels) << (4 * (k & 3));
-#pragma unroll
-          for (int x = 0; x < 8; ++x) *code_half_ptr(p, bh, grow, k0 / 4 + x) = (uint16_t)hw[x];
+        for (int k = 0; k < 32; ++k) {
+          bool tie;
+          const uint32_t c = value_code_nb(v[k], mn[k >> 4], iv[k >> 4], levels, tie);
+          any_tie |= tie && sc[k >> 4] != 0.f;
+          if (vb == 2) hw[k >> 3] += c << (2 * (k & 7));
+          else hw[k >> 2] += c << (4 * (k & 3));
         }
+        if (any_tie) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) hw[j] = 0u;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const uint32_t c = value_code_fast(v[k], mn[k >> 4], sc[k >> 4], iv[k >> 4], levels);
+            if (vb == 2) hw[k >> 3] += c << (2 * (k & 7));
+            else hw[k >> 2] += c << (4 * (k & 3));
+          }
+        }
+        const int nh = 32 / cpw;
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          if (x < nh) *reinterpret_cast<uint16_t*>(cb + s_hofs[part][x]) = (uint16_t)hw[x];
       }
     }
     // ---- 3. codes, E, ||r||
-    bool ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait(&s_mbar[0], ph);
+    bool ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait_sleep(&s_mbar[0], ph);
     if (!ok) s_abort = 1;
     tc::fence_after_sync();
     uint32_t pw[B1];
@@ -996,6 +1084,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       tc_gemm(tmem, sAH, sAL, sTH, sTL);
       tc::mma_commit(smem_u32(&s_mbar[1]));
     }
+    request(tile + gridDim.x);                     // the next tile's, in flight from here
     const bool write = valid && ok;
     if (write) {
       uint8_t* ip = dst_field(p, bh, grow, 0);
@@ -1008,7 +1097,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       }
     }
     // ---- 4. sign bits of z = rho Z
-    ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait(&s_mbar[1], ph);
+    ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait_sleep(&s_mbar[1], ph);
     if (!ok) s_abort = 1;
     tc::fence_after_sync();
     {
@@ -1029,6 +1118,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       // a wait gave up: let the last products finish (bounded) before freeing
       if (lane == 0) {
         atomicExch(&g_quant_tc_err, 1);
+        (void)mbar_wait(&s_mbar[2], 0u);           // the operand copies, if still in flight
+        (void)mbar_wait(&s_mbar[2], 1u);
         if (issued > 0) {
           (void)mbar_wait(&s_mbar[0], (uint32_t)((issued - 1) & 1));
           (void)mbar_wait(&s_mbar[1], (uint32_t)((issued - 1) & 1));
@@ -1052,7 +1143,10 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = tc_smem_bytes();
-    auto kern = p.b1 == 1 ? k_quantize_tc<1> : p.b1 == 2 ? k_quantize_tc<2> : k_quantize_tc<3>;
+    const bool f32 = p.dtype == TQ_F32;
+    auto kern = p.b1 == 1 ? (f32 ? k_quantize_tc<1, true> : k_quantize_tc<1, false>)
+              : p.b1 == 2 ? (f32 ? k_quantize_tc<2, true> : k_quantize_tc<2, false>)
+                          : (f32 ? k_quantize_tc<3, true> : k_quantize_tc<3, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = total < sms ? total : sms;
