@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256) k_prep_mma(Geom g, const void* Q, int Hq,
                                                   float scale_log2, DecodeWs ws) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   pdl_launch_dependents();   // the partial kernel may launch; it waits for this grid
-  prep_mma_body<NV>(g, Q, Hq, Pi, S, cent, scale_log2, ws, blockIdx.x, smem_raw);
+  prep_mma_body<NV>(g, Q, Hq, Pi, S, cent, scale_log2, ws, blockIdx.x >> 1, blockIdx.x & 1, smem_raw);
 }
 
 // ---------------------------------------------------------------- partial
@@ -588,7 +588,7 @@ cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const f
   auto kern = g.d == 256 ? k_prep_mma<2> : k_prep_mma<1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws);
+  kern<<<2 * g.B * g.Hkv, 256, smem, s>>>(g, Q, Hq, Pi, S, cent, scale * kLog2e, ws);   // 2 halves a unit
   return cudaGetLastError();
 }
 

@@ -12,61 +12,69 @@ namespace mmadec {
 __host__ __device__ inline size_t prep_smem_bytes(int d, int m) { return sizeof(float) * MG * (2 * d + m); }
 
 // ---------------------------------------------------------------- prep
-// One CTA per (b, KV head), for its G = 4 queries:
+// For the G = 4 queries of one (b, KV head):
 //  * qf = q in fp32 (for the ring), qr = Pi q, qs = sqrt(pi/2)/m S q, each row of
 //    [Pi; S] read once (a float4 per lane) and dotted with the four queries;
 //  * the Walsh weights of the codebook, the 24-bit fixed-point quantisation of
 //    the query weights and their four int8 slices laid out as the lanes' B
 //    fragments, and the per-head affine constants of the logit (log2 units);
-//  * zeroes the unit's split counter and, in CTA 0, the error flag.
+//  * zeroes the unit's split counter and, in unit 0, the error flag.
+// The MSE half (rows of Pi, the plane fragments, constants kM / CM, qf and the
+// counters) and the QJL half (rows of S, the sign fragments, kQ / CQ) need
+// nothing from each other: part 0 does the first, part 1 the second, part 2
+// both (one CTA of 256 threads per (unit, part)).
 template <int NV>     // float4s of a row per lane: head dim 128 * NV
 __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int Hq, const float* Pi,
                                               const float* S, const float* cent, float scale_log2,
-                                              const DecodeWs& ws, int unit,
+                                              const DecodeWs& ws, int unit, int part,
                                               unsigned char* smem_raw) {
   const int b = unit / g.Hkv, h = unit % g.Hkv;
   const int d = g.d, m = g.m, b1 = g.b1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool do_mse = part != 1, do_qjl = part != 0;
   float* sq = reinterpret_cast<float*>(smem_raw);     // [G][d]
   float* sqr = sq + MG * d;                           // [G][d]
   float* sqs = sqr + MG * d;                          // [G][m]
   __shared__ float s_w[4];                            // Walsh weights of the odd subsets
+  __shared__ float s_cent[8];
   __shared__ unsigned s_maxM[MG], s_maxQ[MG];
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
+  const int rows_pi = b1 > 0 ? d : 0;
+  // this part's rows of [Pi; S]: [r_begin, r_end)
+  const int r_begin = do_mse ? 0 : rows_pi, r_end = do_qjl ? rows_pi + m : rows_pi;
   {
-    // the rows of [Pi; S] are read after the queries: start them towards L2 now
-    const int lines_pi = b1 > 0 ? d * d / 32 : 0, lines = lines_pi + m * d / 32;
-    for (int i = tid; i < lines; i += blockDim.x)
+    // the rows are read after the queries: start them towards L2 now
+    const int l0 = r_begin * d / 32, l1 = r_end * d / 32, lines_pi = rows_pi * d / 32;
+    for (int i = l0 + tid; i < l1; i += blockDim.x)
       prefetch_l2(i < lines_pi ? Pi + 32 * (int64_t)i : S + 32 * (int64_t)(i - lines_pi));
   }
-  if (tid == 0) {
+  if (tid == 0 && do_mse) {
     ws.counter[unit] = 0;
     if (unit == 0) *ws.err = 0;
   }
+  // the codebook and the queries are requested together
+  const int L = b1 > 0 ? 1 << b1 : 0;
+  if (tid < 8) s_cent[tid] = tid < L ? cent[tid] : 0.f;
   for (int i = tid; i < MG * d; i += blockDim.x) {
     const float v = load_f(Q, (int64_t)bq0 * d + i, g.dtype);
     sq[i] = v;
-    ws.qf[(int64_t)bq0 * d + i] = v;
-  }
-  if (tid == 0) {
-    // w_S = (1/L) sum_idx c[idx] (-1)^{popc(idx & S)} for the odd subsets S, in the
-    // order of the feature planes: {0}, {1}, {2}, {0,1,2}.
-    const int L = b1 > 0 ? 1 << b1 : 0;
-    const int subsets[4] = {1, 2, 4, 7};
-    for (int k = 0; k < 4; ++k) {
-      double acc = 0.0;
-      for (int idx = 0; idx < L; ++idx)
-        acc += (double)cent[idx] * ((__popc(idx & subsets[k]) & 1) ? -1.0 : 1.0);
-      s_w[k] = L ? (float)(acc / L) : 0.f;
-    }
+    if (do_mse) ws.qf[(int64_t)bq0 * d + i] = v;
   }
   __syncthreads();
-  const int rows_pi = b1 > 0 ? d : 0;
+  if (tid < 4) {
+    // w_S = (1/L) sum_idx c[idx] (-1)^{popc(idx & S)} for the odd subsets S, in the
+    // order of the feature planes: {0}, {1}, {2}, {0,1,2} (thread k: subset k).
+    const int subset = tid < 3 ? 1 << tid : 7;
+    double acc = 0.0;
+    for (int idx = 0; idx < L; ++idx)
+      acc += (double)s_cent[idx] * ((__popc(idx & subset) & 1) ? -1.0 : 1.0);
+    s_w[tid] = L ? (float)(acc / L) : 0.f;
+  }
   const float qscale = 1.2533141373155003f / (float)m;
-  // Rows of [Pi; S] in passes of 8 per warp: lane l dots float4 l of each row
-  // (coalesced) with columns 4l..4l+3 of the four queries (held in registers);
-  // a reduce-scatter over the warp then leaves the sum of (row l/4, head l%4) in
+  // Rows in passes of 8 per warp: lane l dots float4 l of each row (coalesced)
+  // with columns 4l..4l+3 of the four queries (held in registers); a
+  // reduce-scatter over the warp then leaves the sum of (row l/4, head l%4) in
   // lane l.  (NV float4s per lane per row: columns 128 c + 4 lane.)
   float4 qv[MG][NV];
 #pragma unroll
@@ -74,8 +82,7 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
 #pragma unroll
     for (int c = 0; c < NV; ++c)
       qv[hh][c] = *reinterpret_cast<const float4*>(sq + hh * d + 128 * c + 4 * lane);
-  const int R = rows_pi + m;
-  for (int r0 = 8 * warp; r0 < R; r0 += 8 * (blockDim.x / 32)) {
+  for (int r0 = r_begin + 8 * warp; r0 < r_end; r0 += 8 * (blockDim.x / 32)) {
     float4 wv[8][NV];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -127,13 +134,13 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
     if (warp < 4) {
       float wk = 0.f;
       for (int k = 0; k < F; ++k) wk = fmaxf(wk, fabsf(2.f * s_w[k]));
-      if (F)
+      if (F && do_mse)
         for (int j = lane; j < d; j += 32) {
           const float qr = sqr[hh * d + j];
           mx = fmaxf(mx, wk * fabsf(qr));
           sm += qr;
         }
-    } else {
+    } else if (do_qjl) {
       for (int i = lane; i < m; i += 32) {
         const float qs = sqs[hh * m + i];
         mx = fmaxf(mx, fabsf(2.f * qs));
@@ -159,19 +166,25 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
   const float kFix = 16646144.f;
   if (tid < MG) {
     const float mM = __uint_as_float(s_maxM[tid]), mQ = __uint_as_float(s_maxQ[tid]);
-    const float dM = mM > 0.f ? mM / kFix : 1.f, dQ = mQ > 0.f ? mQ / kFix : 1.f;
-    float wsum = 0.f;
-    for (int k = 0; k < F; ++k) wsum += s_w[k];
     float* c = ws.qconst + ((int64_t)unit * MG + tid) * 4;
-    c[0] = dM / 128.f * scale_log2;
-    c[1] = wsum * s_sumqr[tid] * scale_log2;
-    c[2] = dQ / 128.f * scale_log2;
-    c[3] = -s_sumqs[tid] * scale_log2;
+    if (do_mse) {
+      const float dM = mM > 0.f ? mM / kFix : 1.f;
+      float wsum = 0.f;
+      for (int k = 0; k < F; ++k) wsum += s_w[k];
+      c[0] = dM / 128.f * scale_log2;
+      c[1] = wsum * s_sumqr[tid] * scale_log2;
+    }
+    if (do_qjl) {
+      const float dQ = mQ > 0.f ? mQ / kFix : 1.f;
+      c[2] = dQ / 128.f * scale_log2;
+      c[3] = -s_sumqs[tid] * scale_log2;
+    }
   }
   const int ksM = F * d / 32, ksQ = m / 32;
-  const int words = (ksM + ksQ) * 2 * 2 * 32;
-  uint32_t* fr = ws.frag + (int64_t)unit * words;
-  for (int wi = tid; wi < words; wi += blockDim.x) {
+  const int w0 = do_mse ? 0 : ksM * 128, w1 = do_qjl ? (ksM + ksQ) * 128 : ksM * 128;
+  uint32_t* fr = ws.frag + (int64_t)unit * (ksM + ksQ) * 128;
+  const int kpp = d / 32;                          // k-steps per feature plane
+  for (int wi = w0 + tid; wi < w1; wi += blockDim.x) {
     // word order [ks][lane][ntile][reg]: a lane's four words of a k-step are one uint4
     const int r = wi & 1, nt = (wi >> 1) & 1, ln = (wi >> 2) & 31, ks = wi >> 7;
     const int col = ln >> 2, tg = ln & 3;
@@ -184,15 +197,12 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
       const bool mse = ks < ksM;
       const float mx = __uint_as_float(mse ? s_maxM[hh] : s_maxQ[hh]);
       const float inv_delta = mx > 0.f ? kFix / mx : 1.f;
+      const int plane = mse ? ks / kpp : 0, jb = mse ? (ks - plane * kpp) * 32 : (ks - ksM) * 32;
+      const float wsc = mse ? -2.f * s_w[plane] : 2.f;
+      const float* src = mse ? sqr + hh * d + jb : sqs + hh * m + jb;
       for (int i = 0; i < 4; ++i) {
         const int bit = tg + 8 * i + (r ? 4 : 0);
-        float w;
-        if (mse) {
-          const int plane = ks / (d / 32), j = (ks % (d / 32)) * 32 + bit;
-          w = -2.f * s_w[plane] * sqr[hh * d + j];
-        } else {
-          w = 2.f * sqs[hh * m + (ks - ksM) * 32 + bit];
-        }
+        const float w = wsc * src[bit];
         const int wint = __float2int_rn(w * inv_delta) * (1 << shift);   // |wint| < 2^31
         const int s0 = ((wint + 128) & 255) - 128;
         const int t1 = (wint - s0) >> 8;

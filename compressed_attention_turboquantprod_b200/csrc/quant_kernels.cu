@@ -427,6 +427,34 @@ __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V
 // is a shared-memory broadcast) and reduces rho while Pi x is being formed.
 constexpr int SMALL_THREADS = 256;
 
+// Half a row of a d x d (or m x d) matrix, d <= 128, held in registers: issued
+// early, used later by half_dot.
+struct HalfRowRegs {
+  float4 w[16];
+};
+__device__ __forceinline__ void half_row_load(HalfRowRegs& h, const float* rowp, int d, int half) {
+  const float4* rp = reinterpret_cast<const float4*>(rowp) + half * (d / 8);
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (i < d / 8) h.w[i] = rp[i];
+}
+__device__ __forceinline__ float half_dot(const HalfRowRegs& h, const float* v, int d, int half) {
+  const float* vp = v + half * (d / 2);
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (i < d / 8) {
+      const float4 w = h.w[i];
+      float& a = (i & 1) ? a1 : a0;
+      a = fmaf(w.x, vp[4 * i], a);
+      a = fmaf(w.y, vp[4 * i + 1], a);
+      a = fmaf(w.z, vp[4 * i + 2], a);
+      a = fmaf(w.w, vp[4 * i + 3], a);
+    }
+  const float a = a0 + a1;
+  return a + __shfl_xor_sync(0xffffffffu, a, 1);
+}
+
 __device__ __forceinline__ float half_row_dot(const float* rowp, const float* v, int d, int half) {
   const float4* rp = reinterpret_cast<const float4*>(rowp) + half * (d / 8);
   const float* vp = v + half * (d / 2);
@@ -478,6 +506,10 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
       for (int a = tid >> 1; a < m; a += SMALL_THREADS / 2)
         for (int c = half * (d / 2); c < (half + 1) * (d / 2); c += 32) prefetch_l2(p.T + (int64_t)a * d + c);
     }
+    // d <= 128: this thread's half of Pi row tid / 2 goes out with the key itself
+    const bool regs = d <= 128;
+    HalfRowRegs hr;
+    if (regs && b1 > 0 && (tid >> 1) < d) half_row_load(hr, p.Pi + (int64_t)(tid >> 1) * d, d, tid & 1);
     int64_t e0;
     const void* src = src_row(p, false, bh, row, e0);
     double ss = 0.0;
@@ -500,9 +532,18 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     const float* E = sx;
     const int half = tid & 1;
     if (b1 > 0) {
-      for (int j = tid >> 1; j < d; j += SMALL_THREADS / 2) {
-        const float a = half_row_dot(p.Pi + (int64_t)j * d, sx, d, half);
-        if (half == 0) sy[j] = a * inv;
+      if (regs) {
+        if ((tid >> 1) < d) {
+          const float a = half_dot(hr, sx, d, half);
+          if (half == 0) sy[tid >> 1] = a * inv;
+        }
+        // this thread's half of T row tid / 2, in flight during the codes
+        if ((tid >> 1) < m) half_row_load(hr, p.T + (int64_t)(tid >> 1) * d, d, half);
+      } else {
+        for (int j = tid >> 1; j < d; j += SMALL_THREADS / 2) {
+          const float a = half_row_dot(p.Pi + (int64_t)j * d, sx, d, half);
+          if (half == 0) sy[j] = a * inv;
+        }
       }
       __syncthreads();
       const int L = 1 << b1;
@@ -534,8 +575,10 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     }
     // z = rho T e (or S x), two threads per row; a warp covers 16 rows, so the
     // 32 sign bits of a word come from two warps and are staged in shared memory.
+    if (regs && b1 == 0 && (tid >> 1) < m) half_row_load(hr, p.T + (int64_t)(tid >> 1) * d, d, half);
     for (int a = tid >> 1; a < m; a += SMALL_THREADS / 2) {
-      const float acc = half_row_dot(p.T + (int64_t)a * d, E, d, half);
+      const float acc = (regs && a == (tid >> 1)) ? half_dot(hr, E, d, half)
+                                                  : half_row_dot(p.T + (int64_t)a * d, E, d, half);
       if (half == 0) sz[a] = (b1 > 0) ? acc * rho : acc;
     }
     __syncthreads();
@@ -640,7 +683,8 @@ __global__ void __launch_bounds__(SMALL_THREADS) k_step_pre(QParams p, int nq_ct
     return;
   }
   bid -= nr_ctas;
-  mmadec::prep_mma_body<NV>(sp.g, sp.Q, sp.Hq, sp.Pi, sp.S, sp.cent, sp.scale_log2, sp.ws, bid,
+  mmadec::prep_mma_body<NV>(sp.g, sp.Q, sp.Hq, sp.Pi, sp.S, sp.cent, sp.scale_log2, sp.ws, bid >> 1,
+                            bid & 1,
                             smem_raw);
 }
 
@@ -1279,7 +1323,7 @@ cudaError_t launch_decode_step_pre(const QuantSrc& src, int64_t n_ring_only, con
   auto kern = g.d == 256 ? k_step_pre<2> : k_step_pre<1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<nq + nr + units, SMALL_THREADS, smem, s>>>(p, nq, nr, sp);
+  kern<<<nq + nr + 2 * units, SMALL_THREADS, smem, s>>>(p, nq, nr, sp);   // prep: 2 halves a unit
   return cudaGetLastError();
 }
 
