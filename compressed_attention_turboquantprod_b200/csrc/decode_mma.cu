@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
         const int t = tb + 16 * r + gid + 8 * e;
         float v = B1 > 0 ? rho[t] * fmaf(kM, vM[r][e], CM) + rn[t] * fmaf(kQ, vQ[r][e], CQ)
                          : rho[t] * fmaf(kQ, vQ[r][e], CQ);
-        if (t >= nt_valid) v = -INFINITY;
+        if (nt_valid < kBlockTokens && t >= nt_valid) v = -INFINITY;
         l[r][e] = v;
       }
     if (p.logits) {
@@ -355,15 +355,19 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       {
         const float sa[4] = {sA.x, sA.y, sA.z, sA.w}, sb[4] = {sB.x, sB.y, sB.z, sB.w};
         const float sc[4] = {sC.x, sC.y, sC.z, sC.w}, sd[4] = {sD.x, sD.y, sD.z, sD.w};
+        const float2 pAB = make_float2(pA, pB), pCD = make_float2(pC, pD);
+        const float2 nodd = make_float2(-oddf, -oddf);
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
           // tokens past the end have p = 0 and finite (zeroed or earlier) metadata
-          const float xA = pA * sa[gi], xB = pB * sb[gi], xC = pC * sc[gi], xD = pD * sd[gi];
+          const float2 x0 = mul2(pAB, make_float2(sa[gi], sb[gi]));
+          const float2 x1 = mul2(pCD, make_float2(sc[gi], sd[gi]));
           // column gid even carries fp16(x), odd carries fp16(x - fp16(x))
-          const float2 f0 = __half22float2(__floats2half2_rn(xA, xB));
-          const float2 f1 = __half22float2(__floats2half2_rn(xC, xD));
-          __half2 h0 = __floats2half2_rn(fmaf(-oddf, f0.x, xA), fmaf(-oddf, f0.y, xB));
-          __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
+          const float2 f0 = __half22float2(__floats2half2_rn(x0.x, x0.y));
+          const float2 f1 = __half22float2(__floats2half2_rn(x1.x, x1.y));
+          const float2 l0 = fma2(nodd, f0, x0), l1 = fma2(nodd, f1, x1);
+          __half2 h0 = __floats2half2_rn(l0.x, l0.y);
+          __half2 h1 = __floats2half2_rn(l1.x, l1.y);
           bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
           bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
         }

@@ -321,14 +321,18 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
         {
           const float sa[2] = {sA.x, sA.y}, sb[2] = {sB.x, sB.y};
           const float sc[2] = {sC.x, sC.y}, sd[2] = {sD.x, sD.y};
+          const float2 pAB = make_float2(pA, pB), pCD = make_float2(pC, pD);
+          const float2 nodd = make_float2(-oddf, -oddf);
 #pragma unroll
           for (int gi = 0; gi < 2; ++gi) {
-            const float xA = pA * sa[gi], xB = pB * sb[gi], xC = pC * sc[gi], xD = pD * sd[gi];
+            const float2 x0 = mul2(pAB, make_float2(sa[gi], sb[gi]));
+            const float2 x1 = mul2(pCD, make_float2(sc[gi], sd[gi]));
             // column gid even carries fp16(x), odd carries fp16(x - fp16(x))
-            const float2 f0 = __half22float2(__floats2half2_rn(xA, xB));
-            const float2 f1 = __half22float2(__floats2half2_rn(xC, xD));
-            __half2 h0 = __floats2half2_rn(fmaf(-oddf, f0.x, xA), fmaf(-oddf, f0.y, xB));
-            __half2 h1 = __floats2half2_rn(fmaf(-oddf, f1.x, xC), fmaf(-oddf, f1.y, xD));
+            const float2 f0 = __half22float2(__floats2half2_rn(x0.x, x0.y));
+            const float2 f1 = __half22float2(__floats2half2_rn(x1.x, x1.y));
+            const float2 l0 = fma2(nodd, f0, x0), l1 = fma2(nodd, f1, x1);
+            __half2 h0 = __floats2half2_rn(l0.x, l0.y);
+            __half2 h1 = __floats2half2_rn(l1.x, l1.y);
             bpv[gi][0] = *reinterpret_cast<uint32_t*>(&h0);
             bpv[gi][1] = *reinterpret_cast<uint32_t*>(&h1);
           }
