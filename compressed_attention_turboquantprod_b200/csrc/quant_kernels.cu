@@ -728,10 +728,10 @@ __device__ __forceinline__ void split8(const float (&v)[8], float scale, uint4& 
   uint32_t h[4], l[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float a0 = v[2 * j] * scale, a1 = v[2 * j + 1] * scale;
-    const __half2 hh = __floats2half2_rn(a0, a1);
-    const float2 f = __half22float2(hh);
-    const __half2 ll = __floats2half2_rn(a0 - f.x, a1 - f.y);
+    const float2 a = mmadec::mul2(make_float2(v[2 * j], v[2 * j + 1]), make_float2(scale, scale));
+    const __half2 hh = __floats2half2_rn(a.x, a.y);
+    const float2 lf = mmadec::sub2(a, __half22float2(hh));
+    const __half2 ll = __floats2half2_rn(lf.x, lf.y);
     h[j] = *reinterpret_cast<const uint32_t*>(&hh);
     l[j] = *reinterpret_cast<const uint32_t*>(&ll);
   }
@@ -798,6 +798,22 @@ __device__ __forceinline__ uint32_t value_code_nb(float v, float mn, float inv, 
   tie = fabsf(fabsf(__fsub_rn(x, rr)) - 0.5f) < 1e-5f;
   const uint32_t c = __float_as_uint(t) - __float_as_uint(kRound);
   return c < levels ? c : levels;
+}
+
+// value_code_nb for two channels sharing mn and inv, in packed fp32 pairs (the
+// same IEEE operations, two at a time); `tie` as for value_code_nb, for either.
+__device__ __forceinline__ void value_code_pair(float v0, float v1, float mn, float inv, uint32_t levels,
+                                                uint32_t& c0, uint32_t& c1, bool& tie) {
+  const float2 a = mmadec::sub2(make_float2(v0, v1), make_float2(mn, mn));
+  const float2 x = mmadec::mul2(a, make_float2(inv, inv));
+  const float2 t = mmadec::add2(x, make_float2(kRound, kRound));
+  const float2 rr = mmadec::sub2(t, make_float2(kRound, kRound));
+  const float2 dd = mmadec::sub2(x, rr);
+  tie = fabsf(fabsf(dd.x) - 0.5f) < 1e-5f || fabsf(fabsf(dd.y) - 0.5f) < 1e-5f;
+  const uint32_t k0 = __float_as_uint(t.x) - __float_as_uint(kRound);
+  const uint32_t k1 = __float_as_uint(t.y) - __float_as_uint(kRound);
+  c0 = k0 < levels ? k0 : levels;
+  c1 = k1 < levels ? k1 : levels;
 }
 
 // The issuing thread: D = A B^T over K = 128 as three products per k-step.
@@ -956,7 +972,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
 #pragma unroll
       for (int j = 0; j < 8; ++j) s8[j] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) s8[j & 7] = fmaf(x[j], x[j], s8[j & 7]);
+      for (int j = 0; j < 32; j += 2) {
+        const float2 xx = make_float2(x[j], x[j + 1]);
+        const float2 sp = mmadec::fma2(xx, xx, make_float2(s8[j & 7], s8[(j + 1) & 7]));
+        s8[j & 7] = sp.x;
+        s8[(j + 1) & 7] = sp.y;
+      }
       double ss = 0.0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) ss += (double)s8[j];
@@ -972,7 +993,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       for (int c8 = 0; c8 < 4; ++c8) {
         float v[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = x[8 * c8 + k] * inv;
+        for (int k = 0; k < 8; k += 2) {
+          const float2 u = mmadec::mul2(make_float2(x[8 * c8 + k], x[8 * c8 + k + 1]), make_float2(inv, inv));
+          v[k] = u.x;
+          v[k + 1] = u.y;
+        }
         uint4 hi, lo;
         split8(v, kSplit, hi, lo);
         const int off = tc::operand_off(r, k0 + 8 * c8);
@@ -1051,12 +1076,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
         uint32_t hw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         bool any_tie = false;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
+        for (int k = 0; k < 32; k += 2) {
           bool tie;
-          const uint32_t c = value_code_nb(v[k], mn[k >> 4], iv[k >> 4], levels, tie);
+          uint32_t c0, c1;
+          value_code_pair(v[k], v[k + 1], mn[k >> 4], iv[k >> 4], levels, c0, c1, tie);
           any_tie |= tie && sc[k >> 4] != 0.f;
-          if (vb == 2) hw[k >> 3] += c << (2 * (k & 7));
-          else hw[k >> 2] += c << (4 * (k & 3));
+          if (vb == 2) hw[k >> 3] += (c0 << (2 * (k & 7))) + (c1 << (2 * ((k + 1) & 7)));
+          else hw[k >> 2] += (c0 << (4 * (k & 3))) + (c1 << (4 * ((k + 1) & 3)));
         }
         if (any_tie) {
 #pragma unroll
@@ -1089,20 +1115,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
 #pragma unroll
       for (int j = 0; j < 8; ++j) s8[j] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float y = __uint_as_float(acc[c]) * (1.f / (kSplit * kSplit));
-        int idx = 0;
-        float cv = cen[0];
+      for (int c = 0; c < 32; c += 2) {
+        const float2 y2 = mmadec::mul2(make_float2(__uint_as_float(acc[c]), __uint_as_float(acc[c + 1])),
+                                       make_float2(1.f / (kSplit * kSplit), 1.f / (kSplit * kSplit)));
+        const float yy[2] = {y2.x, y2.y};
+        float cv[2];
 #pragma unroll
-        for (int k = 0; k + 1 < L; ++k)
-          if (bnd[k] < y) {
-            idx = k + 1;
-            cv = cen[k + 1];
-          }
+        for (int u = 0; u < 2; ++u) {
+          int idx = 0;
+          cv[u] = cen[0];
 #pragma unroll
-        for (int pl = 0; pl < B1; ++pl) pw[pl] |= (uint32_t)((idx >> pl) & 1) << c;
-        e[c] = y - cv;
-        s8[c & 7] = fmaf(e[c], e[c], s8[c & 7]);
+          for (int k = 0; k + 1 < L; ++k)
+            if (bnd[k] < yy[u]) {
+              idx = k + 1;
+              cv[u] = cen[k + 1];
+            }
+#pragma unroll
+          for (int pl = 0; pl < B1; ++pl) pw[pl] |= (uint32_t)((idx >> pl) & 1) << (c + u);
+        }
+        const float2 e2 = mmadec::sub2(y2, make_float2(cv[0], cv[1]));
+        e[c] = e2.x;
+        e[c + 1] = e2.y;
+        const float2 sp = mmadec::fma2(e2, e2, make_float2(s8[c & 7], s8[(c + 1) & 7]));
+        s8[c & 7] = sp.x;
+        s8[(c + 1) & 7] = sp.y;
       }
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
