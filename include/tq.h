@@ -300,6 +300,11 @@ int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void
  * Arguments as for tq_append and tq_decode_attention; the workspace is sized for
  * the cache after the append (tq_decode_workspace_bytes of a cache with
  * n_total + n_new tokens; the workspace size does not depend on n_total).
+ * K, V, Q and out may also be pinned (page-locked) host memory from
+ * cudaHostAlloc / cudaMallocHost on a system with unified addressing, where it is
+ * mapped into the device address space at the same pointer: the kernels then
+ * read the new tokens and queries and write the output across the host link,
+ * with no staging copy (the result is identical; only the latency differs).
  * All checks of both parts are made before anything is launched.
  * Errors: INVALID_ARG, CAPACITY, UNSUPPORTED, CUDA.
  */

@@ -64,3 +64,46 @@ def test_decode_step_matches_append_then_decode(kw, n0, steps):
         assert torch.equal(o1, o2), f"outputs differ after step {i}"
         assert torch.equal(l1, l2), f"logits differ after step {i}"
         assert torch.isfinite(o1.float()).all()
+
+
+@pytest.mark.parametrize("kw,n0,steps", [
+    (dict(), 300, [1, 1, 1]),                                           # fused path
+    (dict(W=3), 50, [5]),                                               # the two calls
+])
+def test_decode_step_on_pinned_host_buffers(kw, n0, steps):
+    """The new tokens, the queries and the output of tq_decode_step in pinned host
+    memory (mapped into the device address space; the kernels read and write them
+    across the host link): identical cache, output and logits to device buffers."""
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache, native
+    w = _workload(**kw)
+    total = n0 + sum(steps)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    pj, cbd = _Proj(po), _Cb(cb)
+    K, V = synth.keys_values(w, device="cuda", T=total)
+    caches = [CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
+                                dtype=TORCH_DT[w.dtype]) for _ in range(2)]
+    for c in caches:
+        c.append(K[:, :, :n0].contiguous(), V[:, :, :n0].contiguous(), pj, cbd)
+    scale = 1.0 / math.sqrt(w.d)
+    t = n0
+    for i, n in enumerate(steps):
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        Q = synth.queries(w.scaled(seed=70 + i), device="cuda")
+        kh, vh, qh = k.cpu().pin_memory(), v.cpu().pin_memory(), Q.cpu().pin_memory()
+        outs, logs = [], []
+        for c, (kk, vv, qq, host) in zip(caches, ((k, v, Q, False), (kh, vh, qh, True))):
+            out = torch.empty(w.B, w.Hq, w.d, dtype=TORCH_DT[w.dtype],
+                              device="cpu" if host else "cuda")
+            if host:
+                out = out.pin_memory()
+            lg = torch.empty(w.B, w.Hq, c.n_total + n, dtype=torch.float32, device="cuda")
+            ws = c.workspace(w.Hq)
+            native.tq_decode_step(c.state, kk, vv, qq, scale, pj.Pi, pj.S, pj.T, cbd.centroids,
+                                  cbd.boundaries, out, lg, 0, ws)
+            outs.append(out)
+            logs.append(lg)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0].cpu().view(torch.uint8), outs[1].view(torch.uint8))
+        assert torch.equal(logs[0], logs[1])
+        assert torch.equal(caches[0].buffer, caches[1].buffer)
+        t += n
