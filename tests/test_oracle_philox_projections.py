@@ -89,3 +89,59 @@ def test_rotation_is_haar_distributed():
         acc2 += Q * Q
     assert np.max(np.abs(acc / n)) < 5 * np.sqrt(1.0 / d / n)
     assert abs(np.mean(acc2 / n) - 1.0 / d) < 0.01 / d
+
+
+def _fwht(v):
+    """Plain in-place butterfly Walsh-Hadamard transform (unnormalised), O(d log d)."""
+    v = np.array(v, dtype=np.float64)
+    h = 1
+    while h < v.shape[-1]:
+        for i in range(0, v.shape[-1], 2 * h):
+            a = v[..., i:i + h].copy()
+            b = v[..., i + h:i + 2 * h].copy()
+            v[..., i:i + h] = a + b
+            v[..., i + h:i + 2 * h] = a - b
+        h *= 2
+    return v
+
+
+@pytest.mark.parametrize("d", [2, 8, 64, 256])
+def test_sylvester_hadamard_closed_form(d):
+    """H_d of the recursion has entry (r, c) = (-1)^popcount(r & c)."""
+    H = projections.sylvester_hadamard(d)
+    r = np.arange(d)[:, None]
+    c = np.arange(d)[None, :]
+    par = np.vectorize(lambda x: bin(x).count("1") & 1)(r & c)
+    assert np.array_equal(H, np.where(par == 1, -1.0, 1.0))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_hadamard_rotation_orthogonal_flat_and_fast(d):
+    """Pi = H diag(s) / sqrt(d): orthogonal, every entry of magnitude 1/sqrt(d) (so a
+    single large coordinate is spread evenly over all d), and Pi u equals the fast
+    Walsh-Hadamard transform of s * u divided by sqrt(d)."""
+    seed = projections.layer_seed(3)
+    Pi = projections.hadamard_rotation(d, seed)
+    assert np.max(np.abs(Pi.T @ Pi - np.eye(d))) < 1e-12
+    assert np.allclose(np.abs(Pi), 1.0 / np.sqrt(d), rtol=0, atol=1e-15)
+    s = projections.hadamard_signs(d, seed)
+    rng = np.random.default_rng(5)
+    u = rng.standard_normal((3, d))
+    assert np.max(np.abs(u @ Pi.T - _fwht(u * s) / np.sqrt(d))) < 1e-12
+    e = np.zeros(d)
+    e[d // 3] = 7.0                                    # an outlier coordinate
+    assert np.allclose(np.abs(Pi @ e), 7.0 / np.sqrt(d), rtol=0, atol=1e-12)
+    st = projections.make_projections(d, 32, 3, structured=True)
+    assert np.all(np.abs(st["Pi"]) == np.float32(1.0 / np.sqrt(d)))
+
+
+def test_hadamard_signs_from_philox_stream_2():
+    """s_c = +1 iff the top bit of word 0 of Philox draw c under key (seed, 2) is 0;
+    checked draw by draw against the scalar generator, and balanced."""
+    seed = 42
+    s = projections.hadamard_signs(4096, seed)
+    for c in (0, 1, 777, 4095):
+        w0 = philox.philox4x64_10((np.uint64(c), 0, 0, 0), (seed, 2))[0]
+        assert s[c] == (1.0 if int(w0) >> 63 == 0 else -1.0)
+    assert abs(s.mean()) < 5.0 / np.sqrt(4096)
+    assert not np.array_equal(s, projections.hadamard_signs(4096, seed + 7))

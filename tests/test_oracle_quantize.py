@@ -93,16 +93,19 @@ def test_zero_key():
     assert np.all(pure["bits"] == 1) and pure["rho"][0] == 0
 
 
-@pytest.mark.parametrize("b1,d,m", [(2, 16, 16), (1, 16, 16), (0, 16, 32)])
-def test_estimator_unbiased_over_sketch_draws(b1, d, m):
-    """E_S[estimate] = <q, x> ([TQ] section 4/5).  Draw N independent S matrices;
-    stacking them as one sketch of N*m rows makes the oracle's own estimator
-    return the mean of the N per-draw estimates (its 1/m becomes 1/(N m))."""
+@pytest.mark.parametrize("b1,d,m,structured", [(2, 16, 16, False), (1, 16, 16, False), (0, 16, 32, False),
+                                                (2, 16, 16, True)])
+def test_estimator_unbiased_over_sketch_draws(b1, d, m, structured):
+    """E_S[estimate] = <q, x> ([TQ] section 4/5), with the QR rotation and with the
+    structured Hadamard one.  Draw N independent S matrices; stacking them as one
+    sketch of N*m rows makes the oracle's own estimator return the mean of the N
+    per-draw estimates (its 1/m becomes 1/(N m))."""
     rng = np.random.default_rng(10 + b1)
     x = rng.standard_normal(d)
     q = x + 0.8 * rng.standard_normal(d)             # |<q,x>| well away from 0
     assert abs(q @ x) > 0.5 * np.linalg.norm(q) * np.linalg.norm(x)
-    Pi = projections.rotation(d, 7).astype(np.float32) if b1 else None
+    rot = projections.hadamard_rotation if structured else projections.rotation
+    Pi = rot(d, 7).astype(np.float32) if b1 else None
     c32, b32 = codebook.build(d, b1) if b1 else (None, None)
     N = 100_000
     S = rng.standard_normal((N * m, d)).astype(np.float32)
