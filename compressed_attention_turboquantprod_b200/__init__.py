@@ -43,15 +43,19 @@ class Codebook:
 
 
 class Projections:
-    """Per-layer Pi (d x d), S (m x d) and T = S Pi^T, generated on the GPU."""
+    """Per-layer Pi (d x d), S (m x d) and T = S Pi^T, generated on the GPU.
+    structured: the Hadamard rotation Pi = H diag(s) / sqrt(d) instead of the QR one."""
 
     def __init__(self, d: int, m: int, layer: int, rotation: bool = True, device="cuda",
-                 base_seed: int = 42, stride: int = 7):
+                 base_seed: int = 42, stride: int = 7, structured: bool = False):
         self.d, self.m, self.layer = d, m, layer
         f32 = dict(dtype=torch.float32, device=device)
         self.Pi = torch.empty(d, d, **f32) if rotation else None
         self.S = torch.empty(m, d, **f32)
         self.T = torch.empty(m, d, **f32)
+        if rotation and structured:
+            native.tq_make_projections_hadamard(d, m, layer, self.Pi, self.S, self.T, base_seed, stride)
+            return
         ws = None
         if rotation:
             ws = torch.empty(native.tq_projections_workspace_bytes(d), dtype=torch.uint8, device=device)

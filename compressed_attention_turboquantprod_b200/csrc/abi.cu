@@ -255,6 +255,22 @@ size_t tq_projections_workspace_bytes(int d) {
   return 2 * (size_t)d * d * sizeof(double);
 }
 
+int tq_make_projections_hadamard(int d, int m, int layer, uint64_t base_seed, uint64_t stride,
+                                 float* Pi, float* S, float* T, void* stream) {
+  TQ_FAULT_POINT("tq_make_projections_hadamard");
+  if (!valid_d(d)) return fail(TQ_ERR_UNSUPPORTED, "head dim d=%d not in {64,128,256}", d);
+  if (!valid_m(m)) return fail(TQ_ERR_UNSUPPORTED, "sketch dim m=%d not a multiple of 32 in [32,1024]", m);
+  if (layer < 0) return fail(TQ_ERR_INVALID_ARG, "layer=%d", layer);
+  if (!Pi || !S || !aligned16(Pi) || !aligned16(S) || (T && !aligned16(T)))
+    return fail(TQ_ERR_INVALID_ARG, "Pi and S must be non-null; Pi, S, T 16-byte aligned");
+  int st = check_pending("tq_make_projections_hadamard");
+  if (st != TQ_OK) return st;
+  const uint64_t seed = base_seed + stride * (uint64_t)layer;
+  cudaError_t e = tq::launch_projections_hadamard(d, m, seed, Pi, S, T, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_make_projections_hadamard");
+  return ok();
+}
+
 int tq_make_projections(int d, int m, int layer, uint64_t base_seed, uint64_t stride, float* Pi,
                         float* S, float* T, void* workspace, size_t ws_bytes, void* stream) {
   TQ_FAULT_POINT("tq_make_projections");

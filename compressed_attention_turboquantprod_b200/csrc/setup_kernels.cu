@@ -247,6 +247,22 @@ __global__ void __launch_bounds__(1024) k_qr(double* A, double* Q, int d, float*
   }
 }
 
+// Structured rotation Pi = H diag(s) / sqrt(d) ([NQ] six-stage pipeline, step 4:
+// a Hadamard rotation): H[r][c] = (-1)^popcount(r & c) (Sylvester, d a power of
+// two), s_c = +1 when the top bit of word 0 of Philox draw c (stream 2) is 0.
+// Every entry is +-fl(1/sqrt(d)) (the reciprocal square root taken in float64).
+__global__ void k_hadamard(float* Pi, int d, uint64_t seed) {
+  const int64_t n = (int64_t)d * d;
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= n) return;
+  const int r = (int)(k / d), c = (int)(k % d);
+  uint64_t w[4] = {(uint64_t)c, 0ull, 0ull, 0ull};
+  philox4x64_10(w, seed, 2ull);
+  const float mag = (float)(1.0 / sqrt((double)d));
+  const bool neg = ((__popc((unsigned)(r & c)) & 1) != 0) != ((w[0] >> 63) != 0);
+  Pi[k] = neg ? -mag : mag;
+}
+
 // T = S Pi^T (m x d), float64 accumulation of the stored fp32 values.
 __global__ void k_sketch_rot(const float* S, const float* Pi, float* T, int m, int d) {
   const int a = blockIdx.x;
@@ -258,6 +274,21 @@ __global__ void k_sketch_rot(const float* S, const float* Pi, float* T, int m, i
 }
 
 }  // namespace
+
+cudaError_t launch_projections_hadamard(int d, int m, uint64_t seed, float* Pi, float* S, float* T,
+                                       cudaStream_t s) {
+  const int threads = 256;
+  {
+    const int64_t n = (int64_t)m * d;
+    k_gauss<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(nullptr, S, m, d, seed, 1);
+  }
+  {
+    const int64_t n = (int64_t)d * d;
+    k_hadamard<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(Pi, d, seed);
+  }
+  if (T) k_sketch_rot<<<m, 256, 0, s>>>(S, Pi, T, m, d);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_codebook(int d, int bits, float* cent, float* bnd, cudaStream_t s) {
   k_codebook<<<1, 256, 0, s>>>(d, bits, cent, bnd);

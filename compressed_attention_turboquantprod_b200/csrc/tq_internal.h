@@ -29,6 +29,8 @@ int set_error(int status, const char* fmt, ...);
 
 // ---- setup (setup_kernels.cu) ----
 cudaError_t launch_codebook(int d, int bits, float* cent, float* bnd, cudaStream_t s);
+cudaError_t launch_projections_hadamard(int d, int m, uint64_t seed, float* Pi, float* S, float* T,
+                                       cudaStream_t s);
 cudaError_t launch_projections(int d, int m, uint64_t seed, float* Pi, float* S, float* T,
                                double* ws, cudaStream_t s);
 

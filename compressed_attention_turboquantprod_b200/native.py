@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "tq_codebook_build": (I, [I, I, P, P, P]),
         "tq_projections_workspace_bytes": (SZ, [I]),
         "tq_make_projections": (I, [I, I, I, U64, U64, P, P, P, P, SZ, P]),
+        "tq_make_projections_hadamard": (I, [I, I, I, U64, U64, P, P, P, P]),
         "tq_quantize_keys": (I, [P, I, I64, I, I, I, P, P, P, P, P, P, P, P, P]),
         "tq_quantize_values": (I, [P, I, I64, I, I, I, P, P, P, P]),
         "tq_cache_bytes": (SZ, [D]),
@@ -139,6 +140,13 @@ def tq_make_projections(d: int, m: int, layer: int, Pi, S, T, workspace, base_se
     _check(lib.tq_make_projections(d, m, layer, base_seed, stride, _ptr(Pi), _ptr(S), _ptr(T),
                                    _ptr(workspace), ws_bytes, _stream(stream)),
            "tq_make_projections")
+
+
+def tq_make_projections_hadamard(d: int, m: int, layer: int, Pi, S, T, base_seed: int = 42,
+                                 stride: int = 7, stream=None):
+    _check(lib.tq_make_projections_hadamard(d, m, layer, base_seed, stride, _ptr(Pi), _ptr(S),
+                                            _ptr(T), _stream(stream)),
+           "tq_make_projections_hadamard")
 
 
 # ----------------------------------------------------------------------------- quantise

@@ -9,6 +9,8 @@
  *          ring buffer), 七 (value quantization, known limits).
  *   [AQJL] A-QJL adaptive layer-wise KV compression article
  *          (zingnex.cn/forum/thread/a-qjl-kv): QJL, A-QJL, deployment config.
+ *   [NQ]   KV-cache compression article "无需训练即可将大模型的 KV 缓存压缩 33 倍"
+ *          (explore.n1n.ai): six-stage pipeline, step 4 (Hadamard rotation).
  *
  * Conventions shared by every call:
  *   - Every call returns an int status (enum tq_status).  On failure a
@@ -111,6 +113,24 @@ size_t tq_projections_workspace_bytes(int d);
 int tq_make_projections(int d, int m, int layer, uint64_t base_seed, uint64_t stride,
                         float* Pi, float* S, float* T, void* workspace, size_t ws_bytes,
                         void* stream);
+
+/*
+ * tq_make_projections_hadamard -- the structured rotation ([NQ] the KV-cache
+ * compression page "无需训练即可将大模型的 KV 缓存压缩 33 倍", six-stage pipeline,
+ * step 4: a Hadamard rotation spreads a vector's energy evenly over the
+ * coordinates) in place of the QR one: Pi = H diag(s) / sqrt(d), H the
+ * Sylvester Hadamard matrix (entry (r, c) = (-1)^popcount(r & c)), s_c = +1 when
+ * the top bit of word 0 of Philox4x64-10 draw c under key (seed, 2) is 0, else
+ * -1; every entry is +-fl32(1/sqrt(d)).  S and T = S Pi^T as tq_make_projections
+ * (same seed rule, same S).  Pi is orthogonal, so every call that takes Pi and T
+ * works unchanged with it; Pi u is a fast Walsh-Hadamard transform of s * u.
+ *   Pi  device float[d*d] row-major (written)
+ *   S   device float[m*d] row-major (written)
+ *   T   device float[m*d] row-major (written; may be NULL)
+ * No workspace.  Errors: INVALID_ARG, UNSUPPORTED (d, m), CUDA.
+ */
+int tq_make_projections_hadamard(int d, int m, int layer, uint64_t base_seed, uint64_t stride,
+                                 float* Pi, float* S, float* T, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Quantisation of keys and values (token-major output arrays)              */

@@ -38,9 +38,10 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
 
 
-def oracle_setup(d, b1, m, layer=0):
-    """The oracle's own stored projections and codebook (numpy fp32)."""
-    p = oproj.make_projections(d, m, layer, with_rotation=b1 > 0)
+def oracle_setup(d, b1, m, layer=0, structured=False):
+    """The oracle's own stored projections and codebook (numpy fp32); structured:
+    the Hadamard rotation."""
+    p = oproj.make_projections(d, m, layer, with_rotation=b1 > 0, structured=structured)
     cb = ocb.build(d, b1) if b1 > 0 else (None, None)
     return p, cb
 

@@ -311,6 +311,34 @@ def test_tiny_workload_end_to_end_with_library_projections():
             check_logits(logits.cpu().numpy()[0].astype(np.float64), rl[(0, 0)])
 
 
+def test_hadamard_rotation_end_to_end():
+    """The structured rotation through the whole path: library-made Hadamard
+    projections, GPU append (tensor-core quantise) + decode, vs the oracle with
+    its own Hadamard projections from the same seed."""
+    from compressed_attention_turboquantprod_b200 import Codebook, Projections
+    w = _workload(B=2, Hkv=2, Hq=8, T=700, W=16)
+    K, V = synth.keys_values(w, device="cuda")
+    Q = synth.queries(w, device="cuda")
+    pg, cbg = Projections(w.d, w.m, 2, structured=True), Codebook(w.d, w.b1)
+    gc = _gpu_cache(w, 768)
+    gc.append(K, V, pg, cbg)
+    out, logits = gc.decode(Q, pg, cbg, want_logits=True)
+    torch.cuda.synchronize()
+    po, cb = oracle_setup(w.d, w.b1, w.m, layer=2, structured=True)
+    oc = _oracle_cache(w, 768, po, cb)
+    oc.append(host(K), host(V))
+    ro, rl = oc.decode(host(Q))
+    skipped = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
+    assert skipped <= 4
+    if skipped == 0:                 # identical codes everywhere: outputs and logits too
+        G = w.Hq // w.Hkv
+        check_out(host(out), ro, w.dtype)
+        lg = logits.cpu().numpy().astype(np.float64)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                check_logits(lg[b, h * G:(h + 1) * G], rl[(b, h)])
+
+
 def test_gqa32k_shape_reduced_context_end_to_end():
     from compressed_attention_turboquantprod_b200 import Codebook, Projections
     w = synth.WORKLOADS["gqa32k"].scaled(T=2000)

@@ -57,6 +57,37 @@ def test_projections_match_oracle(d, m, layer, rot):
         assert np.max(np.abs(P64.T @ P64 - np.eye(d))) < 1e-5
 
 
+@pytest.mark.parametrize("d,m,layer", [(128, 128, 0), (256, 256, 3), (64, 96, 1)])
+def test_hadamard_projections_match_oracle(d, m, layer):
+    """The structured rotation: Pi bit-exact (every entry +-fl32(1/sqrt(d)), signs
+    from Philox stream 2), S the same as the QR call's, T = S Pi^T as there."""
+    from compressed_attention_turboquantprod_b200 import Projections
+    pg = Projections(d, m, layer, structured=True)
+    po = oproj.make_projections(d, m, layer, structured=True)
+    assert np.array_equal(pg.Pi.cpu().numpy(), po["Pi"])
+    S = pg.S.cpu().numpy()
+    assert np.all(np.abs(S - po["S"]) <= np.spacing(np.abs(po["S"])))
+    T = pg.T.cpu().numpy()
+    assert np.max(np.abs(T - po["T"])) <= 2e-6 * max(1.0, np.max(np.abs(po["T"])))
+    assert np.array_equal(S, Projections(d, m, layer).S.cpu().numpy())
+
+
+@pytest.mark.parametrize("b1,n", [(2, 1000), (3, 300), (1, 129)])
+def test_quantize_keys_with_hadamard_rotation(b1, n):
+    """Keys quantised with the structured rotation on the tensor-core path: codes,
+    signs and norms against the oracle with the same rotation."""
+    d, m = 128, 128
+    w = synth.Workload("t", B=1, Hq=1, Hkv=1, d=d, T=n, W=0, b1=b1, m=m, vbits=2, group=32,
+                       dtype="bf16", seed=21 + b1, k_outlier_count=3, outlier_scale=8.0)
+    K, _ = synth.keys_values(w, device="cuda")
+    K = K[0, 0].contiguous()
+    po, (c32, b32) = oracle_setup(d, b1, m, structured=True)
+    got = _keys_gpu(K, b1, m, to_dev(po["Pi"]), to_dev(po["T"]), to_dev(c32), to_dev(b32))
+    ref = oq.quantize_keys(host(K), po["Pi"], po["S"], c32, b32, b1)
+    stats = compare_keys(got, ref, d, b1, m, b32)
+    assert stats["skipped_tokens"] <= max(2, n // 200)
+
+
 def _keys_gpu(K, b1, m, Pi, T, c, b):
     n_ = nat()
     n, d = K.shape
