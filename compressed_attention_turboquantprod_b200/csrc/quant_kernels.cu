@@ -787,21 +787,10 @@ __device__ __forceinline__ uint32_t value_code_fast(float v, float mn, float sc,
   return c < levels ? c : levels;
 }
 
-// The same code without the rare exact-division branch: `tie` is set when the
-// product lies within 1e-5 of a half-integer, and the caller recomputes those
-// elements with value_code_fast.
-__device__ __forceinline__ uint32_t value_code_nb(float v, float mn, float inv, uint32_t levels, bool& tie) {
-  const float a = __fsub_rn(v, mn);
-  const float x = __fmul_rn(a, inv);
-  const float t = __fadd_rn(x, kRound);
-  const float rr = __fsub_rn(t, kRound);
-  tie = fabsf(fabsf(__fsub_rn(x, rr)) - 0.5f) < 1e-5f;
-  const uint32_t c = __float_as_uint(t) - __float_as_uint(kRound);
-  return c < levels ? c : levels;
-}
-
-// value_code_nb for two channels sharing mn and inv, in packed fp32 pairs (the
-// same IEEE operations, two at a time); `tie` as for value_code_nb, for either.
+// value_code_fast for two channels sharing mn and inv, in packed fp32 pairs (the
+// same IEEE operations, two at a time), without its rare exact-division branch:
+// `tie` is set when either product lies within 1e-5 of a half-integer, and the
+// caller then recomputes with value_code_fast.
 __device__ __forceinline__ void value_code_pair(float v0, float v1, float mn, float inv, uint32_t levels,
                                                 uint32_t& c0, uint32_t& c1, bool& tie) {
   const float2 a = mmadec::sub2(make_float2(v0, v1), make_float2(mn, mn));
