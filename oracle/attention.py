@@ -15,6 +15,14 @@ compressed tokens plus exact <q, k> over the ring tokens, softmax with scale
 1/sqrt(d) (reading taken: the standard scale), output sum_t p_t v^_t with
 v^ = mn + code * s for compressed tokens and the exact v for ring tokens.  GQA:
 query head hq reads KV head hq // (Hq / Hkv).  All float64, dense softmax.
+
+Multi-token (chunked prefill) attention over the same store ([TQ] §六 for the
+history and the ring; §七 notes that the page's own hybrid path dequantises the
+history for this step): a chunk of n new tokens is scored before it is
+appended.  Readings taken where the pages are silent: query i of the chunk sees
+the compressed history (estimator logits, v^ values), the ring (exact), and the
+chunk's own tokens 0..i (exact keys and values in their input precision, causal
+order, the query's own token included); the softmax scale is the decode's.
 """
 from __future__ import annotations
 
@@ -66,3 +74,23 @@ def decode_group(q, comp_keys, comp_vhat, ring_k, ring_v, Pi32, S32, c32, b1: in
     logits = np.concatenate(parts_l, axis=1)
     values = np.concatenate(parts_v, axis=0)
     return softmax_attention(logits, values, scale), logits
+
+
+def prefill_group(Qg, comp_keys, comp_vhat, ring_k, ring_v, new_k, new_v, Pi32, S32, c32, b1: int,
+                  scale: float):
+    """One (batch, KV head) of a chunk: Qg [n, G, d] the queries of the chunk's n tokens;
+    new_k / new_v [n, d] the chunk's keys and values.  Query i is a decode over the
+    history plus an exact segment of the ring followed by chunk tokens 0..i.
+    Returns out [n, G, d]."""
+    Qg = np.asarray(Qg, dtype=np.float64)
+    n, G, d = Qg.shape
+    new_k = np.asarray(new_k, dtype=np.float64)
+    new_v = np.asarray(new_v, dtype=np.float64)
+    rk0 = np.zeros((0, d)) if ring_k is None else np.asarray(ring_k, dtype=np.float64)
+    rv0 = np.zeros((0, d)) if ring_v is None else np.asarray(ring_v, dtype=np.float64)
+    out = np.zeros((n, G, d))
+    for i in range(n):
+        ek = np.concatenate((rk0, new_k[:i + 1]), axis=0)
+        ev = np.concatenate((rv0, new_v[:i + 1]), axis=0)
+        out[i], _ = decode_group(Qg[i], comp_keys, comp_vhat, ek, ev, Pi32, S32, c32, b1, scale)
+    return out

@@ -117,6 +117,32 @@ class OracleCache:
         return out, logits
 
 
+    def prefill(self, Q, Knew, Vnew, scale=None):
+        """Attention of a chunk of n new tokens before they are appended (the cache is
+        not changed).  Q: [B, n, Hq, d] (token-major); Knew, Vnew: [B, Hkv, n, d] as
+        ``append`` takes them.  Returns out [B, n, Hq, d]."""
+        Q = np.asarray(Q, dtype=np.float64)
+        Knew = np.asarray(Knew, dtype=np.float64)
+        Vnew = np.asarray(Vnew, dtype=np.float64)
+        n, Hq = Q.shape[1], Q.shape[2]
+        G = Hq // self.Hkv
+        scale = 1.0 / np.sqrt(self.d) if scale is None else scale
+        out = np.zeros((self.B, n, Hq, self.d))
+        slots = self.ring_slots()
+        for b in range(self.B):
+            for h in range(self.Hkv):
+                r = self.rec[b][h]
+                vhat = (quantize.dequantize_values(r["codes"], r["scale"], r["vmin"], self.group)
+                        if r is not None else np.zeros((0, self.d)))
+                rk = self.ring_k[b, h, slots] if slots else None
+                rv = self.ring_v[b, h, slots] if slots else None
+                out[b, :, h * G:(h + 1) * G] = attention.prefill_group(
+                    Q[b, :, h * G:(h + 1) * G], r, vhat, rk, rv, Knew[b, h], Vnew[b, h],
+                    self.proj.get("Pi"), self.proj["S"], self.cb[0] if self.cb is not None else None,
+                    self.b1, scale)
+        return out
+
+
 def _to_dtype_bytes(x, dtype: str) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     if dtype == "f32":
