@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantize", action="store_true")
     ap.add_argument("--no-other-decodes", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--workload", default="gqa32k")
     return ap.parse_args()
 
@@ -500,6 +501,11 @@ def run_ours(args):
                "transfer": "tq_decode_step called on pinned host buffers: its kernels read Q, K, V "
                            "and write the output over the host link (mapped pinned memory)"}
 
+    # multi-token (chunked prefill) attention on the same cache: chunks of n tokens
+    prefill = None
+    if not args.no_prefill:
+        prefill = bench_prefill(w, cache, pj, cb, flush_l2, stream, step_bytes()[0], world)
+
     # key/value quantise throughput: 131072 tokens x 8 KV heads in chunks of 4096
     quant = None
     if not args.no_quantize:
@@ -535,6 +541,7 @@ def run_ours(args):
                      "avg_launch_ms": part_avg_ms, "source_hash": src_hash},
         "e2e": e2e,
         "quantize": quant,
+        "prefill": prefill,
         "other_decodes": others,
         "cpu_baseline": cpu,
         "clocks": clk,
@@ -547,6 +554,55 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=(16, 64), reps=20,
+                  warm=3):
+    """tq_prefill_attention on the decode bench's cache (the chunk is scored, not
+    appended), L2 flushed before each call, CUDA events around the call (its four
+    launches).  A plain decode (tq_decode_attention) of the same cache is timed the
+    same way, so that n decodes can be compared with one chunk of n tokens."""
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import native
+    dev = cache.buffer.device
+    scale = 1.0 / math.sqrt(w.d)
+    cent = cb.centroids if cb else None
+
+    def timed(fn):
+        for _ in range(warm):
+            flush_l2()
+            fn()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for k in range(reps):
+            flush_l2()
+            ev[k][0].record(stream)
+            fn()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        return reduce_max(sum(e[0].elapsed_time(e[1]) for e in ev) / reps, world)
+
+    Qd = synth.queries(w, device=dev)
+    outd = torch.empty_like(Qd)
+    wsd = cache.workspace(w.Hq, 0)
+    t_dec = timed(lambda: native.tq_decode_attention(cache.state, Qd, scale, pj.Pi, pj.S, cent,
+                                                     outd, None, 0, wsd))
+    res = []
+    for n in chunks:
+        Q, Kc, Vc = synth.prefill_chunk(w, n, device=dev)
+        out = torch.empty_like(Q)
+        ws = torch.empty(native.tq_prefill_workspace_bytes(cache.state, w.Hq, n, 0),
+                         dtype=torch.uint8, device=dev)
+        t = timed(lambda: native.tq_prefill_attention(cache.state, Q, Kc, Vc, scale, pj.Pi, pj.S,
+                                                      cent, out, 0, ws))
+        native.tq_prefill_check(cache.state, w.Hq, n, 0, ws)
+        toks = reduce_sum(float(w.B * n), world)
+        res.append({"n": n, "ms": t, "query_tokens_per_s": toks / (t * 1e-3),
+                    "history_GB_per_s": reduce_sum(float(hist_bytes), world) / (t * 1e-3) / 1e9,
+                    "vs_n_decodes": n * t_dec / t})
+    return {"chunks": res, "decode_ms": t_dec, "history_bytes": hist_bytes,
+            "timing": "CUDA events around the whole call (prep, history partials, exact segment, "
+                      "merge), L2 flushed before each call, 20 calls after 3 warm-up calls"}
 
 
 def _time_decode(w, layer, dev, reps=10, warm=3):

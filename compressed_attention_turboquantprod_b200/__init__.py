@@ -128,6 +128,23 @@ class CompressedKVCache:
                               cb.boundaries if cb is not None else None, out, logits, num_splits, ws)
         return (out, logits) if want_logits else out
 
+    def prefill(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, proj: Projections,
+                cb: Optional[Codebook], softmax_scale: Optional[float] = None, num_splits: int = 0,
+                out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+        """Attention of a chunk of n new tokens before it is appended: Q [B, n, Hq, d]
+        (token-major), K, V [B, Hkv, n, d]; query i sees the history, the ring and
+        chunk tokens 0..i.  The cache is unchanged (call append(K, V) afterwards)."""
+        B, n, Hq, d = Q.shape
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+        out = torch.empty_like(Q) if out is None else out
+        if workspace is None:
+            need = native.tq_prefill_workspace_bytes(self.state, Hq, n, num_splits)
+            workspace = torch.empty(need, dtype=torch.uint8, device=self.buffer.device)
+        native.tq_prefill_attention(self.state, Q, K, V, scale, proj.Pi, proj.S,
+                                    cb.centroids if cb is not None else None, out, num_splits,
+                                    workspace)
+        return out
+
     def decode(self, Q: torch.Tensor, proj: Projections, cb: Optional[Codebook],
                softmax_scale: Optional[float] = None, want_logits: bool = False,
                num_splits: int = 0, out: Optional[torch.Tensor] = None):

@@ -608,6 +608,128 @@ int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* works
   return ok();
 }
 
+// ---------------------------------------------------------------- chunked prefill
+struct PrefillPlan {
+  tq::Geom g, gv;          // cache geometry; virtual batch B * n
+  int splits = 1, nslots = 2;
+  bool mma = false;
+  tq::DecodeWs ws{};
+};
+
+static int prefill_splits(const tq_cache* c, const tq::Geom& g, int G, int n, bool mma,
+                          int num_splits, int64_t n_comp) {
+  const int64_t nblk = (n_comp + tq::kBlockTokens - 1) / tq::kBlockTokens;
+  int s = num_splits > 0 ? num_splits : tq::prefill_auto_splits(g, G, n_comp, n, mma);
+  (void)c;
+  if (nblk == 0) return 1;
+  if (s > nblk) s = (int)nblk;
+  const int64_t bps = (nblk + s - 1) / s;
+  return (int)((nblk + bps - 1) / bps);
+}
+
+static int prefill_common(const tq_cache* c, int Hq, int n, int num_splits, const char* name) {
+  int st = check_decode_common(c, Hq, num_splits);
+  if (st != TQ_OK) return st;
+  if (n < 1 || n > 65535) return fail(TQ_ERR_INVALID_ARG, "%s: n=%d (1..65535)", name, n);
+  if ((int64_t)c->desc.B * n > (int64_t)1 << 24)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: B * n = %lld query tokens", name, (long long)c->desc.B * n);
+  return TQ_OK;
+}
+
+static tq::Geom virtual_geom(const tq_cache* c, int n) {
+  tq::Geom gv = tq::geom_of(c);
+  gv.B = c->desc.B * n;
+  return gv;
+}
+
+size_t tq_prefill_workspace_bytes(const tq_cache* c, int Hq, int n, int num_splits) {
+  if (prefill_common(c, Hq, n, num_splits, "tq_prefill_workspace_bytes") != TQ_OK) return 0;
+  const tq::Geom g = tq::geom_of(c);
+  const int G = Hq / c->desc.Hkv;
+  const bool mma = tq::prefill_mma_supported(g, G);
+  // the split count at full capacity bounds the one any later length needs
+  const int s = prefill_splits(c, g, G, n, mma, num_splits, c->desc.capacity);
+  const int smax = num_splits > 0 ? num_splits : s;
+  return tq::decode_ws_bytes(virtual_geom(c, n), Hq, smax + 1);
+}
+
+static int prefill_plan(const tq_cache* c, const void* Q, int Hq, int n, const void* K,
+                        const void* V, float softmax_scale, const float* Pi, const float* S,
+                        const float* centroids, void* out, int num_splits, void* workspace,
+                        size_t ws_bytes, const char* name, PrefillPlan& P) {
+  int st = prefill_common(c, Hq, n, num_splits, name);
+  if (st != TQ_OK) return st;
+  const tq_cache_desc& dsc = c->desc;
+  P.g = tq::geom_of(c);
+  P.gv = virtual_geom(c, n);
+  const int G = Hq / dsc.Hkv;
+  P.mma = tq::prefill_mma_supported(P.g, G);
+  if (!P.mma && (int64_t)P.gv.B * dsc.Hkv > 65535)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: B * n * Hkv = %lld above 65535 on this shape's path", name,
+                (long long)P.gv.B * dsc.Hkv);
+  P.splits = prefill_splits(c, P.g, G, n, P.mma, num_splits, n_comp_of(c));
+  P.nslots = P.splits + 1;
+  const size_t need = tq::decode_ws_bytes(P.gv, Hq, P.nslots);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need)
+    return fail(TQ_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed", name, need);
+  if (!Q || !K || !V || !out || !S || !aligned16(S) || (dsc.b1 > 0 && (!Pi || !aligned16(Pi))))
+    return fail(TQ_ERR_INVALID_ARG, "%s: Q, K, V, out, S (and Pi when b1>0) needed", name);
+  if (!std::isfinite(softmax_scale)) return fail(TQ_ERR_INVALID_ARG, "%s: softmax_scale", name);
+  if (dsc.b1 > 0 && !centroids) return fail(TQ_ERR_INVALID_ARG, "%s: centroids needed", name);
+  P.ws = tq::decode_ws_carve(workspace, P.gv, Hq, P.nslots);
+  return TQ_OK;
+}
+
+int tq_prefill_attention(const tq_cache* c, const void* Q, int Hq, int n, const void* K,
+                         const void* V, float softmax_scale, const float* Pi, const float* S,
+                         const float* centroids, void* out, int num_splits, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  TQ_FAULT_POINT("tq_prefill_attention");
+  PrefillPlan P;
+  int st = prefill_plan(c, Q, Hq, n, K, V, softmax_scale, Pi, S, centroids, out, num_splits,
+                        workspace, ws_bytes, "tq_prefill_attention", P);
+  if (st != TQ_OK) return st;
+  st = check_pending("tq_prefill_attention");
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* base = static_cast<const uint8_t*>(c->base);
+  cudaError_t e = P.mma ? tq::launch_decode_prep_mma(P.gv, Q, Hq, Pi, S, centroids, softmax_scale,
+                                                     P.ws, s)
+                        : tq::launch_decode_prep(P.gv, Q, Hq, Pi, S, P.ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: prepare");
+  e = P.mma ? tq::launch_prefill_partial_mma(P.g, base, c->n_total, Hq, n, P.splits, P.nslots, P.ws, s)
+            : tq::launch_decode_partial(P.gv, base, c->n_total, Hq, softmax_scale, centroids, nullptr,
+                                        P.splits, P.ws, s, n, P.nslots, false);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: history");
+  e = tq::launch_prefill_exact(P.g, base, c->n_total, Hq, n, K, V, softmax_scale, P.nslots,
+                               P.splits, P.ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: exact segment");
+  e = tq::launch_decode_combine(P.gv, Hq, out, P.nslots, P.ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: combine");
+  return ok();
+}
+
+int tq_prefill_check(const tq_cache* c, int Hq, int n, int num_splits, const void* workspace,
+                     size_t ws_bytes, void* stream) {
+  int st = prefill_common(c, Hq, n, num_splits, "tq_prefill_check");
+  if (st != TQ_OK) return st;
+  const tq::Geom g = tq::geom_of(c);
+  const tq::Geom gv = virtual_geom(c, n);
+  const int G = Hq / c->desc.Hkv;
+  const int splits = prefill_splits(c, g, G, n, tq::prefill_mma_supported(g, G), num_splits,
+                                    n_comp_of(c));
+  if (!workspace || ws_bytes < tq::decode_ws_bytes(gv, Hq, splits + 1))
+    return fail(TQ_ERR_INVALID_ARG, "tq_prefill_check: workspace too small");
+  tq::DecodeWs ws = tq::decode_ws_carve(const_cast<void*>(workspace), gv, Hq, splits + 1);
+  int flag = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&flag, ws.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_check");
+  if (flag) return fail(TQ_ERR_CUDA, "prefill: a staged load did not complete within its wait limit");
+  return ok();
+}
+
 int tq_quantize_check(void* stream) {
   int flag = 0;
   cudaError_t e = tq::quantize_error_flag(&flag, static_cast<cudaStream_t>(stream));

@@ -28,6 +28,8 @@ struct DParams {
   float* logits;
   int64_t n_log;
   int splits, bps;
+  int qdiv;      // virtual batches per cache batch (query tokens of a chunk; 1 for a decode)
+  int nslots;    // partial slots per (batch, query head); the split index is the slot
   DecodeWs ws;
 };
 
@@ -73,7 +75,7 @@ __global__ void __launch_bounds__(DT) k_decode_partial(DParams p) {
   const int64_t nblk = (p.n_comp + kBlockTokens - 1) / kBlockTokens;
   const int64_t blk0 = (int64_t)split * p.bps;
   const int64_t blk1 = min(nblk, blk0 + p.bps);
-  const uint8_t* region = p.base + (int64_t)bh * g.region_bytes;
+  const uint8_t* region = p.base + (int64_t)((b / p.qdiv) * g.Hkv + h) * g.region_bytes;
   const int vmask = (1 << g.vbits) - 1;
   const int ng = d / g.group;
 
@@ -227,11 +229,11 @@ __global__ void __launch_bounds__(DT) k_decode_partial(DParams p) {
 
   for (int k = 0; k < kMaxG; ++k) {
     const int hh = hs + k * nhs;
-    if (hh < G) p.ws.part_o[((int64_t)(bq0 + hh) * p.splits + split) * d + ch] = acc[k];
+    if (hh < G) p.ws.part_o[((int64_t)(bq0 + hh) * p.nslots + split) * d + ch] = acc[k];
   }
   if (tid < G) {
-    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 0] = sM[tid];
-    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 1] = sLs[tid];
+    p.ws.part_ml[((int64_t)(bq0 + tid) * p.nslots + split) * 2 + 0] = sM[tid];
+    p.ws.part_ml[((int64_t)(bq0 + tid) * p.nslots + split) * 2 + 1] = sLs[tid];
   }
 }
 
@@ -360,13 +362,16 @@ cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float
 
 cudaError_t launch_decode_partial(const Geom& g, const uint8_t* base, int64_t n_total,
                                   int Hq, float scale, const float* cent, float* logits,
-                                  int splits, const DecodeWs& ws, cudaStream_t s) {
+                                  int splits, const DecodeWs& ws, cudaStream_t s, int qdiv,
+                                  int nslots, bool with_ring) {
   DParams p{};
   p.g = g;
   p.base = base;
   p.n_total = n_total;
   p.n_comp = n_total > g.W ? n_total - g.W : 0;
-  p.n_ring = (int)(n_total < g.W ? n_total : g.W);
+  p.n_ring = with_ring ? (int)(n_total < g.W ? n_total : g.W) : 0;
+  p.qdiv = qdiv;
+  p.nslots = nslots > 0 ? nslots : splits;
   p.Hq = Hq;
   p.G = Hq / g.Hkv;
   p.scale_log2 = scale * kLog2e;

@@ -106,9 +106,24 @@ cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float
                                const float* S, const DecodeWs& ws, cudaStream_t s);
 cudaError_t launch_decode_partial(const Geom& g, const uint8_t* base, int64_t n_total,
                                   int Hq, float scale, const float* cent, float* logits,
-                                  int splits, const DecodeWs& ws, cudaStream_t s);
+                                  int splits, const DecodeWs& ws, cudaStream_t s, int qdiv = 1,
+                                  int nslots = 0, bool with_ring = true);
 cudaError_t launch_decode_combine(const Geom& g, int Hq, void* out, int splits,
                                   const DecodeWs& ws, cudaStream_t s);
+
+// ---- multi-token (chunked prefill) attention (prefill_mma.cu) ----
+// The chunk's n query tokens are a virtual batch of B * n decode queries; the
+// history partials take slots 0..splits-1 of splits + 1, the exact segment (ring +
+// chunk tokens 0..i) the last slot, and the decode combine merges them.
+bool prefill_mma_supported(const Geom& g, int G);
+int prefill_mma_warps(const Geom& g, int nq);
+int prefill_auto_splits(const Geom& g, int G, int64_t n_comp, int nq, bool mma);
+cudaError_t launch_prefill_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
+                                       int nq, int splits, int nslots, const DecodeWs& ws,
+                                       cudaStream_t s);
+cudaError_t launch_prefill_exact(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
+                                 int nq, const void* K, const void* V, float scale, int nslots,
+                                 int slot, const DecodeWs& ws, cudaStream_t s);
 
 // Launch with programmatic stream serialisation (programmatic dependent launch):
 // the kernel may begin once the previous kernel of the stream has let its

@@ -87,6 +87,9 @@ def _load() -> ctypes.CDLL:
         "tq_decode_partial": (I, [C, I, F, P, P, P, I, P, SZ, P]),
         "tq_decode_combine": (I, [C, I, P, I, P, SZ, P]),
         "tq_decode_step": (I, [C, P, P, I64, P, I, F, P, P, P, P, P, P, P, I, P, SZ, P]),
+        "tq_prefill_workspace_bytes": (SZ, [C, I, I, I]),
+        "tq_prefill_attention": (I, [C, P, I, I, P, P, F, P, P, P, P, I, P, SZ, P]),
+        "tq_prefill_check": (I, [C, I, I, I, P, SZ, P]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
         "tq_m_for_layer": (I, [ctypes.POINTER(tq_layer_groups), I]),
     }
@@ -226,6 +229,25 @@ def tq_decode_prep(cache: tq_cache, Q, softmax_scale, Pi, S, centroids, num_spli
     _check(lib.tq_decode_prep(ctypes.byref(cache), _ptr(Q), Q.shape[1], softmax_scale, _ptr(Pi),
                               _ptr(S), _ptr(centroids), num_splits, _ptr(workspace),
                               _ws(workspace), _stream(stream)), "tq_decode_prep")
+
+
+def tq_prefill_workspace_bytes(cache: tq_cache, Hq: int, n: int, num_splits: int = 0) -> int:
+    return lib.tq_prefill_workspace_bytes(ctypes.byref(cache), Hq, n, num_splits)
+
+
+def tq_prefill_attention(cache: tq_cache, Q, K, V, softmax_scale: float, Pi, S, centroids, out,
+                         num_splits: int = 0, workspace=None, stream=None):
+    """Q [B, n, Hq, d]; K, V [B, Hkv, n, d]; out [B, n, Hq, d]."""
+    n, Hq = Q.shape[1], Q.shape[2]
+    _check(lib.tq_prefill_attention(ctypes.byref(cache), _ptr(Q), Hq, n, _ptr(K), _ptr(V),
+                                    softmax_scale, _ptr(Pi), _ptr(S), _ptr(centroids), _ptr(out),
+                                    num_splits, _ptr(workspace), _ws(workspace), _stream(stream)),
+           "tq_prefill_attention")
+
+
+def tq_prefill_check(cache: tq_cache, Hq, n, num_splits, workspace, stream=None):
+    _check(lib.tq_prefill_check(ctypes.byref(cache), Hq, n, num_splits, _ptr(workspace),
+                                _ws(workspace), _stream(stream)), "tq_prefill_check")
 
 
 def tq_quantize_check(stream=None):

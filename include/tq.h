@@ -345,6 +345,44 @@ int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* works
                     size_t ws_bytes, void* stream);
 
 /*
+ * tq_prefill_attention -- multi-token (chunked prefill) attention: the n new
+ * tokens of a chunk attend to the cache BEFORE the chunk is appended.  The pages
+ * define the single-token fused decode ([TQ] 六) and note that their hybrid path
+ * dequantises the history for everything else ([TQ] 七); this call scores the
+ * history on the packed cache with the same estimator instead.  Query i (0-based)
+ * of the chunk sees
+ *   - the compressed history: the tq_decode_attention logit and v = mn + code * s,
+ *   - the ring tokens: exact <q, k> and v,
+ *   - the chunk's own tokens 0..i: exact <q, k> and v from K, V (causal),
+ * with p = softmax(softmax_scale * logits) and out = sum_t p_t v_t.  The cache is
+ * not modified: append the chunk afterwards with tq_append(c, K, V, n, ...).
+ *   Q        device [B, n, Hq, d] of desc.dtype (token-major)
+ *   K, V     device [B, Hkv, n, d] of desc.dtype (the layout tq_append takes)
+ *   Pi, S, centroids  as for tq_decode_attention
+ *   out      device [B, n, Hq, d] of desc.dtype (written)
+ *   num_splits  partitions of the history (0 = automatic)
+ *   workspace   device, tq_prefill_workspace_bytes(c, Hq, n, num_splits) bytes;
+ *               it may be reused once the call's stream work has completed
+ * Four launches: query preparation (per query token, as a decode), history
+ * partials (tensor cores for head dim 128, G = 4, 2-bit values in groups of 32,
+ * b1 <= 2; CUDA cores otherwise), the exact segment, and the split merge.
+ * Errors: INVALID_ARG (null pointers, n outside 1..65535, small workspace),
+ * UNSUPPORTED (head mapping, B * n above 2^24), CUDA.
+ */
+size_t tq_prefill_workspace_bytes(const tq_cache* c, int Hq, int n, int num_splits);
+int tq_prefill_attention(const tq_cache* c, const void* Q, int Hq, int n, const void* K,
+                         const void* V, float softmax_scale, const float* Pi, const float* S,
+                         const float* centroids, void* out, int num_splits, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/*
+ * tq_prefill_check -- SYNCHRONOUS: as tq_decode_check, for the last
+ * tq_prefill_attention that used `workspace` (same c, Hq, n, num_splits).
+ */
+int tq_prefill_check(const tq_cache* c, int Hq, int n, int num_splits, const void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/*
  * tq_quantize_check -- SYNCHRONOUS: waits for `stream`, then reports (and
  * clears) the sticky device flag of the batched tensor-core key quantisation
  * (tq_quantize_keys and tq_append with more than 8 tokens, head dim 128,

@@ -178,3 +178,13 @@ def decode_stream(w: Workload, n_steps: int, layer: int = 0, device="cpu"):
     g = _generator(w.seed, 1000 + layer, TENSOR_Q, device)
     Q = torch.randn(n_steps, w.B, w.Hq, w.d, generator=g, device=device).to(w.torch_dtype)
     return Q, Kn, Vn
+
+
+def prefill_chunk(w: Workload, n: int, layer: int = 0, device="cpu"):
+    """Inputs of a chunk of n new tokens scored against the cache: Q [B, n, Hq, d]
+    (token-major) and K, V [B, Hkv, n, d], with the workload's distributions (drawn
+    under layer id ``2000 + layer``)."""
+    K, V = keys_values(w.scaled(T=n), layer=2000 + layer, device=device)
+    g = _generator(w.seed, 2000 + layer, TENSOR_Q, device)
+    Q = torch.randn(w.B, n, w.Hq, w.d, generator=g, device=device).to(w.torch_dtype)
+    return Q, K, V

@@ -163,3 +163,36 @@ def test_layer_groups_from_page_config(nat):
             nat.tq_layer_groups_parse(*bad)
     one = nat.tq_layer_groups_parse("", "256")
     assert nat.tq_m_for_layer(one, 7) == 256
+
+
+def test_prefill_checks(nat):
+    c = _fake_cache(nat)
+    c.n_total = 90
+    L = nat.lib
+    n = 5
+    need = L.tq_prefill_workspace_bytes(ctypes.byref(c), 8, n, 0)
+    assert need > 0
+    assert L.tq_prefill_workspace_bytes(ctypes.byref(c), 7, n, 0) == 0      # Hq % Hkv
+    assert L.tq_prefill_workspace_bytes(ctypes.byref(c), 8, 0, 0) == 0      # empty chunk
+    # more query tokens need more workspace (a virtual batch of B * n queries)
+    assert L.tq_prefill_workspace_bytes(ctypes.byref(c), 8, 2 * n, 0) > need
+
+    def call(Q=FAKE, Hq=8, nn=n, K=FAKE, V=FAKE, scale=0.1, Pi=FAKE, S=FAKE, cent=FAKE, out=FAKE,
+             splits=0, ws=FAKE, wsb=need):
+        return L.tq_prefill_attention(ctypes.byref(c), Q, Hq, nn, K, V, scale, Pi, S, cent, out,
+                                      splits, ws, wsb, None)
+
+    assert call(Hq=7) == nat.TQ_ERR_UNSUPPORTED
+    assert call(nn=0) == nat.TQ_ERR_INVALID_ARG
+    assert call(nn=70000) == nat.TQ_ERR_INVALID_ARG
+    assert call(wsb=64) == nat.TQ_ERR_INVALID_ARG
+    assert call(Q=None) == nat.TQ_ERR_INVALID_ARG
+    assert call(K=None) == nat.TQ_ERR_INVALID_ARG
+    assert call(V=None) == nat.TQ_ERR_INVALID_ARG
+    assert call(out=None) == nat.TQ_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == nat.TQ_ERR_INVALID_ARG
+    assert call(splits=-1) == nat.TQ_ERR_INVALID_ARG
+    # the workspace sized at the current length covers every later length
+    for t in (0, 1, 16, 17, 80, 116):
+        c.n_total = t
+        assert L.tq_prefill_workspace_bytes(ctypes.byref(c), 8, n, 0) == need
