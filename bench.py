@@ -57,6 +57,16 @@ def parse_args():
     return ap.parse_args()
 
 
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak (burst) in TFLOP/s: measured, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -587,6 +597,13 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
     wsd = cache.workspace(w.Hq, 0)
     t_dec = timed(lambda: native.tq_decode_attention(cache.state, Qd, scale, pj.Pi, pj.S, cent,
                                                      outd, None, 0, wsd))
+    # executed tensor work of the history partial per (history token, query token, KV
+    # head): int8 score MMAs (KS k-steps of 32 features x 4 heads x 4 slices) and f16
+    # P V MMAs (128 channels x 4 heads x hi/lo); int8 taken at twice the bf16 peak
+    F = (1 << (w.b1 - 1)) if w.b1 > 0 else 0
+    KS = F * w.d // 32 + w.m // 32
+    bf16, bf16_kind = measured_bf16_tflops()
+    units = w.B * w.Hkv
     res = []
     for n in chunks:
         Q, Kc, Vc = synth.prefill_chunk(w, n, device=dev)
@@ -597,9 +614,16 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
                                                       cent, out, 0, ws))
         native.tq_prefill_check(cache.state, w.Hq, n, 0, ws)
         toks = reduce_sum(float(w.B * n), world)
+        work = float(cache.n_comp) * units * n
+        i8_ops, f16_ops = work * 16 * 32 * KS * 2, work * 128 * 8 * 2
+        ideal_ms = (i8_ops / (2 * bf16 * 1e12) + f16_ops / (bf16 * 1e12)) * 1e3
         res.append({"n": n, "ms": t, "query_tokens_per_s": toks / (t * 1e-3),
                     "history_GB_per_s": reduce_sum(float(hist_bytes), world) / (t * 1e-3) / 1e9,
-                    "vs_n_decodes": n * t_dec / t})
+                    "vs_n_decodes": n * t_dec / t,
+                    "tensor": {"bound": "tensor", "int8_tops": i8_ops / (t * 1e-3) / 1e12,
+                               "f16_tflops": f16_ops / (t * 1e-3) / 1e12,
+                               "ideal_ms_at_peak": ideal_ms, "frac": ideal_ms / t,
+                               "peak_bf16_tflops": bf16, "peak_kind": bf16_kind}})
     return {"chunks": res, "decode_ms": t_dec, "history_bytes": hist_bytes,
             "timing": "CUDA events around the whole call (prep, history partials, exact segment, "
                       "merge), L2 flushed before each call, 20 calls after 3 warm-up calls"}

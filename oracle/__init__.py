@@ -18,7 +18,8 @@ projections and value metadata), no blocking, fusion or reordering.  Sources:
 
 Modules: ``philox`` (counter-based generator), ``projections`` (Pi, S),
 ``codebook`` (Lloyd-Max), ``quantize`` (keys, values), ``layout`` (packed
-byte format), ``attention`` (logits, decode, chunk prefill), ``cache`` (append + ring).
+byte format), ``attention`` (logits, decode, chunk prefill), ``cache`` (append + ring),
+``sensitivity`` (A-QJL layer groups and sketch dims from key variance).
 
 Every function here is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_*.py``; no function is "parity unpinned".
