@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--no-quantize", action="store_true")
     ap.add_argument("--no-other-decodes", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sensitivity", action="store_true")
     ap.add_argument("--workload", default="gqa32k")
     return ap.parse_args()
 
@@ -520,6 +521,9 @@ def run_ours(args):
     quant = None
     if not args.no_quantize:
         quant = bench_quantize(dev, world)
+    sensitivity = None
+    if not args.no_sensitivity:
+        sensitivity = bench_sensitivity(dev, world, peak, flush_l2)
     others = None
     if not args.no_other_decodes:
         del cache, Qs, Kn, Vn
@@ -552,6 +556,7 @@ def run_ours(args):
         "e2e": e2e,
         "quantize": quant,
         "prefill": prefill,
+        "sensitivity": sensitivity,
         "other_decodes": others,
         "cpu_baseline": cpu,
         "clocks": clk,
@@ -627,6 +632,46 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
     return {"chunks": res, "decode_ms": t_dec, "history_bytes": hist_bytes,
             "timing": "CUDA events around the whole call (prep, history partials, exact segment, "
                       "merge), L2 flushed before each call, 20 calls after 3 warm-up calls"}
+
+
+def bench_sensitivity(dev, world, peak, flush_l2, reps=10, warm=3):
+    """Key moments (tq_key_moments) of one layer of calibration keys shaped like the
+    A-QJL workload (batch 16, 8 KV heads, 8192 tokens, d=128, fp16: 268 MB, above
+    L2), L2 flushed before each pass; then the host profile of 32 layers."""
+    import time
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import LayerGroups, native
+    w = synth.WORKLOADS["aqjl"].scaled(T=8192)
+    K, V = synth.keys_values(w, layer=5, device=dev)
+    del V
+    out = torch.empty(2, dtype=torch.float64, device=dev)
+    ws = torch.empty(native.tq_key_moments_workspace_bytes(), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warm):
+        flush_l2()
+        native.tq_key_moments(K, out, ws)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for k in range(reps):
+        flush_l2()
+        ev[k][0].record(stream)
+        native.tq_key_moments(K, out, ws)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    t = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ev) / reps, world)
+    nbytes = K.numel() * K.element_size()
+    gbs = nbytes / (t * 1e-3) / 1e9
+    var = [1.0 + 2.0 * l / 31 for l in range(32)]
+    h0 = time.perf_counter()
+    lg = LayerGroups.from_variances(var, 4, 336)
+    host_ms = (time.perf_counter() - h0) * 1e3
+    del K
+    torch.cuda.empty_cache()
+    return {"keys_bytes": nbytes, "moments_ms": t, "GB_per_s": reduce_sum(gbs, world),
+            "roofline": {"bound": "hbm", "kernel": "k_key_moments", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak},
+            "host_profile_ms_32_layers": host_ms,
+            "profile_of_variance_ramp": {"boundaries": lg.boundaries, "sketch_dims": lg.sketch_dims}}
 
 
 def _time_decode(w, layer, dev, reps=10, warm=3):

@@ -68,8 +68,37 @@ class LayerGroups:
     def __init__(self, boundaries: str, sketch_dims: str):
         self._g = native.tq_layer_groups_parse(boundaries, sketch_dims)
 
+    @classmethod
+    def from_variances(cls, layer_var, num_groups: int, m_avg: int, m_min: int = 32,
+                       m_max: int = 1024) -> "LayerGroups":
+        """Sensitivity profile: groups and sketch dims from per-layer key variances."""
+        obj = cls.__new__(cls)
+        obj._g = native.tq_sensitivity_profile(layer_var, num_groups, m_avg, m_min, m_max)
+        return obj
+
+    @property
+    def boundaries(self):
+        return [int(self._g.bound[i]) for i in range(self._g.n - 1)]
+
+    @property
+    def sketch_dims(self):
+        return [int(self._g.m[i]) for i in range(self._g.n)]
+
     def m_for_layer(self, layer: int) -> int:
         return native.tq_m_for_layer(self._g, layer)
+
+
+def key_variance(K: torch.Tensor, workspace: Optional[torch.Tensor] = None) -> float:
+    """Population variance of every entry of one layer's calibration keys (device
+    moments, one streaming pass; waits for the result)."""
+    out = torch.empty(2, dtype=torch.float64, device=K.device)
+    if workspace is None:
+        workspace = torch.empty(native.tq_key_moments_workspace_bytes(), dtype=torch.uint8,
+                                device=K.device)
+    native.tq_key_moments(K, out, workspace)
+    s1, s2 = out.tolist()
+    n = K.numel()
+    return s2 / n - (s1 / n) ** 2
 
 
 class CompressedKVCache:

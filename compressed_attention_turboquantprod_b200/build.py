@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "libtq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
-         "-Xcompiler", "-fPIC", "-Xcompiler", "-O3", "-shared"]
+         "-Xcompiler", "-fPIC", "-Xcompiler", "-O3", "-Xcompiler", "-ffp-contract=off", "-shared"]
 
 
 def nvcc() -> str:

@@ -760,6 +760,48 @@ static int parse_list(const char* s, int* out, int max_n) {
   return n;
 }
 
+size_t tq_key_moments_workspace_bytes(void) { return tq::key_moments_ws_bytes(); }
+
+int tq_key_moments(const void* K, int dtype, int64_t n, double* out, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  TQ_FAULT_POINT("tq_key_moments");
+  if (!K || !out || !aligned16(K)) return fail(TQ_ERR_INVALID_ARG, "tq_key_moments: K (16-byte aligned) and out needed");
+  if (n < 1) return fail(TQ_ERR_INVALID_ARG, "tq_key_moments: n=%lld", (long long)n);
+  if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16)
+    return fail(TQ_ERR_INVALID_ARG, "tq_key_moments: dtype %d", dtype);
+  if (!workspace || !aligned16(workspace) || ws_bytes < tq::key_moments_ws_bytes())
+    return fail(TQ_ERR_INVALID_ARG, "tq_key_moments: workspace of %zu bytes needed",
+                tq::key_moments_ws_bytes());
+  int st = check_pending("tq_key_moments");
+  if (st != TQ_OK) return st;
+  cudaError_t e = tq::launch_key_moments(K, dtype, n, out, static_cast<double*>(workspace),
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_key_moments");
+  return ok();
+}
+
+int tq_sensitivity_profile(const double* layer_var, int L, int num_groups, int m_avg, int m_min,
+                           int m_max, tq_layer_groups* out) {
+  if (!layer_var || !out) return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: null argument");
+  if (L < 1 || num_groups < 1 || num_groups > 8 || num_groups > L)
+    return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: L=%d num_groups=%d (1..min(8, L))", L,
+                num_groups);
+  if (!valid_m(m_min) || !valid_m(m_max) || m_min > m_max)
+    return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: m range [%d, %d]", m_min, m_max);
+  if (m_avg < m_min) return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: m_avg=%d below m_min", m_avg);
+  for (int i = 0; i < L; ++i)
+    if (!std::isfinite(layer_var[i]) || layer_var[i] < 0.0)
+      return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: variance of layer %d", i);
+  tq_layer_groups g;
+  std::memset(&g, 0, sizeof(g));
+  tq::sensitivity_segment(layer_var, L, num_groups, g.bound);
+  if (tq::sensitivity_allocate(layer_var, L, g.bound, num_groups, m_avg, m_min, m_max, g.m) != 0)
+    return fail(TQ_ERR_INVALID_ARG, "tq_sensitivity_profile: budget below m_min");
+  g.n = num_groups;
+  *out = g;
+  return ok();
+}
+
 int tq_layer_groups_parse(const char* boundaries, const char* sketch_dims, tq_layer_groups* out) {
   if (!boundaries || !sketch_dims || !out) return fail(TQ_ERR_INVALID_ARG, "null argument");
   tq_layer_groups g;

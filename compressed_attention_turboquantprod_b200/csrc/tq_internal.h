@@ -125,6 +125,14 @@ cudaError_t launch_prefill_exact(const Geom& g, const uint8_t* base, int64_t n_t
                                  int nq, const void* K, const void* V, float scale, int nslots,
                                  int slot, const DecodeWs& ws, cudaStream_t s);
 
+// ---- sensitivity profile (sensitivity.cu) ----
+size_t key_moments_ws_bytes();
+cudaError_t launch_key_moments(const void* K, int dtype, int64_t n, double* out, double* part,
+                               cudaStream_t s);
+void sensitivity_segment(const double* var, int L, int k, int* bounds);
+int sensitivity_allocate(const double* var, int L, const int* bounds, int k, int m_avg, int m_min,
+                         int m_max, int* m);
+
 // Launch with programmatic stream serialisation (programmatic dependent launch):
 // the kernel may begin once the previous kernel of the stream has let its
 // dependents launch (griddepcontrol.launch_dependents) instead of after that

@@ -90,6 +90,10 @@ def _load() -> ctypes.CDLL:
         "tq_prefill_workspace_bytes": (SZ, [C, I, I, I]),
         "tq_prefill_attention": (I, [C, P, I, I, P, P, F, P, P, P, P, I, P, SZ, P]),
         "tq_prefill_check": (I, [C, I, I, I, P, SZ, P]),
+        "tq_key_moments_workspace_bytes": (SZ, []),
+        "tq_key_moments": (I, [P, I, I64, P, P, SZ, P]),
+        "tq_sensitivity_profile": (I, [ctypes.POINTER(ctypes.c_double), I, I, I, I, I,
+                                       ctypes.POINTER(tq_layer_groups)]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
         "tq_m_for_layer": (I, [ctypes.POINTER(tq_layer_groups), I]),
     }
@@ -286,6 +290,26 @@ def tq_layer_groups_parse(boundaries: str, sketch_dims: str) -> tq_layer_groups:
     g = tq_layer_groups()
     _check(lib.tq_layer_groups_parse(boundaries.encode(), sketch_dims.encode(), ctypes.byref(g)),
            "tq_layer_groups_parse")
+    return g
+
+
+def tq_key_moments_workspace_bytes() -> int:
+    return lib.tq_key_moments_workspace_bytes()
+
+
+def tq_key_moments(K, out, workspace, stream=None):
+    """out (device float64[2]) = sum and sum of squares of every entry of K."""
+    _check(lib.tq_key_moments(_ptr(K), dtype_code(K.dtype), K.numel(), _ptr(out), _ptr(workspace),
+                              _ws(workspace), _stream(stream)), "tq_key_moments")
+
+
+def tq_sensitivity_profile(layer_var, num_groups: int, m_avg: int, m_min: int = 32,
+                           m_max: int = 1024) -> tq_layer_groups:
+    L = len(layer_var)
+    arr = (ctypes.c_double * L)(*[float(x) for x in layer_var])
+    g = tq_layer_groups()
+    _check(lib.tq_sensitivity_profile(arr, L, num_groups, m_avg, m_min, m_max, ctypes.byref(g)),
+           "tq_sensitivity_profile")
     return g
 
 

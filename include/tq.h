@@ -442,6 +442,38 @@ int tq_layer_groups_parse(const char* boundaries, const char* sketch_dims, tq_la
 /* Sketch dim of `layer`: m of the group containing it (-1 if g is invalid). */
 int tq_m_for_layer(const tq_layer_groups* g, int layer);
 
+/*
+ * Sensitivity profile ([AQJL] sensitivity analyser: each layer's key variance
+ * on calibration data decides the layer groups and their bit allocation; the
+ * pages give no formula, the steps below are this library's reading).
+ *
+ * tq_key_moments -- out[0] = sum and out[1] = sum of squares of the n entries of
+ * K (device, dtype TQ_F32 / TQ_F16 / TQ_BF16, 16-byte aligned), one streaming
+ * pass; the layer's variance is out[1] / n - (out[0] / n)^2.  `out` is a device
+ * double[2]; `workspace` device, tq_key_moments_workspace_bytes() bytes.  The
+ * result does not depend on scheduling (fixed-order reductions).
+ * Errors: INVALID_ARG, CUDA.
+ */
+size_t tq_key_moments_workspace_bytes(void);
+int tq_key_moments(const void* K, int dtype, int64_t n, double* out, void* workspace,
+                   size_t ws_bytes, void* stream);
+
+/*
+ * tq_sensitivity_profile -- host only.  From the per-layer key variances
+ * layer_var[0..L-1] (host), the A-QJL layer groups: num_groups (1..8, <= L)
+ * contiguous groups whose boundaries minimise the summed squared deviation of
+ * the variances from their group means (ties: smallest boundaries first), and
+ * per-group sketch dims, multiples of 32 in [m_min, m_max], minimising
+ * sum_g n_g s_g / m_g (n_g layers, mean variance s_g; the QJL term's variance
+ * is proportional to |k|^2 / m, [TQ] 四) under the sign-bit budget
+ * sum_g n_g m_g <= L * m_avg (greedy 32-steps, largest decrease per bit first,
+ * ties: lower group).  Writes `out` in the form tq_layer_groups_parse gives.
+ * Errors: INVALID_ARG (sizes, m range, negative or non-finite variance, budget
+ * below L * m_min).
+ */
+int tq_sensitivity_profile(const double* layer_var, int L, int num_groups, int m_avg, int m_min,
+                           int m_max, tq_layer_groups* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,6 +29,15 @@ import numpy as np
 STEP = 32
 
 
+def _mean(xs) -> float:
+    """Sequential float64 mean (a fixed summation order: the group decisions below
+    are integers decided by these sums)."""
+    t = 0.0
+    for x in xs:
+        t += float(x)
+    return t / len(xs)
+
+
 def key_variance(K) -> float:
     """Population variance of every entry of one layer's keys, float64."""
     x = np.asarray(K, dtype=np.float64).ravel()
@@ -45,9 +54,12 @@ def segment_layers(var, num_groups: int):
     if not 1 <= num_groups <= L:
         raise ValueError("need 1 <= num_groups <= number of layers")
 
-    def sse(a, b):          # layers a..b-1
-        seg = v[a:b]
-        return float(((seg - seg.mean()) ** 2).sum())
+    def sse(a, b):          # layers a..b-1, sequential float64 sums
+        mu = _mean(v[a:b])
+        t = 0.0
+        for x in v[a:b]:
+            t += (float(x) - mu) * (float(x) - mu)
+        return t
 
     INF = float("inf")
     # best[g][l]: minimal cost of the first l layers in g groups, with its boundaries
@@ -74,7 +86,7 @@ def allocate_sketch_dims(var, bounds, m_avg: int, m_min: int = 32, m_max: int = 
     L = v.size
     edges = [0] + list(bounds) + [L]
     n = [edges[i + 1] - edges[i] for i in range(len(edges) - 1)]
-    s = [float(v[edges[i]:edges[i + 1]].mean()) for i in range(len(n))]
+    s = [_mean(v[edges[i]:edges[i + 1]]) for i in range(len(n))]
     m = [m_min] * len(n)
     left = L * m_avg - sum(ng * m_min for ng in n)
     if left < 0:

@@ -196,3 +196,45 @@ def test_prefill_checks(nat):
     for t in (0, 1, 16, 17, 80, 116):
         c.n_total = t
         assert L.tq_prefill_workspace_bytes(ctypes.byref(c), 8, n, 0) == need
+
+
+def test_sensitivity_profile_equals_oracle(nat):
+    """Host-only call: the groups and sketch dims equal the oracle's exactly (both
+    take the integer decisions in sequential IEEE double sums)."""
+    import numpy as np
+    from oracle import sensitivity as sens
+    rng = np.random.default_rng(7)
+    for trial in range(120):
+        L = int(rng.integers(1, 33))
+        k = int(rng.integers(1, min(8, L) + 1))
+        kind = trial % 3
+        v = (rng.gamma(2.0, 1.0, size=L) if kind == 0 else
+             np.full(L, 1.5) if kind == 1 else 1 + 2 * np.arange(L) / max(L - 1, 1))
+        m_min = int(rng.choice([32, 64]))
+        m_max = int(rng.choice([256, 512, 1024]))
+        m_avg = int(rng.integers(m_min, m_max + 1))
+        b, m = sens.profile(v, k, m_avg, m_min, m_max)
+        g = nat.tq_sensitivity_profile(v, k, m_avg, m_min, m_max)
+        assert g.n == k
+        assert [g.bound[i] for i in range(k - 1)] == list(b)
+        assert [g.m[i] for i in range(k)] == list(m)
+        for layer in range(L):
+            gi = sum(1 for x in b if layer >= x)
+            assert nat.tq_m_for_layer(g, layer) == m[gi]
+
+
+def test_sensitivity_profile_checks(nat):
+    import numpy as np
+    v = np.linspace(1.0, 3.0, 32)
+    for args in ((v, 0, 256), (v, 9, 256), (v[:3], 4, 256), (v, 4, 16)):
+        with pytest.raises(nat.TQError):
+            nat.tq_sensitivity_profile(*args)
+    with pytest.raises(nat.TQError):
+        nat.tq_sensitivity_profile(v, 4, 256, 48, 512)           # m_min not a multiple of 32
+    with pytest.raises(nat.TQError):
+        nat.tq_sensitivity_profile(np.r_[v[:-1], -1.0], 4, 256)  # negative variance
+    L = nat.lib
+    assert L.tq_key_moments(None, 2, 10, FAKE, FAKE, 1 << 20, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_key_moments(FAKE, 2, 0, FAKE, FAKE, 1 << 20, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_key_moments(FAKE, 7, 10, FAKE, FAKE, 1 << 20, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_key_moments(FAKE, 2, 10, FAKE, FAKE, 8, None) == nat.TQ_ERR_INVALID_ARG

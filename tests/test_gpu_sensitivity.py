@@ -1,0 +1,50 @@
+"""GPU parity of the sensitivity profile's key moments against the oracle, and the
+profile of synthetic calibration layers (the A-QJL variance ramp)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_common import host
+from oracle import sensitivity as sens
+
+pytestmark = pytest.mark.gpu
+
+# fp32 sums of the entries of one 16-byte load, fp64 beyond: a few fp32 ulp at most
+VAR_REL = 1e-7
+
+
+@pytest.mark.parametrize("shape,dtype", [
+    ((2, 2, 257, 128), torch.bfloat16), ((3, 1, 1001, 64), torch.float16),
+    ((1, 4, 333, 128), torch.float32), ((1, 1, 1, 7), torch.bfloat16),
+    ((16, 8, 512, 128), torch.float16), ((1, 1, 5, 3), torch.float32),
+])
+def test_key_moments_match_oracle(shape, dtype):
+    from compressed_attention_turboquantprod_b200 import key_variance
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    K = (torch.randn(*shape, generator=g, device="cuda") * 1.7 + 0.3).to(dtype)
+    got = key_variance(K)
+    want = sens.key_variance(host(K))
+    assert abs(got - want) <= VAR_REL * want, (got, want)
+
+
+def test_profile_of_synthetic_calibration_layers():
+    """32 layers of synthetic calibration keys with variance 1 + 2 l / 31: the
+    device variances give the oracle's profile (boundaries 8, 16, 24), and the
+    library's host step equals the oracle's on the same variances."""
+    from compressed_attention_turboquantprod_b200 import LayerGroups, key_variance
+    w = synth.WORKLOADS["aqjl"].scaled(B=2, T=512)
+    gpu_v, ref_v = [], []
+    for layer in range(32):
+        K, _ = synth.keys_values(w, layer=layer, device="cuda")
+        gpu_v.append(key_variance(K))
+        ref_v.append(sens.key_variance(host(K)))
+    gpu_v, ref_v = np.array(gpu_v), np.array(ref_v)
+    assert np.all(np.abs(gpu_v - ref_v) <= VAR_REL * ref_v)
+    b_ref, m_ref = sens.profile(ref_v, 4, 336)
+    lg = LayerGroups.from_variances(gpu_v, 4, 336)
+    assert b_ref == [8, 16, 24]
+    assert lg.boundaries == b_ref and lg.sketch_dims == m_ref
+    b2, m2 = sens.profile(gpu_v, 4, 336)
+    assert lg.boundaries == b2 and lg.sketch_dims == m2
