@@ -616,11 +616,10 @@ struct PrefillPlan {
   tq::DecodeWs ws{};
 };
 
-static int prefill_splits(const tq_cache* c, const tq::Geom& g, int G, int n, bool mma,
-                          int num_splits, int64_t n_comp) {
+static int prefill_splits(const tq::Geom& g, int G, int n, bool mma, int num_splits,
+                          int64_t n_comp) {
   const int64_t nblk = (n_comp + tq::kBlockTokens - 1) / tq::kBlockTokens;
   int s = num_splits > 0 ? num_splits : tq::prefill_auto_splits(g, G, n_comp, n, mma);
-  (void)c;
   if (nblk == 0) return 1;
   if (s > nblk) s = (int)nblk;
   const int64_t bps = (nblk + s - 1) / s;
@@ -648,7 +647,7 @@ size_t tq_prefill_workspace_bytes(const tq_cache* c, int Hq, int n, int num_spli
   const int G = Hq / c->desc.Hkv;
   const bool mma = tq::prefill_mma_supported(g, G);
   // the split count at full capacity bounds the one any later length needs
-  const int s = prefill_splits(c, g, G, n, mma, num_splits, c->desc.capacity);
+  const int s = prefill_splits(g, G, n, mma, num_splits, c->desc.capacity);
   const int smax = num_splits > 0 ? num_splits : s;
   return tq::decode_ws_bytes(virtual_geom(c, n), Hq, smax + 1);
 }
@@ -667,7 +666,7 @@ static int prefill_plan(const tq_cache* c, const void* Q, int Hq, int n, const v
   if (!P.mma && (int64_t)P.gv.B * dsc.Hkv > 65535)
     return fail(TQ_ERR_UNSUPPORTED, "%s: B * n * Hkv = %lld above 65535 on this shape's path", name,
                 (long long)P.gv.B * dsc.Hkv);
-  P.splits = prefill_splits(c, P.g, G, n, P.mma, num_splits, n_comp_of(c));
+  P.splits = prefill_splits(P.g, G, n, P.mma, num_splits, n_comp_of(c));
   P.nslots = P.splits + 1;
   const size_t need = tq::decode_ws_bytes(P.gv, Hq, P.nslots);
   if (!workspace || !aligned16(workspace) || ws_bytes < need)
@@ -716,7 +715,7 @@ int tq_prefill_check(const tq_cache* c, int Hq, int n, int num_splits, const voi
   const tq::Geom g = tq::geom_of(c);
   const tq::Geom gv = virtual_geom(c, n);
   const int G = Hq / c->desc.Hkv;
-  const int splits = prefill_splits(c, g, G, n, tq::prefill_mma_supported(g, G), num_splits,
+  const int splits = prefill_splits(g, G, n, tq::prefill_mma_supported(g, G), num_splits,
                                     n_comp_of(c));
   if (!workspace || ws_bytes < tq::decode_ws_bytes(gv, Hq, splits + 1))
     return fail(TQ_ERR_INVALID_ARG, "tq_prefill_check: workspace too small");

@@ -12,7 +12,7 @@
 //       weights as four int8 slices; f16 P V MMAs over the token-pair value
 //       words), but every warp owns QG = 2 query tokens (2 x 4 heads) and walks
 //       all 64 tokens of every staged block, so one masked key operand serves two
-//       query tokens and one staged block serves up to 16 (8 warps).  Each warp's
+//       query tokens and one staged block serves up to 8 (4 warps).  Each warp's
 //       softmax state covers all tokens of the split, so its (m, l, o) go straight
 //       to the partial slots without a cross-warp merge.
 //   k_prefill_exact        the exact segment of every query (ring + chunk tokens
@@ -30,7 +30,11 @@ using namespace mmadec;
 
 constexpr int MD = 128;
 constexpr int QG = 2;            // query tokens per warp
-constexpr int PNW = 8;           // warps per CTA at most
+#ifndef TQ_PREFILL_WARPS
+#define TQ_PREFILL_WARPS 4
+#endif
+constexpr int PNW = TQ_PREFILL_WARPS;   // warps per CTA at most
+constexpr int kPrefillRegs = 232;       // registers per thread of the partial kernel (bound)
 constexpr int PNST = 4;          // staged blocks in flight
 constexpr int kPairBytes = 2 * MD * 2 / 8;   // value codes of a token pair (2-bit)
 
@@ -568,9 +572,16 @@ int prefill_auto_splits(const Geom& g, int G, int64_t n_comp, int nq, bool mma) 
     int64_t s = (148 * 4 + (int64_t)units * nq - 1) / ((int64_t)units * nq);
     return (int)max((int64_t)1, min(nblk, s));
   }
-  const int qpc = QG * prefill_mma_warps(g, nq);
+  const int nw = prefill_mma_warps(g, nq);
+  const int qpc = QG * nw;
   const int64_t base = (int64_t)units * ((nq + qpc - 1) / qpc);
-  const int slots = 148;                   // one CTA per SM (shared memory)
+  // resident CTAs per SM: registers and shared memory (staged blocks + query slices)
+  const int F = g.b1 > 0 ? 1 << (g.b1 - 1) : 0;
+  const int KS = F * MD / 32 + g.m / 32;
+  const size_t smem = (size_t)PNST * g.block_bytes + (size_t)nw * QG * KS * 128 * sizeof(uint32_t);
+  const int by_regs = 65536 / (nw * 32 * kPrefillRegs);
+  const int by_smem = (int)((size_t)(227 * 1024) / (smem + 1024));
+  const int slots = 148 * max(1, min(by_regs, by_smem));
   // the split count whose grid fills its last wave best, at least 4 blocks a split
   int best = 1;
   double best_score = -1.0;
