@@ -14,7 +14,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["native", "TQError", "Codebook", "Projections", "CompressedKVCache", "LayerGroups"]
+__all__ = ["native", "TQError", "Codebook", "Projections", "CompressedKVCache", "LayerGroups",
+           "key_variance", "stack_partials", "gather_partials", "merge_partials"]
 
 
 def __getattr__(name):
@@ -174,6 +175,20 @@ class CompressedKVCache:
                                     workspace)
         return out
 
+    def decode_partials(self, Q: torch.Tensor, proj: Projections, cb: Optional[Codebook],
+                        softmax_scale: Optional[float] = None, num_splits: int = 0,
+                        workspace: Optional[torch.Tensor] = None):
+        """This cache's share of a context-sharded decode: query preparation and the
+        split partials, not merged.  Returns (part_ml [B*Hq, S, 2], part_o
+        [B*Hq, S, d]), float32 views into the workspace (valid until it is reused)."""
+        B, Hq, d = Q.shape
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+        ws = self.workspace(Hq, num_splits) if workspace is None else workspace
+        cent = cb.centroids if cb is not None else None
+        native.tq_decode_prep(self.state, Q, scale, proj.Pi, proj.S, cent, num_splits, ws)
+        native.tq_decode_partial(self.state, Hq, scale, cent, None, num_splits, ws)
+        return native.tq_decode_partials_view(self.state, Hq, num_splits, ws)
+
     def decode(self, Q: torch.Tensor, proj: Projections, cb: Optional[Codebook],
                softmax_scale: Optional[float] = None, want_logits: bool = False,
                num_splits: int = 0, out: Optional[torch.Tensor] = None):
@@ -188,3 +203,44 @@ class CompressedKVCache:
                                    cb.centroids if cb is not None else None, out, logits,
                                    num_splits, ws)
         return (out, logits) if want_logits else out
+
+
+# ----------------------------------------------------------------------------- sharded context
+def stack_partials(parts, slots: int):
+    """Split partials of several context shards side by side: parts = [(part_ml
+    [rows, S_i, 2], part_o [rows, S_i, d]), ...] with S_i <= slots; a shard with
+    fewer splits is padded with empty slots (m = -inf, l = 0, o = 0).  Returns
+    (part_ml [rows, R * slots, 2], part_o [rows, R * slots, d]), contiguous."""
+    mls, os_ = [], []
+    for ml, o in parts:
+        rows, s, d = o.shape
+        if s > slots:
+            raise ValueError(f"a shard has {s} splits, more than slots={slots}")
+        pm = torch.zeros(rows, slots, 2, dtype=torch.float32, device=ml.device)
+        pm[:, :, 0] = float("-inf")
+        pm[:, :s] = ml
+        po = torch.zeros(rows, slots, d, dtype=torch.float32, device=o.device)
+        po[:, :s] = o
+        mls.append(pm)
+        os_.append(po)
+    return torch.cat(mls, dim=1).contiguous(), torch.cat(os_, dim=1).contiguous()
+
+
+def gather_partials(part_ml: torch.Tensor, part_o: torch.Tensor, slots: int, group=None):
+    """All-gather every rank's split partials of one decode (each rank holds one shard
+    of the context) and stack them as ``stack_partials`` does.  Every rank passes
+    the same ``slots`` (at least its own split count)."""
+    import torch.distributed as dist
+    ml, o = stack_partials([(part_ml, part_o)], slots)
+    R = dist.get_world_size(group)
+    mls = [torch.empty_like(ml) for _ in range(R)]
+    os_ = [torch.empty_like(o) for _ in range(R)]
+    dist.all_gather(mls, ml, group=group)
+    dist.all_gather(os_, o, group=group)
+    return torch.cat(mls, dim=1).contiguous(), torch.cat(os_, dim=1).contiguous()
+
+
+def merge_partials(part_ml: torch.Tensor, part_o: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+    """out [rows, d] (any float dtype): the softmax merge of the slots of each row."""
+    native.tq_merge_partials(part_ml, part_o, out)
+    return out

@@ -590,6 +590,47 @@ int tq_decode_combine(const tq_cache* c, int Hq, void* out, int num_splits, void
                       workspace, ws_bytes, stream, false, false, true, "tq_decode_combine");
 }
 
+int tq_decode_partials_view(const tq_cache* c, int Hq, int num_splits, void* workspace,
+                            size_t ws_bytes, float** part_ml, float** part_o, int* splits) {
+  int st = check_decode_common(c, Hq, num_splits);
+  if (st != TQ_OK) return st;
+  if (!part_ml || !part_o || !splits)
+    return fail(TQ_ERR_INVALID_ARG, "tq_decode_partials_view: null output pointer");
+  const tq::Geom g = tq::geom_of(c);
+  const int s = eff_splits(g, Hq / c->desc.Hkv, n_comp_of(c), num_splits);
+  if (!workspace || ws_bytes < tq::decode_ws_bytes(g, Hq, s))
+    return fail(TQ_ERR_INVALID_ARG, "tq_decode_partials_view: workspace too small");
+  const tq::DecodeWs ws = tq::decode_ws_carve(workspace, g, Hq, s);
+  *part_ml = ws.part_ml;
+  *part_o = ws.part_o;
+  *splits = s;
+  return ok();
+}
+
+int tq_merge_partials(const float* part_ml, const float* part_o, int64_t rows, int slots, int d,
+                      int dtype, void* out, void* stream) {
+  TQ_FAULT_POINT("tq_merge_partials");
+  if (!part_ml || !part_o || !out) return fail(TQ_ERR_INVALID_ARG, "tq_merge_partials: null pointer");
+  if (rows < 1 || rows > ((int64_t)1 << 31) - 1 || slots < 1 || d < 1 || d > 1024)
+    return fail(TQ_ERR_INVALID_ARG, "tq_merge_partials: rows=%lld slots=%d d=%d", (long long)rows,
+                slots, d);
+  if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16)
+    return fail(TQ_ERR_INVALID_ARG, "tq_merge_partials: dtype %d", dtype);
+  int st = check_pending("tq_merge_partials");
+  if (st != TQ_OK) return st;
+  // the decode merge kernel over an explicit partial array: rows x 1 "heads"
+  tq::Geom g{};
+  g.B = (int)rows;
+  g.d = d;
+  g.dtype = dtype;
+  tq::DecodeWs ws{};
+  ws.part_ml = const_cast<float*>(part_ml);
+  ws.part_o = const_cast<float*>(part_o);
+  cudaError_t e = tq::launch_decode_combine(g, 1, out, slots, ws, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_merge_partials");
+  return ok();
+}
+
 int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* workspace,
                     size_t ws_bytes, void* stream) {
   int st = check_decode_common(c, Hq, num_splits);

@@ -94,6 +94,9 @@ def _load() -> ctypes.CDLL:
         "tq_key_moments": (I, [P, I, I64, P, P, SZ, P]),
         "tq_sensitivity_profile": (I, [ctypes.POINTER(ctypes.c_double), I, I, I, I, I,
                                        ctypes.POINTER(tq_layer_groups)]),
+        "tq_decode_partials_view": (I, [C, I, I, P, SZ, ctypes.POINTER(P), ctypes.POINTER(P),
+                                        ctypes.POINTER(I)]),
+        "tq_merge_partials": (I, [P, P, I64, I, I, I, P, P]),
         "tq_layer_groups_parse": (I, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(tq_layer_groups)]),
         "tq_m_for_layer": (I, [ctypes.POINTER(tq_layer_groups), I]),
     }
@@ -283,6 +286,27 @@ def tq_decode_step(cache: tq_cache, K, V, Q, softmax_scale, Pi, S, T, centroids,
 def tq_decode_combine(cache: tq_cache, Hq, out, num_splits, workspace, stream=None):
     _check(lib.tq_decode_combine(ctypes.byref(cache), Hq, _ptr(out), num_splits, _ptr(workspace),
                                  _ws(workspace), _stream(stream)), "tq_decode_combine")
+
+
+def tq_decode_partials_view(cache: tq_cache, Hq, num_splits, workspace):
+    """(part_ml, part_o) as torch views of the workspace: [B*Hq, S, 2] and [B*Hq, S, d]."""
+    ml, o, s = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_int()
+    _check(lib.tq_decode_partials_view(ctypes.byref(cache), Hq, num_splits, _ptr(workspace),
+                                       _ws(workspace), ctypes.byref(ml), ctypes.byref(o),
+                                       ctypes.byref(s)), "tq_decode_partials_view")
+    rows, S, d = cache.desc.B * Hq, s.value, cache.desc.d
+    base = workspace.data_ptr()
+    f = workspace.view(torch.uint8)
+    ml_t = f[ml.value - base: ml.value - base + rows * S * 2 * 4].view(torch.float32).view(rows, S, 2)
+    o_t = f[o.value - base: o.value - base + rows * S * d * 4].view(torch.float32).view(rows, S, d)
+    return ml_t, o_t
+
+
+def tq_merge_partials(part_ml, part_o, out, stream=None):
+    """out [rows, d] from part_ml [rows, slots, 2] and part_o [rows, slots, d] (float32)."""
+    rows, slots, d = part_o.shape
+    _check(lib.tq_merge_partials(_ptr(part_ml), _ptr(part_o), rows, slots, d, dtype_code(out.dtype),
+                                 _ptr(out), _stream(stream)), "tq_merge_partials")
 
 
 # ----------------------------------------------------------------------------- layer groups

@@ -383,6 +383,34 @@ int tq_prefill_check(const tq_cache* c, int Hq, int n, int num_splits, const voi
                      size_t ws_bytes, void* stream);
 
 /*
+ * Context-sharded decode (one exchange step).  A context too long for one GPU
+ * can be split by token ranges over several caches (one per GPU: the earlier
+ * ranges in caches with W = 0, the range holding the newest tokens with the
+ * ring).  Each GPU runs tq_decode_prep + tq_decode_partial (out = NULL) on its
+ * shard; the split partials of all shards are gathered (an all-gather over
+ * NCCL, outside this library) and merged.  Because the softmax partials
+ * (m, l, o) of disjoint token sets merge exactly, the result is the decode of the
+ * whole context ([TQ] 六 online softmax).
+ *
+ * tq_decode_partials_view -- where tq_decode_partial leaves its partials in
+ * `workspace` (same c, Hq, num_splits): *part_ml = device float
+ * [B*Hq][*splits][2] (m in log2 units of softmax_scale * logit, then l),
+ * *part_o = device float [B*Hq][*splits][d] (sum of p v, unnormalised), and
+ * *splits = the split count that call uses.  No launch.  Errors: INVALID_ARG,
+ * UNSUPPORTED.
+ *
+ * tq_merge_partials -- out[r] = sum_s 2^(m_rs - M_r) o_rs / sum_s 2^(m_rs - M_r) l_rs
+ * with M_r = max_s m_rs (slots with m = -inf are empty; a row with no token gives
+ * 0) for part_ml [rows][slots][2] and part_o [rows][slots][d] (device, the
+ * layout above with the shards' splits side by side); out device [rows][d] of
+ * dtype.  Errors: INVALID_ARG, CUDA.
+ */
+int tq_decode_partials_view(const tq_cache* c, int Hq, int num_splits, void* workspace,
+                            size_t ws_bytes, float** part_ml, float** part_o, int* splits);
+int tq_merge_partials(const float* part_ml, const float* part_o, int64_t rows, int slots, int d,
+                      int dtype, void* out, void* stream);
+
+/*
  * tq_quantize_check -- SYNCHRONOUS: waits for `stream`, then reports (and
  * clears) the sticky device flag of the batched tensor-core key quantisation
  * (tq_quantize_keys and tq_append with more than 8 tokens, head dim 128,

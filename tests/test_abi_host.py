@@ -238,3 +238,24 @@ def test_sensitivity_profile_checks(nat):
     assert L.tq_key_moments(FAKE, 2, 0, FAKE, FAKE, 1 << 20, None) == nat.TQ_ERR_INVALID_ARG
     assert L.tq_key_moments(FAKE, 7, 10, FAKE, FAKE, 1 << 20, None) == nat.TQ_ERR_INVALID_ARG
     assert L.tq_key_moments(FAKE, 2, 10, FAKE, FAKE, 8, None) == nat.TQ_ERR_INVALID_ARG
+
+
+def test_sharded_decode_calls_checked_on_the_host(nat):
+    c = _fake_cache(nat)
+    c.n_total = 90
+    L = nat.lib
+    need = L.tq_decode_workspace_bytes(ctypes.byref(c), 8, 0)
+    ml, o, s = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_int()
+    ws = ctypes.c_void_p(1 << 24)
+    assert L.tq_decode_partials_view(ctypes.byref(c), 8, 0, ws, need, ctypes.byref(ml),
+                                     ctypes.byref(o), ctypes.byref(s)) == nat.TQ_OK
+    assert s.value == L.tq_decode_auto_splits(ctypes.byref(c), 8)
+    assert (1 << 24) < ml.value < o.value < (1 << 24) + need
+    assert L.tq_decode_partials_view(ctypes.byref(c), 8, 0, ws, 64, ctypes.byref(ml),
+                                     ctypes.byref(o), ctypes.byref(s)) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_decode_partials_view(ctypes.byref(c), 7, 0, ws, need, ctypes.byref(ml),
+                                     ctypes.byref(o), ctypes.byref(s)) == nat.TQ_ERR_UNSUPPORTED
+    for args in ((None, FAKE, 4, 3, 128, 2), (FAKE, FAKE, 0, 3, 128, 2), (FAKE, FAKE, 4, 0, 128, 2),
+                 (FAKE, FAKE, 4, 3, 2048, 2), (FAKE, FAKE, 4, 3, 128, 9)):
+        assert L.tq_merge_partials(*args, FAKE, None) == nat.TQ_ERR_INVALID_ARG
+    assert L.tq_merge_partials(FAKE, FAKE, 4, 3, 128, 2, None, None) == nat.TQ_ERR_INVALID_ARG
