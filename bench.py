@@ -274,6 +274,57 @@ def oracle_decode_sample(w, K1, V1, Q_steps, Kn, Vn, budget_s=12.0, min_reps=2, 
     return statistics.mean(times), statistics.mean(nbytes), i, threads
 
 
+def oracle_prefill_sample(w, n=16, context=4096, reps=2):
+    """Time the oracle's multi-token attention on one (batch, KV head) unit of workload
+    w: a cache of `context` tokens (quantised untimed), then `reps` timed calls that
+    score a chunk of n tokens.  Inputs are drawn on the host.  Returns (seconds per
+    call, compressed tokens of the sample, threads)."""
+    import numpy as np
+    import synth
+    from oracle import cache as ocache
+    from oracle import codebook as ocb
+    from oracle import projections as oproj
+    G = w.Hq // w.Hkv
+    w1 = w.scaled(B=1, Hkv=1, Hq=G, T=context)
+    K, V = synth.keys_values(w1, device="cpu")
+    Q, Kc, Vc = synth.prefill_chunk(w1, n, device="cpu")
+    po = oproj.make_projections(w.d, w.m, 0, with_rotation=w.b1 > 0)
+    cb = ocb.build(w.d, w.b1) if w.b1 else None
+    oc = ocache.OracleCache(1, 1, w.d, w.b1, w.m, w.vbits, w.group, w.W, context + 64, w.dtype, po, cb)
+    f = lambda t: t.double().numpy()
+    oc.append(f(K), f(V))
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oc.prefill(f(Q), f(Kc), f(Vc))
+        times.append(time.perf_counter() - t0)
+    return statistics.mean(times), oc.n_comp, _oracle_threads()
+
+
+def oracle_moments_sample(w, tokens=8192, reps=2):
+    """Time the oracle's key variance on one batch row of a calibration layer shaped
+    like workload w (all KV heads, `tokens` tokens), drawn on the host.  Returns
+    (seconds per pass, bytes of the sample in the workload dtype, threads)."""
+    import synth
+    from oracle import sensitivity as osens
+    K, _ = synth.keys_values(w.scaled(B=1, T=tokens), layer=5, device="cpu")
+    x = K.double().numpy()
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        osens.key_variance(x)
+        times.append(time.perf_counter() - t0)
+    return statistics.mean(times), K.numel() * K.element_size(), _oracle_threads()
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
 def _host_unit(w, device):
     """K, V of unit (b=0, h=0) at full context and per-step inputs, as float64 numpy."""
     import numpy as np
@@ -538,6 +589,25 @@ def run_ours(args):
                "sample": f"1 of {w.B * w.Hkv} (batch, KV-head) units at full context, {reps} steps "
                          "(append one token + decode its query heads), NumPy float64; GB/s of "
                          "that unit's packed bytes"}
+        if prefill is not None:
+            n0 = prefill["chunks"][0]["n"]
+            sec_p, comp_s, thr = oracle_prefill_sample(w, n=n0)
+            # the oracle's time is linear in the history and in the units: scaled to the
+            # bench's history length and its B * Hkv units
+            hist = prefill["history_tokens"]
+            t_full = sec_p * (hist / comp_s) * (w.B * w.Hkv)
+            prefill["cpu_baseline"] = {
+                "kind": "oracle", "value": w.B * n0 / t_full, "unit": "query tokens/s",
+                "cores": thr,
+                "sample": f"one (batch, KV-head) unit, {comp_s}-token history, a {n0}-token chunk, "
+                          f"NumPy float64, scaled by {hist}/{comp_s} history and "
+                          f"{w.B * w.Hkv} units"}
+        if sensitivity is not None:
+            sec_m, nb_m, thr = oracle_moments_sample(synth.WORKLOADS["aqjl"])
+            sensitivity["cpu_baseline"] = {
+                "kind": "oracle", "value": nb_m / sec_m / 1e9, "unit": "GB/s", "cores": thr,
+                "sample": "key variance of one batch row (8 KV heads x 8192 tokens x 128, fp16 "
+                          "bytes) of the calibration layer, NumPy float64"}
 
     # per timed step (tq_decode_step): one grid for the quantise of the token leaving
     # the ring + ring write + query preparation, one partial kernel
@@ -630,6 +700,7 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
                                "ideal_ms_at_peak": ideal_ms, "frac": ideal_ms / t,
                                "peak_bf16_tflops": bf16, "peak_kind": bf16_kind}})
     return {"chunks": res, "decode_ms": t_dec, "history_bytes": hist_bytes,
+            "history_tokens": int(cache.n_comp),
             "timing": "CUDA events around the whole call (prep, history partials, exact segment, "
                       "merge), L2 flushed before each call, 20 calls after 3 warm-up calls"}
 

@@ -76,3 +76,16 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
                               no_cpu_baseline=True, no_quantize=True, workload="gqa32k")
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_oracle_samples_of_the_bench_legs_run_on_the_host():
+    """The CPU oracle timings beside the multi-token and key-moments legs draw their
+    inputs on the host and run the oracle only."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.WORKLOADS["gqa32k"].scaled(seed=0)
+    sec, comp, thr = bench.oracle_prefill_sample(w, n=4, context=512, reps=1)
+    assert sec > 0 and comp == 512 - w.W and thr >= 1
+    sec, nb, thr = bench.oracle_moments_sample(synth.WORKLOADS["aqjl"], tokens=64, reps=1)
+    assert sec > 0 and nb == 8 * 64 * 128 * 2 and thr >= 1
