@@ -38,6 +38,14 @@ def test_every_declared_symbol_is_exported(nat):
     assert nat.lib.tq_version() == 1
 
 
+def test_every_declared_call_has_a_binding(nat):
+    """The Python binding marshals every call the header declares (same names)."""
+    import inspect
+    src = inspect.getsource(nat)
+    bound = set(re.findall(r'"(tq_[a-z0-9_]+)": \(', src))
+    assert [n for n in _declared() if n not in bound] == []
+
+
 @pytest.mark.parametrize("cfg", [
     (8, 8, 128, 2, 128, 2, 32, 16, 32768, "bf16"),
     (4, 4, 256, 3, 256, 4, 64, 16, 262144, "bf16"),
