@@ -569,9 +569,10 @@ def run_ours(args):
         prefill = bench_prefill(w, cache, pj, cb, flush_l2, stream, step_bytes()[0], world)
 
     # key/value quantise throughput: 131072 tokens x 8 KV heads in chunks of 4096
-    quant = None
+    quant = qsample = None
     if not args.no_quantize:
-        quant = bench_quantize(dev, world)
+        quant, qsample = bench_quantize(
+            dev, world, keep_sample=rank == 0 and world == 1 and not args.no_cpu_baseline)
     sensitivity = None
     if not args.no_sensitivity:
         sensitivity = bench_sensitivity(dev, world, peak, flush_l2)
@@ -602,6 +603,8 @@ def run_ours(args):
                 "sample": f"one (batch, KV-head) unit, {comp_s}-token history, a {n0}-token chunk, "
                           f"NumPy float64, scaled by {hist}/{comp_s} history and "
                           f"{w.B * w.Hkv} units"}
+        if qsample is not None:
+            quant["parity_vs_oracle"] = oracle_quantize_counts(qsample)
         if sensitivity is not None:
             sec_m, nb_m, thr = oracle_moments_sample(synth.WORKLOADS["aqjl"])
             sensitivity["cpu_baseline"] = {
@@ -828,7 +831,10 @@ def bench_other_decodes(dev, world, peak):
     return res
 
 
-def bench_quantize(dev, world, reps=3):
+def bench_quantize(dev, world, reps=3, keep_sample=False):
+    """Chunked append of the quantise workload; with keep_sample, the inputs and
+    the packed region of (batch 0, KV head 0) on the host (for the oracle check
+    of the CPU-baseline leg)."""
     import torch
     import synth
     from compressed_attention_turboquantprod_b200 import Codebook, CompressedKVCache, Projections
@@ -837,6 +843,9 @@ def bench_quantize(dev, world, reps=3):
     K, V = synth.keys_values(w, device=dev)
     chunks = [(K[:, :, t:t + w.chunk].contiguous(), V[:, :, t:t + w.chunk].contiguous())
               for t in range(0, w.T, w.chunk)]
+    sample = None
+    if keep_sample:
+        sample = {"K": K[0, 0].double().cpu().numpy(), "V": V[0, 0].double().cpu().numpy()}
     del K, V
     cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
                               dtype=w.torch_dtype, device=dev)
@@ -861,12 +870,45 @@ def bench_quantize(dev, world, reps=3):
     ms_h = timed(Projections(w.d, w.m, 0, device=dev, structured=True))
     keys = reduce_sum(float(w.T * w.Hkv * w.B), world)
     tb = cache.state.token_bytes
+    if sample is not None:
+        # the Hadamard pass ran last: append once more with the QR projections
+        cache.state.n_total = 0
+        for k, v in chunks:
+            cache.append(k, v, pj, cb)
+        torch.cuda.synchronize()
+        sample["region"] = cache.buffer[:cache.state.region_bytes].cpu().numpy()
     nbytes = w.T * w.Hkv * w.B * (2 * w.d * 2 + tb)
-    return {"Mkeys_per_s": keys / (ms * 1e-3) / 1e6, "ms": ms, "keys": int(keys),
+    res = {"Mkeys_per_s": keys / (ms * 1e-3) / 1e6, "ms": ms, "keys": int(keys),
             "Mkeys_per_s_hadamard_rotation": keys / (ms_h * 1e-3) / 1e6,
             "GB_per_s": reduce_sum(float(nbytes), world) / (ms * 1e-3) / 1e9,
             "workload": "quant: 131072 tokens x 8 KV heads, d=128, bf16, appended in chunks of 4096; "
                         "keys b1=2 + m=128, values 2-bit g=32 (key + value per key)"}
+    return res, sample
+
+
+def oracle_quantize_counts(sample):
+    """The oracle's one-shot quantisation of the sampled unit's 131072 tokens
+    against the library's chunked append of them: near-boundary exemption counts
+    of the key codes and sign bits, and value fields (must be bit-exact)."""
+    import numpy as np
+    import synth
+    from oracle import cache as ocache, codebook as ocb, layout as olayout
+    from oracle import projections as oproj, quantize as oq
+    w = synth.WORKLOADS["quant"]
+    po, cb = oproj.make_projections(w.d, w.m, 0), ocb.build(w.d, w.b1)
+    oc = ocache.OracleCache(1, 1, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T, w.dtype, po, cb)
+    oc.append(sample["K"][None, None], sample["V"][None, None])
+    r = oc.rec[0][0]
+    n = r["rho"].shape[0]
+    buf = np.zeros(oc.lay.total_bytes, np.uint8)
+    buf[:oc.lay.region_bytes] = sample["region"][:oc.lay.region_bytes]
+    fg = olayout.decode_fields(olayout.read_region(buf, oc.lay, 0, 0, n), oc.lay)
+    counts = oq.band_agreement(fg["idx"], fg["bits"], r, cb[1])
+    counts["value_field_mismatches"] = int(
+        np.sum(fg["codes"] != r["codes"]) + np.sum(fg["scale"] != r["scale"].astype(np.float32))
+        + np.sum(fg["vmin"] != r["vmin"].astype(np.float32)))
+    counts["sample"] = "batch 0, KV head 0: all 131072 tokens of the chunked append"
+    return counts
 
 
 def main():

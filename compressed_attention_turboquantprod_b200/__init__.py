@@ -90,16 +90,14 @@ class LayerGroups:
 
 
 def key_variance(K: torch.Tensor, workspace: Optional[torch.Tensor] = None) -> float:
-    """Population variance of every entry of one layer's calibration keys (device
-    moments, one streaming pass; waits for the result)."""
+    """Population variance of every entry of one layer's calibration keys
+    (tq_key_moments, one streaming pass on the device; waits for the result)."""
     out = torch.empty(2, dtype=torch.float64, device=K.device)
     if workspace is None:
         workspace = torch.empty(native.tq_key_moments_workspace_bytes(), dtype=torch.uint8,
                                 device=K.device)
     native.tq_key_moments(K, out, workspace)
-    s1, s2 = out.tolist()
-    n = K.numel()
-    return s2 / n - (s1 / n) ** 2
+    return float(out[1].item())
 
 
 class CompressedKVCache:

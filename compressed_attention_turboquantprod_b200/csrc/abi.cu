@@ -218,6 +218,17 @@ Geom geom_of(const tq_cache* c) {
 }
 }  // namespace tq
 
+namespace tq {
+// Scratch bytes a decode of the cache's current state needs: the split count is
+// the one decode_plan takes (clamped to the cache's blocks), 0 for invalid
+// arguments.
+size_t decode_ws_bytes_now(const tq_cache* c, int Hq, int num_splits) {
+  if (check_decode_common(c, Hq, num_splits) != TQ_OK) return 0;
+  const Geom g = geom_of(c);
+  return decode_ws_bytes(g, Hq, eff_splits(g, Hq / c->desc.Hkv, n_comp_of(c), num_splits));
+}
+}  // namespace tq
+
 extern "C" {
 
 const char* tq_last_error(void) { return g_err.c_str(); }
@@ -439,6 +450,7 @@ size_t tq_decode_workspace_bytes(const tq_cache* c, int Hq, int num_splits) {
   return tq::decode_ws_bytes(tq::geom_of(c), Hq, max_splits(c, Hq, num_splits));
 }
 
+
 struct DecodePlan {
   tq::Geom g;
   int splits = 1;
@@ -637,7 +649,14 @@ int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* works
   if (st != TQ_OK) return st;
   tq::Geom g = tq::geom_of(c);
   const int splits = eff_splits(g, Hq / c->desc.Hkv, n_comp_of(c), num_splits);
-  if (!workspace || ws_bytes < tq::decode_ws_bytes(g, Hq, splits))
+  if (!workspace) {       // the static scratch of tq_decode_attention_noalloc
+    void* p = nullptr;
+    st = tq::noalloc_scratch(&p);
+    if (st != TQ_OK) return st;
+    workspace = p;
+    ws_bytes = (size_t)TQ_NOALLOC_SCRATCH_BYTES;
+  }
+  if (ws_bytes < tq::decode_ws_bytes(g, Hq, splits))
     return fail(TQ_ERR_INVALID_ARG, "tq_decode_check: workspace too small");
   tq::DecodeWs ws = tq::decode_ws_carve(const_cast<void*>(workspace), g, Hq, splits);
   int flag = 0;

@@ -23,8 +23,11 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
+}  // namespace
+
+namespace tq {
 // Device address of the scratch array on the current device (set up on first use).
-int scratch_address(void** out) {
+int noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return tq::set_error(TQ_ERR_CUDA, "tq_decode_attention_noalloc: cudaGetDevice failed");
@@ -41,25 +44,23 @@ int scratch_address(void** out) {
   *out = g_scratch_addr[dev];
   return TQ_OK;
 }
-
-}  // namespace
+}  // namespace tq
 
 extern "C" int tq_decode_attention_noalloc(const tq_cache* c, const void* Q, int Hq,
                                            float softmax_scale, const float* Pi, const float* S,
                                            const float* centroids, void* out, float* logits,
                                            int num_splits, void* stream) {
-  // Scratch the decode would need with these arguments (0 when they are invalid:
-  // tq_decode_attention below then reports why).
-  int splits = num_splits;
-  if (splits == 0 && c) splits = tq_decode_auto_splits(c, Hq);
-  const size_t need = splits > 0 ? tq_decode_workspace_bytes(c, Hq, splits) : 0;
+  // Scratch the decode needs with these arguments and the cache's current length,
+  // from the split count the decode itself takes (0 when the arguments are
+  // invalid: tq_decode_attention below then reports why).
+  const size_t need = tq::decode_ws_bytes_now(c, Hq, num_splits);
   if (need > (size_t)TQ_NOALLOC_SCRATCH_BYTES)
     return tq::set_error(TQ_ERR_UNSUPPORTED,
                          "tq_decode_attention_noalloc: needs %zu bytes of scratch, more than the "
                          "static maximum of %zu bytes (use tq_decode_attention with a workspace)",
                          need, (size_t)TQ_NOALLOC_SCRATCH_BYTES);
   void* ws = nullptr;
-  int st = scratch_address(&ws);
+  int st = tq::noalloc_scratch(&ws);
   if (st != TQ_OK) return st;
   return tq_decode_attention(c, Q, Hq, softmax_scale, Pi, S, centroids, out, logits, num_splits,
                              ws, (size_t)TQ_NOALLOC_SCRATCH_BYTES, stream);

@@ -2,11 +2,16 @@
 // sensitivity analyser: each layer's key variance on calibration data decides
 // the layer groups and their bit allocation).
 //
-// Device: the first two moments of a layer's calibration keys (sum and sum of
-// squares of every entry), one streaming pass at HBM speed: 16-byte loads, the
-// entries of a load summed in fp32 (exact for bf16 squares; a few ulp for
-// fp16/fp32), fp64 across loads, fixed-order block and grid reductions (the
-// result does not depend on scheduling).
+// Device: the mean and population variance of every entry of a layer's
+// calibration keys, one streaming pass at HBM speed.  Entries are taken
+// relative to a shift c (the fp32 mean of the first min(n, 32) entries, the
+// same in every CTA), so the sums stay of the size of the spread and not of
+// the mean: d = x - c, S1 = sum d, S2 = sum d^2, mean = c + S1/n, variance =
+// S2/n - (S1/n)^2 (shifted-data formula; the one-pass sum of squares, which
+// cancels catastrophically for keys whose mean is large against their spread,
+// is never formed).  16-byte loads, the entries of a load summed in fp32, fp64
+// across loads, fixed-order block and grid reductions (the result does not
+// depend on scheduling).
 //
 // Host: the groups and sketch dims from the per-layer variances.
 //   * contiguous groups whose boundaries minimise the summed squared deviation
@@ -29,12 +34,12 @@ constexpr int kMomBlocks = 148 * 4;
 constexpr int kMomThreads = 256;
 constexpr int kMomUnroll = 4;     // 16-byte loads in flight per thread
 
-__device__ __forceinline__ void moments16(uint4 u, int dtype, float& s1, float& s2) {
+__device__ __forceinline__ void moments16(uint4 u, int dtype, float c, float& s1, float& s2) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
   if (dtype == TQ_F32) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float x = __uint_as_float(w[i]);
+      const float x = __uint_as_float(w[i]) - c;
       s1 += x;
       s2 = fmaf(x, x, s2);
     }
@@ -51,14 +56,33 @@ __device__ __forceinline__ void moments16(uint4 u, int dtype, float& s1, float& 
         lo = f.x;
         hi = f.y;
       }
+      lo -= c;
+      hi -= c;
       s1 += lo + hi;
       s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
     }
   }
 }
 
+// The shift: fp32 mean of the first min(n, 32) entries (one warp, fixed order;
+// every caller gets the same value).
+__device__ __forceinline__ float moments_shift(const void* K, int dtype, int64_t n, int lane) {
+  const int k = n < 32 ? (int)n : 32;
+  float x = lane < k ? load_f(K, lane, dtype) : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x / (float)k;
+}
+
 __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int dtype, int64_t n,
                                                             double* part) {
+  __shared__ float s_c;
+  if (threadIdx.x < 32) {
+    const float c = moments_shift(K, dtype, n, threadIdx.x);
+    if (threadIdx.x == 0) s_c = c;
+  }
+  __syncthreads();
+  const float c = s_c;
   const int per = dtype == TQ_F32 ? 4 : 8;              // entries per 16-byte load
   const int64_t nv = n / per;
   const int64_t nth = (int64_t)gridDim.x * kMomThreads;
@@ -74,13 +98,13 @@ __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int 
     for (int k = 0; k < kMomUnroll; ++k)
       if (i + k * nth < nv) {
         float s1 = 0.f, s2 = 0.f;
-        moments16(u[k], dtype, s1, s2);
+        moments16(u[k], dtype, c, s1, s2);
         d1 += (double)s1;
         d2 += (double)s2;
       }
   }
   for (int64_t i = nv * per + t0; i < n; i += nth) {     // ragged tail
-    const double x = (double)load_f(K, i, dtype);
+    const double x = (double)(load_f(K, i, dtype) - c);
     d1 += x;
     d2 += x * x;
   }
@@ -108,8 +132,11 @@ __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int 
   }
 }
 
-__global__ void k_moments_final(const double* part, int nb, double* out) {
+// out[0] = mean, out[1] = population variance (>= 0), from the blocks' shifted sums.
+__global__ void k_moments_final(const void* K, int dtype, int64_t n, const double* part, int nb,
+                                double* out) {
   const int lane = threadIdx.x;
+  const float c = moments_shift(K, dtype, n, lane);
   double a = 0.0, b = 0.0;
   for (int i = lane; i < nb; i += 32) {
     a += part[2 * i];
@@ -121,8 +148,10 @@ __global__ void k_moments_final(const double* part, int nb, double* out) {
     b += __shfl_xor_sync(0xffffffffu, b, o);
   }
   if (lane == 0) {
-    out[0] = a;
-    out[1] = b;
+    const double dn = (double)n, m1 = a / dn;
+    const double var = b / dn - m1 * m1;
+    out[0] = (double)c + m1;
+    out[1] = var > 0.0 ? var : 0.0;
   }
 }
 
@@ -152,7 +181,7 @@ cudaError_t launch_key_moments(const void* K, int dtype, int64_t n, double* out,
   k_key_moments<<<(unsigned)nb, kMomThreads, 0, s>>>(K, dtype, n, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_moments_final<<<1, 32, 0, s>>>(part, (int)nb, out);
+  k_moments_final<<<1, 32, 0, s>>>(K, dtype, n, part, (int)nb, out);
   return cudaGetLastError();
 }
 

@@ -89,6 +89,11 @@ struct DecodeWs {
   float* part_o;    // [B*Hq, splits, d]
 };
 size_t decode_ws_bytes(const Geom& g, int Hq, int splits);
+// Scratch of a decode of c's current state with these arguments (abi.cu; 0 when
+// they are invalid), and the device address of the static scratch array of
+// tq_decode_attention_noalloc on the current device (noalloc_decode.cu).
+size_t decode_ws_bytes_now(const tq_cache* c, int Hq, int num_splits);
+int noalloc_scratch(void** out);
 DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits);
 int decode_auto_splits(const Geom& g, int G, int64_t n_comp);
 

@@ -264,8 +264,10 @@ def tq_quantize_check(stream=None):
 
 
 def tq_decode_check(cache: tq_cache, Hq, num_splits, workspace, stream=None):
+    """workspace None: the static scratch of tq_decode_attention_noalloc."""
     _check(lib.tq_decode_check(ctypes.byref(cache), Hq, num_splits, _ptr(workspace),
-                               _ws(workspace), _stream(stream)), "tq_decode_check")
+                               _ws(workspace) if workspace is not None else 0, _stream(stream)),
+           "tq_decode_check")
 
 
 def tq_decode_partial(cache: tq_cache, Hq, softmax_scale, centroids, logits, num_splits,

@@ -339,7 +339,8 @@ int tq_decode_step(tq_cache* c, const void* K, const void* V, int64_t n_new, con
  * kernel whose bounded wait on a shared-memory load gives up (it never should)
  * skips its work and raises a flag instead of hanging; this call returns
  * TQ_ERR_CUDA when the flag is set, TQ_OK otherwise.  Arguments as for
- * tq_decode_attention.
+ * tq_decode_attention; workspace == NULL (ws_bytes ignored) reads the flag of
+ * the static scratch of tq_decode_attention_noalloc on the current device.
  */
 int tq_decode_check(const tq_cache* c, int Hq, int num_splits, const void* workspace,
                     size_t ws_bytes, void* stream);
@@ -439,8 +440,11 @@ int tq_quantize_check(void* stream);
  *   serialised by the caller.  Each call overwrites every scratch byte it reads,
  *   so nothing needs clearing between calls.
  *   Arguments as tq_decode_attention, without the workspace.
+ *   A kernel whose bounded wait gave up leaves its flag in the static scratch:
+ *   tq_decode_check(c, Hq, num_splits, NULL, 0, stream) reads it.
  * Errors: those of tq_decode_attention; UNSUPPORTED when the decode needs more
- *   scratch than TQ_NOALLOC_SCRATCH_BYTES (e.g. very large B * Hq); CUDA when
+ *   scratch than TQ_NOALLOC_SCRATCH_BYTES (sized from the split count the decode
+ *   takes for the cache's current length: e.g. very large B * Hq); CUDA when
  *   the address lookup fails.
  */
 #define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -475,9 +479,13 @@ int tq_m_for_layer(const tq_layer_groups* g, int layer);
  * on calibration data decides the layer groups and their bit allocation; the
  * pages give no formula, the steps below are this library's reading).
  *
- * tq_key_moments -- out[0] = sum and out[1] = sum of squares of the n entries of
- * K (device, dtype TQ_F32 / TQ_F16 / TQ_BF16, 16-byte aligned), one streaming
- * pass; the layer's variance is out[1] / n - (out[0] / n)^2.  `out` is a device
+ * tq_key_moments -- out[0] = mean and out[1] = population variance of the n
+ * entries of K (device, dtype TQ_F32 / TQ_F16 / TQ_BF16, 16-byte aligned), the
+ * statistic of the [AQJL] sensitivity analyser, in one streaming pass.  The
+ * entries are summed relative to a shift (the fp32 mean of the first min(n, 32)
+ * entries): S1 = sum (x - c), S2 = sum (x - c)^2, in fp32 within a 16-byte load
+ * and fp64 beyond, and variance = S2/n - (S1/n)^2 in fp64, so keys whose mean
+ * is large against their spread keep their precision.  `out` is a device
  * double[2]; `workspace` device, tq_key_moments_workspace_bytes() bytes.  The
  * result does not depend on scheduling (fixed-order reductions).
  * Errors: INVALID_ARG, CUDA.

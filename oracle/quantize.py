@@ -103,3 +103,27 @@ def sign_exempt(z, rel: float = 1e-5):
     z = np.asarray(z, dtype=np.float64)
     m = z.shape[1]
     return np.abs(z) <= rel * np.sqrt(np.sum(z * z, axis=1, keepdims=True)) / np.sqrt(m)
+
+
+def band_agreement(idx_got, bits_got, ref: dict, beta32) -> dict:
+    """Codes and sign bits decided elsewhere (idx_got [n, d] or None for pure QJL,
+    bits_got [n, m]) against this oracle's (``ref``: the quantize_keys output,
+    with its fp32 y and its z).  A code may differ only where ``code_exempt``
+    holds and a sign bit only where ``sign_exempt`` holds; a token with a
+    differing code has its sign bits left out (they depend on the code).
+    Returns the counts; ``outside_band`` > 0 means a disagreement."""
+    n = ref["bits"].shape[0]
+    flipped = np.zeros(n, bool)
+    code_mis = code_out = 0
+    if idx_got is not None:
+        mis = np.asarray(idx_got) != ref["idx"]
+        ex = code_exempt(ref["y32"], beta32)
+        code_mis = int(mis.sum())
+        code_out = int((mis & ~ex).sum())
+        flipped = np.any(mis, axis=1)
+    smis = (np.asarray(bits_got) != ref["bits"]) & ~flipped[:, None]
+    sign_out = int((smis & ~sign_exempt(ref["z"])).sum())
+    return {"tokens": int(n), "code_mismatch_in_band": code_mis - code_out,
+            "sign_mismatch_in_band": int(smis.sum()) - sign_out,
+            "tokens_with_a_flipped_code": int(flipped.sum()),
+            "outside_band": code_out + sign_out}

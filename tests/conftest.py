@@ -31,3 +31,19 @@ def page_figures():
         k, v = (s.strip() for s in row.split("=", 1))
         out[k] = v
     return out
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the near-boundary exemption counts the GPU parity tests recorded."""
+    gc = sys.modules.get("gpu_common")
+    rows = getattr(gc, "PARITY_COUNTS", None) if gc else None
+    if not rows:
+        return
+    tr = terminalreporter
+    tr.section("near-boundary exemptions (codes / sign bits inside the 1e-5 band)")
+    tot = {}
+    for label, counts in rows:
+        tr.write_line(f"{label}: " + ", ".join(f"{k}={v}" for k, v in counts.items()))
+        for k, v in counts.items():
+            tot[k] = tot.get(k, 0) + v
+    tr.write_line("total: " + ", ".join(f"{k}={v}" for k, v in tot.items()))

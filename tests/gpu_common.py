@@ -16,13 +16,19 @@ from oracle import quantize as oq
 #  - rho: 4 ulp; ||r||: 2e-6 relative (fp32 rounding of y = Pi x / rho feeds
 #    e = y - c[idx]; ~1e-8 absolute on entries of size ~3e-2 over d terms);
 #  - logits given identical codes: 1e-3 relative or 1e-4 absolute;
-#  - attention outputs: 2e-3 max-abs, plus half an ulp of the output dtype at
-#    |o| (the output is stored in the cache dtype; bf16 alone rounds |o| = 4 by
-#    up to 7.8e-3, which no arithmetic can beat).
+#  - attention outputs: 2e-3 max-abs, or, where the output dtype's own rounding
+#    of |o| exceeds that (bf16 at |o| >= 1: half an ulp is 3.9e-3 and more),
+#    half an ulp of the output dtype at |o| plus 64 fp32 ulp of |o| for the
+#    kernel's arithmetic.  Below |o| = 1 the bound is 2e-3 itself.
 RHO_ULP = 4
 RNORM_ULP = 4
 LOGIT_REL, LOGIT_ABS = 1e-3, 1e-4
 OUT_ABS = 2e-3
+OUT_ARITH_F32_ULP = 64
+
+# Near-boundary exemptions seen by compare_keys calls given a label: (label, counts).
+# The session summary (conftest.py) prints them, so every GPU test log carries them.
+PARITY_COUNTS = []
 
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
@@ -54,9 +60,10 @@ def unpack_bits_dev(packed: torch.Tensor, nbits: int) -> np.ndarray:
     return olayout.unpack_bits(packed.cpu().numpy(), nbits)
 
 
-def compare_keys(gpu: dict, ref: dict, d: int, b1: int, m: int, beta32):
+def compare_keys(gpu: dict, ref: dict, d: int, b1: int, m: int, beta32, label=None):
     """gpu: dict of host numpy arrays (idx planes bytes, signs bytes, rho, rnorm);
-    ref: oracle quantize_keys output.  Asserts parity; returns counts."""
+    ref: oracle quantize_keys output.  Asserts parity; returns counts (recorded
+    in PARITY_COUNTS under `label` when one is given)."""
     n = ref["rho"].shape[0]
     bits_g = olayout.unpack_bits(gpu["signs"], m)
     skip_tok = np.zeros(n, bool)
@@ -87,9 +94,18 @@ def compare_keys(gpu: dict, ref: dict, d: int, b1: int, m: int, beta32):
             ref["rho"].astype(np.float64) * np.sqrt(d) * 2.0 ** -21
         ok = np.abs(rn_g - rn_r) <= tol
         assert np.all(ok | skip_tok), f"rnorm max err / tol {np.max((np.abs(rn_g - rn_r) / tol)[~skip_tok])}"
-    return {"code_mismatch": n_code_mis, "code_exempt": n_code_ex,
-            "sign_mismatch": int(smis.sum()), "sign_exempt": int(sex.sum()),
-            "skipped_tokens": int(skip_tok.sum())}
+    counts = {"tokens": int(n), "code_mismatch": n_code_mis, "code_exempt": n_code_ex,
+              "sign_mismatch": int(smis.sum()), "sign_exempt": int(sex.sum()),
+              "skipped_tokens": int(skip_tok.sum())}
+    if label is not None:
+        PARITY_COUNTS.append((label, counts))
+    return counts
+
+
+def record(label, **counts):
+    """Record a count that is not a key comparison (e.g. units whose end-to-end
+    output check was skipped because a code flipped inside the boundary band)."""
+    PARITY_COUNTS.append((label, counts))
 
 
 def check_logits(got: np.ndarray, want: np.ndarray):
@@ -107,11 +123,18 @@ def storage_half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
     return 0.5 * np.exp2(e - (HALF_ULP_BITS[dtype] - 1))
 
 
+def out_tolerance(want: np.ndarray, dtype: str) -> np.ndarray:
+    """max(2e-3, half an ulp of the output dtype at |o| + 64 fp32 ulp of |o|)."""
+    f32_ulp = np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
+    return np.maximum(OUT_ABS, storage_half_ulp(want, dtype) + OUT_ARITH_F32_ULP * f32_ulp)
+
+
 def check_out(got: np.ndarray, want: np.ndarray, dtype: str = "bf16"):
     if not got.size:
         return 0.0
     err = np.abs(got - want)
-    tol = OUT_ABS + storage_half_ulp(want, dtype)
-    assert np.all(err <= tol), (f"output error {np.max(err - tol) + OUT_ABS:.3g} over "
-                                f"{OUT_ABS} + storage rounding (max |o| {np.max(np.abs(want)):.3g})")
+    tol = out_tolerance(want, dtype)
+    i = int(np.argmax(err - tol))
+    assert np.all(err <= tol), (f"output error {err.flat[i]:.3g} over its bound {tol.flat[i]:.3g} "
+                                f"at |o| = {abs(want.flat[i]):.3g} (max |o| {np.max(np.abs(want)):.3g})")
     return float(np.max(err))

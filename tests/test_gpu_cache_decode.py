@@ -7,7 +7,7 @@ import torch
 
 import synth
 from gpu_common import (TORCH_DT, check_logits, check_out, compare_keys, host, nat, oracle_setup,
-                        to_dev)
+                        record, to_dev)
 from oracle import cache as ocache
 from oracle import layout as olayout
 
@@ -42,11 +42,17 @@ def _oracle_cache(w, capacity, po, cb):
                               w.dtype, po, cb if w.b1 > 0 else None)
 
 
-def _compare_cache_bytes(gpu_buf: np.ndarray, oc: ocache.OracleCache):
+def _compare_cache_bytes(gpu_buf: np.ndarray, oc: ocache.OracleCache, per_unit=False,
+                         label=None):
+    """Packed cache vs the oracle's: total tokens with a flipped code, or with
+    per_unit, {(b, h): tokens with a flipped code}."""
     ref = oc.to_bytes()
     assert gpu_buf.shape == ref.shape
+    units = {(b, h): 0 for b in range(oc.B) for h in range(oc.Hkv)}
     if np.array_equal(gpu_buf, ref):
-        return 0
+        if label is not None:
+            record(label, code_mismatch=0, sign_mismatch=0, skipped_tokens=0)
+        return units if per_unit else 0
     lay = oc.lay
     # rings and value fields must match exactly; key fields may differ only on exempt elements
     assert np.array_equal(gpu_buf[lay.ring_k_off:], ref[lay.ring_k_off:])
@@ -64,9 +70,11 @@ def _compare_cache_bytes(gpu_buf: np.ndarray, oc: ocache.OracleCache):
             got = {"idx": fg["idx"], "signs": fg["sign"],
                    "rho": np.ascontiguousarray(fg["rho"]).view("<f4").ravel(),
                    "rnorm": np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel() if oc.b1 else None}
-            st = compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None)
+            st = compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None,
+                              label=None if label is None else f"{label} unit ({b},{h})")
             skipped += st["skipped_tokens"]
-    return skipped
+            units[(b, h)] = st["skipped_tokens"]
+    return units if per_unit else skipped
 
 
 def test_append_packed_bytes_match_oracle_across_chunks():
@@ -264,7 +272,7 @@ def test_decode_empty_cache_is_zero():
     assert torch.count_nonzero(out).item() == 0
 
 
-def _flips(gc, oc, b, h, W_unit=None):
+def _flips(gc, oc, b, h, W_unit=None, label=None):
     """Number of tokens of GPU unit (b, h) whose key codes differ from the oracle's
     (each difference is asserted to lie in the boundary band)."""
     lay = oc.lay
@@ -278,7 +286,8 @@ def _flips(gc, oc, b, h, W_unit=None):
     got = {"idx": fg["idx"], "signs": fg["sign"],
            "rho": np.ascontiguousarray(fg["rho"]).view("<f4").ravel(),
            "rnorm": np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel() if oc.b1 else None}
-    return compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None)["skipped_tokens"]
+    return compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None,
+                        label=label)["skipped_tokens"]
 
 
 # End-to-end output checks (library quantisation + library decode against the
@@ -293,6 +302,7 @@ def test_tiny_workload_end_to_end_with_library_projections():
     its own projections from the same seed."""
     from compressed_attention_turboquantprod_b200 import Codebook, Projections
     w = synth.WORKLOADS["tiny"]
+    checked = 0
     for W in (0, 16):
         wl = w.scaled(W=W)
         K, V = synth.keys_values(wl, device="cuda")
@@ -306,9 +316,12 @@ def test_tiny_workload_end_to_end_with_library_projections():
         oc = _oracle_cache(wl, 512, po, cb)
         oc.append(host(K), host(V))
         ro, rl = oc.decode(host(Q))
-        if _flips(gc, oc, 0, 0) == 0:
+        if _flips(gc, oc, 0, 0, label=f"tiny W={W}") == 0:
             check_out(host(out), ro, wl.dtype)
             check_logits(logits.cpu().numpy()[0].astype(np.float64), rl[(0, 0)])
+            checked += 1
+    record("tiny end-to-end output checks", cases_checked=checked, cases_skipped=2 - checked)
+    assert checked >= 1
 
 
 def test_hadamard_rotation_end_to_end():
@@ -328,15 +341,23 @@ def test_hadamard_rotation_end_to_end():
     oc = _oracle_cache(w, 768, po, cb)
     oc.append(host(K), host(V))
     ro, rl = oc.decode(host(Q))
-    skipped = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
-    assert skipped <= 4
-    if skipped == 0:                 # identical codes everywhere: outputs and logits too
-        G = w.Hq // w.Hkv
-        check_out(host(out), ro, w.dtype)
-        lg = logits.cpu().numpy().astype(np.float64)
-        for b in range(w.B):
-            for h in range(w.Hkv):
-                check_logits(lg[b, h * G:(h + 1) * G], rl[(b, h)])
+    flips = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc, per_unit=True,
+                                 label="hadamard rotation")
+    assert sum(flips.values()) <= 4
+    # outputs and logits of every unit whose codes came out identical
+    G = w.Hq // w.Hkv
+    lg = logits.cpu().numpy().astype(np.float64)
+    o, r = host(out), ro
+    checked = 0
+    for (b, h), f in flips.items():
+        if f == 0:
+            hs = slice(h * G, (h + 1) * G)
+            check_out(o[b:b + 1, hs], r[b:b + 1, hs], w.dtype)
+            check_logits(lg[b, hs], rl[(b, h)])
+            checked += 1
+    record("hadamard end-to-end output checks", units_checked=checked,
+           units_skipped=len(flips) - checked)
+    assert checked >= 1
 
 
 def test_gqa32k_shape_reduced_context_end_to_end():

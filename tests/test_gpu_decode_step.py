@@ -1,14 +1,20 @@
 """tq_decode_step (append + decode as one call) against tq_append followed by
 tq_decode_attention on a twin cache: the packed cache, the ring, the outputs and
 the logits must be identical after every step, whichever path the call takes
-(the fused two-launch path, or the two calls)."""
+(the fused two-launch path, or the two calls).  The fused step's cache and
+output are also compared with the oracle's own append and decode of the same
+tokens after every step."""
 import math
 
+import numpy as np
 import pytest
 import torch
 
 import synth
-from gpu_common import TORCH_DT, oracle_setup, to_dev
+from gpu_common import (TORCH_DT, check_logits, check_out, compare_keys, host, oracle_setup,
+                        record, to_dev)
+from oracle import cache as ocache
+from oracle import layout as olayout
 
 pytestmark = pytest.mark.gpu
 
@@ -21,6 +27,49 @@ class _Proj:
 class _Cb:
     def __init__(self, cb):
         self.centroids, self.boundaries = to_dev(cb[0]), to_dev(cb[1])
+
+
+def _unit_flips(gpu_buf, oc, b, h, label):
+    """Tokens of unit (b, h) whose key codes differ from the oracle's (each
+    difference inside the boundary band); value fields and ring bit-exact."""
+    lay = oc.lay
+    ref = oc.to_bytes()
+    r = oc.rec[b][h]
+    if r is None:
+        return 0
+    n = r["rho"].shape[0]
+    fg = olayout.read_region(gpu_buf, lay, b, h, n)
+    fr = olayout.read_region(ref, lay, b, h, n)
+    for name in ("vcode", "vscale", "vmin"):
+        assert np.array_equal(fg[name], fr[name]), name
+    got = {"idx": fg["idx"], "signs": fg["sign"],
+           "rho": np.ascontiguousarray(fg["rho"]).view("<f4").ravel(),
+           "rnorm": np.ascontiguousarray(fg["rnorm"]).view("<f4").ravel() if oc.b1 else None}
+    return compare_keys(got, r, oc.d, oc.b1, oc.m, oc.cb[1] if oc.b1 else None,
+                        label=label)["skipped_tokens"]
+
+
+def _check_against_oracle(cache, oc, out, logits, Q, w, label):
+    """The GPU cache after a step vs the oracle's, then the step's output and
+    logits vs the oracle's decode for every unit whose codes are identical.
+    Returns the number of units checked."""
+    buf = cache.buffer.cpu().numpy()
+    lay = oc.lay
+    ref = oc.to_bytes()
+    assert np.array_equal(buf[lay.ring_k_off:], ref[lay.ring_k_off:]), "ring differs"
+    ro, rl = oc.decode(host(Q))
+    G = w.Hq // w.Hkv
+    o = host(out)
+    lg = logits.cpu().numpy().astype(np.float64)
+    checked = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            if _unit_flips(buf, oc, b, h, f"{label} unit ({b},{h})") == 0:
+                hs = slice(h * G, (h + 1) * G)
+                check_out(o[b:b + 1, hs], ro[b:b + 1, hs], w.dtype)
+                check_logits(lg[b, hs], rl[(b, h)])
+                checked += 1
+    return checked
 
 
 def _workload(**kw):
@@ -48,15 +97,20 @@ def test_decode_step_matches_append_then_decode(kw, n0, steps):
     K, V = synth.keys_values(w, device="cuda", T=total)
     caches = [CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
                                 dtype=TORCH_DT[w.dtype]) for _ in range(2)]
+    oc = ocache.OracleCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
+                            w.dtype, po, cb if w.b1 else None)
     for c in caches:
         c.append(K[:, :, :n0].contiguous(), V[:, :, :n0].contiguous(), pj, cbd)
+    oc.append(host(K[:, :, :n0]), host(V[:, :, :n0]))
     t = n0
+    checked = 0
     for i, n in enumerate(steps):
         k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
         Q = synth.queries(w.scaled(seed=50 + i), device="cuda")
         o1, l1 = caches[0].decode_step(k, v, Q, pj, cbd, want_logits=True)
         caches[1].append(k, v, pj, cbd)
         o2, l2 = caches[1].decode(Q, pj, cbd, want_logits=True)
+        oc.append(host(k), host(v))
         torch.cuda.synchronize()
         t += n
         assert caches[0].n_total == caches[1].n_total == t
@@ -64,6 +118,10 @@ def test_decode_step_matches_append_then_decode(kw, n0, steps):
         assert torch.equal(o1, o2), f"outputs differ after step {i}"
         assert torch.equal(l1, l2), f"logits differ after step {i}"
         assert torch.isfinite(o1.float()).all()
+        checked += _check_against_oracle(caches[0], oc, o1, l1, Q, w, f"decode step {i}")
+    record(f"decode step {kw} vs oracle", unit_steps_checked=checked,
+           unit_steps_skipped=len(steps) * w.B * w.Hkv - checked)
+    assert checked >= 1
 
 
 @pytest.mark.parametrize("kw,n0,steps", [

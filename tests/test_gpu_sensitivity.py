@@ -29,6 +29,25 @@ def test_key_moments_match_oracle(shape, dtype):
     assert abs(got - want) <= VAR_REL * want, (got, want)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+def test_key_variance_large_mean_small_spread(dtype):
+    """Mean 1e3 and standard deviation 1: the one-pass sum of squares would lose
+    about six digits here; the library's shifted sums match the oracle's
+    two-pass variance to 1e-9 relative."""
+    from compressed_attention_turboquantprod_b200 import key_variance, native
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    K = (torch.randn(4, 8, 1024, 128, generator=g, device="cuda") + 1000.0).to(dtype)
+    got = key_variance(K)
+    want = sens.key_variance(host(K))
+    assert abs(got - want) <= 1e-9 * want, (got, want)
+    out = torch.empty(2, dtype=torch.float64, device="cuda")
+    ws = torch.empty(native.tq_key_moments_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    native.tq_key_moments(K, out, ws)
+    mean = float(out[0].item())
+    assert abs(mean - float(host(K).mean())) <= 1e-12 * 1000.0
+
+
 def test_profile_of_synthetic_calibration_layers():
     """32 layers of synthetic calibration keys with variance 1 + 2 l / 31: the
     device variances give the oracle's profile (boundaries 8, 16, 24), and the

@@ -212,3 +212,32 @@ def test_exemption_masks():
     assert ex.tolist() == [[True, True, True, False]]
     z = np.array([[1.0, -1.0, 1e-7, 0.0]])
     assert quantize.sign_exempt(z).tolist() == [[False, False, True, True]]
+
+
+def test_band_agreement_counts_planted_mismatches():
+    """The comparison rule of the parity checks: a code flipped at an element
+    inside the boundary band counts as in-band (and its token's signs are left
+    out), a code flipped elsewhere and a sign flipped away from zero count as
+    outside the band."""
+    d, m, b1 = 16, 32, 2
+    p, (c32, b32) = _setup(d, m, b1)
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((50, d))
+    ref = quantize.quantize_keys(X, p["Pi"], p["S"], c32, b32, b1)
+    same = quantize.band_agreement(ref["idx"].copy(), ref["bits"].copy(), ref, b32)
+    assert same["outside_band"] == 0 and same["code_mismatch_in_band"] == 0
+    # plant y exactly on a boundary for token 3, coordinate 2: that element is exempt
+    ref2 = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in ref.items()}
+    ref2["y32"][3, 2] = b32[1]
+    idx = ref2["idx"].copy()
+    idx[3, 2] ^= 1
+    bits = ref2["bits"].copy()
+    bits[3, 0] ^= 1                         # dropped: token 3 has a flipped code
+    c = quantize.band_agreement(idx, bits, ref2, b32)
+    assert c["code_mismatch_in_band"] == 1 and c["tokens_with_a_flipped_code"] == 1
+    assert c["outside_band"] == 0
+    idx[7, 5] = (idx[7, 5] + 2) % 4          # far from any boundary (checked below)
+    assert not quantize.code_exempt(ref2["y32"], b32)[7, 5]
+    bits[9, np.argmax(np.abs(ref2["z"][9]))] ^= 1     # the largest |z|: never exempt
+    c = quantize.band_agreement(idx, bits, ref2, b32)
+    assert c["outside_band"] == 2
