@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-sensitivity", action="store_true")
     ap.add_argument("--workload", default="gqa32k")
+    ap.add_argument("--case", choices=sorted(CASES), default=None,
+                    help="run one small per-kernel workload (for a profiler capture) instead "
+                         "of the bench")
     return ap.parse_args()
 
 
@@ -573,6 +576,9 @@ def run_ours(args):
     if not args.no_quantize:
         quant, qsample = bench_quantize(
             dev, world, keep_sample=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    structured = None
+    if not args.no_quantize:
+        structured = bench_structured_rotation(dev, world)
     sensitivity = None
     if not args.no_sensitivity:
         sensitivity = bench_sensitivity(dev, world, peak, flush_l2)
@@ -628,6 +634,7 @@ def run_ours(args):
                      "avg_launch_ms": part_avg_ms, "source_hash": src_hash},
         "e2e": e2e,
         "quantize": quant,
+        "structured_rotation": structured,
         "prefill": prefill,
         "sensitivity": sensitivity,
         "other_decodes": others,
@@ -680,6 +687,7 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
     # P V MMAs (128 channels x 4 heads x hi/lo); int8 taken at twice the bf16 peak
     F = (1 << (w.b1 - 1)) if w.b1 > 0 else 0
     KS = F * w.d // 32 + w.m // 32
+    G = w.Hq // w.Hkv
     bf16, bf16_kind = measured_bf16_tflops()
     units = w.B * w.Hkv
     res = []
@@ -693,15 +701,24 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
         native.tq_prefill_check(cache.state, w.Hq, n, 0, ws)
         toks = reduce_sum(float(w.B * n), world)
         work = float(cache.n_comp) * units * n
+        # the method's own work per (history token, query token, KV head): for each of
+        # the G query heads the MSE dot (d), the QJL dot (m) and the P V row (d)
+        algo_flops = work * 2 * G * ((w.d if w.b1 > 0 else 0) + w.m + w.d)
+        algo_tflops = algo_flops / (t * 1e-3) / 1e12
         i8_ops, f16_ops = work * 16 * 32 * KS * 2, work * 128 * 8 * 2
         ideal_ms = (i8_ops / (2 * bf16 * 1e12) + f16_ops / (bf16 * 1e12)) * 1e3
         res.append({"n": n, "ms": t, "query_tokens_per_s": toks / (t * 1e-3),
                     "history_GB_per_s": reduce_sum(float(hist_bytes), world) / (t * 1e-3) / 1e9,
                     "vs_n_decodes": n * t_dec / t,
-                    "tensor": {"bound": "tensor", "int8_tops": i8_ops / (t * 1e-3) / 1e12,
-                               "f16_tflops": f16_ops / (t * 1e-3) / 1e12,
-                               "ideal_ms_at_peak": ideal_ms, "frac": ideal_ms / t,
-                               "peak_bf16_tflops": bf16, "peak_kind": bf16_kind}})
+                    "tensor": {"bound": "tensor", "achieved": algo_tflops, "peak": bf16,
+                               "unit": "TFLOP/s", "frac": algo_tflops / bf16,
+                               "flops": "algorithmic: 2 G (d + m + d) per (history token, query "
+                                        "token, KV head)",
+                               "peak_kind": bf16_kind,
+                               "executed": {"int8_tops": i8_ops / (t * 1e-3) / 1e12,
+                                            "f16_tflops": f16_ops / (t * 1e-3) / 1e12,
+                                            "ideal_ms_at_peak": ideal_ms,
+                                            "frac_of_executed_ideal": ideal_ms / t}}})
     return {"chunks": res, "decode_ms": t_dec, "history_bytes": hist_bytes,
             "history_tokens": int(cache.n_comp),
             "timing": "CUDA events around the whole call (prep, history partials, exact segment, "
@@ -886,6 +903,72 @@ def bench_quantize(dev, world, reps=3, keep_sample=False):
     return res, sample
 
 
+def bench_structured_rotation(dev, world, reps=5):
+    """What the fast Walsh-Hadamard transform buys where the rotation runs on CUDA
+    cores: the tile quantiser on the 262K wide-head shape (d = 256, no tensor-core
+    path; 4 KV heads x 16384 tokens per append) and the single-token append of a
+    decode step on the 32K GQA shape, each with the dense QR rotation and with the
+    structured one (same data)."""
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import Codebook, CompressedKVCache, Projections
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return reduce_max(e0.elapsed_time(e1) / reps, world)
+
+    res = {}
+    w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+    K, V = synth.keys_values(w, device=dev)
+    cb = Codebook(w.d, w.b1, device=dev)
+    keys = w.B * w.Hkv * w.T
+    for structured in (False, True):
+        pj = Projections(w.d, w.m, 0, device=dev, structured=structured)
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, 0, w.T,
+                                  dtype=w.torch_dtype, device=dev, structured=structured)
+
+        def call():
+            cache.state.n_total = 0
+            cache.append(K, V, pj, cb)
+        ms = timed(call)
+        res["tile_quantise_wide_Mkeys_per_s_" + ("hadamard" if structured else "dense")] = \
+            reduce_sum(keys / (ms * 1e-3) / 1e6, world)
+        del cache
+    del K, V
+    w = synth.WORKLOADS["gqa32k"].scaled(T=4096)
+    K, V = synth.keys_values(w, device=dev)
+    cb = Codebook(w.d, w.b1, device=dev)
+    n_calls = reps + 1
+    _, Kn, Vn = synth.decode_stream(w, n_calls, device=dev)
+    for structured in (False, True):
+        pj = Projections(w.d, w.m, 0, device=dev, structured=structured)
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W,
+                                  w.T + n_calls + 64, dtype=w.torch_dtype, device=dev,
+                                  structured=structured)
+        cache.append(K, V, pj, cb)
+        state = {"i": 0}
+
+        def step():
+            i = state["i"]
+            state["i"] = i + 1
+            cache.append(Kn[i], Vn[i], pj, cb)
+        ms = timed(step)
+        res["single_token_append_us_" + ("hadamard" if structured else "dense")] = ms * 1e3
+        del cache
+    res["workloads"] = ("tile quantiser: d=256, b1=3, m=256, 4-bit values g=64, 4 KV heads x 16384 "
+                        "bf16 tokens per append; single-token append: batch 8, 8 KV heads, d=128, "
+                        "b1=2, m=128, 16-token ring (the token leaving the ring is quantised)")
+    return res
+
+
 def oracle_quantize_counts(sample):
     """The oracle's one-shot quantisation of the sampled unit's 131072 tokens
     against the library's chunked append of them: near-boundary exemption counts
@@ -911,8 +994,128 @@ def oracle_quantize_counts(sample):
     return counts
 
 
+# --------------------------------------------------------------------------- per-kernel cases
+# Small workloads (inputs above L2 where the kernel streams, a few GB at most), one
+# call repeated, each reaching one or two kernels that the main bench does not
+# time on its own; `bench.py --case NAME` prints one JSON line with the mean call
+# time (CUDA events, L2 flushed before each call).
+CASES = {
+    "decode_cuda_core": "CUDA-core decode (k_decode_prep, k_decode_partial, k_decode_combine): "
+                        "batch 8, 16 query heads over 8 KV heads (G = 2: no tensor-core path), "
+                        "d = 64, context 32768, keys b1 = 2 + QJL m = 64, 2-bit values g = 32, bf16",
+    "quantize_sgemm": "64-token SGEMM tile quantise (k_quantize): the 262K wide-head shape (d = 256, "
+                      "b1 = 3, m = 256, 4-bit values g = 64, bf16), 4 KV heads x 16384 tokens per call",
+    "quantize_sgemm_hadamard": "the same with the structured rotation (the per-row fast "
+                               "Walsh-Hadamard transform instead of the rotation GEMM)",
+    "append_small": "single-token append (k_quantize_small, k_ring_write): the 32K GQA cache "
+                    "(batch 8, 8 KV heads, d = 128, 16-token ring), one token per sequence per call",
+    "prefill": "multi-token call (k_prefill_partial_mma, k_prefill_exact, merge) on the 32K GQA "
+               "cache, 16-token chunk",
+}
+
+
+def run_case(args):
+    import torch
+    import synth
+    from compressed_attention_turboquantprod_b200 import (Codebook, CompressedKVCache, Projections,
+                                                           native)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=args.steps, warm=args.warmup):
+        for _ in range(warm):
+            flush_w.zero_()
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush_w.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps
+
+    name = args.case
+    out = {"case": name, "what": CASES[name]}
+    if name == "decode_cuda_core":
+        w = synth.Workload("decode_cuda_core", B=8, Hq=16, Hkv=8, d=64, T=32768, W=16, b1=2, m=64,
+                           vbits=2, group=32, dtype="bf16", k_outlier_frac=0.02,
+                           v_outlier_frac=0.02, outlier_scale=8.0)
+        pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
+                                  dtype=w.torch_dtype, device=dev)
+        K, V = synth.keys_values(w, device=dev)
+        cache.append(K, V, pj, cb)
+        del K, V
+        Q = synth.queries(w, device=dev)
+        o = torch.empty_like(Q)
+        ws = cache.workspace(w.Hq)
+        scale = 1.0 / math.sqrt(w.d)
+        ms = timed(lambda: native.tq_decode_attention(cache.state, Q, scale, pj.Pi, pj.S,
+                                                      cb.centroids, o, None, 0, ws))
+        nb = w.B * w.Hkv * (cache.n_comp * cache.state.token_bytes + 2 * cache.n_ring * w.d * 2)
+        out.update(ms=ms, packed_bytes=nb, GB_per_s=nb / (ms * 1e-3) / 1e9)
+    elif name.startswith("quantize_sgemm"):
+        w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+        structured = name.endswith("hadamard")
+        pj = Projections(w.d, w.m, 0, device=dev, structured=structured)
+        cb = Codebook(w.d, w.b1, device=dev)
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, 0, w.T,
+                                  dtype=w.torch_dtype, device=dev, structured=structured)
+        K, V = synth.keys_values(w, device=dev)
+
+        def call():
+            cache.state.n_total = 0
+            cache.append(K, V, pj, cb)
+        ms = timed(call)
+        keys = w.B * w.Hkv * w.T
+        out.update(ms=ms, keys=keys, Mkeys_per_s=keys / (ms * 1e-3) / 1e6)
+    elif name == "append_small":
+        w = synth.WORKLOADS["gqa32k"]
+        pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)
+        n_calls = args.warmup + args.steps
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W,
+                                  w.T + n_calls + 64, dtype=w.torch_dtype, device=dev)
+        K, V = synth.keys_values(w, device=dev)
+        cache.append(K, V, pj, cb)
+        del K, V
+        _, Kn, Vn = synth.decode_stream(w, n_calls, device=dev)
+        it = iter(range(n_calls))
+
+        def call():
+            i = next(it)
+            cache.append(Kn[i], Vn[i], pj, cb)
+        ms = timed(call)
+        out.update(ms=ms, tokens_per_call=w.B * w.Hkv)
+    elif name == "prefill":
+        w = synth.WORKLOADS["gqa32k"]
+        pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)
+        cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
+                                  dtype=w.torch_dtype, device=dev)
+        K, V = synth.keys_values(w, device=dev)
+        cache.append(K, V, pj, cb)
+        del K, V
+        Q, Kc, Vc = synth.prefill_chunk(w, 16, device=dev)
+        o = torch.empty_like(Q)
+        ws = torch.empty(native.tq_prefill_workspace_bytes(cache.state, w.Hq, 16, 0),
+                         dtype=torch.uint8, device=dev)
+        scale = 1.0 / math.sqrt(w.d)
+        ms = timed(lambda: native.tq_prefill_attention(cache.state, Q, Kc, Vc, scale, pj.Pi, pj.S,
+                                                       cb.centroids, o, 0, ws))
+        native.tq_prefill_check(cache.state, w.Hq, 16, 0, ws)
+        out.update(ms=ms, query_tokens=w.B * 16)
+    torch.cuda.synchronize()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -104,8 +104,11 @@ class CompressedKVCache:
     """A packed cache of B x Hkv sequences plus its full-precision ring."""
 
     def __init__(self, B, Hkv, d, b1, m, vbits, group, W, capacity, dtype=torch.bfloat16,
-                 device="cuda"):
-        self.desc = native.make_desc(B, Hkv, d, b1, m, vbits, group, W, capacity, dtype)
+                 device="cuda", structured: bool = False):
+        """structured: the projections come from Projections(..., structured=True);
+        the rotations on CUDA cores then run as fast Walsh-Hadamard transforms."""
+        rot = native.TQ_ROTATION_HADAMARD if structured else native.TQ_ROTATION_DENSE
+        self.desc = native.make_desc(B, Hkv, d, b1, m, vbits, group, W, capacity, dtype, rot)
         self.dtype = dtype
         nbytes = native.tq_cache_bytes(self.desc)
         if nbytes == 0:

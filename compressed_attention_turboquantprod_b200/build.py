@@ -17,6 +17,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtq.so")
+# The bounds-checked build (every computed address checked on the device, failures
+# recorded, never trapped): the same sources with -DTQ_DEBUG_BOUNDS.
+LIB_BOUNDS = os.path.join(PKG, "libtq_bounds.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
@@ -34,21 +37,24 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
     deps.append(os.path.join(INCLUDE, "tq.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile libtq.so if needed; returns its path."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          bounds: bool = False) -> str:
+    """Compile libtq.so (bounds: libtq_bounds.so) if needed; returns its path."""
+    lib = LIB_BOUNDS if bounds else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp"
+    extra = ["-DTQ_DEBUG_BOUNDS"] if bounds else []
+    cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
@@ -58,10 +64,10 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose or ptxas_info:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv,
+                bounds="--bounds" in sys.argv))

@@ -92,6 +92,8 @@ int layout_status(const tq_cache_desc* dsc, tq_cache* out) {
     return fail(TQ_ERR_INVALID_ARG, "bad descriptor (B=%d Hkv=%d capacity=%lld W=%d)", dsc->B,
                 dsc->Hkv, (long long)dsc->capacity, dsc->W);
   if (!valid_dtype(dsc->dtype)) return fail(TQ_ERR_INVALID_ARG, "bad dtype %d", dsc->dtype);
+  if (dsc->rotation != TQ_ROTATION_DENSE && dsc->rotation != TQ_ROTATION_HADAMARD)
+    return fail(TQ_ERR_INVALID_ARG, "bad rotation %d", dsc->rotation);
   int st = check_shape(dsc->d, dsc->b1, dsc->m, dsc->vbits, dsc->group, true);
   if (st != TQ_OK) return st;
   const int d = dsc->d, b1 = dsc->b1;
@@ -197,11 +199,13 @@ Geom geom_of(const tq_cache* c) {
   g.group = d.group;
   g.W = d.W;
   g.dtype = d.dtype;
+  g.hadamard = d.rotation == TQ_ROTATION_HADAMARD && d.b1 > 0;
   g.capacity = d.capacity;
   g.block_bytes = c->block_bytes;
   g.region_bytes = c->region_bytes;
   g.ring_k_off = c->ring_k_off;
   g.ring_v_off = c->ring_v_off;
+  g.total_bytes = (int64_t)c->bytes;
   g.f_idx = d.b1 * d.d / 8;
   g.f_sign = d.m / 8;
   g.f_rnorm = d.b1 > 0 ? 4 : 0;
@@ -232,6 +236,39 @@ size_t decode_ws_bytes_now(const tq_cache* c, int Hq, int num_splits) {
 extern "C" {
 
 const char* tq_last_error(void) { return g_err.c_str(); }
+
+int tq_debug_bounds_enabled(void) {
+#ifdef TQ_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int tq_debug_bounds_check(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "tq_debug_bounds_check");
+  const struct {
+    const char* file;
+    int (*read)();
+  } files[] = {{"quant_kernels", tq::bounds_flag_quant},    {"decode_kernels", tq::bounds_flag_decode},
+               {"decode_tc", tq::bounds_flag_decode_tc},   {"decode_mma", tq::bounds_flag_decode_mma},
+               {"decode_mma_wide", tq::bounds_flag_wide}, {"prefill_mma", tq::bounds_flag_prefill}};
+  int first = 0;
+  const char* where = "";
+  for (const auto& f : files) {
+    const int v = f.read();
+    if (v != 0 && first == 0) {
+      first = v;
+      where = f.file;
+    }
+  }
+  if (first == -1) return fail(TQ_ERR_CUDA, "tq_debug_bounds_check: a flag could not be read");
+  if (first != 0)
+    return fail(TQ_ERR_CUDA, "bounds check %d failed in %s (an access outside its buffer was skipped)",
+                first, where);
+  return ok();
+}
 
 int tq_version(void) { return 1; }
 

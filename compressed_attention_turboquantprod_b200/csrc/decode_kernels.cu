@@ -107,7 +107,9 @@ __global__ void __launch_bounds__(DT) k_decode_partial(DParams p) {
     {
       const uint4* src = reinterpret_cast<const uint4*>(region + blk * g.block_bytes);
       uint4* dst = reinterpret_cast<uint4*>(sBuf);
-      for (int i = tid; i < (int)(g.block_bytes / 16); i += DT) dst[i] = src[i];
+      const bool inb = TQ_CHECKED(src, g.block_bytes, p.base, g.total_bytes, 501);
+      for (int i = tid; i < (int)(g.block_bytes / 16); i += DT)
+        dst[i] = inb ? src[i] : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
     const int nt = (int)min((int64_t)kBlockTokens, p.n_comp - blk * kBlockTokens);
@@ -191,8 +193,9 @@ __global__ void __launch_bounds__(DT) k_decode_partial(DParams p) {
         const int rr = i / d, c = i % d;
         const int64_t slot = (first + r0 + rr) % g.W;
         const int64_t e = ((int64_t)bh * g.W + slot) * d + c;
-        sK[rr * d + c] = load_f(p.base + g.ring_k_off, e, g.dtype);
-        sV[rr * d + c] = load_f(p.base + g.ring_v_off, e, g.dtype);
+        const bool inb = TQ_CHECKED(p.base + g.ring_v_off + e * es, es, p.base, g.total_bytes, 502);
+        sK[rr * d + c] = inb ? load_f(p.base + g.ring_k_off, e, g.dtype) : 0.f;
+        sV[rr * d + c] = inb ? load_f(p.base + g.ring_v_off, e, g.dtype) : 0.f;
       }
       (void)es;
       __syncthreads();
@@ -251,7 +254,9 @@ __global__ void __launch_bounds__(256) k_decode_prep(Geom g, const void* Q, int 
   __syncthreads();
   const float qscale = 1.2533141373155003f / (float)m;   // sqrt(pi/2) / m
   const int rows_pi = (g.b1 > 0) ? d : 0;
-  for (int r = warp; r < rows_pi + m; r += blockDim.x / 32) {
+  if (g.hadamard && warp == 0)      // Pi q as a butterfly: H (Pi[0,:] * q)
+    warp_hadamard_rotate(Pi, sq, 1.f, ws.qr + (int64_t)bq * d, d, lane);
+  for (int r = g.hadamard ? rows_pi + warp : warp; r < rows_pi + m; r += blockDim.x / 32) {
     const float* row = (r < rows_pi) ? Pi + (int64_t)r * d : S + (int64_t)(r - rows_pi) * d;
     float a = 0.f;
     for (int i = lane; i < d; i += 32) a = fmaf(row[i], sq[i], a);
@@ -396,5 +401,7 @@ cudaError_t launch_decode_combine(const Geom& g, int Hq, void* out, int splits,
   k_decode_combine<<<g.B * Hq, g.d, 0, s>>>(g, splits, out, ws);
   return cudaGetLastError();
 }
+
+TQ_BOUNDS_READER(bounds_flag_decode)
 
 }  // namespace tq

@@ -39,6 +39,7 @@
 // {0, 1, 2}, m in {64, 128, 192, 256, 384, 512}.  Other shapes use
 // decode_kernels.cu.
 #include <cfloat>
+#include <cstdlib>
 
 #include "mma_common.cuh"
 #include "prep_mma.cuh"
@@ -616,6 +617,7 @@ cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_
   p.ws = ws;
   p.err = ws.err;
   if (g.d == 256) return launch_partial_wide(p, s);
+  if (!getenv("TQ_LEGACY_DECODE")) return launch_partial_tc(p, s);
   const int ksq = g.m / 32;
   switch (g.b1 * 32 + ksq) {
     case 0 * 32 + 2: return launch_partial_t<0, 2>(p, s);
@@ -639,5 +641,7 @@ cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_
     default: return cudaErrorInvalidValue;
   }
 }
+
+TQ_BOUNDS_READER(bounds_flag_decode_mma)
 
 }  // namespace tq

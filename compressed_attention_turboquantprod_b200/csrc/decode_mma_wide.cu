@@ -102,13 +102,13 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
     if (ring_split) {
       const uint32_t nbytes = (uint32_t)(min(RC, p.n_ring) * WD * es);
       mbar_expect_tx(&ringbar, 2 * nbytes);
-      bulk_load(s_rk, ring_k, nbytes, &ringbar);
-      bulk_load(s_rv, ring_v, nbytes, &ringbar);
+      cache_bulk_load(s_rk, ring_k, nbytes, &ringbar, p.base, g.total_bytes, 202);
+      cache_bulk_load(s_rv, ring_v, nbytes, &ringbar, p.base, g.total_bytes, 203);
     }
     for (int s = 0; s < WNST; ++s) s_iss[s] = 0;
     for (int s = 0; s < WNST && s < nb; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
-      bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 204);
       s_iss[s] = 1;
     }
   }
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
         if (j + WNST < nb && !s_abort) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[st], (uint32_t)bb);
-          bulk_load(stage + (size_t)st * bb, region + (blk0 + j + WNST) * bb, (uint32_t)bb, &full[st]);
+          cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + WNST) * bb, (uint32_t)bb, &full[st], p.base, g.total_bytes, 205);
           s_iss[st] += 1;
         }
       }
@@ -403,8 +403,8 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
       if (ci > 0 && tid == 0) {
         const uint32_t nbytes = (uint32_t)(nc * WD * es);
         mbar_expect_tx(&ringbar, 2 * nbytes);
-        bulk_load(s_rk, ring_k + (int64_t)c0 * WD * es, nbytes, &ringbar);
-        bulk_load(s_rv, ring_v + (int64_t)c0 * WD * es, nbytes, &ringbar);
+        cache_bulk_load(s_rk, ring_k + (int64_t)c0 * WD * es, nbytes, &ringbar, p.base, g.total_bytes, 206);
+        cache_bulk_load(s_rv, ring_v + (int64_t)c0 * WD * es, nbytes, &ringbar, p.base, g.total_bytes, 207);
       }
       const bool rok = __all_sync(0xffffffffu, mbar_wait(&ringbar, (uint32_t)(ci & 1)));
       if (!rok && lane == 0) {
@@ -559,4 +559,7 @@ cudaError_t launch_partial_wide(const MParams& p, cudaStream_t s) {
 }
 
 }  // namespace mmadec
+
+TQ_BOUNDS_READER(bounds_flag_wide)
+
 }  // namespace tq

@@ -99,6 +99,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// A bulk copy out of the cache buffer [base, base + total); in the bounds-checked
+// build a source range outside it is recorded under `code` and not copied.
+__device__ __forceinline__ void cache_bulk_load(void* dst, const uint8_t* src, uint32_t bytes,
+                                                uint64_t* bar, const uint8_t* base, int64_t total,
+                                                int code) {
+  if (TQ_CHECKED(src, bytes, base, total, code)) bulk_load(dst, src, bytes, bar);
+}
+
 // Packed fp32 pairs (sm_100): one instruction for two IEEE products / fused
 // multiply-adds, each rounded exactly as the scalar operation.
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
@@ -168,6 +176,9 @@ __device__ __forceinline__ float slices_to_float(int s0, int s1, int s2, int s3)
   const int lo = s0 + 256 * s1, hi = s2 + 256 * s3;
   return fmaf(65536.f, __int2float_rn(hi), __int2float_rn(lo));
 }
+
+// The head-dim-128 partial kernel with the scores on tcgen05 (decode_tc.cu).
+cudaError_t launch_partial_tc(const MParams& p, cudaStream_t s);
 
 // The head-dim-256 kernel (decode_mma_wide.cu).
 bool decode_wide_supported(const Geom& g, int G);

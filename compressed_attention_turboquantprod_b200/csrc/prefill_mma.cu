@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(PNW * 32, 1) k_prefill_partial_mma(PParams p) 
     for (int s = 0; s < PNST; ++s) s_iss[s] = 0;
     for (int s = 0; s < PNST && s < nb; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
-      bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 302);
       s_iss[s] = 1;
     }
   }
@@ -362,8 +362,8 @@ __global__ void __launch_bounds__(PNW * 32, 1) k_prefill_partial_mma(PParams p) 
         if (j + PNST < nb && !s_abort) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[st], (uint32_t)bb);
-          bulk_load(stage + (size_t)st * bb, region + (blk0 + j + PNST) * bb, (uint32_t)bb,
-                    &full[st]);
+          cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + PNST) * bb, (uint32_t)bb,
+                    &full[st], p.base, g.total_bytes, 303);
           s_iss[st] += 1;
         }
       }
@@ -660,5 +660,7 @@ cudaError_t launch_prefill_exact(const Geom& g, const uint8_t* base, int64_t n_t
   k_prefill_exact<<<grid, ET, 0, s>>>(p);
   return cudaGetLastError();
 }
+
+TQ_BOUNDS_READER(bounds_flag_prefill)
 
 }  // namespace tq

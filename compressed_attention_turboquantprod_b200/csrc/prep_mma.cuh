@@ -41,8 +41,9 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
   __shared__ float s_sumqr[MG], s_sumqs[MG];
   const int bq0 = b * Hq + h * MG;
   const int rows_pi = b1 > 0 ? d : 0;
-  // this part's rows of [Pi; S]: [r_begin, r_end)
-  const int r_begin = do_mse ? 0 : rows_pi, r_end = do_qjl ? rows_pi + m : rows_pi;
+  // this part's rows of [Pi; S]: [r_begin, r_end) (with the structured rotation, Pi q
+  // is a butterfly instead: no rows of Pi are read but row 0)
+  const int r_begin = do_mse && !g.hadamard ? 0 : rows_pi, r_end = do_qjl ? rows_pi + m : rows_pi;
   {
     // the rows are read after the queries: start them towards L2 now
     const int l0 = r_begin * d / 32, l1 = r_end * d / 32, lines_pi = rows_pi * d / 32;
@@ -76,6 +77,10 @@ __device__ __forceinline__ void prep_mma_body(const Geom& g, const void* Q, int 
   // with columns 4l..4l+3 of the four queries (held in registers); a
   // reduce-scatter over the warp then leaves the sum of (row l/4, head l%4) in
   // lane l.  (NV float4s per lane per row: columns 128 c + 4 lane.)
+  if (g.hadamard && do_mse && warp < MG) {   // Pi q = H (Pi[0,:] * q), head = warp
+    warp_hadamard_rotate(Pi, sq + warp * d, 1.f, sqr + warp * d, d, lane);
+    for (int j = lane; j < d; j += 32) ws.qr[(int64_t)(bq0 + warp) * d + j] = sqr[warp * d + j];
+  }
   float4 qv[MG][NV];
 #pragma unroll
   for (int hh = 0; hh < MG; ++hh)

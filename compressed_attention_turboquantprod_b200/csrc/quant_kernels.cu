@@ -41,6 +41,7 @@ struct QParams {
   // shapes
   int d, b1, m, vbits, group;
   bool do_keys, do_values;
+  bool hadamard;      // Pi = H diag(s) / sqrt(d): y = H (Pi[0,:] * x) / rho as a butterfly
   const float* Pi;
   const float* T;
   const float* cent;
@@ -97,33 +98,52 @@ __device__ Smem carve(unsigned char* raw, int d) {
 }
 
 // Element pointer base + index of row i (token t_first + i) of (b, h) in the source.
+// (Bounds-checked build: a row outside its buffer reads from the sink.)
 __device__ __forceinline__ const void* src_row(const QParams& p, bool values, int bh, int64_t i,
                                                int64_t& elem) {
   const int d = p.d;
+  const int es = p.dtype == TQ_F32 ? 4 : 2;
   const void* chunk = values ? p.V : p.K;
+  const void* base = chunk;
+  int64_t rows;
   if (!p.cache_mode) {
     elem = i * d;
-    return chunk;
+    rows = p.t_first + p.n;
+  } else {
+    const int64_t t = p.t_first + i;
+    if (t < p.n_old) {
+      elem = ((int64_t)bh * p.g.W + t % p.g.W) * d;
+      base = values ? p.ringV : p.ringK;
+      rows = (int64_t)p.g.B * p.g.Hkv * p.g.W;
+    } else {
+      elem = ((int64_t)bh * p.n_new + (t - p.n_old)) * d;
+      rows = (int64_t)p.g.B * p.g.Hkv * p.n_new;
+    }
   }
-  const int64_t t = p.t_first + i;
-  if (t < p.n_old) {
-    elem = ((int64_t)bh * p.g.W + t % p.g.W) * d;
-    return values ? p.ringV : p.ringK;
+  if (!TQ_CHECKED(static_cast<const char*>(base) + elem * es, (int64_t)d * es, base,
+                  rows * d * es, values ? 402 : 401)) {
+    elem = 0;
+    return TQ_SINK(const void*);
   }
-  elem = ((int64_t)bh * p.n_new + (t - p.n_old)) * d;
-  return chunk;
+  return base;
 }
 
 // 16-bit half x (codes of channels (16/vbits) x ...) of the value codes of row i:
 // token-major in the standalone arrays, token-pair records in the cache.
 __device__ __forceinline__ uint16_t* code_half_ptr(const QParams& p, int bh, int64_t i, int x) {
+  uint16_t* r;
   if (p.cache_mode) {
     const Geom& g = p.g;
     const int64_t t = p.t_first + i;
     uint8_t* blk = p.base + (int64_t)bh * g.region_bytes + (t / kBlockTokens) * g.block_bytes;
-    return reinterpret_cast<uint16_t*>(blk + g.o_vcode + vcode_half_off(g, (int)(t % kBlockTokens), x));
+    r = reinterpret_cast<uint16_t*>(blk + g.o_vcode + vcode_half_off(g, (int)(t % kBlockTokens), x));
+    if (!TQ_CHECKED(r, 2, p.base, g.total_bytes, 403)) r = TQ_SINK(uint16_t*);
+  } else {
+    r = reinterpret_cast<uint16_t*>(p.arr.codes + (p.t_first + i) * (p.d * p.vbits / 8)) + x;
+    if (!TQ_CHECKED(r, 2, p.arr.codes, (p.t_first + p.n) * (p.d * p.vbits / 8), 404))
+      r = TQ_SINK(uint16_t*);
   }
-  return reinterpret_cast<uint16_t*>(p.arr.codes + (p.t_first + i) * (p.d * p.vbits / 8)) + x;
+  return r;
 }
 
 // Base of row i's value codes and the byte offset of its 16-bit half x from that
@@ -141,7 +161,7 @@ __device__ __forceinline__ int code_half_off(const QParams& p, int x) {
   return p.cache_mode ? vcode_half_off(p.g, 0, x) : 2 * x;
 }
 
-__device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t i, int which) {
+__device__ __forceinline__ uint8_t* dst_field_raw(const QParams& p, int bh, int64_t i, int which) {
   // which: 0 idx, 1 sign, 2 rho, 3 rnorm, 5 vscale, 6 vmin (value codes: code_half_ptr)
   if (p.cache_mode) {
     const Geom& g = p.g;
@@ -165,6 +185,30 @@ __device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t 
     case 5: return reinterpret_cast<uint8_t*>(p.arr.vscale + ti * (d / p.group));
     default: return reinterpret_cast<uint8_t*>(p.arr.vmin + ti * (d / p.group));
   }
+}
+
+// Field `which` of row i (bounds-checked build: the sink when it falls outside
+// the cache buffer or the caller's array).
+__device__ __forceinline__ uint8_t* dst_field(const QParams& p, int bh, int64_t i, int which) {
+  uint8_t* r = dst_field_raw(p, bh, i, which);
+#ifdef TQ_DEBUG_BOUNDS
+  const int d = p.d;
+  const int fsz = which == 0 ? p.b1 * d / 8 : which == 1 ? p.m / 8 : which <= 3 ? 4 : 4 * (d / p.group);
+  const void* lo;
+  int64_t ext;
+  if (p.cache_mode) {
+    lo = p.base;
+    ext = p.g.total_bytes;
+  } else {
+    const int64_t rows = p.t_first + p.n;
+    lo = which == 0 ? (const void*)p.arr.idx : which == 1 ? (const void*)p.arr.signs
+       : which == 2 ? (const void*)p.arr.rho : which == 3 ? (const void*)p.arr.rnorm
+       : which == 5 ? (const void*)p.arr.vscale : (const void*)p.arr.vmin;
+    ext = rows * fsz;
+  }
+  if (!TQ_CHECKED(r, fsz, lo, ext, 410 + which)) r = TQ_SINK(uint8_t*);
+#endif
+  return r;
 }
 
 // code = clamp(rint(fl((v - mn) / s)), 0, levels) with fl the IEEE fp32 quotient.
@@ -275,16 +319,21 @@ __device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int6
   __syncthreads();
   const float* E = s.X;
   if (b1 > 0) {
-    for (int col0 = 0; col0 < d; col0 += NC) {
-      float acc[4][8];
-      gemm_pass(s.X, sx, p.Pi, d, col0, d, s.B, acc);
+    if (p.hadamard) {      // a butterfly per row, one warp each
+      for (int r = warp; r < NT; r += THREADS / 32)
+        warp_hadamard_rotate(p.Pi, s.X + r * sx, s.inv[r], s.Y + r * sx, d, lane);
+    } else {
+      for (int col0 = 0; col0 < d; col0 += NC) {
+        float acc[4][8];
+        gemm_pass(s.X, sx, p.Pi, d, col0, d, s.B, acc);
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int col = col0 + tx + 16 * c;
-          if (col < d) s.Y[(4 * ty + r) * sx + col] = acc[r][c] * s.inv[4 * ty + r];
-        }
+          for (int c = 0; c < 8; ++c) {
+            const int col = col0 + tx + 16 * c;
+            if (col < d) s.Y[(4 * ty + r) * sx + col] = acc[r][c] * s.inv[4 * ty + r];
+          }
+      }
     }
     __syncthreads();
     const int L = 1 << b1;
@@ -416,7 +465,9 @@ __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V
                           ((int64_t)bh * n_new + (t - n_old)) * row_words;
     uint32_t* dst = reinterpret_cast<uint32_t*>(base + (which ? g.ring_v_off : g.ring_k_off)) +
                     ((int64_t)bh * g.W + t % g.W) * row_words;
-    dst[w] = src[w];
+    if (TQ_CHECKED(src + w, 4, which ? V : K, (int64_t)g.B * g.Hkv * n_new * row_words * 4, 420) &&
+        TQ_CHECKED(dst + w, 4, base, g.total_bytes, 421))
+      dst[w] = src[w];
   }
 }
 
@@ -501,7 +552,7 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
       // this thread's halves of its rows of Pi and T are read after the norm
       const int half = tid & 1;
       for (int j = tid >> 1; j < d; j += SMALL_THREADS / 2)
-        if (b1 > 0)
+        if (b1 > 0 && !p.hadamard)
           for (int c = half * (d / 2); c < (half + 1) * (d / 2); c += 32) prefetch_l2(p.Pi + (int64_t)j * d + c);
       for (int a = tid >> 1; a < m; a += SMALL_THREADS / 2)
         for (int c = half * (d / 2); c < (half + 1) * (d / 2); c += 32) prefetch_l2(p.T + (int64_t)a * d + c);
@@ -509,7 +560,8 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     // d <= 128: this thread's half of Pi row tid / 2 goes out with the key itself
     const bool regs = d <= 128;
     HalfRowRegs hr;
-    if (regs && b1 > 0 && (tid >> 1) < d) half_row_load(hr, p.Pi + (int64_t)(tid >> 1) * d, d, tid & 1);
+    if (regs && b1 > 0 && !p.hadamard && (tid >> 1) < d)
+      half_row_load(hr, p.Pi + (int64_t)(tid >> 1) * d, d, tid & 1);
     int64_t e0;
     const void* src = src_row(p, false, bh, row, e0);
     double ss = 0.0;
@@ -521,7 +573,8 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     ss = warp_sum_d(ss);
     if (lane == 0) s_red[warp] = ss;
     __syncthreads();
-    if (ring_new)    // the token is in shared memory: its ring slot takes the new one
+    if (ring_new &&  // the token is in shared memory: its ring slot takes the new one
+        TQ_CHECKED(static_cast<const char*>(src) + e0 * es, d * es, p.base, p.g.total_bytes, 422))
       copy_row16(reinterpret_cast<char*>(const_cast<void*>(src)) + e0 * es, ring_new, d * es, tid,
                  SMALL_THREADS);
     double t = 0.0;
@@ -532,7 +585,10 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     const float* E = sx;
     const int half = tid & 1;
     if (b1 > 0) {
-      if (regs) {
+      if (p.hadamard) {       // y = H (Pi[0,:] * x) / rho as a butterfly in warp 0
+        if (warp == 0) warp_hadamard_rotate(p.Pi, sx, inv, sy, d, lane);
+        if (regs && (tid >> 1) < m) half_row_load(hr, p.T + (int64_t)(tid >> 1) * d, d, half);
+      } else if (regs) {
         if ((tid >> 1) < d) {
           const float a = half_dot(hr, sx, d, half);
           if (half == 0) sy[tid >> 1] = a * inv;
@@ -598,7 +654,8 @@ __device__ __forceinline__ void quantize_small_body(const QParams& p, int64_t ro
     const void* src = src_row(p, true, bh, row, e0);
     for (int c = tid; c < d; c += SMALL_THREADS) sx[c] = load_f(src, e0 + c, p.dtype);
     __syncthreads();
-    if (ring_new)
+    if (ring_new &&
+        TQ_CHECKED(static_cast<const char*>(src) + e0 * es, d * es, p.base, p.g.total_bytes, 423))
       copy_row16(reinterpret_cast<char*>(const_cast<void*>(src)) + e0 * es, ring_new, d * es, tid,
                  SMALL_THREADS);
     float* vs = sz;            // [ng] scales, [ng] minima
@@ -1086,7 +1143,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
         const int nh = 32 / cpw;
 #pragma unroll
         for (int x = 0; x < 8; ++x)
-          if (x < nh) *reinterpret_cast<uint16_t*>(cb + s_hofs[part][x]) = (uint16_t)hw[x];
+          if (x < nh && TQ_CHECKED(cb + s_hofs[part][x], 2, p.cache_mode ? p.base : p.arr.codes,
+                                   p.cache_mode ? p.g.total_bytes
+                                                : (p.t_first + p.n) * (p.d * p.vbits / 8), 424))
+            *reinterpret_cast<uint16_t*>(cb + s_hofs[part][x]) = (uint16_t)hw[x];
       }
     }
     // ---- 3. codes, E, ||r||
@@ -1301,6 +1361,7 @@ cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* b
   p.bnd = bnd;
   p.base = base;
   p.g = g;
+  p.hadamard = g.hadamard;
   return run_quantize(p, g.B * g.Hkv, s);
 }
 
@@ -1339,6 +1400,7 @@ cudaError_t launch_decode_step_pre(const QuantSrc& src, int64_t n_ring_only, con
   p.bnd = bnd;
   p.base = base;
   p.g = g;
+  p.hadamard = g.hadamard;
   const int units = g.B * g.Hkv;
   const int nq = (int)(src.n * units * 2), nr = (int)(n_ring_only * units);
   StepPrep sp{g, Q, Hq, Pi, S, cent, softmax_scale * mmadec::kLog2e, ws};
@@ -1351,5 +1413,7 @@ cudaError_t launch_decode_step_pre(const QuantSrc& src, int64_t n_ring_only, con
   kern<<<nq + nr + 2 * units, SMALL_THREADS, smem, s>>>(p, nq, nr, sp);   // prep: 2 halves a unit
   return cudaGetLastError();
 }
+
+TQ_BOUNDS_READER(bounds_flag_quant)
 
 }  // namespace tq

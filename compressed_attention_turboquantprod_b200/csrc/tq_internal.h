@@ -16,13 +16,25 @@ constexpr int kMaxLevels = 16;    // 2^b1 for b1 <= 4 (codebook build)
 // Geometry of the packed cache, as plain values for kernels.
 struct Geom {
   int B, Hkv, d, b1, m, vbits, group, W, dtype;
+  bool hadamard;      // Pi = H diag(s) / sqrt(d): rotations on CUDA cores as a butterfly
   int64_t capacity;
   int64_t block_bytes, region_bytes, ring_k_off, ring_v_off;
+  int64_t total_bytes;  // the cache buffer's extent (bounds-checked build)
   int f_idx, f_sign, f_rnorm, f_vcode, f_vmeta;        // bytes per token per field
   int o_idx, o_sign, o_rho, o_rnorm, o_vcode, o_vscale, o_vmin;  // field offsets in a block
 };
 
 Geom geom_of(const tq_cache* c);
+
+// Bounds-checked build: each kernel file's flag (the code of its first failed
+// check, 0 if none; -1 if it could not be read), read and cleared.  In the normal
+// build these return 0.
+int bounds_flag_quant();
+int bounds_flag_decode();
+int bounds_flag_decode_tc();
+int bounds_flag_decode_mma();
+int bounds_flag_wide();
+int bounds_flag_prefill();
 
 // Record a thread-local error message (printf-style) and return `status`.
 int set_error(int status, const char* fmt, ...);

@@ -14,7 +14,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtq.so")
+# TQ_LIBRARY=bounds loads the bounds-checked build (libtq_bounds.so) instead.
+LIB_PATH = os.path.join(_HERE, "libtq_bounds.so" if os.environ.get("TQ_LIBRARY") == "bounds"
+                        else "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CAPACITY, TQ_ERR_CUDA, TQ_ERR_NOT_CONVERGED = range(6)
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
@@ -35,7 +37,7 @@ class tq_cache_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("b1", ctypes.c_int32), ("m", ctypes.c_int32), ("vbits", ctypes.c_int32),
                 ("group", ctypes.c_int32), ("W", ctypes.c_int32), ("capacity", ctypes.c_int64),
-                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("rotation", ctypes.c_int32)]
 
 
 class tq_cache(ctypes.Structure):
@@ -65,6 +67,8 @@ def _load() -> ctypes.CDLL:
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_version": (I, []),
         "tq_debug_fail_next": (I, [ctypes.c_char_p]),
+        "tq_debug_bounds_enabled": (I, []),
+        "tq_debug_bounds_check": (I, []),
         "tq_codebook_build": (I, [I, I, P, P, P]),
         "tq_projections_workspace_bytes": (SZ, [I]),
         "tq_make_projections": (I, [I, I, I, U64, U64, P, P, P, P, SZ, P]),
@@ -175,9 +179,13 @@ def tq_quantize_values(V: torch.Tensor, vbits: int, group: int, codes, scale, vm
 
 
 # ----------------------------------------------------------------------------- cache
-def make_desc(B, Hkv, d, b1, m, vbits, group, W, capacity, dtype) -> tq_cache_desc:
+TQ_ROTATION_DENSE, TQ_ROTATION_HADAMARD = 0, 1
+
+
+def make_desc(B, Hkv, d, b1, m, vbits, group, W, capacity, dtype,
+              rotation=TQ_ROTATION_DENSE) -> tq_cache_desc:
     return tq_cache_desc(B, Hkv, d, b1, m, vbits, group, W, capacity,
-                         dtype if isinstance(dtype, int) else dtype_code(dtype), 0)
+                         dtype if isinstance(dtype, int) else dtype_code(dtype), rotation)
 
 
 def tq_cache_bytes(desc: tq_cache_desc) -> int:
@@ -345,3 +353,11 @@ def tq_m_for_layer(groups: tq_layer_groups, layer: int) -> int:
 
 def tq_debug_fail_next(name: Optional[str]):
     lib.tq_debug_fail_next(name.encode() if name else None)
+
+
+def tq_debug_bounds_enabled() -> int:
+    return lib.tq_debug_bounds_enabled()
+
+
+def tq_debug_bounds_check():
+    _check(lib.tq_debug_bounds_check(), "tq_debug_bounds_check")

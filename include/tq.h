@@ -124,6 +124,12 @@ int tq_make_projections(int d, int m, int layer, uint64_t base_seed, uint64_t st
  * -1; every entry is +-fl32(1/sqrt(d)).  S and T = S Pi^T as tq_make_projections
  * (same seed rule, same S).  Pi is orthogonal, so every call that takes Pi and T
  * works unchanged with it; Pi u is a fast Walsh-Hadamard transform of s * u.
+ * A cache whose descriptor says rotation = TQ_ROTATION_HADAMARD reads only row 0
+ * of Pi (= s / sqrt(d)) where the rotation runs on CUDA cores -- the append of up
+ * to 8 tokens per sequence (a decode step), the tile quantiser of shapes without
+ * the tensor-core path, and the query preparation of every decode and prefill --
+ * and applies Pi u = H (Pi[0,:] * u) as an O(d log d) butterfly; the tensor-core
+ * tile quantiser multiplies by the dense Pi.
  *   Pi  device float[d*d] row-major (written)
  *   S   device float[m*d] row-major (written)
  *   T   device float[m*d] row-major (written; may be NULL)
@@ -185,8 +191,15 @@ typedef struct tq_cache_desc {
   int32_t W;          /* full-precision ring size, 0..1024                    */
   int64_t capacity;   /* max compressed tokens per (b, kv head)              */
   int32_t dtype;      /* dtype of K, V, Q, the ring and the output           */
-  int32_t reserved;
+  int32_t rotation;   /* TQ_ROTATION_DENSE (0): Pi any orthogonal matrix;
+                         TQ_ROTATION_HADAMARD (1): Pi from
+                         tq_make_projections_hadamard, applied as a fast
+                         Walsh-Hadamard transform where the rotation runs on
+                         CUDA cores (see tq_make_projections_hadamard)      */
 } tq_cache_desc;
+
+#define TQ_ROTATION_DENSE 0
+#define TQ_ROTATION_HADAMARD 1
 
 /*
  * Cache state.  Layout of the device buffer (also defined by the CPU oracle):
@@ -509,6 +522,22 @@ int tq_key_moments(const void* K, int dtype, int64_t n, double* out, void* works
  */
 int tq_sensitivity_profile(const double* layer_var, int L, int num_groups, int m_avg, int m_min,
                            int m_max, tq_layer_groups* out);
+
+/*
+ * Bounds-checked build (libtq_bounds.so, compiled with -DTQ_DEBUG_BOUNDS; not a
+ * method step).  In that build every kernel checks each address it computes from
+ * cache geometry, token positions or split ranges against the buffer it belongs
+ * to (the cache buffer, the caller's arrays, the workspace); a failing check
+ * records its code in a device flag and the access is not made (stores go to a
+ * sink, loads read zeros, a bulk copy is skipped and the consumer's bounded wait
+ * reports it).  No check traps.
+ * tq_debug_bounds_enabled -- 1 in the bounds-checked build, 0 otherwise.
+ * tq_debug_bounds_check -- SYNCHRONOUS (device-wide): reads and clears every
+ *   kernel file's flag; TQ_ERR_CUDA naming the first failed check's code when one
+ *   is set, TQ_OK otherwise (always TQ_OK in the normal build).
+ */
+int tq_debug_bounds_enabled(void);
+int tq_debug_bounds_check(void);
 
 #ifdef __cplusplus
 }

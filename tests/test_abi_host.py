@@ -266,3 +266,16 @@ def test_sharded_decode_calls_checked_on_the_host(nat):
                  (FAKE, FAKE, 4, 3, 2048, 2), (FAKE, FAKE, 4, 3, 128, 9)):
         assert L.tq_merge_partials(*args, FAKE, None) == nat.TQ_ERR_INVALID_ARG
     assert L.tq_merge_partials(FAKE, FAKE, 4, 3, 128, 2, None, None) == nat.TQ_ERR_INVALID_ARG
+
+
+def test_rotation_field_of_the_descriptor(nat):
+    """rotation 0 (dense) and 1 (Hadamard) give the same layout; anything else is
+    rejected before any device work."""
+    base = (2, 2, 128, 2, 128, 2, 32, 16, 1000, 2)
+    dense = nat.tq_cache_bytes(nat.make_desc(*base, rotation=nat.TQ_ROTATION_DENSE))
+    had = nat.tq_cache_bytes(nat.make_desc(*base, rotation=nat.TQ_ROTATION_HADAMARD))
+    assert dense == had > 0
+    assert nat.tq_cache_bytes(nat.make_desc(*base, rotation=2)) == 0
+    with pytest.raises(nat.TQError) as ei:
+        nat.tq_cache_layout(nat.make_desc(*base, rotation=-1))
+    assert ei.value.status == nat.TQ_ERR_INVALID_ARG and "rotation" in ei.value.message

@@ -382,3 +382,55 @@ def test_gqa32k_shape_reduced_context_end_to_end():
             check_out(host(out[b:b + 1, 4 * h:4 * h + 4]), ro, w.dtype)
             checked += 1
     assert checked >= 2
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),                                                          # d=128: tensor-core paths
+    dict(d=256, b1=3, m=256, vbits=4, group=64, Hq=8, Hkv=2),        # d=256: tile quantiser + wide
+    dict(d=64, b1=2, m=64, Hq=4, Hkv=2, dtype="f32"),                # CUDA-core decode (G = 2)
+])
+def test_hadamard_fast_transform_every_rotation_site(kw):
+    """A cache flagged with the structured rotation applies Pi = H diag(s)/sqrt(d)
+    as a fast Walsh-Hadamard transform wherever the rotation runs on CUDA cores:
+    the append of up to 8 tokens, the tile quantiser of shapes without the
+    tensor-core path, the fused decode step and the query preparation.  Given the
+    oracle's (dense) Hadamard projections, the packed cache agrees with the
+    oracle's outside the boundary band and the outputs with the oracle's decode."""
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache
+    w = _workload(T=400, **kw)
+    po, cb = oracle_setup(w.d, w.b1, w.m, layer=3, structured=True)
+    pj, cbd = _Proj(po), _Cb(cb)
+    K, V = synth.keys_values(w, device="cuda")
+    cap = 448
+    gc = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, cap,
+                           dtype=TORCH_DT[w.dtype], structured=True)
+    oc = _oracle_cache(w, cap, po, cb)
+    G = w.Hq // w.Hkv
+    t, checked, units = 0, 0, 0
+    for i, (n, how) in enumerate(((300, "append"), (5, "append"), (1, "step"), (3, "step"),
+                                  (1, "append"), (2, "step"))):
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        Q = synth.queries(w.scaled(seed=200 + i), device="cuda")
+        if how == "append":
+            gc.append(k, v, pj, cbd)
+            oc.append(host(k), host(v))
+            out, lg = gc.decode(Q, pj, cbd, want_logits=True)
+        else:
+            out, lg = gc.decode_step(k, v, Q, pj, cbd, want_logits=True)
+            oc.append(host(k), host(v))
+        torch.cuda.synchronize()
+        t += n
+        flips = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc, per_unit=True,
+                                     label=f"hadamard transform {w.d} step {i}")
+        ro, rl = oc.decode(host(Q))
+        o, lgs = host(out), lg.cpu().numpy().astype(np.float64)
+        for (b, h), f in flips.items():
+            units += 1
+            if f == 0:
+                hs = slice(h * G, (h + 1) * G)
+                check_out(o[b:b + 1, hs], ro[b:b + 1, hs], w.dtype)
+                check_logits(lgs[b, hs], rl[(b, h)])
+                checked += 1
+    record(f"hadamard transform d={w.d} end-to-end checks", unit_steps_checked=checked,
+           unit_steps_skipped=units - checked)
+    assert checked >= 1
