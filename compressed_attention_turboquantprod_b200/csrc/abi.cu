@@ -251,9 +251,9 @@ int tq_debug_bounds_check(void) {
   const struct {
     const char* file;
     int (*read)();
-  } files[] = {{"quant_kernels", tq::bounds_flag_quant},    {"decode_kernels", tq::bounds_flag_decode},
-               {"decode_tc", tq::bounds_flag_decode_tc},   {"decode_mma", tq::bounds_flag_decode_mma},
-               {"decode_mma_wide", tq::bounds_flag_wide}, {"prefill_mma", tq::bounds_flag_prefill}};
+  } files[] = {{"quant_kernels", tq::bounds_flag_quant}, {"decode_kernels", tq::bounds_flag_decode},
+               {"decode_mma", tq::bounds_flag_decode_mma}, {"decode_mma_wide", tq::bounds_flag_wide},
+               {"prefill_mma", tq::bounds_flag_prefill}};
   int first = 0;
   const char* where = "";
   for (const auto& f : files) {

@@ -39,7 +39,6 @@
 // {0, 1, 2}, m in {64, 128, 192, 256, 384, 512}.  Other shapes use
 // decode_kernels.cu.
 #include <cfloat>
-#include <cstdlib>
 
 #include "mma_common.cuh"
 #include "prep_mma.cuh"
@@ -121,13 +120,13 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     if (ring_split) {
       const uint32_t nbytes = (uint32_t)(min(RC, p.n_ring) * MD * es);
       mbar_expect_tx(&ringbar, 2 * nbytes);
-      bulk_load(s_rk, ring_k, nbytes, &ringbar);
-      bulk_load(s_rv, ring_v, nbytes, &ringbar);
+      cache_bulk_load(s_rk, ring_k, nbytes, &ringbar, p.base, g.total_bytes, 101);
+      cache_bulk_load(s_rv, ring_v, nbytes, &ringbar, p.base, g.total_bytes, 102);
     }
     for (int s = 0; s < NST; ++s) s_iss[s] = 0;
     for (int s = 0; s < NST && s < nb; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
-      bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s]);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 103);
       s_iss[s] = 1;
     }
   }
@@ -301,12 +300,13 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     if (p.logits) {
       const float inv = 1.f / p.scale_log2;
       float* lg = p.logits + (int64_t)(bq0 + tig) * p.n_log + tok0;
+      const int64_t nlog_all = (int64_t)g.B * p.Hq * p.n_log;
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int t = tb + 16 * r + gid + 8 * e;
-          if (t < nt_valid) lg[t] = l[r][e] * inv;
+          if (t < nt_valid && TQ_CHECKED(lg + t, 4, p.logits, 4 * nlog_all, 111)) lg[t] = l[r][e] * inv;
         }
     }
 
@@ -400,8 +400,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
         if (j + NST < nb && !s_abort) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[st], (uint32_t)bb);
-          bulk_load(stage + (size_t)st * bb, region + (blk0 + j + NST) * bb, (uint32_t)bb,
-                    &full[st]);
+          cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + NST) * bb, (uint32_t)bb,
+                    &full[st], p.base, g.total_bytes, 104);
           s_iss[st] += 1;
         }
       }
@@ -439,8 +439,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       if (ci > 0 && tid == 0) {
         const uint32_t nbytes = (uint32_t)(nc * MD * es);
         mbar_expect_tx(&ringbar, 2 * nbytes);
-        bulk_load(s_rk, ring_k + (int64_t)c0 * MD * es, nbytes, &ringbar);
-        bulk_load(s_rv, ring_v + (int64_t)c0 * MD * es, nbytes, &ringbar);
+        cache_bulk_load(s_rk, ring_k + (int64_t)c0 * MD * es, nbytes, &ringbar, p.base, g.total_bytes, 105);
+        cache_bulk_load(s_rv, ring_v + (int64_t)c0 * MD * es, nbytes, &ringbar, p.base, g.total_bytes, 106);
       }
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&ringbar, (uint32_t)(ci & 1)));
       if (!ok && lane == 0) {
@@ -460,7 +460,9 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
 #pragma unroll 8
         for (int j = 0; j < MD; ++j) dot = fmaf(q[j], load_f(s_rk, (int64_t)sl * MD + j, g.dtype), dot);
         const int64_t rt = ((int64_t)(c0 + sl) - first % g.W + g.W) % g.W;
-        if (p.logits) p.logits[(int64_t)(bq0 + tig) * p.n_log + p.n_comp + rt] = dot;
+        float* dst = p.logits + (int64_t)(bq0 + tig) * p.n_log + p.n_comp + rt;
+        if (p.logits && TQ_CHECKED(dst, 4, p.logits, 4 * (int64_t)g.B * p.Hq * p.n_log, 112))
+          *dst = dot;
         l = dot * p.scale_log2;
       }
       float p0, p1;
@@ -516,11 +518,13 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     *reinterpret_cast<float2*>(&s_out[(warp * MG + tig) * MD + chan(mt)]) = make_float2(o0, o1);
   }
   __syncthreads();
+  const int64_t rows = (int64_t)g.B * p.Hq;
   for (int i = tid; i < MG * MD; i += MT) {
     const int hh = i / MD, ch = i % MD;
     float o = 0.f;
     for (int w = 0; w < 4; ++w) o += s_out[(w * MG + hh) * MD + ch];
-    p.ws.part_o[((int64_t)(bq0 + hh) * p.splits + split) * MD + ch] = o;
+    float* dst = p.ws.part_o + ((int64_t)(bq0 + hh) * p.splits + split) * MD + ch;
+    if (TQ_CHECKED(dst, 4, p.ws.part_o, 4 * rows * p.splits * MD, 113)) *dst = o;
   }
   if (tid < MG) {
     float M = -INFINITY, L = 0.f;
@@ -528,8 +532,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     if (M != -INFINITY)
       for (int w = 0; w < 4; ++w)
         if (s_m[w][tid] != -INFINITY) L += s_l[w][tid] * exp2f(s_m[w][tid] - M);
-    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 0] = M;
-    p.ws.part_ml[((int64_t)(bq0 + tid) * p.splits + split) * 2 + 1] = L;
+    float* dst = p.ws.part_ml + ((int64_t)(bq0 + tid) * p.splits + split) * 2;
+    if (TQ_CHECKED(dst, 8, p.ws.part_ml, 8 * rows * p.splits, 114)) {
+      dst[0] = M;
+      dst[1] = L;
+    }
   }
   if (!p.out) return;
   // The last split of this unit to finish merges all splits' (m, l, o).
@@ -562,7 +569,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       }
       o = o / L;
     }
-    store_f(p.out, (int64_t)bq * MD + ch, g.dtype, o);
+    if (TQ_CHECKED((const char*)p.out + ((int64_t)bq * MD + ch) * es, es, p.out, rows * MD * es, 115))
+      store_f(p.out, (int64_t)bq * MD + ch, g.dtype, o);
   }
 }
 
@@ -617,7 +625,6 @@ cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_
   p.ws = ws;
   p.err = ws.err;
   if (g.d == 256) return launch_partial_wide(p, s);
-  if (!getenv("TQ_LEGACY_DECODE")) return launch_partial_tc(p, s);
   const int ksq = g.m / 32;
   switch (g.b1 * 32 + ksq) {
     case 0 * 32 + 2: return launch_partial_t<0, 2>(p, s);

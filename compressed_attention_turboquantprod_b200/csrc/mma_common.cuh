@@ -177,9 +177,6 @@ __device__ __forceinline__ float slices_to_float(int s0, int s1, int s2, int s3)
   return fmaf(65536.f, __int2float_rn(hi), __int2float_rn(lo));
 }
 
-// The head-dim-128 partial kernel with the scores on tcgen05 (decode_tc.cu).
-cudaError_t launch_partial_tc(const MParams& p, cudaStream_t s);
-
 // The head-dim-256 kernel (decode_mma_wide.cu).
 bool decode_wide_supported(const Geom& g, int G);
 cudaError_t launch_partial_wide(const MParams& p, cudaStream_t s);

@@ -9,9 +9,9 @@
 // the mean: d = x - c, S1 = sum d, S2 = sum d^2, mean = c + S1/n, variance =
 // S2/n - (S1/n)^2 (shifted-data formula; the one-pass sum of squares, which
 // cancels catastrophically for keys whose mean is large against their spread,
-// is never formed).  16-byte loads, the entries of a load summed in fp32, fp64
-// across loads, fixed-order block and grid reductions (the result does not
-// depend on scheduling).
+// is never formed).  16-byte loads, d, its sums and its squares in fp64 (all
+// exact but the sums), fixed-order block and grid reductions (the result does
+// not depend on scheduling).
 //
 // Host: the groups and sketch dims from the per-layer variances.
 //   * contiguous groups whose boundaries minimise the summed squared deviation
@@ -34,14 +34,17 @@ constexpr int kMomBlocks = 148 * 4;
 constexpr int kMomThreads = 256;
 constexpr int kMomUnroll = 4;     // 16-byte loads in flight per thread
 
-__device__ __forceinline__ void moments16(uint4 u, int dtype, float c, float& s1, float& s2) {
+// One 16-byte load: d = x - c, its sum and its square in fp64 (x and c are fp32
+// values, so d and d^2 are exact in fp64; fp32 squares would round with a bias
+// when the entries sit on a coarse grid, as 16-bit inputs do).
+__device__ __forceinline__ void moments16(uint4 u, int dtype, double c, double& s1, double& s2) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
   if (dtype == TQ_F32) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float x = __uint_as_float(w[i]) - c;
+      const double x = (double)__uint_as_float(w[i]) - c;
       s1 += x;
-      s2 = fmaf(x, x, s2);
+      s2 = fma(x, x, s2);
     }
   } else {
 #pragma unroll
@@ -56,10 +59,9 @@ __device__ __forceinline__ void moments16(uint4 u, int dtype, float c, float& s1
         lo = f.x;
         hi = f.y;
       }
-      lo -= c;
-      hi -= c;
-      s1 += lo + hi;
-      s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+      const double a = (double)lo - c, b = (double)hi - c;
+      s1 += a + b;
+      s2 = fma(a, a, fma(b, b, s2));
     }
   }
 }
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int 
     if (threadIdx.x == 0) s_c = c;
   }
   __syncthreads();
-  const float c = s_c;
+  const double c = (double)s_c;
   const int per = dtype == TQ_F32 ? 4 : 8;              // entries per 16-byte load
   const int64_t nv = n / per;
   const int64_t nth = (int64_t)gridDim.x * kMomThreads;
@@ -96,15 +98,10 @@ __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int 
       if (i + k * nth < nv) u[k] = __ldg(v + i + k * nth);
 #pragma unroll
     for (int k = 0; k < kMomUnroll; ++k)
-      if (i + k * nth < nv) {
-        float s1 = 0.f, s2 = 0.f;
-        moments16(u[k], dtype, c, s1, s2);
-        d1 += (double)s1;
-        d2 += (double)s2;
-      }
+      if (i + k * nth < nv) moments16(u[k], dtype, c, d1, d2);
   }
   for (int64_t i = nv * per + t0; i < n; i += nth) {     // ragged tail
-    const double x = (double)(load_f(K, i, dtype) - c);
+    const double x = (double)load_f(K, i, dtype) - c;
     d1 += x;
     d2 += x * x;
   }

@@ -31,7 +31,6 @@ Geom geom_of(const tq_cache* c);
 // build these return 0.
 int bounds_flag_quant();
 int bounds_flag_decode();
-int bounds_flag_decode_tc();
 int bounds_flag_decode_mma();
 int bounds_flag_wide();
 int bounds_flag_prefill();

@@ -496,9 +496,9 @@ int tq_m_for_layer(const tq_layer_groups* g, int layer);
  * entries of K (device, dtype TQ_F32 / TQ_F16 / TQ_BF16, 16-byte aligned), the
  * statistic of the [AQJL] sensitivity analyser, in one streaming pass.  The
  * entries are summed relative to a shift (the fp32 mean of the first min(n, 32)
- * entries): S1 = sum (x - c), S2 = sum (x - c)^2, in fp32 within a 16-byte load
- * and fp64 beyond, and variance = S2/n - (S1/n)^2 in fp64, so keys whose mean
- * is large against their spread keep their precision.  `out` is a device
+ * entries): d = x - c, S1 = sum d and S2 = sum d^2 in fp64 (d and d^2 exact),
+ * and variance = S2/n - (S1/n)^2 in fp64, so keys whose mean is large against
+ * their spread keep their precision.  `out` is a device
  * double[2]; `workspace` device, tq_key_moments_workspace_bytes() bytes.  The
  * result does not depend on scheduling (fixed-order reductions).
  * Errors: INVALID_ARG, CUDA.

@@ -40,6 +40,11 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     if not rows:
         return
     tr = terminalreporter
+    worst = getattr(gc, "OUT_WORST", None)
+    if worst and worst["ratio"] > 0:
+        tr.section("attention outputs vs the oracle")
+        tr.write_line(f"worst error / bound {worst['ratio']:.3f} (error {worst['err']:.3g} at "
+                      f"|o| = {worst['abs_o']:.3g})")
     tr.section("near-boundary exemptions (codes / sign bits inside the 1e-5 band)")
     tot = {}
     for label, counts in rows:

@@ -16,15 +16,18 @@ from oracle import quantize as oq
 #  - rho: 4 ulp; ||r||: 2e-6 relative (fp32 rounding of y = Pi x / rho feeds
 #    e = y - c[idx]; ~1e-8 absolute on entries of size ~3e-2 over d terms);
 #  - logits given identical codes: 1e-3 relative or 1e-4 absolute;
-#  - attention outputs: 2e-3 max-abs, or, where the output dtype's own rounding
-#    of |o| exceeds that (bf16 at |o| >= 1: half an ulp is 3.9e-3 and more),
-#    half an ulp of the output dtype at |o| plus 64 fp32 ulp of |o| for the
-#    kernel's arithmetic.  Below |o| = 1 the bound is 2e-3 itself.
+#  - attention outputs: max(2e-3, half an ulp of the output dtype at |o| + 1e-3).
+#    2e-3 is the budget, half of it allowed to the kernel's arithmetic (whose
+#    error scales with the values averaged, not with |o|: logits within their
+#    own 1e-4 tolerance move an output over ~20-sized outlier values by several
+#    1e-4), so the bound is 2e-3 itself wherever the dtype's rounding leaves
+#    room (bf16 below |o| = 0.5, every f32 output) and the correctly rounded
+#    value plus that allowance elsewhere (2.95e-3 at bf16 |o| in [0.5, 1)).
 RHO_ULP = 4
 RNORM_ULP = 4
 LOGIT_REL, LOGIT_ABS = 1e-3, 1e-4
 OUT_ABS = 2e-3
-OUT_ARITH_F32_ULP = 64
+OUT_ARITH = 1e-3
 
 # Near-boundary exemptions seen by compare_keys calls given a label: (label, counts).
 # The session summary (conftest.py) prints them, so every GPU test log carries them.
@@ -94,9 +97,12 @@ def compare_keys(gpu: dict, ref: dict, d: int, b1: int, m: int, beta32, label=No
             ref["rho"].astype(np.float64) * np.sqrt(d) * 2.0 ** -21
         ok = np.abs(rn_g - rn_r) <= tol
         assert np.all(ok | skip_tok), f"rnorm max err / tol {np.max((np.abs(rn_g - rn_r) / tol)[~skip_tok])}"
+    # tokens whose stored codes or sign bits differ (inside the band): their logits
+    # legitimately differ from the oracle's, so end-to-end checks skip their units
+    flip_tok = skip_tok | np.any(smis, axis=1)
     counts = {"tokens": int(n), "code_mismatch": n_code_mis, "code_exempt": n_code_ex,
               "sign_mismatch": int(smis.sum()), "sign_exempt": int(sex.sum()),
-              "skipped_tokens": int(skip_tok.sum())}
+              "skipped_tokens": int(flip_tok.sum())}
     if label is not None:
         PARITY_COUNTS.append((label, counts))
     return counts
@@ -124,9 +130,12 @@ def storage_half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def out_tolerance(want: np.ndarray, dtype: str) -> np.ndarray:
-    """max(2e-3, half an ulp of the output dtype at |o| + 64 fp32 ulp of |o|)."""
-    f32_ulp = np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
-    return np.maximum(OUT_ABS, storage_half_ulp(want, dtype) + OUT_ARITH_F32_ULP * f32_ulp)
+    """max(2e-3, half an ulp of the output dtype at |o| + 1e-3)."""
+    return np.maximum(OUT_ABS, storage_half_ulp(want, dtype) + OUT_ARITH)
+
+
+# worst error / bound seen by check_out in this session (printed with the counts)
+OUT_WORST = {"ratio": 0.0, "err": 0.0, "abs_o": 0.0}
 
 
 def check_out(got: np.ndarray, want: np.ndarray, dtype: str = "bf16"):
@@ -134,7 +143,10 @@ def check_out(got: np.ndarray, want: np.ndarray, dtype: str = "bf16"):
         return 0.0
     err = np.abs(got - want)
     tol = out_tolerance(want, dtype)
-    i = int(np.argmax(err - tol))
+    i = int(np.argmax(err / tol))
+    if err.flat[i] / tol.flat[i] > OUT_WORST["ratio"]:
+        OUT_WORST.update(ratio=float(err.flat[i] / tol.flat[i]), err=float(err.flat[i]),
+                         abs_o=float(abs(want.flat[i])))
     assert np.all(err <= tol), (f"output error {err.flat[i]:.3g} over its bound {tol.flat[i]:.3g} "
                                 f"at |o| = {abs(want.flat[i]):.3g} (max |o| {np.max(np.abs(want)):.3g})")
     return float(np.max(err))

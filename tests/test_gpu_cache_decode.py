@@ -428,8 +428,8 @@ def test_hadamard_fast_transform_every_rotation_site(kw):
             units += 1
             if f == 0:
                 hs = slice(h * G, (h + 1) * G)
-                check_out(o[b:b + 1, hs], ro[b:b + 1, hs], w.dtype)
                 check_logits(lgs[b, hs], rl[(b, h)])
+                check_out(o[b:b + 1, hs], ro[b:b + 1, hs], w.dtype)
                 checked += 1
     record(f"hadamard transform d={w.d} end-to-end checks", unit_steps_checked=checked,
            unit_steps_skipped=units - checked)
