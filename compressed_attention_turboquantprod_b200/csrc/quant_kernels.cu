@@ -855,11 +855,39 @@ __device__ __forceinline__ void value_code_pair(float v0, float v1, float mn, fl
   const float2 t = mmadec::add2(x, make_float2(kRound, kRound));
   const float2 rr = mmadec::sub2(t, make_float2(kRound, kRound));
   const float2 dd = mmadec::sub2(x, rr);
-  tie = fabsf(fabsf(dd.x) - 0.5f) < 1e-5f || fabsf(fabsf(dd.y) - 0.5f) < 1e-5f;
+  // |x - rint(x)| <= 1/2 here, so "within 1e-5 of a half-integer" is one compare
+  tie = fabsf(dd.x) > 0.5f - 1e-5f || fabsf(dd.y) > 0.5f - 1e-5f;
   const uint32_t k0 = __float_as_uint(t.x) - __float_as_uint(kRound);
   const uint32_t k1 = __float_as_uint(t.y) - __float_as_uint(kRound);
   c0 = k0 < levels ? k0 : levels;
   c1 = k1 < levels ? k1 : levels;
+}
+
+// idx = #{k : beta_k < y} (ascending boundaries beta_0 .. beta_{L-2}) and c[idx], by a
+// binary search: bit b1-1 first, each compare choosing between the boundaries of
+// the half it selects (selects only: the tables stay in registers).
+template <int B1>
+__device__ __forceinline__ void code_search(float y, const float* bnd, const float* cen, int& idx,
+                                            float& cv) {
+  if constexpr (B1 == 1) {
+    const bool b0 = bnd[0] < y;
+    idx = b0;
+    cv = b0 ? cen[1] : cen[0];
+  } else if constexpr (B1 == 2) {
+    const bool b1 = bnd[1] < y;
+    const bool b0 = (b1 ? bnd[2] : bnd[0]) < y;
+    idx = 2 * b1 + b0;
+    cv = b1 ? (b0 ? cen[3] : cen[2]) : (b0 ? cen[1] : cen[0]);
+  } else {
+    const bool b2 = bnd[3] < y;
+    const bool b1 = (b2 ? bnd[5] : bnd[1]) < y;
+    const float t0 = b2 ? (b1 ? bnd[6] : bnd[4]) : (b1 ? bnd[2] : bnd[0]);
+    const bool b0 = t0 < y;
+    idx = 4 * b2 + 2 * b1 + b0;
+    const float lo = b1 ? (b0 ? cen[3] : cen[2]) : (b0 ? cen[1] : cen[0]);
+    const float hi = b1 ? (b0 ? cen[7] : cen[6]) : (b0 ? cen[5] : cen[4]);
+    cv = b2 ? hi : lo;
+  }
 }
 
 // The issuing thread: D = A B^T over K = 128 as three products per k-step.
@@ -1171,14 +1199,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
         float cv[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          int idx = 0;
-          cv[u] = cen[0];
-#pragma unroll
-          for (int k = 0; k + 1 < L; ++k)
-            if (bnd[k] < yy[u]) {
-              idx = k + 1;
-              cv[u] = cen[k + 1];
-            }
+          // idx = #{k : beta_k < y} by binary search over the ascending boundaries
+          // (the same count: the predicate is monotone in k), bits high to low
+          int idx;
+          code_search<B1>(yy[u], bnd, cen, idx, cv[u]);
 #pragma unroll
           for (int pl = 0; pl < B1; ++pl) pw[pl] |= (uint32_t)((idx >> pl) & 1) << (c + u);
         }
@@ -1233,9 +1257,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       uint32_t acc[32];
       tc::tmem_ld32(trow, acc);
       tc::tmem_wait_ld();
-      uint32_t w = 0u;
+      // bit = [rho Z >= 0]: for rho > 0 that is [Z >= 0] (a set-on-compare mask per
+      // column); a zero rho makes z = 0, every bit 1
+      uint32_t pos = 0u;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) w |= (uint32_t)(__uint_as_float(acc[c]) * rhof >= 0.f) << c;
+      for (int c = 0; c < 32; ++c) {
+        uint32_t m;
+        asm("set.ge.u32.f32 %0, %1, 0f00000000;" : "=r"(m) : "f"(__uint_as_float(acc[c])));
+        pos |= m & (1u << c);
+      }
+      const uint32_t w = rhof > 0.f ? pos : 0xFFFFFFFFu;
       if (valid && ok) *reinterpret_cast<uint32_t*>(dst_field(p, bh, grow, 1) + 4 * part) = w;
     }
     tc::fence_before_sync();
