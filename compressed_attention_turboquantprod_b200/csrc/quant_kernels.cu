@@ -23,7 +23,8 @@
 namespace tq {
 namespace {
 
-constexpr int NT = 64;        // tokens per tile
+// Tokens per tile of the SGEMM tile quantiser: 64, or 32 where the fp32 tiles of 64
+// would leave room for only one CTA per SM (rotated shapes at d >= 128, d = 256).
 constexpr int THREADS = 256;
 constexpr int NC = 128;       // output columns per GEMM pass
 constexpr int KC = 32;        // k-chunk staged in shared memory
@@ -53,46 +54,46 @@ struct QParams {
 };
 
 struct Smem {
-  float* X;      // [NT][d+4]
-  float* Y;      // [NT][d+4]
+  float* X;      // [nt][d+4]
+  float* Y;      // [nt][d+4]   (rotated rows; absent when b1 == 0)
   float* B;      // [KC][SBS]
-  float* Z;      // [NT][SBS]
-  double* rho64; // [NT]
-  float* rho;    // [NT]
-  float* inv;    // [NT]
+  float* Z;      // [nt][SBS]
+  double* rho64; // [nt]
+  float* rho;    // [nt]
+  float* inv;    // [nt]
   float* cb;     // [16] centroids, [16] boundaries
-  float* vs;     // [NT * 16] value scales
-  float* vm;     // [NT * 16] value minima
+  float* vs;     // [nt * 16] value scales
+  float* vm;     // [nt * 16] value minima
 };
 
-__host__ __device__ inline size_t smem_bytes(int d) {
+__host__ __device__ inline size_t smem_bytes(int d, int nt, int b1) {
   const int sx = d + 4;
-  return sizeof(float) * (2 * NT * sx + KC * SBS + NT * SBS) + sizeof(double) * NT +
-         sizeof(float) * (2 * NT + 32 + 2 * NT * 16);
+  return sizeof(float) * ((b1 > 0 ? 2 : 1) * nt * sx + KC * SBS + nt * SBS) + sizeof(double) * nt +
+         sizeof(float) * (2 * nt + 32 + 2 * nt * 16);
 }
 
-__device__ Smem carve(unsigned char* raw, int d) {
+__device__ Smem carve(unsigned char* raw, int d, int nt, int b1) {
   Smem s;
   const int sx = d + 4;
   double* dp = reinterpret_cast<double*>(raw);
   s.rho64 = dp;
-  float* f = reinterpret_cast<float*>(dp + NT);
+  float* f = reinterpret_cast<float*>(dp + nt);
   s.X = f;
-  f += NT * sx;
-  s.Y = f;
-  f += NT * sx;
+  f += nt * sx;
+  s.Y = b1 > 0 ? f : nullptr;
+  if (b1 > 0) f += nt * sx;
   s.B = f;
   f += KC * SBS;
   s.Z = f;
-  f += NT * SBS;
+  f += nt * SBS;
   s.rho = f;
-  f += NT;
+  f += nt;
   s.inv = f;
-  f += NT;
+  f += nt;
   s.cb = f;
   f += 32;
   s.vs = f;
-  f += NT * 16;
+  f += nt * 16;
   s.vm = f;
   return s;
 }
@@ -249,6 +250,7 @@ __device__ __forceinline__ void load4(const void* base, int64_t e, int dtype, fl
 
 // Load rows [row0, row0+NT) of the key or value source into X (fp32, zero past n):
 // a warp per row, the source address computed once per row, 4 elements per lane.
+template <int NT>
 __device__ void load_tile(const QParams& p, bool values, int bh, int64_t row0, float* X) {
   const int d = p.d, sx = d + 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -264,13 +266,15 @@ __device__ void load_tile(const QParams& p, bool values, int bh, int64_t row0, f
   }
 }
 
-// acc[r][c] = sum_k A[4ty+r][k] * Bg[col0 + tx + 16c][k], k < kdim; Bg row-major
-// [ncols][kdim], rows past ncols read as zero.
+// acc[r][c] = sum_k A[RT ty + r][k] * Bg[col0 + tx + 16c][k], k < kdim (RT = NT/16 rows
+// per thread); Bg row-major [ncols][kdim], rows past ncols read as zero.
+template <int NT>
 __device__ void gemm_pass(const float* A, int sa, const float* Bg, int kdim, int col0, int ncols,
-                          float* sB, float acc[4][8]) {
+                          float* sB, float (&acc)[NT / 16][8]) {
+  constexpr int RT = NT / 16;
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int r = 0; r < RT; ++r)
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
   for (int k0 = 0; k0 < kdim; k0 += KC) {
@@ -282,13 +286,13 @@ __device__ void gemm_pass(const float* A, int sa, const float* Bg, int kdim, int
     __syncthreads();
 #pragma unroll 4
     for (int kk = 0; kk < KC; ++kk) {
-      float a[4], b[8];
+      float a[RT], b[8];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = A[(4 * ty + r) * sa + k0 + kk];
+      for (int r = 0; r < RT; ++r) a[r] = A[(RT * ty + r) * sa + k0 + kk];
 #pragma unroll
       for (int c = 0; c < 8; ++c) b[c] = sB[kk * SBS + tx + 16 * c];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < RT; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
     }
@@ -296,11 +300,13 @@ __device__ void gemm_pass(const float* A, int sa, const float* Bg, int kdim, int
   }
 }
 
+template <int NT>
 __device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int64_t row0) {
+  constexpr int RT = NT / 16;
   const int d = p.d, sx = d + 4, b1 = p.b1, m = p.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ty = tid / 16, tx = tid % 16;
-  load_tile(p, false, bh, row0, s.X);
+  load_tile<NT>(p, false, bh, row0, s.X);
   __syncthreads();
   for (int r = warp; r < NT; r += THREADS / 32) {
     double ss = 0.0;
@@ -324,14 +330,14 @@ __device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int6
         warp_hadamard_rotate(p.Pi, s.X + r * sx, s.inv[r], s.Y + r * sx, d, lane);
     } else {
       for (int col0 = 0; col0 < d; col0 += NC) {
-        float acc[4][8];
-        gemm_pass(s.X, sx, p.Pi, d, col0, d, s.B, acc);
+        float acc[RT][8];
+        gemm_pass<NT>(s.X, sx, p.Pi, d, col0, d, s.B, acc);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RT; ++r)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const int col = col0 + tx + 16 * c;
-            if (col < d) s.Y[(4 * ty + r) * sx + col] = acc[r][c] * s.inv[4 * ty + r];
+            if (col < d) s.Y[(RT * ty + r) * sx + col] = acc[r][c] * s.inv[RT * ty + r];
           }
       }
     }
@@ -362,14 +368,14 @@ __device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int6
     E = s.Y;
   }
   for (int col0 = 0; col0 < m; col0 += NC) {
-    float acc[4][8];
-    gemm_pass(E, sx, p.T, d, col0, m, s.B, acc);
+    float acc[RT][8];
+    gemm_pass<NT>(E, sx, p.T, d, col0, m, s.B, acc);
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < RT; ++r)
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float z = (b1 > 0) ? acc[r][c] * s.rho[4 * ty + r] : acc[r][c];
-        s.Z[(4 * ty + r) * SBS + tx + 16 * c] = z;
+        const float z = (b1 > 0) ? acc[r][c] * s.rho[RT * ty + r] : acc[r][c];
+        s.Z[(RT * ty + r) * SBS + tx + 16 * c] = z;
       }
     __syncthreads();
     for (int r = warp; r < NT; r += THREADS / 32) {
@@ -386,11 +392,12 @@ __device__ void quantize_keys_tile(const QParams& p, const Smem& s, int bh, int6
     if (row0 + r < p.n) *reinterpret_cast<float*>(dst_field(p, bh, row0 + r, 2)) = s.rho[r];
 }
 
+template <int NT>
 __device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, int64_t row0) {
   const int d = p.d, sx = d + 4, g = p.group, ng = d / g, vb = p.vbits;
   const float levels = (float)((1 << vb) - 1);
   const int tid = threadIdx.x;
-  load_tile(p, true, bh, row0, s.X);
+  load_tile<NT>(p, true, bh, row0, s.X);
   __syncthreads();
   for (int pr = tid; pr < NT * ng; pr += blockDim.x) {
     const int r = pr / ng, gi = pr % ng;
@@ -428,9 +435,10 @@ __device__ void quantize_values_tile(const QParams& p, const Smem& s, int bh, in
   __syncthreads();
 }
 
+template <int NT>
 __global__ void __launch_bounds__(THREADS) k_quantize(QParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  Smem s = carve(smem_raw, p.d);
+  Smem s = carve(smem_raw, p.d, NT, p.do_keys ? p.b1 : 0);
   const int bh = blockIdx.y;
   const int64_t row0 = (int64_t)blockIdx.x * NT;
   if (threadIdx.x < 16) {
@@ -439,9 +447,9 @@ __global__ void __launch_bounds__(THREADS) k_quantize(QParams p) {
     s.cb[16 + threadIdx.x] = (threadIdx.x + 1 < L) ? p.bnd[threadIdx.x] : 0.f;
   }
   __syncthreads();
-  if (p.do_keys) quantize_keys_tile(p, s, bh, row0);
+  if (p.do_keys) quantize_keys_tile<NT>(p, s, bh, row0);
   __syncthreads();
-  if (p.do_values) quantize_values_tile(p, s, bh, row0);
+  if (p.do_values) quantize_values_tile<NT>(p, s, bh, row0);
 }
 
 __global__ void k_ring_write(Geom g, uint8_t* base, const void* K, const void* V, int64_t n_old,
@@ -1177,6 +1185,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
             *reinterpret_cast<uint16_t*>(cb + s_hofs[part][x]) = (uint16_t)hw[x];
       }
     }
+    // the next tile's key and value rows: both register copies are consumed, so the
+    // loads have the codes, the second product and the signs to land
+    request(tile + gridDim.x);
     // ---- 3. codes, E, ||r||
     bool ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait_sleep(&s_mbar[0], ph);
     if (!ok) s_abort = 1;
@@ -1237,7 +1248,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       tc_gemm(tmem, sAH, sAL, sTH, sTL);
       tc::mma_commit(smem_u32(&s_mbar[1]));
     }
-    request(tile + gridDim.x);                     // the next tile's, in flight from here
     const bool write = valid && ok;
     if (write) {
       uint8_t* ip = dst_field(p, bh, grow, 0);
@@ -1320,12 +1330,15 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     k_quantize_small<<<grid, SMALL_THREADS, smem, s>>>(p);
     return cudaGetLastError();
   }
-  const size_t smem = smem_bytes(p.d);
-  cudaError_t e = cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  // 64-token tiles where two CTAs fit an SM, else 32
+  const int kb1 = p.do_keys ? p.b1 : 0;
+  const int nt = smem_bytes(p.d, 64, kb1) <= (110u << 10) ? 64 : 32;
+  const size_t smem = smem_bytes(p.d, nt, kb1);
+  auto kern = nt == 32 ? k_quantize<32> : k_quantize<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((p.n + NT - 1) / NT), (unsigned)bh_count);
-  k_quantize<<<grid, THREADS, smem, s>>>(p);
+  dim3 grid((unsigned)((p.n + nt - 1) / nt), (unsigned)bh_count);
+  kern<<<grid, THREADS, smem, s>>>(p);
   return cudaGetLastError();
 }
 
