@@ -780,7 +780,19 @@ def _time_decode(w, layer, dev, reps=10, warm=3):
     cache = CompressedKVCache(wl.B, wl.Hkv, wl.d, wl.b1, m, wl.vbits, wl.group, wl.W, wl.T,
                               dtype=wl.torch_dtype, device=dev)
     K, V = synth.keys_values(wl, layer=layer, device=dev)
-    cache.append(K, V, pj, cb)
+    # the cache fill is a one-shot quantise-and-append of every token: timed on its
+    # second run (the first one grows the stream-ordered pool of the operand image)
+    stream = torch.cuda.current_stream(dev)
+    fill_ms = 0.0
+    for rep in range(2):
+        cache.state.n_total = 0
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.append(K, V, pj, cb)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fill_ms = e0.elapsed_time(e1)
     del K, V
     torch.cuda.empty_cache()
     Q = synth.queries(wl, layer=layer, device=dev)
@@ -788,7 +800,6 @@ def _time_decode(w, layer, dev, reps=10, warm=3):
     out = torch.empty(wl.B, wl.Hq, wl.d, dtype=wl.torch_dtype, device=dev)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
     scale = 1.0 / math.sqrt(wl.d)
     cent = cb.centroids if cb else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
@@ -809,9 +820,14 @@ def _time_decode(w, layer, dev, reps=10, warm=3):
     whole = sum(a[0].elapsed_time(a[2]) for a in ev) / reps
     es = 4 if wl.dtype == "f32" else 2
     nbytes = wl.B * wl.Hkv * (cache.n_comp * cache.state.token_bytes + 2 * cache.n_ring * wl.d * es)
+    keys = wl.B * wl.Hkv * wl.T
+    fill = {"ms": fill_ms, "keys": keys, "Mkeys_per_s": keys / (fill_ms * 1e-3) / 1e6,
+            # reads of K and V, writes of the packed records (and the ring)
+            "bytes": keys * 2 * wl.d * es + wl.B * wl.Hkv * (cache.n_comp * cache.state.token_bytes
+                                                             + 2 * cache.n_ring * wl.d * es)}
     del cache, ws, out, flush_w, flush_r
     torch.cuda.empty_cache()
-    return part, whole, nbytes
+    return part, whole, nbytes, fill
 
 
 def bench_other_decodes(dev, world, peak):
@@ -822,12 +838,13 @@ def bench_other_decodes(dev, world, peak):
     w = synth.WORKLOADS["aqjl"]
     groups, tot_ms, tot_bytes = [], 0.0, 0.0
     for layer in (0, 8, 16, 24):
-        part, whole, nb = _time_decode(w, layer, dev)
+        part, whole, nb, fill = _time_decode(w, layer, dev)
         part, whole = reduce_max(part, world), reduce_max(whole, world)
         nb_all = reduce_sum(float(nb), world)
         groups.append({"layers": f"{layer}-{layer + 7}", "m": w.m_for_layer(layer),
                        "partial_ms": part, "decode_ms": whole, "GB_per_s": nb_all / (part * 1e-3) / 1e9,
-                       "frac_of_peak": nb / (part * 1e-3) / 1e9 / peak})
+                       "frac_of_peak": nb / (part * 1e-3) / 1e9 / peak,
+                       "cache_fill": _fill_entry(fill, world, peak)})
         tot_ms += 8 * whole
         tot_bytes += 8 * nb_all
     res["aqjl"] = {"workload": "A-QJL: 32 layers, batch 16, 32 query heads over 8 KV heads, d=128, "
@@ -837,15 +854,25 @@ def bench_other_decodes(dev, world, peak):
                    "tokens_per_s": reduce_sum(16.0, world) / (tot_ms * 1e-3),
                    "ms_per_token_step": tot_ms}
     w = synth.WORKLOADS["wide"]
-    part, whole, nb = _time_decode(w, 0, dev)
+    part, whole, nb, fill = _time_decode(w, 0, dev)
     part, whole = reduce_max(part, world), reduce_max(whole, world)
     nb_all = reduce_sum(float(nb), world)
     res["wide"] = {"workload": "wide: batch 4, 16 query heads over 4 KV heads, d=256, context 262144, "
                                "keys b1=3 + m=256, 4-bit values g=64",
                    "partial_ms": part, "decode_ms": whole, "GB_per_s": nb_all / (part * 1e-3) / 1e9,
                    "frac_of_peak": nb / (part * 1e-3) / 1e9 / peak,
-                   "tokens_per_s": reduce_sum(4.0, world) / (whole * 1e-3)}
+                   "tokens_per_s": reduce_sum(4.0, world) / (whole * 1e-3),
+                   "cache_fill": _fill_entry(fill, world, peak)}
     return res
+
+
+def _fill_entry(fill, world, peak):
+    """The one-shot cache fill (every token quantised and appended in one call, on
+    the tensor cores at these shapes) as Mkeys/s and HBM fraction of its bytes."""
+    ms = reduce_max(fill["ms"], world)
+    return {"ms": ms, "Mkeys_per_s": reduce_sum(float(fill["keys"]), world) / (ms * 1e-3) / 1e6,
+            "GB_per_s": reduce_sum(float(fill["bytes"]), world) / (ms * 1e-3) / 1e9,
+            "frac_of_peak": fill["bytes"] / (ms * 1e-3) / 1e9 / peak}
 
 
 def bench_quantize(dev, world, reps=3, keep_sample=False):
@@ -905,8 +932,8 @@ def bench_quantize(dev, world, reps=3, keep_sample=False):
 
 def bench_structured_rotation(dev, world, reps=5):
     """What the fast Walsh-Hadamard transform buys where the rotation runs on CUDA
-    cores: the tile quantiser on the 262K wide-head shape (d = 256, no tensor-core
-    path; 4 KV heads x 16384 tokens per append) and the single-token append of a
+    cores: the SGEMM tile quantiser (d = 64, the head dim without a tensor-core
+    path; 8 KV heads x 16384 tokens per append) and the single-token append of a
     decode step on the 32K GQA shape, each with the dense QR rotation and with the
     structured one (same data)."""
     import torch
@@ -926,7 +953,7 @@ def bench_structured_rotation(dev, world, reps=5):
         return reduce_max(e0.elapsed_time(e1) / reps, world)
 
     res = {}
-    w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+    w = _sgemm_workload()
     K, V = synth.keys_values(w, device=dev)
     cb = Codebook(w.d, w.b1, device=dev)
     keys = w.B * w.Hkv * w.T
@@ -939,7 +966,7 @@ def bench_structured_rotation(dev, world, reps=5):
             cache.state.n_total = 0
             cache.append(K, V, pj, cb)
         ms = timed(call)
-        res["tile_quantise_wide_Mkeys_per_s_" + ("hadamard" if structured else "dense")] = \
+        res["tile_quantise_d64_Mkeys_per_s_" + ("hadamard" if structured else "dense")] = \
             reduce_sum(keys / (ms * 1e-3) / 1e6, world)
         del cache
     del K, V
@@ -963,10 +990,18 @@ def bench_structured_rotation(dev, world, reps=5):
         ms = timed(step)
         res["single_token_append_us_" + ("hadamard" if structured else "dense")] = ms * 1e3
         del cache
-    res["workloads"] = ("tile quantiser: d=256, b1=3, m=256, 4-bit values g=64, 4 KV heads x 16384 "
+    res["workloads"] = ("tile quantiser: d=64, b1=2, m=64, 2-bit values g=32, 8 KV heads x 16384 "
                         "bf16 tokens per append; single-token append: batch 8, 8 KV heads, d=128, "
                         "b1=2, m=128, 16-token ring (the token leaving the ring is quantised)")
     return res
+
+
+def _sgemm_workload():
+    """A shape the tile quantiser keeps on the CUDA-core SGEMM (d = 64)."""
+    import synth
+    return synth.Workload("quantize_sgemm", B=1, Hq=16, Hkv=8, d=64, T=16384, W=0, b1=2, m=64,
+                          vbits=2, group=32, dtype="bf16", k_outlier_frac=0.02,
+                          v_outlier_frac=0.02, outlier_scale=8.0)
 
 
 def oracle_quantize_counts(sample):
@@ -1003,10 +1038,16 @@ CASES = {
     "decode_cuda_core": "CUDA-core decode (k_decode_prep, k_decode_partial, k_decode_combine): "
                         "batch 8, 16 query heads over 8 KV heads (G = 2: no tensor-core path), "
                         "d = 64, context 32768, keys b1 = 2 + QJL m = 64, 2-bit values g = 32, bf16",
-    "quantize_sgemm": "64-token SGEMM tile quantise (k_quantize): the 262K wide-head shape (d = 256, "
-                      "b1 = 3, m = 256, 4-bit values g = 64, bf16), 4 KV heads x 16384 tokens per call",
+    "quantize_sgemm": "64-token SGEMM tile quantise (k_quantize, the shapes without a tensor-core "
+                      "path): d = 64, b1 = 2, m = 64, 2-bit values g = 32, bf16, 8 KV heads x 16384 "
+                      "tokens per call",
     "quantize_sgemm_hadamard": "the same with the structured rotation (the per-row fast "
                                "Walsh-Hadamard transform instead of the rotation GEMM)",
+    "quantize_tc_wide": "tcgen05 tile quantise on streamed operand pieces (k_operand_image, "
+                        "k_quantize_tcg): the 262K wide-head shape (d = 256, b1 = 3, m = 256, 4-bit "
+                        "values g = 64, bf16), 4 KV heads x 16384 tokens per call",
+    "quantize_tc_aqjl": "the same kernel on the A-QJL shape of layers 0-7 (pure QJL, d = 128, "
+                        "m = 512, fp16 keys, 2-bit values g = 32), 8 KV heads x 16384 tokens per call",
     "append_small": "single-token append (k_quantize_small, k_ring_write): the 32K GQA cache "
                     "(batch 8, 8 KV heads, d = 128, 16-token ring), one token per sequence per call",
     "prefill": "multi-token call (k_prefill_partial_mma, k_prefill_exact, merge) on the 32K GQA "
@@ -1058,11 +1099,16 @@ def run_case(args):
                                                       cb.centroids, o, None, 0, ws))
         nb = w.B * w.Hkv * (cache.n_comp * cache.state.token_bytes + 2 * cache.n_ring * w.d * 2)
         out.update(ms=ms, packed_bytes=nb, GB_per_s=nb / (ms * 1e-3) / 1e9)
-    elif name.startswith("quantize_sgemm"):
-        w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+    elif name.startswith("quantize_"):
+        if name.startswith("quantize_sgemm"):
+            w = _sgemm_workload()
+        elif name == "quantize_tc_wide":
+            w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+        else:
+            w = synth.WORKLOADS["aqjl"].scaled(B=1, T=16384, m=512)
         structured = name.endswith("hadamard")
-        pj = Projections(w.d, w.m, 0, device=dev, structured=structured)
-        cb = Codebook(w.d, w.b1, device=dev)
+        pj = Projections(w.d, w.m, 0, device=dev, rotation=w.b1 > 0, structured=structured)
+        cb = Codebook(w.d, w.b1, device=dev) if w.b1 else None
         cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, 0, w.T,
                                   dtype=w.torch_dtype, device=dev, structured=structured)
         K, V = synth.keys_values(w, device=dev)
@@ -1072,7 +1118,9 @@ def run_case(args):
             cache.append(K, V, pj, cb)
         ms = timed(call)
         keys = w.B * w.Hkv * w.T
-        out.update(ms=ms, keys=keys, Mkeys_per_s=keys / (ms * 1e-3) / 1e6)
+        nbytes = keys * (2 * w.d * (4 if w.dtype == "f32" else 2) + cache.state.token_bytes)
+        out.update(ms=ms, keys=keys, Mkeys_per_s=keys / (ms * 1e-3) / 1e6,
+                   GB_per_s=nbytes / (ms * 1e-3) / 1e9)
     elif name == "append_small":
         w = synth.WORKLOADS["gqa32k"]
         pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)

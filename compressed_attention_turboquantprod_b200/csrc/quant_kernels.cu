@@ -1301,6 +1301,568 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     tc::tmem_dealloc(tmem, TC_COLS);
   }
 }
+
+// ---------------------------------------------------------------- tcgen05 tiles, general shapes
+// The same pipeline for head dim D in {128, 256}, sketch dim m a multiple of 32 up
+// to 512 (the accumulator takes at most the 512 tensor-memory columns) and b1 in
+// 0..3 (b1 = 0: pure QJL, z = S x with T = S).  At these shapes Pi and T do not
+// fit in shared memory beside the A operand, so they are streamed:
+// k_operand_image writes them once per call into a device scratch as f16 hi + lo
+// (x kSplit) "pieces" of 128 output rows x 64 K in the canonical K-major layout,
+// in the order a tile consumes them (Pi by N-chunk then K-chunk, then T the same
+// way); a tensor warp copies the pieces into shared-memory stages (bulk copies
+// completing on an mbarrier), issues each piece's MMAs (three hi/lo products per
+// 16-wide k-step) and commits them to the barrier that frees the stage, running
+// ahead into the next tile while the epilogue works.  The 16 epilogue warps hold
+// one token row per thread as in k_quantize_tc, D/4 coordinates (D/128 words of
+// 32) per thread:
+//   U -> A;  [b1 > 0: Y = U Pi^T; codes, E -> A];  Z = A T^T;  sign bits.
+constexpr int TG_EPI = 512;                   // epilogue threads (16 warps)
+constexpr int TG_THREADS = TG_EPI + 32;       // and the tensor warp
+constexpr int TG_KC = 64;                     // K of one operand piece
+constexpr int TG_PIECE = 128 * TG_KC * 4;     // bytes of a full piece (f16 hi + lo)
+constexpr int TG_OPS = 192 * 1024;            // shared memory of A and the stages
+
+__host__ __device__ constexpr int tg_stages(int D) { return (TG_OPS - 512 * D) / TG_PIECE; }
+__host__ __device__ inline size_t tg_smem_bytes() {
+  return (size_t)TG_OPS + (sizeof(double) * 2 + sizeof(float2)) * TC_PARTS * TCM;
+}
+// Bytes of the operand image: Pi (b1 > 0) and T, 4 bytes (hi + lo) per element.
+__host__ __device__ inline size_t tg_image_bytes(int D, int b1, int m) {
+  return (size_t)4 * D * ((b1 > 0 ? D : 0) + m);
+}
+// Tensor-memory columns: a power of two >= max(D (b1 > 0), m, 32).
+__host__ __device__ inline uint32_t tg_tmem_cols(int D, int b1, int m) {
+  const int need = (b1 > 0 && D > m) ? D : m;
+  uint32_t c = 32;
+  while ((int)c < need) c <<= 1;
+  return c;
+}
+
+// Piece c of a tile's sequence (nY = pieces of Pi): its byte offset in the image,
+// rows (the MMA's N), first accumulator column and K chunk.  Every N-chunk but the
+// last of T has 128 rows; a piece of r rows takes 256 r bytes.
+struct TgPiece {
+  uint32_t off;
+  int nr, dcol, kc;
+};
+__host__ __device__ inline TgPiece tg_piece(int c, int D, int m, int nY) {
+  const int kpn = D / TG_KC;
+  TgPiece pc;
+  if (c < nY) {
+    pc.kc = c % kpn;
+    pc.nr = 128;
+    pc.dcol = 128 * (c / kpn);
+    pc.off = (uint32_t)c * TG_PIECE;
+  } else {
+    const int j = c - nY, nc = j / kpn;
+    pc.kc = j % kpn;
+    pc.nr = m - 128 * nc < 128 ? m - 128 * nc : 128;
+    pc.dcol = 128 * nc;
+    pc.off = (uint32_t)(nY + nc * kpn) * TG_PIECE + (uint32_t)(pc.kc * pc.nr * 256);
+  }
+  return pc;
+}
+
+// One thread per 8 consecutive K of a row of Pi (b1 > 0) or T: f16 hi + lo
+// (x kSplit), hi at the row's place in its piece, lo r * 128 bytes further.
+__global__ void k_operand_image(const float* Pi, const float* T, int D, int b1, int m,
+                                uint8_t* img, int64_t img_bytes) {
+  pdl_launch_dependents();     // the quantiser may start its own prologue
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int k8 = D / 8, rowsY = b1 > 0 ? D : 0;
+  if (i >= (int64_t)(rowsY + m) * k8) return;
+  const int row = (int)(i / k8), k = 8 * (int)(i % k8);
+  const bool isY = row < rowsY;
+  const int n = isY ? row : row - rowsY;
+  const float4* src = reinterpret_cast<const float4*>((isY ? Pi : T) + (int64_t)n * D + k);
+  const float4 f0 = src[0], f1 = src[1];
+  const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+  uint4 hi, lo;
+  split8(v, kSplit, hi, lo);
+  const int kpn = D / TG_KC, nY = rowsY > 0 ? (D / 128) * kpn : 0;
+  const int rl = n % 128, kl = k % TG_KC;
+  const TgPiece pc = tg_piece((isY ? 0 : nY) + (n / 128) * kpn + k / TG_KC, D, m, nY);
+  const uint32_t o = pc.off + (uint32_t)((((rl >> 3) * 8) + (kl >> 3)) * 128 + (rl & 7) * 16);
+  if (TQ_CHECKED(img + o, 16, img, img_bytes, 431)) *reinterpret_cast<uint4*>(img + o) = hi;
+  if (TQ_CHECKED(img + o + pc.nr * 128, 16, img, img_bytes, 432))
+    *reinterpret_cast<uint4*>(img + o + pc.nr * 128) = lo;
+}
+
+template <int D, int B1, bool F32>
+__global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const uint8_t* img,
+                                                               int64_t img_bytes, int64_t tiles_per_bh,
+                                                               int64_t total_tiles) {
+  using mmadec::mbar_init;
+  using mmadec::mbar_wait;
+  using mmadec::mbar_wait_sleep;
+  using mmadec::smem_u32;
+  constexpr int NW = D / 128;                  // 32-coordinate words per thread
+  constexpr int NS = tg_stages(D);             // piece stages
+  constexpr int KPN = D / TG_KC;               // pieces per N-chunk
+  constexpr int NY = B1 > 0 ? (D / 128) * KPN : 0;
+  constexpr int L = B1 > 0 ? 1 << B1 : 2;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_full[NS], s_empty[NS];
+  __shared__ __align__(8) uint64_t s_aready, s_ydone, s_zdone, s_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_hofs[TC_PARTS][16];         // value-code half offsets of each part
+  unsigned char* AH = smem_raw;
+  unsigned char* AL = AH + 256 * D;
+  unsigned char* ST = AL + 256 * D;            // [NS][TG_PIECE]
+  double* ssp = reinterpret_cast<double*>(smem_raw + TG_OPS);      // [part][row] sums of x^2
+  double* sep = ssp + TC_PARTS * TCM;                                // [part][row] sums of e^2
+  float2* vmm = reinterpret_cast<float2*>(sep + TC_PARTS * TCM);    // [part][row] value min / max
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int m = p.m;
+  const int nC = NY + ((m + 127) / 128) * KPN;
+  const uint32_t tcols = tg_tmem_cols(D, B1, m);
+  const int vb = p.vbits;
+  const int hpp = 2 * NW * vb;                 // 16-bit code halves per part
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    mbar_init(&s_aready, TG_EPI);
+    mbar_init(&s_ydone, 1);
+    mbar_init(&s_zdone, 1);
+    mbar_init(&s_drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_abort = 0;
+  }
+  if (tid < TC_PARTS * 16) {
+    const int pp = tid >> 4, x = tid & 15;
+    s_hofs[pp][x] = x < hpp ? code_half_off(p, pp * hpp + x) : 0;
+  }
+  if (warp == TG_EPI / 32) {
+    tc::tmem_alloc(smem_u32(&s_tmem), tcols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  const int64_t my_tiles = blockIdx.x < total_tiles ? (total_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (warp == TG_EPI / 32) {
+    // ------------------------------------------------ the tensor warp (one thread)
+    if (lane == 0) {
+      const uint32_t sAH = smem_u32(AH), sAL = smem_u32(AL), sST = smem_u32(ST);
+      const int64_t total_p = my_tiles * nC;
+      pdl_wait();                                // the image is written by the previous kernel
+      int64_t loaded = 0, gp = 0;
+      bool ok = true;
+      auto load = [&](int64_t gpc) {
+        const int st = (int)(gpc % NS);
+        const TgPiece pc = tg_piece((int)(gpc % nC), D, m, NY);
+        const uint32_t bytes = (uint32_t)pc.nr * 256u;
+        mmadec::mbar_expect_tx(&s_full[st], bytes);
+        if (TQ_CHECKED(img + pc.off, bytes, img, img_bytes, 430))
+          mmadec::bulk_load(ST + (size_t)st * TG_PIECE, img + pc.off, bytes, &s_full[st]);
+      };
+      for (; loaded < NS && loaded < total_p; ++loaded) load(loaded);
+      uint32_t aph = 0;
+      for (int64_t t = 0; t < my_tiles && ok; ++t) {
+        for (int pass = B1 > 0 ? 0 : 1; pass < 2 && ok; ++pass) {
+          // operand A (U, or E) written by all epilogue threads
+          if (!mbar_wait_sleep(&s_aready, aph) || *reinterpret_cast<volatile int*>(&s_abort)) {
+            ok = false;
+            break;
+          }
+          aph ^= 1u;
+          tc::fence_after_sync();
+          const int c0 = pass == 0 ? 0 : NY, c1 = pass == 0 ? NY : nC;
+          for (int c = c0; c < c1; ++c, ++gp) {
+            const int st = (int)(gp % NS);
+            if (!mbar_wait(&s_full[st], (uint32_t)((gp / NS) & 1))) {
+              ok = false;
+              break;
+            }
+            const TgPiece pc = tg_piece(c, D, m, NY);
+            const uint32_t idesc = tc::idesc_f16(TCM, pc.nr);
+            const uint32_t bh = sST + (uint32_t)st * TG_PIECE, bl = bh + (uint32_t)pc.nr * 128u;
+            const uint32_t dt = tmem + (uint32_t)pc.dcol;
+#pragma unroll
+            for (int ks = 0; ks < TG_KC / 16; ++ks) {
+              const uint32_t ao = (uint32_t)pc.kc * 1024u + 256u * ks, bo = 256u * ks;
+              const uint64_t dah = tc::smem_desc_sbo(sAH + ao, 16 * D), dal = tc::smem_desc_sbo(sAL + ao, 16 * D);
+              const uint64_t dbh = tc::smem_desc_sbo(bh + bo, 1024), dbl = tc::smem_desc_sbo(bl + bo, 1024);
+              tc::mma_f16(dt, dah, dbh, idesc, (pc.kc | ks) ? 1u : 0u);
+              tc::mma_f16(dt, dah, dbl, idesc, 1u);
+              tc::mma_f16(dt, dal, dbh, idesc, 1u);
+            }
+            tc::mma_commit(smem_u32(&s_empty[st]));
+            if (gp >= 1 && loaded < total_p) {
+              // refill the previous piece's stage once its products are done
+              const int64_t pr = gp - 1;
+              if (!mbar_wait(&s_empty[pr % NS], (uint32_t)((pr / NS) & 1))) {
+                ++gp;
+                ok = false;
+                break;
+              }
+              load(loaded);
+              ++loaded;
+            }
+          }
+          if (!ok) break;
+          tc::mma_commit(smem_u32(pass == 0 ? &s_ydone : &s_zdone));
+        }
+      }
+      if (!ok) {
+        // a wait gave up: let every product and copy in flight finish (bounded)
+        s_abort = 1;
+        atomicExch(&g_quant_tc_err, 1);
+        tc::mma_commit(smem_u32(&s_drain));
+        (void)mbar_wait(&s_drain, 0u);
+        for (int64_t q = gp; q < loaded; ++q) (void)mbar_wait(&s_full[q % NS], (uint32_t)((q / NS) & 1));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ the epilogue warps
+    const int q = warp & 3, part = warp >> 2;
+    const int r = 32 * q + lane;                 // this thread's row of every tile
+    const int kw0 = part * NW;                   // and its first 32-wide word
+    const int g = p.group;
+    const uint32_t levels = (1u << vb) - 1u;
+    const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+    float bnd[L - 1], cen[L];
+#pragma unroll
+    for (int k = 0; k < L; ++k) cen[k] = B1 > 0 ? p.cent[k] : 0.f;
+#pragma unroll
+    for (int k = 0; k + 1 < L; ++k) bnd[k] = B1 > 0 ? p.bnd[k] : 0.f;
+    // source rows of a tile: this thread's key and value segments (register copies
+    // one tile ahead at D = 128; requests towards L2 at D = 256)
+    RawSeg<F32> xr[NW], vr[NW];
+    auto row_src = [&](int64_t t, bool values, int64_t& e) -> const void* {
+      const int tbh = (int)(t / tiles_per_bh);
+      const int64_t ti = (t % tiles_per_bh) * TCM + r;
+      if (t >= total_tiles || ti >= p.n || (values && !p.do_values)) return nullptr;
+      return src_row(p, values, tbh, ti, e);
+    };
+    auto request = [&](int64_t t) {
+      int64_t ek = 0, ev = 0;
+      const void* ks = row_src(t, false, ek);
+      const void* vs = row_src(t, true, ev);
+      if constexpr (NW == 1) {
+        raw_load(xr[0], ks, ek + 32 * kw0, ks != nullptr);
+        raw_load(vr[0], vs, ev + 32 * kw0, vs != nullptr);
+      } else {
+        const int es = F32 ? 4 : 2;
+        if (ks) prefetch_l2(static_cast<const char*>(ks) + (ek + 32 * kw0) * es);
+        if (vs) prefetch_l2(static_cast<const char*>(vs) + (ev + 32 * kw0) * es);
+      }
+    };
+    request(blockIdx.x);
+    int64_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      const int bh = (int)(tile / tiles_per_bh);
+      const int64_t grow = (tile % tiles_per_bh) * TCM + r;
+      const bool valid = grow < p.n;
+      const uint32_t ph = (uint32_t)(it & 1);
+      if constexpr (NW > 1) {
+        int64_t ek = 0;
+        const void* ks = row_src(tile, false, ek);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) raw_load(xr[w], ks, ek + 32 * (kw0 + w), ks != nullptr);
+      }
+      // ---- 1. rho and U = X / rho
+      float rhof;
+      double rho64;
+      {
+        double ss = 0.0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          float x[32], s8[8];
+          raw_to_float(xr[w], p.dtype, x);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) s8[j] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 xx = make_float2(x[j], x[j + 1]);
+            const float2 sp = mmadec::fma2(xx, xx, make_float2(s8[j & 7], s8[(j + 1) & 7]));
+            s8[j & 7] = sp.x;
+            s8[(j + 1) & 7] = sp.y;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss += (double)s8[j];
+        }
+        ssp[part * TCM + r] = ss;
+        tc::bar_sync(1, TG_EPI);
+        ss = (ssp[r] + ssp[TCM + r]) + (ssp[2 * TCM + r] + ssp[3 * TCM + r]);
+        const double rs = ss > 0.0 ? rsqrt(ss) : 0.0;
+        rho64 = ss * rs;
+        rhof = (float)rho64;
+        const float inv = (float)rs;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          float x[32];
+          raw_to_float(xr[w], p.dtype, x);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+              const float2 u = mmadec::mul2(make_float2(x[8 * c8 + k], x[8 * c8 + k + 1]), make_float2(inv, inv));
+              v[k] = u.x;
+              v[k + 1] = u.y;
+            }
+            uint4 hi, lo;
+            split8(v, kSplit, hi, lo);
+            const int k = 32 * (kw0 + w) + 8 * c8;
+            const int off = (((r >> 3) * (D / 8)) + (k >> 3)) * 128 + (r & 7) * 16;
+            *reinterpret_cast<uint4*>(AH + off) = hi;
+            *reinterpret_cast<uint4*>(AL + off) = lo;
+          }
+        }
+      }
+      tc::fence_async_shared();
+      tc::fence_before_sync();
+      mmadec::mbar_arrive(&s_aready);
+      // ---- 2. values of this thread's 32 NW channels, while the first product runs
+      if (p.do_values) {
+        if constexpr (NW > 1) {
+          int64_t ev = 0;
+          const void* vs = row_src(tile, true, ev);
+#pragma unroll
+          for (int w = 0; w < NW; ++w) raw_load(vr[w], vs, ev + 32 * (kw0 + w), vs != nullptr);
+        }
+        constexpr int NCH = 2 * NW;                // 16-channel chunks of this thread
+        float mn[NCH], mx[NCH];
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          float v[32];
+          raw_to_float(vr[w], p.dtype, v);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float a = v[16 * c], b = v[16 * c];
+#pragma unroll
+            for (int k = 1; k < 16; ++k) {
+              a = fminf(a, v[16 * c + k]);
+              b = fmaxf(b, v[16 * c + k]);
+            }
+            mn[2 * w + c] = a;
+            mx[2 * w + c] = b;
+          }
+        }
+        const int gc = g / 16;                     // chunks per group
+        if (gc <= NCH) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            const int c0 = c - c % gc;
+            float a = mn[c0], b = mx[c0];
+            for (int j = 1; j < gc; ++j) {
+              a = fminf(a, mn[c0 + j]);
+              b = fmaxf(b, mx[c0 + j]);
+            }
+            // in place: rewriting a group's first chunk with the group's extremes
+            // leaves the later chunks of the group with the same result
+            mn[c] = a;
+            mx[c] = b;
+          }
+        } else {
+          float a = mn[0], b = mx[0];
+#pragma unroll
+          for (int c = 1; c < NCH; ++c) {
+            a = fminf(a, mn[c]);
+            b = fmaxf(b, mx[c]);
+          }
+          vmm[part * TCM + r] = make_float2(a, b);
+          tc::bar_sync(1, TG_EPI);
+          const int np = gc / NCH, p0 = part - part % np;
+          a = FLT_MAX;
+          b = -FLT_MAX;
+          for (int j = 0; j < np; ++j) {
+            const float2 m2 = vmm[(p0 + j) * TCM + r];
+            a = fminf(a, m2.x);
+            b = fmaxf(b, m2.y);
+          }
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            mn[c] = a;
+            mx[c] = b;
+          }
+        }
+        if (valid) {
+          float sc[NCH], iv[NCH];
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            sc[c] = __fdiv_rn(__fsub_rn(mx[c], mn[c]), (float)levels);
+            iv[c] = sc[c] != 0.f ? __frcp_rn(sc[c]) : 0.f;
+          }
+          float* vsp = reinterpret_cast<float*>(dst_field(p, bh, grow, 5));
+          float* vmp = reinterpret_cast<float*>(dst_field(p, bh, grow, 6));
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            const int ch = 32 * kw0 + 16 * c;
+            if (ch % g == 0) {
+              vsp[ch / g] = sc[c];
+              vmp[ch / g] = mn[c];
+            }
+          }
+          uint8_t* cb = code_base(p, bh, grow);
+          uint32_t hw[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hw[j] = 0u;
+          bool any_tie = false;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            float v[32];
+            raw_to_float(vr[w], p.dtype, v);
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              const int c = 2 * w + (k >> 4);
+              bool tie;
+              uint32_t c0, c1;
+              value_code_pair(v[k], v[k + 1], mn[c], iv[c], levels, c0, c1, tie);
+              any_tie |= tie && sc[c] != 0.f;
+              const int ch = 32 * w + k;             // channel within this thread's range
+              if (vb == 2) hw[ch >> 3] += (c0 << (2 * (ch & 7))) + (c1 << (2 * ((ch + 1) & 7)));
+              else hw[ch >> 2] += (c0 << (4 * (ch & 3))) + (c1 << (4 * ((ch + 1) & 3)));
+            }
+          }
+          if (any_tie) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) hw[j] = 0u;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+              float v[32];
+              raw_to_float(vr[w], p.dtype, v);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                const int c = 2 * w + (k >> 4), ch = 32 * w + k;
+                const uint32_t cd = value_code_fast(v[k], mn[c], sc[c], iv[c], levels);
+                if (vb == 2) hw[ch >> 3] += cd << (2 * (ch & 7));
+                else hw[ch >> 2] += cd << (4 * (ch & 3));
+              }
+            }
+          }
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            if (x < hpp && TQ_CHECKED(cb + s_hofs[part][x], 2, p.cache_mode ? p.base : p.arr.codes,
+                                      p.cache_mode ? p.g.total_bytes
+                                                   : (p.t_first + p.n) * (p.d * p.vbits / 8), 433))
+              *reinterpret_cast<uint16_t*>(cb + s_hofs[part][x]) = (uint16_t)hw[x];
+        }
+      }
+      // the next tile's rows: this tile's register copies are consumed
+      request(tile + gridDim.x);
+      bool ok = true;
+      // ---- 3. codes, E, ||r||
+      if constexpr (B1 > 0) {
+        ok = !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait_sleep(&s_ydone, ph);
+        if (!ok) {
+          s_abort = 1;
+          atomicExch(&g_quant_tc_err, 1);
+        }
+        tc::fence_after_sync();
+        uint32_t pw[B1][NW];
+        double se = 0.0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          uint32_t acc[32];
+          tc::tmem_ld32(trow + (uint32_t)(32 * (kw0 + w)), acc);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int pl = 0; pl < B1; ++pl) pw[pl][w] = 0u;
+          float e[32], s8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) s8[j] = 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 y2 = mmadec::mul2(make_float2(__uint_as_float(acc[c]), __uint_as_float(acc[c + 1])),
+                                           make_float2(1.f / (kSplit * kSplit), 1.f / (kSplit * kSplit)));
+            const float yy[2] = {y2.x, y2.y};
+            float cv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              int idx;
+              code_search<B1>(yy[u], bnd, cen, idx, cv[u]);
+#pragma unroll
+              for (int pl = 0; pl < B1; ++pl) pw[pl][w] |= (uint32_t)((idx >> pl) & 1) << (c + u);
+            }
+            const float2 e2 = mmadec::sub2(y2, make_float2(cv[0], cv[1]));
+            e[c] = e2.x;
+            e[c + 1] = e2.y;
+            const float2 sp = mmadec::fma2(e2, e2, make_float2(s8[c & 7], s8[(c + 1) & 7]));
+            s8[c & 7] = sp.x;
+            s8[(c + 1) & 7] = sp.y;
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = e[8 * c8 + k];
+            uint4 hi, lo;
+            split8(v, kSplit, hi, lo);
+            const int k = 32 * (kw0 + w) + 8 * c8;
+            const int off = (((r >> 3) * (D / 8)) + (k >> 3)) * 128 + (r & 7) * 16;
+            *reinterpret_cast<uint4*>(AH + off) = hi;
+            *reinterpret_cast<uint4*>(AL + off) = lo;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) se += (double)s8[j];
+        }
+        tc::fence_async_shared();
+        tc::fence_before_sync();
+        mmadec::mbar_arrive(&s_aready);
+        sep[part * TCM + r] = se;
+        tc::bar_sync(3, TG_EPI);
+        if (valid && ok) {
+          uint8_t* ip = dst_field(p, bh, grow, 0);
+#pragma unroll
+          for (int pl = 0; pl < B1; ++pl)
+#pragma unroll
+            for (int w = 0; w < NW; ++w)
+              *reinterpret_cast<uint32_t*>(ip + pl * (D / 8) + 4 * (kw0 + w)) = pw[pl][w];
+          if (part == 0) {
+            const double sev = (sep[r] + sep[TCM + r]) + (sep[2 * TCM + r] + sep[3 * TCM + r]);
+            *reinterpret_cast<float*>(dst_field(p, bh, grow, 3)) = (float)(rho64 * sqrt(sev));
+          }
+        }
+      }
+      // ---- 4. sign bits of z (rho Z for b1 > 0, S x = rho Z for b1 = 0)
+      ok = ok && !*reinterpret_cast<volatile int*>(&s_abort) && mbar_wait_sleep(&s_zdone, ph);
+      if (!ok) {
+        s_abort = 1;
+        atomicExch(&g_quant_tc_err, 1);
+      }
+      tc::fence_after_sync();
+      {
+        uint8_t* sp = valid && ok ? dst_field(p, bh, grow, 1) : nullptr;
+        for (int w = part; w < m / 32; w += TC_PARTS) {
+          uint32_t acc[32];
+          tc::tmem_ld32(trow + (uint32_t)(32 * w), acc);
+          tc::tmem_wait_ld();
+          // bit = [z >= 0]: [Z >= 0] for rho > 0 (a set-on-compare mask per column);
+          // a zero rho makes z = 0, every bit 1
+          uint32_t pos = 0u;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            uint32_t mk;
+            asm("set.ge.u32.f32 %0, %1, 0f00000000;" : "=r"(mk) : "f"(__uint_as_float(acc[c])));
+            pos |= mk & (1u << c);
+          }
+          if (sp) *reinterpret_cast<uint32_t*>(sp + 4 * w) = rhof > 0.f ? pos : 0xFFFFFFFFu;
+        }
+        if (sp && part == 0) *reinterpret_cast<float*>(dst_field(p, bh, grow, 2)) = rhof;
+      }
+      tc::fence_before_sync();
+      tc::bar_sync(4, TG_EPI);
+      if (*reinterpret_cast<volatile int*>(&s_abort)) break;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == TG_EPI / 32) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, tcols);
+  }
+}
+
 }  // namespace
 
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
@@ -1322,6 +1884,46 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     const int64_t grid = total < sms ? total : sms;
     kern<<<(unsigned)grid, TC_THREADS, smem, s>>>(p, tiles_per_bh, total);
     return cudaGetLastError();
+  }
+  if (p.n > 8 && p.do_keys && (p.d == 128 || p.d == 256) && p.m % 32 == 0 && p.m <= 512 &&
+      p.b1 >= 0 && p.b1 <= 3) {
+    // the same on streamed operand pieces: Pi and T written once into a scratch image
+    const int64_t tiles_per_bh = (p.n + TCM - 1) / TCM;
+    const int64_t total = tiles_per_bh * bh_count;
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t ib = (int64_t)tg_image_bytes(p.d, p.b1, p.m);
+    void* img = nullptr;
+    cudaError_t e = cudaMallocAsync(&img, (size_t)ib, s);
+    if (e != cudaSuccess) return e;
+    const int64_t chunks = (int64_t)((p.b1 > 0 ? p.d : 0) + p.m) * (p.d / 8);
+    k_operand_image<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(p.Pi, p.T, p.d, p.b1, p.m,
+                                                                     static_cast<uint8_t*>(img), ib);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+      const bool f32 = p.dtype == TQ_F32, wide = p.d == 256;
+      using KFn = void (*)(QParams, const uint8_t*, int64_t, int64_t, int64_t);
+      static const KFn table[2][4][2] = {
+          {{k_quantize_tcg<128, 0, false>, k_quantize_tcg<128, 0, true>},
+           {k_quantize_tcg<128, 1, false>, k_quantize_tcg<128, 1, true>},
+           {k_quantize_tcg<128, 2, false>, k_quantize_tcg<128, 2, true>},
+           {k_quantize_tcg<128, 3, false>, k_quantize_tcg<128, 3, true>}},
+          {{k_quantize_tcg<256, 0, false>, k_quantize_tcg<256, 0, true>},
+           {k_quantize_tcg<256, 1, false>, k_quantize_tcg<256, 1, true>},
+           {k_quantize_tcg<256, 2, false>, k_quantize_tcg<256, 2, true>},
+           {k_quantize_tcg<256, 3, false>, k_quantize_tcg<256, 3, true>}}};
+      const KFn kern = table[wide][p.b1][f32];
+      const size_t smem = tg_smem_bytes();
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) {
+        const int64_t grid = total < sms ? total : sms;
+        e = launch_pdl(kern, dim3((unsigned)grid), dim3(TG_THREADS), smem, s, p,
+                       static_cast<const uint8_t*>(img), ib, tiles_per_bh, total);
+      }
+    }
+    const cudaError_t ef = cudaFreeAsync(img, s);
+    return e != cudaSuccess ? e : ef;
   }
   if (p.n <= 8) {
     // a few tokens per (b, kv head): one CTA per token

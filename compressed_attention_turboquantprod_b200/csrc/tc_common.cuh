@@ -31,6 +31,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
          ((uint64_t)(kRowBytes >> 4) << 32) | (1ull << 46);
 }
 
+// The same for an operand whose consecutive 8-row groups are `sbo` bytes apart
+// (K = 8 sbo / 128 f16 per row: sbo = 1024 for K = 64, 4096 for K = 256).
+__device__ __forceinline__ uint64_t smem_desc_sbo(uint32_t saddr, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(kChunkBytes >> 4) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // Instruction descriptor of kind::f16: f16 A and B, fp32 D, both K-major, M x N.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);

@@ -162,6 +162,63 @@ def test_append_quantize_variants(b1, m, vb, g, dt):
     _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
 
 
+@pytest.mark.parametrize("d,b1,m,vb,g,dt,chunks", [
+    (256, 3, 256, 4, 64, "bf16", (9, 300)),          # the wide shape: Pi and T streamed
+    (256, 0, 128, 2, 128, "f16", (130, 140)),        # pure QJL at d = 256, a group over two parts
+    (256, 1, 96, 2, 16, "f32", (128, 129)),          # an N tail of 96 rows, 16-channel groups
+    (256, 2, 512, 4, 32, "bf16", (200,)),            # 512 accumulator columns
+    (128, 0, 512, 2, 32, "f16", (9, 257, 300)),      # the A-QJL shapes: m = 512 / 384 / 192
+    (128, 0, 384, 2, 32, "f16", (129,)),
+    (128, 0, 192, 4, 64, "bf16", (64, 300)),
+    (128, 3, 64, 4, 128, "bf16", (150,)),            # one N-chunk of 64 rows, a group of 128
+    (128, 2, 32, 2, 32, "f32", (12,)),
+])
+def test_append_tensor_core_general_shapes(d, b1, m, vb, g, dt, chunks):
+    """Chunks of more than 8 tokens at shapes outside d = m = 128 run on the tensor
+    cores with the operands streamed from a per-call image: packed bytes equal the
+    oracle's (codes and signs outside the boundary band), values bit-exact, and the
+    kernel's wait flag clear."""
+    T = sum(chunks) + 7
+    w = _workload(B=1, Hkv=2, d=d, b1=b1, m=m, vbits=vb, group=g, dtype=dt, W=7, T=T,
+                  seed=31 + d + m + b1)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda")
+    gc = _gpu_cache(w, T)
+    oc = _oracle_cache(w, T, po, cb)
+    t = 0
+    for n in chunks + (7,):
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        gc.append(k, v, _Proj(po), _Cb(cb) if b1 else None)
+        oc.append(host(k), host(v))
+        t += n
+    torch.cuda.synchronize()
+    nat().tq_quantize_check()
+    skipped = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc,
+                                   label=f"tensor-core append d={d} b1={b1} m={m}")
+    assert skipped <= max(2, T // 100)
+
+
+def test_append_tensor_core_many_tiles_per_cta():
+    """More 128-token tiles than SMs, so persistent CTAs stream the operand pieces of
+    several tiles in a row (the stages wrap across tiles): d = 256, b1 = 3, m = 256
+    and pure QJL m = 512 against the oracle."""
+    for (d, b1, m, vb, g, dt) in ((256, 3, 256, 4, 64, "bf16"), (128, 0, 512, 2, 32, "f16")):
+        T = 128 * 40 + 19
+        w = _workload(B=1, Hkv=4, d=d, b1=b1, m=m, vbits=vb, group=g, dtype=dt, W=16, T=T,
+                      seed=77 + b1)
+        po, cb = oracle_setup(w.d, w.b1, w.m)
+        K, V = synth.keys_values(w, device="cuda")
+        gc = _gpu_cache(w, T)
+        oc = _oracle_cache(w, T, po, cb)
+        gc.append(K, V, _Proj(po), _Cb(cb) if b1 else None)
+        oc.append(host(K), host(V))
+        torch.cuda.synchronize()
+        nat().tq_quantize_check()
+        skipped = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc,
+                                       label=f"tensor-core append, many tiles, d={d} m={m}")
+        assert skipped <= max(2, w.Hkv * T // 200)
+
+
 def _decode_identical_codes(w, n_tokens, capacity, num_splits=0, Hq=None):
     """Oracle-built cache bytes decoded by the GPU with the oracle's projections."""
     Hq = Hq or w.Hq
