@@ -1045,9 +1045,9 @@ CASES = {
                                "Walsh-Hadamard transform instead of the rotation GEMM)",
     "quantize_tc_wide": "tcgen05 tile quantise on streamed operand pieces (k_operand_image, "
                         "k_quantize_tcg): the 262K wide-head shape (d = 256, b1 = 3, m = 256, 4-bit "
-                        "values g = 64, bf16), 4 KV heads x 16384 tokens per call",
+                        "values g = 64, bf16), 4 KV heads x 32768 tokens per call",
     "quantize_tc_aqjl": "the same kernel on the A-QJL shape of layers 0-7 (pure QJL, d = 128, "
-                        "m = 512, fp16 keys, 2-bit values g = 32), 8 KV heads x 16384 tokens per call",
+                        "m = 512, fp16 keys, 2-bit values g = 32), 8 KV heads x 65536 tokens per call",
     "append_small": "single-token append (k_quantize_small, k_ring_write): the 32K GQA cache "
                     "(batch 8, 8 KV heads, d = 128, 16-token ring), one token per sequence per call",
     "prefill": "multi-token call (k_prefill_partial_mma, k_prefill_exact, merge) on the 32K GQA "
@@ -1103,9 +1103,9 @@ def run_case(args):
         if name.startswith("quantize_sgemm"):
             w = _sgemm_workload()
         elif name == "quantize_tc_wide":
-            w = synth.WORKLOADS["wide"].scaled(B=1, T=16384)
+            w = synth.WORKLOADS["wide"].scaled(B=1, T=32768)
         else:
-            w = synth.WORKLOADS["aqjl"].scaled(B=1, T=16384, m=512)
+            w = synth.WORKLOADS["aqjl"].scaled(B=1, T=65536, m=512)
         structured = name.endswith("hadamard")
         pj = Projections(w.d, w.m, 0, device=dev, rotation=w.b1 > 0, structured=structured)
         cb = Codebook(w.d, w.b1, device=dev) if w.b1 else None

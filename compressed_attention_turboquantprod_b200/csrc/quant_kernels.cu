@@ -15,6 +15,8 @@
 //   * every other shape: 64-token tiles with the contractions as a register-tiled
 //     fp32 SGEMM (k_quantize).
 #include <cfloat>
+#include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "prep_mma.cuh"
@@ -1426,7 +1428,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
     }
-    mbar_init(&s_aready, TG_EPI);
+    mbar_init(&s_aready, TG_EPI / 32);           // one arrival per epilogue warp
     mbar_init(&s_ydone, 1);
     mbar_init(&s_zdone, 1);
     mbar_init(&s_drain, 1);
@@ -1451,7 +1453,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
     // ------------------------------------------------ the tensor warp (one thread)
     if (lane == 0) {
       const uint32_t sAH = smem_u32(AH), sAL = smem_u32(AL), sST = smem_u32(ST);
-      const int64_t total_p = my_tiles * nC;
+      // when a tile's pieces all fit in the stages they are loaded once and stay
+      const bool resident = nC <= NS;
+      const int64_t total_p = resident ? nC : my_tiles * nC;
       pdl_wait();                                // the image is written by the previous kernel
       int64_t loaded = 0, gp = 0;
       bool ok = true;
@@ -1467,8 +1471,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
       uint32_t aph = 0;
       for (int64_t t = 0; t < my_tiles && ok; ++t) {
         for (int pass = B1 > 0 ? 0 : 1; pass < 2 && ok; ++pass) {
-          // operand A (U, or E) written by all epilogue threads
-          if (!mbar_wait_sleep(&s_aready, aph) || *reinterpret_cast<volatile int*>(&s_abort)) {
+          // operand A (U, or E) written by all epilogue threads (polled without a
+          // sleep hint: this handoff is on every tile's critical path)
+          if (!mbar_wait(&s_aready, aph) || *reinterpret_cast<volatile int*>(&s_abort)) {
             ok = false;
             break;
           }
@@ -1476,8 +1481,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
           tc::fence_after_sync();
           const int c0 = pass == 0 ? 0 : NY, c1 = pass == 0 ? NY : nC;
           for (int c = c0; c < c1; ++c, ++gp) {
-            const int st = (int)(gp % NS);
-            if (!mbar_wait(&s_full[st], (uint32_t)((gp / NS) & 1))) {
+            const int st = resident ? c : (int)(gp % NS);
+            if ((!resident || gp < nC) && !mbar_wait(&s_full[st], (uint32_t)((gp / NS) & 1))) {
               ok = false;
               break;
             }
@@ -1494,6 +1499,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
               tc::mma_f16(dt, dah, dbl, idesc, 1u);
               tc::mma_f16(dt, dal, dbh, idesc, 1u);
             }
+            if (resident) continue;
             tc::mma_commit(smem_u32(&s_empty[st]));
             if (gp >= 1 && loaded < total_p) {
               // refill the previous piece's stage once its products are done
@@ -1621,7 +1627,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
       }
       tc::fence_async_shared();
       tc::fence_before_sync();
-      mmadec::mbar_arrive(&s_aready);
+      __syncwarp();
+      if (lane == 0) mmadec::mbar_arrive(&s_aready);
       // ---- 2. values of this thread's 32 NW channels, while the first product runs
       if (p.do_values) {
         if constexpr (NW > 1) {
@@ -1808,7 +1815,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
         }
         tc::fence_async_shared();
         tc::fence_before_sync();
-        mmadec::mbar_arrive(&s_aready);
+        __syncwarp();
+        if (lane == 0) mmadec::mbar_arrive(&s_aready);
         sep[part * TCM + r] = se;
         tc::bar_sync(3, TG_EPI);
         if (valid && ok) {
@@ -1865,6 +1873,39 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
 
 }  // namespace
 
+// A private stream-ordered memory pool per device for the operand images: freed
+// blocks stay in the pool (no release threshold), so the per-call allocation is a
+// stream-ordered reuse, never a new mapping.
+static cudaError_t image_pool(cudaMemPool_t* out) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = UINT64_MAX;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
   if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0 && p.b1 <= 3) {
@@ -1895,7 +1936,9 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t ib = (int64_t)tg_image_bytes(p.d, p.b1, p.m);
     void* img = nullptr;
-    cudaError_t e = cudaMallocAsync(&img, (size_t)ib, s);
+    cudaMemPool_t pool;
+    cudaError_t e = image_pool(&pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&img, (size_t)ib, pool, s);
     if (e != cudaSuccess) return e;
     const int64_t chunks = (int64_t)((p.b1 > 0 ? p.d : 0) + p.m) * (p.d / 8);
     k_operand_image<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(p.Pi, p.T, p.d, p.b1, p.m,
