@@ -1050,8 +1050,9 @@ CASES = {
                         "m = 512, fp16 keys, 2-bit values g = 32), 8 KV heads x 65536 tokens per call",
     "append_small": "single-token append (k_quantize_small, k_ring_write): the 32K GQA cache "
                     "(batch 8, 8 KV heads, d = 128, 16-token ring), one token per sequence per call",
-    "prefill": "multi-token call (k_prefill_partial_mma, k_prefill_exact, merge) on the 32K GQA "
+    "prefill": "multi-token call (history partial, k_prefill_exact, merge) on the 32K GQA "
                "cache, 16-token chunk",
+    "prefill64": "the same with a 64-token chunk",
 }
 
 
@@ -1138,7 +1139,8 @@ def run_case(args):
             cache.append(Kn[i], Vn[i], pj, cb)
         ms = timed(call)
         out.update(ms=ms, tokens_per_call=w.B * w.Hkv)
-    elif name == "prefill":
+    elif name.startswith("prefill"):
+        nq = 64 if name == "prefill64" else 16
         w = synth.WORKLOADS["gqa32k"]
         pj, cb = Projections(w.d, w.m, 0, device=dev), Codebook(w.d, w.b1, device=dev)
         cache = CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, w.T,
@@ -1146,15 +1148,15 @@ def run_case(args):
         K, V = synth.keys_values(w, device=dev)
         cache.append(K, V, pj, cb)
         del K, V
-        Q, Kc, Vc = synth.prefill_chunk(w, 16, device=dev)
+        Q, Kc, Vc = synth.prefill_chunk(w, nq, device=dev)
         o = torch.empty_like(Q)
-        ws = torch.empty(native.tq_prefill_workspace_bytes(cache.state, w.Hq, 16, 0),
+        ws = torch.empty(native.tq_prefill_workspace_bytes(cache.state, w.Hq, nq, 0),
                          dtype=torch.uint8, device=dev)
         scale = 1.0 / math.sqrt(w.d)
         ms = timed(lambda: native.tq_prefill_attention(cache.state, Q, Kc, Vc, scale, pj.Pi, pj.S,
                                                        cb.centroids, o, 0, ws))
-        native.tq_prefill_check(cache.state, w.Hq, 16, 0, ws)
-        out.update(ms=ms, query_tokens=w.B * 16)
+        native.tq_prefill_check(cache.state, w.Hq, nq, 0, ws)
+        out.update(ms=ms, query_tokens=w.B * nq)
     torch.cuda.synchronize()
     print(json.dumps(out), flush=True)
     return 0

@@ -253,7 +253,7 @@ int tq_debug_bounds_check(void) {
     int (*read)();
   } files[] = {{"quant_kernels", tq::bounds_flag_quant}, {"decode_kernels", tq::bounds_flag_decode},
                {"decode_mma", tq::bounds_flag_decode_mma}, {"decode_mma_wide", tq::bounds_flag_wide},
-               {"prefill_mma", tq::bounds_flag_prefill}};
+               {"prefill_mma", tq::bounds_flag_prefill}, {"prefill_tc", tq::bounds_flag_prefill_tc}};
   int first = 0;
   const char* where = "";
   for (const auto& f : files) {
@@ -718,6 +718,12 @@ static int prefill_splits(const tq::Geom& g, int G, int n, bool mma, int num_spl
   const int64_t nblk = (n_comp + tq::kBlockTokens - 1) / tq::kBlockTokens;
   int s = num_splits > 0 ? num_splits : tq::prefill_auto_splits(g, G, n_comp, n, mma);
   if (nblk == 0) return 1;
+  if (mma && tq::prefill_tc_supported(g, G, n)) {
+    // the tcgen05 partial splits whole 128-token tiles and runs empty splits as
+    // empty partials: any count up to the tile count (monotone in n_comp)
+    const int64_t ntiles = (nblk + 1) / 2;
+    return (int)(s < ntiles ? s : ntiles);
+  }
   if (s > nblk) s = (int)nblk;
   const int64_t bps = (nblk + s - 1) / s;
   return (int)((nblk + bps - 1) / bps);
@@ -793,7 +799,10 @@ int tq_prefill_attention(const tq_cache* c, const void* Q, int Hq, int n, const 
                                                      P.ws, s)
                         : tq::launch_decode_prep(P.gv, Q, Hq, Pi, S, P.ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: prepare");
-  e = P.mma ? tq::launch_prefill_partial_mma(P.g, base, c->n_total, Hq, n, P.splits, P.nslots, P.ws, s)
+  const bool tc = P.mma && tq::prefill_tc_supported(P.g, Hq / c->desc.Hkv, n);
+  e = tc      ? tq::launch_prefill_partial_tc(P.g, base, c->n_total, Hq, n, P.splits, P.nslots,
+                                              centroids, P.ws, s)
+    : P.mma ? tq::launch_prefill_partial_mma(P.g, base, c->n_total, Hq, n, P.splits, P.nslots, P.ws, s)
             : tq::launch_decode_partial(P.gv, base, c->n_total, Hq, softmax_scale, centroids, nullptr,
                                         P.splits, P.ws, s, n, P.nslots, false);
   if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention: history");

@@ -567,6 +567,7 @@ int prefill_auto_splits(const Geom& g, int G, int64_t n_comp, int nq, bool mma) 
   const int64_t nblk = (n_comp + kBlockTokens - 1) / kBlockTokens;
   if (nblk <= 1) return 1;
   const int units = g.B * g.Hkv;
+  if (mma && prefill_tc_supported(g, G, nq)) return prefill_tc_splits(g, n_comp, nq);
   if (!mma) {
     // the CUDA-core partial runs per virtual (query token) batch: one wave or so
     int64_t s = (148 * 4 + (int64_t)units * nq - 1) / ((int64_t)units * nq);

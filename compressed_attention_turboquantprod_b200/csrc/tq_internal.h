@@ -34,6 +34,7 @@ int bounds_flag_decode();
 int bounds_flag_decode_mma();
 int bounds_flag_wide();
 int bounds_flag_prefill();
+int bounds_flag_prefill_tc();
 
 // Record a thread-local error message (printf-style) and return `status`.
 int set_error(int status, const char* fmt, ...);
@@ -132,6 +133,13 @@ cudaError_t launch_decode_combine(const Geom& g, int Hq, void* out, int splits,
 // history partials take slots 0..splits-1 of splits + 1, the exact segment (ring +
 // chunk tokens 0..i) the last slot, and the decode combine merges them.
 bool prefill_mma_supported(const Geom& g, int G);
+// the tcgen05 history partial (prefill_tc.cu): chunks of >= 8 tokens on the
+// tensor-core shapes whose operands fit
+bool prefill_tc_supported(const Geom& g, int G, int nq);
+int prefill_tc_splits(const Geom& g, int64_t n_comp, int nq);
+cudaError_t launch_prefill_partial_tc(const Geom& g, const uint8_t* base, int64_t n_total, int Hq, int nq,
+                                      int splits, int nslots, const float* cent, const DecodeWs& ws,
+                                      cudaStream_t s);
 int prefill_mma_warps(const Geom& g, int nq);
 int prefill_auto_splits(const Geom& g, int G, int64_t n_comp, int nq, bool mma);
 cudaError_t launch_prefill_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
