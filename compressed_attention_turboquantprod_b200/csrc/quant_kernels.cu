@@ -780,7 +780,8 @@ constexpr float kSplit = 1024.f;
 constexpr int TCM = 128;                   // rows of a tile (MMA M)
 constexpr int TC_PARTS = 4;                // 32-coordinate parts of a row
 constexpr int TC_THREADS = TCM * TC_PARTS; // 16 warps
-constexpr uint32_t TC_COLS = 128;          // tensor-memory columns: one 128 x 128 fp32 tile
+constexpr uint32_t TC_COLS = 256;          // tensor-memory columns: the 128 x 128 fp32 tile of the
+                                           // hi*hi products, then that of the hi/lo corrections
 constexpr int TC_OPB = TCM * QD * 2;       // bytes of one f16 operand (32 KB)
 constexpr float kRound = 12582912.f;       // 1.5 * 2^23: x + kRound rounds x (|x| < 2^22) to an integer
 
@@ -900,7 +901,10 @@ __device__ __forceinline__ void code_search(float y, const float* bnd, const flo
   }
 }
 
-// The issuing thread: D = A B^T over K = 128 as three products per k-step.
+// The issuing thread: D = A B^T over K = 128 as three products per k-step, the
+// hi*hi products into columns 0..127 and the hi*lo + lo*hi corrections into
+// 128..255 (the epilogue adds them in fp32: the large partial sums then take one
+// accumulation per k-step instead of three).
 __device__ __forceinline__ void tc_gemm(uint32_t d_tmem, uint32_t ah, uint32_t al, uint32_t bh,
                                         uint32_t bl) {
   constexpr uint32_t idesc = tc::idesc_f16(TCM, QD);
@@ -908,8 +912,22 @@ __device__ __forceinline__ void tc_gemm(uint32_t d_tmem, uint32_t ah, uint32_t a
   for (int ks = 0; ks < QD / 16; ++ks) {
     const uint32_t o = 256u * ks;
     tc::mma_f16(d_tmem, tc::smem_desc(ah + o), tc::smem_desc(bh + o), idesc, ks > 0 ? 1u : 0u);
-    tc::mma_f16(d_tmem, tc::smem_desc(ah + o), tc::smem_desc(bl + o), idesc, 1u);
-    tc::mma_f16(d_tmem, tc::smem_desc(al + o), tc::smem_desc(bh + o), idesc, 1u);
+    tc::mma_f16(d_tmem + QD, tc::smem_desc(ah + o), tc::smem_desc(bl + o), idesc, ks > 0 ? 1u : 0u);
+    tc::mma_f16(d_tmem + QD, tc::smem_desc(al + o), tc::smem_desc(bh + o), idesc, 1u);
+  }
+}
+
+// 32 columns of this thread's accumulator row: the hi*hi sums plus the corrections.
+__device__ __forceinline__ void tc_ld_sum32(uint32_t taddr, uint32_t (&acc)[32]) {
+  tc::tmem_ld32(taddr, acc);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {       // the corrections 16 columns at a time (registers)
+    uint32_t cor[16];
+    tc::tmem_ld16(taddr + QD + 16 * h, cor);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      acc[16 * h + c] = __float_as_uint(__uint_as_float(acc[16 * h + c]) + __uint_as_float(cor[c]));
   }
 }
 
@@ -1197,8 +1215,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     uint32_t pw[B1];
     {
       uint32_t acc[32];
-      tc::tmem_ld32(trow, acc);
-      tc::tmem_wait_ld();
+      tc_ld_sum32(trow, acc);
 #pragma unroll
       for (int pl = 0; pl < B1; ++pl) pw[pl] = 0u;
       float e[32], s8[8];
@@ -1267,8 +1284,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     tc::fence_after_sync();
     {
       uint32_t acc[32];
-      tc::tmem_ld32(trow, acc);
-      tc::tmem_wait_ld();
+      tc_ld_sum32(trow, acc);
       // bit = [rho Z >= 0]: for rho > 0 that is [Z >= 0] (a set-on-compare mask per
       // column); a zero rho makes z = 0, every bit 1
       uint32_t pos = 0u;
@@ -1333,12 +1349,24 @@ __host__ __device__ inline size_t tg_smem_bytes() {
 __host__ __device__ inline size_t tg_image_bytes(int D, int b1, int m) {
   return (size_t)4 * D * ((b1 > 0 ? D : 0) + m);
 }
-// Tensor-memory columns: a power of two >= max(D (b1 > 0), m, 32).
+// With b1 > 0 the hi*hi products accumulate apart from the hi*lo + lo*hi
+// corrections (two accumulators, summed in fp32 by the epilogue), so that the
+// large partial sums take one accumulation per k-step instead of three: the
+// residual e = y - c[idx] is an order of magnitude below y, and its sketch
+// z = T e carries y's absolute error times sqrt(d), so y needs close to fp32
+// accuracy (measured at d = 256: sign decisions within 7e-6 of the rms |z| with
+// one accumulator, against 1.3e-6 for the fp32 CUDA-core product).  Pure QJL
+// (z = S u, no residual) keeps one.
+__host__ __device__ inline bool tg_split_acc(int D, int b1, int m) {
+  return b1 > 0 && 2 * (D > m ? D : m) <= 512;
+}
+// Tensor-memory columns: a power of two >= max(D (b1 > 0), m, 32), twice that
+// with split accumulators (the corrections at + half).
 __host__ __device__ inline uint32_t tg_tmem_cols(int D, int b1, int m) {
   const int need = (b1 > 0 && D > m) ? D : m;
   uint32_t c = 32;
   while ((int)c < need) c <<= 1;
-  return c;
+  return tg_split_acc(D, b1, m) ? 2 * c : c;
 }
 
 // Piece c of a tile's sequence (nY = pieces of Pi): its byte offset in the image,
@@ -1420,6 +1448,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
   const int m = p.m;
   const int nC = NY + ((m + 127) / 128) * KPN;
   const uint32_t tcols = tg_tmem_cols(D, B1, m);
+  const bool split = tg_split_acc(D, B1, m);
   const int vb = p.vbits;
   const int hpp = 2 * NW * vb;                 // 16-bit code halves per part
 
@@ -1490,14 +1519,16 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
             const uint32_t idesc = tc::idesc_f16(TCM, pc.nr);
             const uint32_t bh = sST + (uint32_t)st * TG_PIECE, bl = bh + (uint32_t)pc.nr * 128u;
             const uint32_t dt = tmem + (uint32_t)pc.dcol;
+            const uint32_t dc = split ? dt + tcols / 2 : dt;     // corrections
 #pragma unroll
             for (int ks = 0; ks < TG_KC / 16; ++ks) {
               const uint32_t ao = (uint32_t)pc.kc * 1024u + 256u * ks, bo = 256u * ks;
               const uint64_t dah = tc::smem_desc_sbo(sAH + ao, 16 * D), dal = tc::smem_desc_sbo(sAL + ao, 16 * D);
               const uint64_t dbh = tc::smem_desc_sbo(bh + bo, 1024), dbl = tc::smem_desc_sbo(bl + bo, 1024);
-              tc::mma_f16(dt, dah, dbh, idesc, (pc.kc | ks) ? 1u : 0u);
-              tc::mma_f16(dt, dah, dbl, idesc, 1u);
-              tc::mma_f16(dt, dal, dbh, idesc, 1u);
+              const uint32_t first = (pc.kc | ks) ? 1u : 0u;
+              tc::mma_f16(dt, dah, dbh, idesc, first);
+              tc::mma_f16(dc, dah, dbl, idesc, split ? first : 1u);
+              tc::mma_f16(dc, dal, dbh, idesc, 1u);
             }
             if (resident) continue;
             tc::mma_commit(smem_u32(&s_empty[st]));
@@ -1772,6 +1803,17 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
         for (int w = 0; w < NW; ++w) {
           uint32_t acc[32];
           tc::tmem_ld32(trow + (uint32_t)(32 * (kw0 + w)), acc);
+          if (split) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {   // the corrections 16 columns at a time
+              uint32_t cor[16];
+              tc::tmem_ld16(trow + tcols / 2 + (uint32_t)(32 * (kw0 + w)) + 16 * hh, cor);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                acc[16 * hh + c] = __float_as_uint(__uint_as_float(acc[16 * hh + c]) + __uint_as_float(cor[c]));
+            }
+          }
           tc::tmem_wait_ld();
 #pragma unroll
           for (int pl = 0; pl < B1; ++pl) pw[pl][w] = 0u;
@@ -1844,6 +1886,17 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
         for (int w = part; w < m / 32; w += TC_PARTS) {
           uint32_t acc[32];
           tc::tmem_ld32(trow + (uint32_t)(32 * w), acc);
+          if (split) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {   // the corrections 16 columns at a time
+              uint32_t cor[16];
+              tc::tmem_ld16(trow + tcols / 2 + (uint32_t)(32 * w) + 16 * hh, cor);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                acc[16 * hh + c] = __float_as_uint(__uint_as_float(acc[16 * hh + c]) + __uint_as_float(cor[c]));
+            }
+          }
           tc::tmem_wait_ld();
           // bit = [z >= 0]: [Z >= 0] for rho > 0 (a set-on-compare mask per column);
           // a zero rho makes z = 0, every bit 1
