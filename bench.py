@@ -683,8 +683,9 @@ def bench_prefill(w, cache, pj, cb, flush_l2, stream, hist_bytes, world, chunks=
     t_dec = timed(lambda: native.tq_decode_attention(cache.state, Qd, scale, pj.Pi, pj.S, cent,
                                                      outd, None, 0, wsd))
     # executed tensor work of the history partial per (history token, query token, KV
-    # head): int8 score MMAs (KS k-steps of 32 features x 4 heads x 4 slices) and f16
-    # P V MMAs (128 channels x 4 heads x hi/lo); int8 taken at twice the bf16 peak
+    # head): int8 score MMAs (KS k-steps of 32 features x 4 heads x 4 slices; tcgen05
+    # for chunks of 8 or more tokens) and f16 P V MMAs (128 channels x 4 heads x
+    # hi/lo); int8 taken at twice the bf16 peak
     F = (1 << (w.b1 - 1)) if w.b1 > 0 else 0
     KS = F * w.d // 32 + w.m // 32
     G = w.Hq // w.Hkv
