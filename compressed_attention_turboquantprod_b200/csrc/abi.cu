@@ -466,13 +466,16 @@ int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const fl
   tq::Geom g = tq::geom_of(c);
   uint8_t* base = static_cast<uint8_t*>(c->base);
   cudaError_t e = cudaSuccess;
+  bool ring_written = false;
   if (c_new > c_old) {
     tq::QuantSrc src{K, V, c_new - c_old, c_old, n_old, n_new};
-    e = tq::launch_quantize_cache(src, g, base, Pi, T, centroids, boundaries, s);
+    e = tq::launch_quantize_cache(src, g, base, Pi, T, centroids, boundaries, s, &ring_written);
     if (e != cudaSuccess) return cuda_fail(e, "tq_append: quantize");
   }
-  e = tq::launch_ring_write(g, base, K, V, n_old, n_new, s);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_append: ring");
+  if (!ring_written) {
+    e = tq::launch_ring_write(g, base, K, V, n_old, n_new, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_append: ring");
+  }
   c->n_total = n_tot;
   return ok();
 }

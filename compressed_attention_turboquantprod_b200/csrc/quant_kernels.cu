@@ -39,6 +39,7 @@ struct QParams {
   int dtype;
   int64_t n, t_first, n_old, n_new;
   bool cache_mode;
+  bool fuse_ring;     // cache mode, n_new >= W: the tile kernel also writes the new ring
   const void* ringK;
   const void* ringV;
   // shapes
@@ -108,7 +109,7 @@ __device__ __forceinline__ const void* src_row(const QParams& p, bool values, in
   const int es = p.dtype == TQ_F32 ? 4 : 2;
   const void* chunk = values ? p.V : p.K;
   const void* base = chunk;
-  int64_t rows;
+  [[maybe_unused]] int64_t rows;   // read by the bounds-checked build
   if (!p.cache_mode) {
     elem = i * d;
     rows = p.t_first + p.n;
@@ -979,6 +980,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
   // this thread's key and value segments of a tile, requested one tile ahead (the
   // first before the operand staging, so that its latency overlaps the staging)
   RawSeg<F32> xr, vr;
+  // Launched programmatically (cache appends that write the ring themselves): the
+  // kernel before may still run.  Nothing here touches its data except the ring
+  // slots (read by a (b, h)'s first tile, which holds the tokens leaving the ring,
+  // then rewritten by the same CTA): those tiles wait for it first.
   auto request = [&](int64_t t) {
     bool ok_row = false;
     const void* ks = nullptr;
@@ -986,7 +991,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     int64_t ek = 0, ev = 0;
     if (t < total_tiles) {
       const int tbh = (int)(t / tiles_per_bh);
-      const int64_t trow_i = (t % tiles_per_bh) * TCM + r;
+      const int64_t tr0 = (t % tiles_per_bh) * TCM;
+      if (p.cache_mode && p.t_first + tr0 < p.n_old) pdl_wait();     // uniform per tile
+      const int64_t trow_i = tr0 + r;
       ok_row = trow_i < p.n;
       if (ok_row) {
         ks = src_row(p, false, tbh, trow_i, ek);
@@ -996,6 +1003,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     raw_load(xr, ks, ek + k0, ok_row);
     raw_load(vr, vs, ev + k0, ok_row && p.do_values);
   };
+  // the next append's tile kernel may launch (its CTAs take the SMs this grid leaves)
+  if (p.fuse_ring) pdl_launch_dependents();
   request(blockIdx.x);
 
   constexpr int kStage = QD * 4 + 16;
@@ -1266,6 +1275,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       tc::fence_after_sync();
       tc_gemm(tmem, sAH, sAL, sTH, sTL);
       tc::mma_commit(smem_u32(&s_mbar[1]));
+    }
+    if (p.fuse_ring && row0 == 0) {
+      // a (b, h)'s first tile: every thread has used its rows (the old ring slots
+      // included) before the barrier above, so the new ring (the chunk's last W
+      // tokens, token t into slot t mod W) is written now, 16 bytes a thread
+      const Geom& gg = p.g;
+      const int rb = QD * es / 16;                      // 16-byte words of a row
+      for (int i = tid; i < 2 * gg.W * rb; i += TC_THREADS) {
+        const int which = i / (gg.W * rb), rem = i % (gg.W * rb), rr = rem / rb, wd = rem % rb;
+        const int64_t t = p.n_old + p.n_new - gg.W + rr;            // absolute token
+        const uint4* src = reinterpret_cast<const uint4*>(which ? p.V : p.K) +
+                           ((int64_t)bh * p.n_new + (t - p.n_old)) * rb + wd;
+        uint4* dst = reinterpret_cast<uint4*>(p.base + (which ? gg.ring_v_off : gg.ring_k_off)) +
+                     ((int64_t)bh * gg.W + t % gg.W) * rb + wd;
+        if (TQ_CHECKED(src, 16, which ? p.V : p.K, (int64_t)gg.B * gg.Hkv * p.n_new * rb * 16, 425) &&
+            TQ_CHECKED(dst, 16, p.base, gg.total_bytes, 426))
+          *dst = *src;
+      }
     }
     const bool write = valid && ok;
     if (write) {
@@ -1600,6 +1627,18 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
       const int64_t grow = (tile % tiles_per_bh) * TCM + r;
       const bool valid = grow < p.n;
       const uint32_t ph = (uint32_t)(it & 1);
+      {
+        // the rows of the tile after next towards L2 (this thread's segments)
+        int64_t ek = 0, ev = 0;
+        const void* ks = row_src(tile + 2 * (int64_t)gridDim.x, false, ek);
+        const void* vs = row_src(tile + 2 * (int64_t)gridDim.x, true, ev);
+        const int es = F32 ? 4 : 2;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          if (ks) prefetch_l2(static_cast<const char*>(ks) + (ek + 32 * (kw0 + w)) * es);
+          if (vs) prefetch_l2(static_cast<const char*>(vs) + (ev + 32 * (kw0 + w)) * es);
+        }
+      }
       if constexpr (NW > 1) {
         int64_t ek = 0;
         const void* ks = row_src(tile, false, ek);
@@ -1976,6 +2015,10 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = total < sms ? total : sms;
+    // a cache append whose chunk replaces the whole ring writes the ring in this
+    // kernel, which is then launched programmatically: consecutive appends overlap
+    p.fuse_ring = p.cache_mode && p.g.W > 0 && p.n_new >= p.g.W;
+    if (p.fuse_ring) return launch_pdl(kern, dim3((unsigned)grid), dim3(TC_THREADS), smem, s, p, tiles_per_bh, total);
     kern<<<(unsigned)grid, TC_THREADS, smem, s>>>(p, tiles_per_bh, total);
     return cudaGetLastError();
   }
@@ -2078,7 +2121,7 @@ cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1
 
 cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* base,
                                   const float* Pi, const float* T, const float* cent,
-                                  const float* bnd, cudaStream_t s) {
+                                  const float* bnd, cudaStream_t s, bool* ring_written) {
   QParams p{};
   p.K = src.K;
   p.V = src.V;
@@ -2104,7 +2147,9 @@ cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* b
   p.base = base;
   p.g = g;
   p.hadamard = g.hadamard;
-  return run_quantize(p, g.B * g.Hkv, s);
+  const cudaError_t e = run_quantize(p, g.B * g.Hkv, s);
+  if (ring_written) *ring_written = e == cudaSuccess && p.fuse_ring;
+  return e;
 }
 
 cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,

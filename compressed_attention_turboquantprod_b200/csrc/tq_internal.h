@@ -73,9 +73,11 @@ cudaError_t launch_quantize_arrays(const QuantSrc& src, int dtype, int d, int b1
                                    int vbits, int group, bool do_keys, bool do_values,
                                    const float* Pi, const float* T, const float* cent,
                                    const float* bnd, const QuantDst& dst, cudaStream_t s);
+// *ring_written (may be null): the launch also wrote the new ring (then no ring
+// write may follow it)
 cudaError_t launch_quantize_cache(const QuantSrc& src, const Geom& g, uint8_t* base,
                                   const float* Pi, const float* T, const float* cent,
-                                  const float* bnd, cudaStream_t s);
+                                  const float* bnd, cudaStream_t s, bool* ring_written);
 cudaError_t launch_ring_write(const Geom& g, uint8_t* base, const void* K, const void* V,
                               int64_t n_old, int64_t n_new, cudaStream_t s);
 // Decode step (tq_decode_step): quantise of the tokens leaving the ring with the

@@ -156,6 +156,11 @@ int tq_make_projections_hadamard(int d, int m, int layer, uint64_t base_seed, ui
  *   signs       device uint8[n * m/8], bit i at byte i>>3, bit i&7
  *   norm_x      device float[n] (rho)
  *   norm_r      device float[n] (||r||; NULL if b1 == 0)
+ * More than 8 keys at head dim 128 or 256 with m a multiple of 32 up to 512 run
+ * on the tensor cores (the rotation and sketch products as f16 hi + lo splits,
+ * fp32 accumulation); other shapes on a CUDA-core fp32 tile kernel.  Outside
+ * d = m = 128 the call takes a per-call operand scratch of 4 d (d [b1 > 0] + m)
+ * bytes from a library-owned stream-ordered pool on the current device.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
  */
 int tq_quantize_keys(const void* K, int dtype, int64_t n, int d, int b1, int m,
@@ -256,7 +261,10 @@ int64_t tq_cache_ring_tokens(const tq_cache* c);
  * into a flat cache; recent tokens kept at full precision in a ring).  Tokens
  * leaving the ring and tokens of the chunk older than the last W are quantised
  * (keys as tq_quantize_keys, values as tq_quantize_values) straight into the
- * packed blocks; the last W go to the ring.  Two kernels, in stream order.
+ * packed blocks; the last W go to the ring.  Two kernels, in stream order; one
+ * at d = m = 128 with b1 >= 1 when the chunk has more than 8 tokens per (b, kv
+ * head) and at least W, which writes the ring itself and may start while the
+ * previous append's kernel finishes (consecutive chunks overlap).
  *   K, V     device [B, Hkv, n_new, d] of desc.dtype, contiguous
  *   Pi, T, centroids, boundaries  as for tq_quantize_keys
  * Errors: INVALID_ARG, CAPACITY (nothing written), CUDA.
@@ -427,10 +435,10 @@ int tq_merge_partials(const float* part_ml, const float* part_o, int64_t rows, i
 /*
  * tq_quantize_check -- SYNCHRONOUS: waits for `stream`, then reports (and
  * clears) the sticky device flag of the batched tensor-core key quantisation
- * (tq_quantize_keys and tq_append with more than 8 tokens, head dim 128,
- * m = 128, b1 >= 1).  That kernel waits, with a bound, for its tensor-core
- * products to complete; if a wait gives up (it never should) it stops and sets
- * the flag instead of hanging.  Returns TQ_ERR_CUDA when the flag was set,
+ * (tq_quantize_keys and tq_append with more than 8 tokens, head dim 128 or 256,
+ * m a multiple of 32 up to 512).  Those kernels wait, with a bound, for their
+ * operand copies and tensor-core products to complete; if a wait gives up (it
+ * never should) they stop and set the flag instead of hanging.  Returns TQ_ERR_CUDA when the flag was set,
  * TQ_OK otherwise.  The pages have no counterpart: this is a diagnostic of this
  * library.
  */

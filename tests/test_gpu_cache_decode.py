@@ -96,6 +96,38 @@ def test_append_packed_bytes_match_oracle_across_chunks():
         _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
 
 
+def test_append_chunks_that_write_the_ring_in_the_tile_kernel():
+    """Chunks of at least W tokens are quantised by a tile kernel that also writes
+    the new ring and may start before the previous append's kernel has finished:
+    a first chunk into an empty cache, chunks that replace the ring after
+    tile-kernel and ring-kernel appends, a chunk of exactly W, and appends that
+    take the separate ring kernel in between, issued back to back (no
+    synchronisation between appends, so the kernels do overlap); packed bytes
+    (ring included) equal the oracle's at the end."""
+    w = _workload(B=2, Hkv=3, d=128, T=700, W=16, seed=5)
+    cap = 700
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    K, V = synth.keys_values(w, device="cuda")
+    gc = _gpu_cache(w, cap)
+    oc = _oracle_cache(w, cap, po, cb)
+    pj, cbd = _Proj(po), _Cb(cb)
+    chunks, t = [], 0
+    for n in (40, 20, 16, 9, 30, 3, 200, 17, 300, 12):
+        chunks.append((K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()))
+        t += n
+    torch.cuda.synchronize()
+    for k, v in chunks:
+        gc.append(k, v, pj, cbd)
+    torch.cuda.synchronize()
+    for k, v in chunks:
+        oc.append(host(k), host(v))
+    assert gc.n_total == oc.n_total == t
+    skipped = _compare_cache_bytes(gc.buffer.cpu().numpy(), oc)
+    nat().tq_quantize_check()
+    record("appends writing the ring in the tile kernel", tokens=t, skipped_tokens=skipped)
+    assert skipped <= 3
+
+
 def test_append_degenerate_tokens_every_quantise_path():
     """Zero keys, constant value rows (s = 0), exact half-step value ties and zero
     value rows through the tensor-core tile kernel (a 300-token chunk), the
