@@ -911,6 +911,36 @@ def bench_quantize(dev, world, reps=3, keep_sample=False):
                 times.append(e0.elapsed_time(e1))
         return reduce_max(min(times), world)
     ms = timed(pj)
+    region = cache.buffer[:cache.state.region_bytes]
+    ref_sum = int(region.view(torch.int32).sum().item())
+    # the same 32 appends captured once as a CUDA graph and replayed: the device
+    # time without the host's per-call launch work (same kernels, same bytes)
+    graph = {}
+    try:
+        g = torch.cuda.CUDAGraph()
+        cache.state.n_total = 0
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for k, v in chunks:
+                cache.append(k, v, pj, cb)
+        times = []
+        for r in range(reps + 1):
+            region.zero_()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if r > 0:
+                times.append(e0.elapsed_time(e1))
+        gms = reduce_max(min(times), world)
+        graph = {"Mkeys_per_s": reduce_sum(float(w.T * w.Hkv * w.B), world) / (gms * 1e-3) / 1e6,
+                 "ms": gms, "same_bytes_as_the_calls": int(region.view(torch.int32).sum().item()) == ref_sum}
+        del g
+    except Exception as ex:          # a capture the runtime refuses: report, do not fail
+        graph = {"unavailable": str(ex)[:200]}
+    torch.cuda.synchronize()
     # the same append with the structured (Hadamard) rotation
     ms_h = timed(Projections(w.d, w.m, 0, device=dev, structured=True))
     keys = reduce_sum(float(w.T * w.Hkv * w.B), world)
@@ -924,6 +954,7 @@ def bench_quantize(dev, world, reps=3, keep_sample=False):
         sample["region"] = cache.buffer[:cache.state.region_bytes].cpu().numpy()
     nbytes = w.T * w.Hkv * w.B * (2 * w.d * 2 + tb)
     res = {"Mkeys_per_s": keys / (ms * 1e-3) / 1e6, "ms": ms, "keys": int(keys),
+            "graph": graph,
             "Mkeys_per_s_hadamard_rotation": keys / (ms_h * 1e-3) / 1e6,
             "GB_per_s": reduce_sum(float(nbytes), world) / (ms * 1e-3) / 1e9,
             "workload": "quant: 131072 tokens x 8 KV heads, d=128, bf16, appended in chunks of 4096; "
