@@ -32,8 +32,8 @@ def _w(**kw):
 
 CASES = [
     # name, workload, appends (chunk sizes), decode steps, prefill chunk, structured rotation
-    ("tensor_core", _w(), (300, 5), (1, 2), 7, False),
-    ("tensor_core_hadamard", _w(T=140), (120, 3), (1,), 0, True),
+    ("tensor_core", _w(), (300, 5), (1, 2), 12, False),
+    ("tensor_core_hadamard", _w(T=140), (120, 3), (1,), 7, True),
     ("wide", _w(d=256, b1=3, m=256, vbits=4, group=64, T=150), (130, 1), (1,), 3, False),
     ("cuda_core", _w(d=64, Hq=6, Hkv=2, dtype="f32", W=5, T=77, m=64), (70, 2), (1,), 3, False),
     ("pure_qjl", _w(b1=0, m=192, dtype="f16", T=100), (90,), (2,), 0, False),
