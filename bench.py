@@ -878,8 +878,9 @@ def _aqjl_32_layer_step(w, dev, reps=5, warm=2):
 
 
 def bench_other_decodes(dev, world, peak):
-    """The A-QJL (32 layers; one layer per sketch-size group timed, x8) and the
-    wide-head 262K decodes at full size."""
+    """The A-QJL decodes (one layer of each sketch-size group timed alone, then a
+    whole 32-layer token step over all resident layer caches) and the wide-head
+    262K decode, at full size."""
     import synth
     res = {}
     w = synth.WORKLOADS["aqjl"]
