@@ -273,15 +273,35 @@ __global__ void k_decode_combine(Geom g, int splits, void* out, DecodeWs ws) {
   const float* ml = ws.part_ml + (int64_t)bq * splits * 2;
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
+  const float* po = ws.part_o + (int64_t)bq * splits * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float o = 0.f, L = 0.f;
     if (M != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float ms = ml[2 * s];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
+      // the same sums in the same order; four splits' values are loaded before
+      // any is used, so that their loads are in flight together
+      int s = 0;
+      for (; s + 4 <= splits; s += 4) {
+        float v[4], ms[4], ls[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          ms[u] = ml[2 * (s + u)];
+          ls[u] = ml[2 * (s + u) + 1];
+          v[u] = po[(int64_t)(s + u) * d + c];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (ms[u] != -INFINITY) {
+            const float w = exp2f(ms[u] - M);
+            L = fmaf(ls[u], w, L);
+            o = fmaf(v[u], w, o);
+          }
+      }
+      for (; s < splits; ++s) {
+        const float m1 = ml[2 * s];
+        if (m1 == -INFINITY) continue;
+        const float w = exp2f(m1 - M);
         L = fmaf(ml[2 * s + 1], w, L);
-        o = fmaf(ws.part_o[((int64_t)bq * splits + s) * d + c], w, o);
+        o = fmaf(po[(int64_t)s * d + c], w, o);
       }
       o = o / L;
     }

@@ -551,6 +551,11 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // the split weights go to the (free again) s_out area when they fit there
+  if (MG * p.splits <= 4 * MG * MD) {
+    merge_splits<MD, MT>(p, bq0, s_out);
+    return;
+  }
   for (int i = tid; i < MG * MD; i += MT) {
     const int hh = i / MD, ch = i % MD;
     const int bq = bq0 + hh;

@@ -505,6 +505,11 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // the split weights go to the (free again) s_out area when they fit there
+  if (MG * p.splits <= 2 * MG * WD) {
+    merge_splits<WD, WT>(p, bq0, s_out);
+    return;
+  }
   for (int i = tid; i < MG * WD; i += WT) {
     const int hh = i / WD, ch = i % WD;
     const int bq = bq0 + hh;

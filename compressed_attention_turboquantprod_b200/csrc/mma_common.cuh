@@ -174,6 +174,77 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// The output of a unit from its splits' (m, l, o), run by the CTA of the split that
+// finishes last (NT = 32 MG threads).  Warp hh turns the (m, l) of head hh in every
+// split into the weights exp2(m_s - M) / L, kept in s_wgt[MG][splits] (shared
+// memory of at least MG * splits floats); then thread t sums the channels
+// t + NT c of all MG heads as sum_s w_s o_s, loading the values of several splits
+// before using any, so that 16 loads are in flight per round trip to L2.
+template <int D, int NT>
+__device__ __forceinline__ void merge_splits(const MParams& p, int bq0, float* s_wgt) {
+  static_assert(NT == 32 * MG && D % NT == 0, "one warp per head, whole channels per thread");
+  constexpr int CPT = D / NT;                 // channels per thread
+  constexpr int U = 4 / CPT;                  // splits per round
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = p.splits;
+  {
+    const volatile float* ml = p.ws.part_ml + (int64_t)(bq0 + warp) * S * 2;
+    float M = -INFINITY;
+    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, ml[2 * sp]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int sp = lane; sp < S; sp += 32) {
+      const float ms = ml[2 * sp];
+      if (ms != -INFINITY) L = fmaf(ml[2 * sp + 1], exp2f(ms - M), L);
+    }
+    L = warp_sum(L);
+    for (int sp = lane; sp < S; sp += 32) {
+      const float ms = ml[2 * sp];
+      s_wgt[warp * S + sp] = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M) / L;
+    }
+  }
+  __syncthreads();
+  const float* po = p.ws.part_o + (int64_t)bq0 * S * D + tid;
+  const int64_t hs = (int64_t)S * D;          // stride between heads
+  float o[MG][CPT];
+#pragma unroll
+  for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) o[hh][c] = 0.f;
+  int sp = 0;
+  for (; sp + U <= S; sp += U) {
+    float v[U][MG][CPT];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) v[u][hh][c] = __ldcg(po + hh * hs + (int64_t)(sp + u) * D + c * NT);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) o[hh][c] = fmaf(v[u][hh][c], s_wgt[hh * S + sp + u], o[hh][c]);
+  }
+  for (; sp < S; ++sp)
+#pragma unroll
+    for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+      for (int c = 0; c < CPT; ++c)
+        o[hh][c] = fmaf(__ldcg(po + hh * hs + (int64_t)sp * D + c * NT), s_wgt[hh * S + sp], o[hh][c]);
+  const int es = p.g.dtype == TQ_F32 ? 4 : 2;
+  const int64_t rows = (int64_t)p.g.B * p.Hq;
+#pragma unroll
+  for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      const int64_t e = (int64_t)(bq0 + hh) * D + tid + c * NT;
+      if (TQ_CHECKED(static_cast<const char*>(p.out) + e * es, es, p.out, rows * D * es, 117))
+        store_f(p.out, e, p.g.dtype, o[hh][c]);
+    }
+}
+
 // s0 + 2^8 s1 + 2^16 s2 + 2^24 s3 for the four slice sums of a score (each below
 // 2^23 in magnitude): the pairs are joined exactly in 32-bit integers (< 2^31),
 // then converted once each; the result carries fp32 rounding only.

@@ -932,6 +932,15 @@ __device__ __forceinline__ void tc_ld_sum32(uint32_t taddr, uint32_t (&acc)[32])
   }
 }
 
+// (b, kv head) and first row of tile t of a call: 32-bit division (the host sends a
+// call to the tile kernels only when its tiles number below 2^31).
+__device__ __forceinline__ int tile_bh(int64_t t, int64_t tiles_per_bh, int64_t& row0) {
+  const uint32_t tt = (uint32_t)t, tp = (uint32_t)tiles_per_bh;
+  const uint32_t q = tt / tp;
+  row0 = (int64_t)(tt - q * tp) * TCM;
+  return (int)q;
+}
+
 template <int B1, bool F32>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_t tiles_per_bh,
                                                               int64_t total_tiles) {
@@ -990,8 +999,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     const void* vs = nullptr;
     int64_t ek = 0, ev = 0;
     if (t < total_tiles) {
-      const int tbh = (int)(t / tiles_per_bh);
-      const int64_t tr0 = (t % tiles_per_bh) * TCM;
+      int64_t tr0;
+      const int tbh = tile_bh(t, tiles_per_bh, tr0);
       if (p.cache_mode && p.t_first + tr0 < p.n_old) pdl_wait();     // uniform per tile
       const int64_t trow_i = tr0 + r;
       ok_row = trow_i < p.n;
@@ -1051,8 +1060,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
   uint32_t it = 0;
   const int64_t tiles_here = *reinterpret_cast<volatile int*>(&s_abort) ? 0 : total_tiles;
   for (int64_t tile = blockIdx.x; tile < tiles_here; tile += gridDim.x, ++it) {
-    const int bh = (int)(tile / tiles_per_bh);
-    const int64_t row0 = (tile % tiles_per_bh) * TCM;
+    int64_t row0;
+    const int bh = tile_bh(tile, tiles_per_bh, row0);
     const uint32_t ph = it & 1u;
     const int64_t grow = row0 + r;
     const bool valid = grow < p.n;
@@ -1060,8 +1069,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       // the rows of the tile after next towards L2
       const int64_t nt = tile + 2 * (int64_t)gridDim.x;
       if (nt < tiles_here) {
-        const int nbh = (int)(nt / tiles_per_bh);
-        const int64_t nrow = (nt % tiles_per_bh) * TCM + r;
+        int64_t nrow;
+        const int nbh = tile_bh(nt, tiles_per_bh, nrow);
+        nrow += r;
         if (nrow < p.n) {
           int64_t e0;
           const void* src = src_row(p, false, nbh, nrow, e0);
@@ -1602,9 +1612,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
     // one tile ahead at D = 128; requests towards L2 at D = 256)
     RawSeg<F32> xr[NW], vr[NW];
     auto row_src = [&](int64_t t, bool values, int64_t& e) -> const void* {
-      const int tbh = (int)(t / tiles_per_bh);
-      const int64_t ti = (t % tiles_per_bh) * TCM + r;
-      if (t >= total_tiles || ti >= p.n || (values && !p.do_values)) return nullptr;
+      if (t >= total_tiles) return nullptr;
+      int64_t ti;
+      const int tbh = tile_bh(t, tiles_per_bh, ti);
+      ti += r;
+      if (ti >= p.n || (values && !p.do_values)) return nullptr;
       return src_row(p, values, tbh, ti, e);
     };
     auto request = [&](int64_t t) {
@@ -1623,8 +1635,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_quantize_tcg(QParams p, const
     request(blockIdx.x);
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const int bh = (int)(tile / tiles_per_bh);
-      const int64_t grow = (tile % tiles_per_bh) * TCM + r;
+      int64_t grow;
+      const int bh = tile_bh(tile, tiles_per_bh, grow);
+      grow += r;
       const bool valid = grow < p.n;
       const uint32_t ph = (uint32_t)(it & 1);
       {
@@ -2000,7 +2013,9 @@ static cudaError_t image_pool(cudaMemPool_t* out) {
 
 static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
-  if (p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0 && p.b1 <= 3) {
+  // the tile kernels index a call's tiles in 32 bits
+  const bool tiles32 = (p.n + TCM - 1) / TCM * bh_count < (int64_t)1 << 31;
+  if (tiles32 && p.n > 8 && p.do_keys && p.d == QD && p.m == QM && p.b1 > 0 && p.b1 <= 3) {
     // fifth-generation tensor cores: one persistent CTA per SM over 128-token tiles
     const int64_t tiles_per_bh = (p.n + TCM - 1) / TCM;
     const int64_t total = tiles_per_bh * bh_count;
@@ -2022,7 +2037,7 @@ static cudaError_t run_quantize(QParams& p, int bh_count, cudaStream_t s) {
     kern<<<(unsigned)grid, TC_THREADS, smem, s>>>(p, tiles_per_bh, total);
     return cudaGetLastError();
   }
-  if (p.n > 8 && p.do_keys && (p.d == 128 || p.d == 256) && p.m % 32 == 0 && p.m <= 512 &&
+  if (tiles32 && p.n > 8 && p.do_keys && (p.d == 128 || p.d == 256) && p.m % 32 == 0 && p.m <= 512 &&
       p.b1 >= 0 && p.b1 <= 3) {
     // the same on streamed operand pieces: Pi and T written once into a scratch image
     const int64_t tiles_per_bh = (p.n + TCM - 1) / TCM;
