@@ -3,6 +3,7 @@
 // nothing and writes nothing.
 #include <cctype>
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -527,10 +528,14 @@ static int decode_plan(const tq_cache* c, const void* Q, int Hq, float softmax_s
   return TQ_OK;
 }
 
+// early_blk: packed blocks [0, early_blk) of every unit that the kernel launched just
+// before the partial kernel does not write (the partial may request them before it
+// waits for that kernel); the preparation launched here writes none of them.
 static int decode_launch(const tq_cache* c, const DecodePlan& P, const void* Q, int Hq,
                          float softmax_scale, const float* Pi, const float* S,
                          const float* centroids, void* out, float* logits, cudaStream_t s,
-                         bool prep, bool partial, bool combine, const char* name) {
+                         bool prep, bool partial, bool combine, const char* name,
+                         int64_t early_blk = 0) {
   cudaError_t e = cudaSuccess;
   if (prep) {
     e = P.mma ? tq::launch_decode_prep_mma(P.g, Q, Hq, Pi, S, centroids, softmax_scale, P.ws, s)
@@ -541,7 +546,8 @@ static int decode_launch(const tq_cache* c, const DecodePlan& P, const void* Q, 
     // the tensor-core partial kernel merges the splits itself when given `out`
     void* fused_out = (P.mma && combine) ? out : nullptr;
     e = P.mma ? tq::launch_decode_partial_mma(P.g, static_cast<const uint8_t*>(c->base), c->n_total,
-                                              Hq, softmax_scale, logits, P.splits, P.ws, fused_out, s)
+                                              Hq, softmax_scale, logits, P.splits, P.ws, fused_out,
+                                              prep ? INT64_MAX : early_blk, s)
               : tq::launch_decode_partial(P.g, static_cast<const uint8_t*>(c->base), c->n_total, Hq,
                                           softmax_scale, centroids, logits, P.splits, P.ws, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
@@ -614,8 +620,9 @@ int tq_decode_step(tq_cache* c, const void* K, const void* V, int64_t n_new, con
                                              centroids, boundaries, Q, Hq, S, softmax_scale, P.ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step: quantise + prepare");
   c->n_total = n_tot;
+  // the fused quantise writes the packed blocks from the one holding token c_old on
   return decode_launch(c, P, Q, Hq, softmax_scale, Pi, S, centroids, out, logits, s, false, true,
-                       true, "tq_decode_step");
+                       true, "tq_decode_step", c_old / tq::kBlockTokens);
 }
 
 int tq_decode_prep(const tq_cache* c, const void* Q, int Hq, float softmax_scale,

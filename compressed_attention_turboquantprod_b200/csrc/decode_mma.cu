@@ -113,8 +113,18 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
     mbar_init(&ringbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // Launched programmatically after the preparation kernel: nothing that kernel or
-  // an earlier one writes is touched before this wait.
+  // Launched programmatically after the preparation kernel (or the fused quantise
+  // and preparation of a decode step): of what that grid may write, only the packed
+  // blocks below p.early_blk are touched before the wait for it, where they fill
+  // the first stages while it runs.
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) s_iss[s] = 0;
+    for (int s = 0; s < NST && s < nb && blk0 + s < p.early_blk; ++s) {
+      mbar_expect_tx(&full[s], (uint32_t)bb);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 107);
+      s_iss[s] = 1;
+    }
+  }
   pdl_wait();
   if (tid == 0) {
     if (ring_split) {
@@ -123,8 +133,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       cache_bulk_load(s_rk, ring_k, nbytes, &ringbar, p.base, g.total_bytes, 101);
       cache_bulk_load(s_rv, ring_v, nbytes, &ringbar, p.base, g.total_bytes, 102);
     }
-    for (int s = 0; s < NST; ++s) s_iss[s] = 0;
     for (int s = 0; s < NST && s < nb; ++s) {
+      if (s_iss[s]) continue;
       mbar_expect_tx(&full[s], (uint32_t)bb);
       cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 103);
       s_iss[s] = 1;
@@ -551,9 +561,8 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // the split weights go to the (free again) s_out area when they fit there
-  if (MG * p.splits <= 4 * MG * MD) {
-    merge_splits<MD, MT>(p, bq0, s_out);
+  if (p.splits <= 32) {
+    merge_splits<MD, MT>(p, bq0);
     return;
   }
   for (int i = tid; i < MG * MD; i += MT) {
@@ -612,9 +621,10 @@ cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const f
 
 cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
                                       float scale, float* logits, int splits, const DecodeWs& ws,
-                                      void* out, cudaStream_t s) {
+                                      void* out, int64_t early_blk, cudaStream_t s) {
   MParams p{};
   p.out = out;
+  p.early_blk = early_blk;
   p.g = g;
   p.base = base;
   p.n_total = n_total;

@@ -95,8 +95,17 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
     mbar_init(&ringbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // launched programmatically after the preparation kernel: nothing that kernel or
-  // an earlier one writes is touched before this wait
+  // launched programmatically after the preparation kernel (or the fused quantise
+  // and preparation of a decode step): of what that grid may write, only the packed
+  // blocks below p.early_blk are touched before the wait for it
+  if (tid == 0) {
+    for (int s = 0; s < WNST; ++s) s_iss[s] = 0;
+    for (int s = 0; s < WNST && s < nb && blk0 + s < p.early_blk; ++s) {
+      mbar_expect_tx(&full[s], (uint32_t)bb);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 205);
+      s_iss[s] = 1;
+    }
+  }
   pdl_wait();
   if (tid == 0) {
     if (ring_split) {
@@ -105,8 +114,8 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
       cache_bulk_load(s_rk, ring_k, nbytes, &ringbar, p.base, g.total_bytes, 202);
       cache_bulk_load(s_rv, ring_v, nbytes, &ringbar, p.base, g.total_bytes, 203);
     }
-    for (int s = 0; s < WNST; ++s) s_iss[s] = 0;
     for (int s = 0; s < WNST && s < nb; ++s) {
+      if (s_iss[s]) continue;
       mbar_expect_tx(&full[s], (uint32_t)bb);
       cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 204);
       s_iss[s] = 1;
@@ -505,9 +514,8 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // the split weights go to the (free again) s_out area when they fit there
-  if (MG * p.splits <= 2 * MG * WD) {
-    merge_splits<WD, WT>(p, bq0, s_out);
+  if (p.splits <= 32) {
+    merge_splits<WD, WT>(p, bq0);
     return;
   }
   for (int i = tid; i < MG * WD; i += WT) {

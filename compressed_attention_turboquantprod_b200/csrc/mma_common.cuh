@@ -23,6 +23,9 @@ struct MParams {
   DecodeWs ws;
   int* err;
   void* out;        // when non-null, the last split of a unit also writes the output
+  int64_t early_blk;  // packed blocks [0, early_blk) of every unit are not written by the
+                      // grid this kernel is launched programmatically after: their stages
+                      // may be requested before the wait for that grid
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -175,64 +178,63 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // The output of a unit from its splits' (m, l, o), run by the CTA of the split that
-// finishes last (NT = 32 MG threads).  Warp hh turns the (m, l) of head hh in every
-// split into the weights exp2(m_s - M) / L, kept in s_wgt[MG][splits] (shared
-// memory of at least MG * splits floats); then thread t sums the channels
-// t + NT c of all MG heads as sum_s w_s o_s, loading the values of several splits
-// before using any, so that 16 loads are in flight per round trip to L2.
+// finishes last (NT = 32 MG threads, at most 32 splits: a lane per split).  Every
+// warp reads the (m, l) of all MG heads, lane s those of split s, and turns them
+// into the weights exp2(m_s - M) / L with warp reductions (no shared memory, no
+// barrier); thread t sums the channels t + NT c of all heads as sum_s w_s o_s.
+// The values of the first eight splits are requested together with (m, l), the
+// rest eight splits at a time, so that the merge takes few round trips to L2.
 template <int D, int NT>
-__device__ __forceinline__ void merge_splits(const MParams& p, int bq0, float* s_wgt) {
+__device__ __forceinline__ void merge_splits(const MParams& p, int bq0) {
   static_assert(NT == 32 * MG && D % NT == 0, "one warp per head, whole channels per thread");
   constexpr int CPT = D / NT;                 // channels per thread
-  constexpr int U = 4 / CPT;                  // splits per round
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int U = 8;                        // splits per round
+  const int tid = threadIdx.x, lane = tid & 31;
   const int S = p.splits;
-  {
-    const volatile float* ml = p.ws.part_ml + (int64_t)(bq0 + warp) * S * 2;
-    float M = -INFINITY;
-    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, ml[2 * sp]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int sp = lane; sp < S; sp += 32) {
-      const float ms = ml[2 * sp];
-      if (ms != -INFINITY) L = fmaf(ml[2 * sp + 1], exp2f(ms - M), L);
-    }
-    L = warp_sum(L);
-    for (int sp = lane; sp < S; sp += 32) {
-      const float ms = ml[2 * sp];
-      s_wgt[warp * S + sp] = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M) / L;
-    }
-  }
-  __syncthreads();
   const float* po = p.ws.part_o + (int64_t)bq0 * S * D + tid;
   const int64_t hs = (int64_t)S * D;          // stride between heads
+  float v[U][MG][CPT];
+  auto request = [&](int sp0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int hh = 0; hh < MG; ++hh)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c)
+          v[u][hh][c] = sp0 + u < S ? __ldcg(po + hh * hs + (int64_t)(sp0 + u) * D + c * NT) : 0.f;
+  };
+  request(0);
+  float w[MG];                                // lane s: the weight of split s, per head
+#pragma unroll
+  for (int hh = 0; hh < MG; ++hh) {
+    float ms = -INFINITY, ls = 0.f;
+    if (lane < S) {
+      const float* ml = p.ws.part_ml + ((int64_t)(bq0 + hh) * S + lane) * 2;
+      ms = __ldcg(ml);
+      ls = __ldcg(ml + 1);
+    }
+    const float M = warp_max(ms);
+    const float e = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    const float L = warp_sum(ls * e);
+    w[hh] = e == 0.f ? 0.f : e / L;
+  }
   float o[MG][CPT];
 #pragma unroll
   for (int hh = 0; hh < MG; ++hh)
 #pragma unroll
     for (int c = 0; c < CPT; ++c) o[hh][c] = 0.f;
-  int sp = 0;
-  for (; sp + U <= S; sp += U) {
-    float v[U][MG][CPT];
+  for (int sp0 = 0; sp0 < S; sp0 += U) {
+    if (sp0 > 0) request(sp0);
 #pragma unroll
     for (int u = 0; u < U; ++u)
+      if (sp0 + u < S)
 #pragma unroll
-      for (int hh = 0; hh < MG; ++hh)
+        for (int hh = 0; hh < MG; ++hh) {
+          const float wt = __shfl_sync(0xffffffffu, w[hh], sp0 + u);
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) v[u][hh][c] = __ldcg(po + hh * hs + (int64_t)(sp + u) * D + c * NT);
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int hh = 0; hh < MG; ++hh)
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) o[hh][c] = fmaf(v[u][hh][c], s_wgt[hh * S + sp + u], o[hh][c]);
+          for (int c = 0; c < CPT; ++c) o[hh][c] = fmaf(v[u][hh][c], wt, o[hh][c]);
+        }
   }
-  for (; sp < S; ++sp)
-#pragma unroll
-    for (int hh = 0; hh < MG; ++hh)
-#pragma unroll
-      for (int c = 0; c < CPT; ++c)
-        o[hh][c] = fmaf(__ldcg(po + hh * hs + (int64_t)sp * D + c * NT), s_wgt[hh * S + sp], o[hh][c]);
   const int es = p.g.dtype == TQ_F32 ? 4 : 2;
   const int64_t rows = (int64_t)p.g.B * p.Hq;
 #pragma unroll

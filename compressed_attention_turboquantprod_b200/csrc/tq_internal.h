@@ -117,9 +117,11 @@ int decode_mma_ctas_per_sm(const Geom& g);      // resident CTAs per SM of the p
 cudaError_t launch_decode_prep_mma(const Geom& g, const void* Q, int Hq, const float* Pi,
                                    const float* S, const float* cent, float scale,
                                    const DecodeWs& ws, cudaStream_t s);
+// early_blk: packed blocks [0, early_blk) of every unit are not written by the kernel
+// launched just before on the stream (0 when that is not known)
 cudaError_t launch_decode_partial_mma(const Geom& g, const uint8_t* base, int64_t n_total, int Hq,
                                       float scale, float* logits, int splits, const DecodeWs& ws,
-                                      void* out, cudaStream_t s);
+                                      void* out, int64_t early_blk, cudaStream_t s);
 
 cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float* Pi,
                                const float* S, const DecodeWs& ws, cudaStream_t s);
