@@ -162,7 +162,7 @@ int eff_splits(const tq::Geom& g, int G, int64_t n_comp, int num_splits) {
 int max_splits(const tq_cache* c, int Hq, int num_splits) {
   if (num_splits > 0) return num_splits;
   tq::Geom g = tq::geom_of(c);
-  return tq::decode_auto_splits(g, Hq / c->desc.Hkv, c->desc.capacity);
+  return tq::decode_max_auto_splits(g, Hq / c->desc.Hkv, c->desc.capacity);
 }
 
 int check_decode_common(const tq_cache* c, int Hq, int num_splits) {

@@ -364,19 +364,40 @@ DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits) {
   return w;
 }
 
+// The tensor-core kernel's CTAs of a unit split its blocks evenly; the SM that ends
+// last carries about ceil(units s / 148) CTAs of ceil(nblk / s) blocks (CTAs that
+// finish early are backfilled by waiting ones), the per-SM load this returns.
+static int64_t sm_load(int64_t units, int64_t s, int64_t nblk) {
+  return ((units * s + 147) / 148) * ((nblk + s - 1) / s);
+}
+
 int decode_auto_splits(const Geom& g, int G, int64_t n_comp) {
   const int64_t nblk = (n_comp + kBlockTokens - 1) / kBlockTokens;
   const int units = g.B * g.Hkv;
   int64_t s;
   if (decode_mma_supported(g, G)) {
-    // one wave of the tensor-core kernel (148 SMs x its resident CTAs), never more
-    s = (int64_t)(148 * decode_mma_ctas_per_sm(g)) / units;
+    // one wave of the kernel (148 SMs x its resident CTAs); twice that many smaller
+    // CTAs when the wave leaves the SMs' loads uneven (e.g. 128 units x 4 splits in
+    // 592 slots: 4 CTAs on some SMs, 3 on others) and the halves balance them at
+    // least 5 % better
+    const int64_t s1 = (int64_t)(148 * decode_mma_ctas_per_sm(g)) / units;
+    s = s1;
+    if (s1 >= 1 && 2 * s1 <= nblk && sm_load(units, 2 * s1, nblk) * 20 < sm_load(units, s1, nblk) * 19)
+      s = 2 * s1;
   } else {
     s = (kTargetCtas + units - 1) / units;
   }
   if (s > nblk) s = nblk;
   if (s < 1) s = 1;
   return (int)s;
+}
+
+int decode_max_auto_splits(const Geom& g, int G, int64_t capacity) {
+  if (!decode_mma_supported(g, G)) return decode_auto_splits(g, G, capacity);   // grows with n
+  const int64_t nblk = (capacity + kBlockTokens - 1) / kBlockTokens;
+  int64_t s = 2 * ((int64_t)(148 * decode_mma_ctas_per_sm(g)) / (g.B * g.Hkv));
+  if (s > nblk) s = nblk;
+  return s < 1 ? 1 : (int)s;
 }
 
 cudaError_t launch_decode_prep(const Geom& g, const void* Q, int Hq, const float* Pi,

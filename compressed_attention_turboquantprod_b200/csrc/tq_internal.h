@@ -110,6 +110,8 @@ size_t decode_ws_bytes_now(const tq_cache* c, int Hq, int num_splits);
 int noalloc_scratch(void** out);
 DecodeWs decode_ws_carve(void* base, const Geom& g, int Hq, int splits);
 int decode_auto_splits(const Geom& g, int G, int64_t n_comp);
+// The largest decode_auto_splits(g, G, n) for n <= capacity (workspace sizing).
+int decode_max_auto_splits(const Geom& g, int G, int64_t capacity);
 
 // tensor-core path (decode_mma.cu)
 bool decode_mma_supported(const Geom& g, int G);
