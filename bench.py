@@ -503,7 +503,7 @@ def run_ours(args):
     part_avg_ms = sum(t_part) / len(t_part)
     part_bytes = sum(part_bytes_list) / len(part_bytes_list)
     peak, peak_kind = measured_peak()
-    src_hash = source_hash("decode_mma.cu")
+    src_hash = source_hash("decode_mma.cu", "mma_common.cuh")
     traffic = profiled_traffic("decode_partial_gqa32k.json", src_hash)
     achieved = part_bytes / (part_avg_ms * 1e-3) / 1e9
 
