@@ -146,6 +146,33 @@ def test_decode_checks(nat):
         assert L.tq_decode_workspace_bytes(ctypes.byref(c), 8, 0) == need
 
 
+def test_auto_splits_balance_the_sms(nat):
+    """The tensor-core decode takes one wave of CTAs (148 SMs x 4 at head dim 128,
+    x 2 at 256) when that loads the SMs evenly, and twice the splits when the wave
+    leaves some SMs a whole CTA ahead: the most loaded SM carries about
+    ceil(units s / 148) CTAs of ceil(blocks / s) blocks."""
+    L = nat.lib
+    cases = [
+        # 64 units x 9 = 576 CTAs: 4 x 57 blocks; 18 splits give 8 x 29, no better
+        (dict(B=8, Hkv=8, capacity=32768), 32, 9),
+        # 128 units x 4 = 512 CTAs in 592 slots: 4 x 256 blocks; 8 splits: 7 x 128
+        (dict(B=16, Hkv=8, b1=0, m=512, dtype=1, capacity=65536), 32, 8),
+        # 16 units x 18 = 288 CTAs: 2 x 228 blocks; 36 splits give 4 x 114, no better
+        (dict(B=4, Hkv=4, d=256, b1=3, m=256, vbits=4, group=64, capacity=262144), 16, 18),
+    ]
+    for geo, Hq, want in cases:
+        c = _fake_cache(nat, **geo)
+        need = L.tq_decode_workspace_bytes(ctypes.byref(c), Hq, 0)
+        c.n_total = geo["capacity"]
+        assert L.tq_decode_auto_splits(ctypes.byref(c), Hq) == want
+        # the workspace sized for the capacity covers every length's automatic count
+        for n in (0, 17, 4096, geo["capacity"] // 2, geo["capacity"]):
+            c.n_total = n
+            s = L.tq_decode_auto_splits(ctypes.byref(c), Hq)
+            assert 1 <= s <= 2 * want
+            assert L.tq_decode_workspace_bytes(ctypes.byref(c), Hq, s) <= need
+
+
 def test_fault_injection_is_host_side_and_one_shot(nat):
     c = _fake_cache(nat)
     nat.tq_debug_fail_next("tq_append")
