@@ -79,6 +79,43 @@ def _workload(**kw):
     return synth.Workload(**base)
 
 
+@pytest.mark.parametrize("n0", [100, 150, 220])
+def test_decode_step_single_split_early_stages(n0):
+    """One split per unit: the partial kernel requests the packed blocks below the one
+    that receives the token leaving the ring before it waits for the fused quantise,
+    and the others after.  n0 = 100 / 150 / 220 puts that boundary after the first /
+    second / third of its four stages."""
+    from compressed_attention_turboquantprod_b200 import CompressedKVCache
+    w = _workload()
+    steps = [1, 1, 2]
+    total = n0 + sum(steps)
+    po, cb = oracle_setup(w.d, w.b1, w.m)
+    pj, cbd = _Proj(po), _Cb(cb)
+    K, V = synth.keys_values(w, device="cuda", T=total)
+    caches = [CompressedKVCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
+                                dtype=TORCH_DT[w.dtype]) for _ in range(2)]
+    oc = ocache.OracleCache(w.B, w.Hkv, w.d, w.b1, w.m, w.vbits, w.group, w.W, total + 64,
+                            w.dtype, po, cb)
+    for c in caches:
+        c.append(K[:, :, :n0].contiguous(), V[:, :, :n0].contiguous(), pj, cbd)
+    oc.append(host(K[:, :, :n0]), host(V[:, :, :n0]))
+    t, checked = n0, 0
+    for i, n in enumerate(steps):
+        k, v = K[:, :, t:t + n].contiguous(), V[:, :, t:t + n].contiguous()
+        Q = synth.queries(w.scaled(seed=70 + i), device="cuda")
+        o1, l1 = caches[0].decode_step(k, v, Q, pj, cbd, want_logits=True, num_splits=1)
+        caches[1].append(k, v, pj, cbd)
+        o2, l2 = caches[1].decode(Q, pj, cbd, want_logits=True, num_splits=1)
+        oc.append(host(k), host(v))
+        torch.cuda.synchronize()
+        t += n
+        assert torch.equal(caches[0].buffer, caches[1].buffer), f"cache bytes differ after step {i}"
+        assert torch.equal(o1, o2), f"outputs differ after step {i}"
+        assert torch.equal(l1, l2), f"logits differ after step {i}"
+        checked += _check_against_oracle(caches[0], oc, o1, l1, Q, w, f"single-split step {i}")
+    assert checked >= 1
+
+
 @pytest.mark.parametrize("kw,n0,steps", [
     (dict(), 300, [1, 1, 1, 1, 1]),                                     # full ring, one token a step
     (dict(), 5, [3, 8, 8, 1]),                                          # ring filling up
