@@ -79,6 +79,7 @@ __device__ __forceinline__ float moments_shift(const void* K, int dtype, int64_t
 __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int dtype, int64_t n,
                                                             double* part) {
   __shared__ float s_c;
+  pdl_launch_dependents();      // the merge kernel may launch; it waits for this grid
   if (threadIdx.x < 32) {
     const float c = moments_shift(K, dtype, n, threadIdx.x);
     if (threadIdx.x == 0) s_c = c;
@@ -130,10 +131,13 @@ __global__ void __launch_bounds__(kMomThreads) k_key_moments(const void* K, int 
 }
 
 // out[0] = mean, out[1] = population variance (>= 0), from the blocks' shifted sums.
+// Launched programmatically after k_key_moments: the shift (from K, which that
+// kernel does not write) is formed before the wait for its partial sums.
 __global__ void k_moments_final(const void* K, int dtype, int64_t n, const double* part, int nb,
                                 double* out) {
   const int lane = threadIdx.x;
   const float c = moments_shift(K, dtype, n, lane);
+  pdl_wait();
   double a = 0.0, b = 0.0;
   for (int i = lane; i < nb; i += 32) {
     a += part[2 * i];
@@ -178,8 +182,8 @@ cudaError_t launch_key_moments(const void* K, int dtype, int64_t n, double* out,
   k_key_moments<<<(unsigned)nb, kMomThreads, 0, s>>>(K, dtype, n, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_moments_final<<<1, 32, 0, s>>>(K, dtype, n, part, (int)nb, out);
-  return cudaGetLastError();
+  return launch_pdl(k_moments_final, dim3(1), dim3(32), 0, s, K, dtype, n,
+                    static_cast<const double*>(part), (int)nb, out);
 }
 
 void sensitivity_segment(const double* var, int L, int k, int* bounds) {
