@@ -277,7 +277,13 @@ int tq_append(tq_cache* c, const void* K, const void* V, int64_t n_new, const fl
 /* Decode attention                                                          */
 /* ------------------------------------------------------------------------ */
 
-/* Number of split-K partitions tq_decode_attention uses when num_splits == 0. */
+/* Number of split-K partitions tq_decode_attention uses when num_splits == 0: on
+ * the tensor-core paths one wave of CTAs (148 SMs x the CTAs an SM holds) divided
+ * among the (b, kv head) units, or twice that when the wave would leave some SMs
+ * a whole CTA ahead of others (the most loaded SM's share, about
+ * ceil(units s / 148) CTAs of ceil(blocks / s) blocks, at least 5 % smaller);
+ * at most the number of 64-token blocks.  tq_decode_workspace_bytes(c, Hq, 0)
+ * covers the count at every length up to the capacity. */
 int tq_decode_auto_splits(const tq_cache* c, int Hq);
 
 /* Bytes of device workspace for a decode with Hq query heads and num_splits
