@@ -973,11 +973,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
     s_abort = 0;
   }
   __syncthreads();
-  // resident B operands: Pi, then T, brought in fp32 by bulk copies into the (not
-  // yet used) A area at a 528-byte row stride (eight consecutive rows fall in
-  // distinct bank groups), then split there into f16 hi/lo in the operand layout:
-  // row n (output coordinate) over K = 128, a 16-byte chunk (8 consecutive k) per
-  // thread and step, eight consecutive rows per eight threads (conflict-free)
+  // resident B operands: Pi and T, brought in fp32 by bulk copies (Pi at a
+  // 528-byte row stride, so that eight consecutive rows fall in distinct bank
+  // groups), then split into f16 hi/lo in the operand layout: row n (output
+  // coordinate) over K = 128, a 16-byte chunk (8 consecutive k) per thread and
+  // step, eight consecutive rows per eight threads (conflict-free stores)
   const int q = warp & 3, part = warp >> 2;
   const int r = 32 * q + lane;                     // this thread's row of every tile
   const int k0 = 32 * part;                        // and its first coordinate / channel
@@ -1016,19 +1016,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
   if (p.fuse_ring) pdl_launch_dependents();
   request(blockIdx.x);
 
+  // Both matrices in one round of bulk copies: Pi's rows into the (not yet used) A
+  // area at a 528-byte stride, T's rows unpadded into the Pi operand area; T is
+  // split first (into its own operand area), then Pi (into the area T's rows held).
   constexpr int kStage = QD * 4 + 16;
-  for (int mat = 0; mat < 2; ++mat) {
-    if (tid == 0) mmadec::mbar_expect_tx(&s_mbar[2], QD * QD * 4);
-    __syncthreads();
-    if (tid < QD) {                                  // one row copy per thread
-      tc::fence_async_shared();                      // the area's earlier reads come first
-      mmadec::bulk_load(AH + tid * kStage, (mat ? p.T : p.Pi) + tid * QD, QD * 4, &s_mbar[2]);
-    }
-    if (!mbar_wait_sleep(&s_mbar[2], (uint32_t)mat)) s_abort = 1;
+  if (tid == 0) mmadec::mbar_expect_tx(&s_mbar[2], 2 * QD * QD * 4);
+  __syncthreads();
+  if (tid < 2 * QD) {                                // one row copy per thread
+    tc::fence_async_shared();
+    if (tid < QD) mmadec::bulk_load(AH + tid * kStage, p.Pi + tid * QD, QD * 4, &s_mbar[2]);
+    else mmadec::bulk_load(PH + (tid - QD) * (QD * 4), p.T + (tid - QD) * QD, QD * 4, &s_mbar[2]);
+  }
+  if (!mbar_wait_sleep(&s_mbar[2], 0u)) s_abort = 1;
+  for (int mat = 1; mat >= 0; --mat) {
+    // T (unpadded rows): the eight threads of a 16-byte load phase take eight
+    // consecutive k chunks (two-way bank conflicts instead of eight-way); the
+    // stores stay conflict-free (eight consecutive rows)
+    const unsigned char* srcb = mat ? PH : AH;
+    const int stride = mat ? QD * 4 : kStage;
     for (int c = tid; c < QD * (QD / 8); c += TC_THREADS) {
-      const int n = (c & 7) + 8 * (c >> 7), kc = (c >> 3) & 15;
-      const float4 f0 = *reinterpret_cast<const float4*>(AH + n * kStage + 32 * kc);
-      const float4 f1 = *reinterpret_cast<const float4*>(AH + n * kStage + 32 * kc + 16);
+      const int n = (c & 7) + 8 * (c >> 7);
+      const int kc = mat ? (((c >> 3) + (c & 7)) & 15) : ((c >> 3) & 15);
+      const float4 f0 = *reinterpret_cast<const float4*>(srcb + n * stride + 32 * kc);
+      const float4 f1 = *reinterpret_cast<const float4*>(srcb + n * stride + 32 * kc + 16);
       const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
       uint4 hi, lo;
       split8(v, kSplit, hi, lo);
@@ -1344,7 +1354,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_quantize_tc(QParams p, int64_
       if (lane == 0) {
         atomicExch(&g_quant_tc_err, 1);
         (void)mbar_wait(&s_mbar[2], 0u);           // the operand copies, if still in flight
-        (void)mbar_wait(&s_mbar[2], 1u);
         if (issued > 0) {
           (void)mbar_wait(&s_mbar[0], (uint32_t)((issued - 1) & 1));
           (void)mbar_wait(&s_mbar[1], (uint32_t)((issued - 1) & 1));
