@@ -75,7 +75,6 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   __shared__ int s_abort;
   __shared__ float s_m[4][MG], s_l[4][MG];
   __shared__ float s_mn[4][MG][4];
-  __shared__ int s_cnt[NST];
   __shared__ int s_iss[NST];       // copies issued into each stage (for the error-path drain)
   __shared__ __align__(16) uint32_t s_frag[KS * 128];
   __shared__ __align__(8) uint64_t ringbar;
@@ -151,7 +150,6 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
   }
   const float* qc = p.ws.qconst + ((int64_t)unit * MG + tig) * 4;
   const float kM = qc[0], CM = qc[1], kQ = qc[2], CQ = qc[3];
-  if (tid < NST) s_cnt[tid] = 0;
   __syncthreads();
   const uint4* bfr = reinterpret_cast<const uint4*>(s_frag) + lane;
 
@@ -398,25 +396,19 @@ __global__ void __launch_bounds__(MT, 4) k_decode_partial_mma(MParams p) {
       }
     }
     }  // ok
-    // Release the stage: the second warp of the pair to finish it refills it
-    // with block j + NST (same parity, so the same pair consumes it).
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      const int done = atomicAdd(&s_cnt[st], 1);
-      if (done == 1) {
-        __threadfence_block();
-        s_cnt[st] = 0;
-        if (j + NST < nb && !s_abort) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_expect_tx(&full[st], (uint32_t)bb);
-          cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + NST) * bb, (uint32_t)bb,
-                    &full[st], p.base, g.total_bytes, 104);
-          s_iss[st] += 1;
-        }
-      }
+    // Release the stage: the two warps of the pair meet at their named barrier,
+    // which also ORs their view of the abort flag (so that both leave the loop
+    // together and every barrier is met by both); then the pair's first warp
+    // refills the stage with block j + NST (same parity, so the same pair
+    // consumes it).
+    if (pair_release(pair, *((volatile int*)&s_abort) != 0)) break;
+    if ((warp & 1) == 0 && lane == 0 && j + NST < nb) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&full[st], (uint32_t)bb);
+      cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + NST) * bb, (uint32_t)bb,
+                &full[st], p.base, g.total_bytes, 104);
+      s_iss[st] += 1;
     }
-    if (*((volatile int*)&s_abort)) break;
   }
   __syncthreads();
 

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   __shared__ __align__(8) uint64_t full[WNST];
   __shared__ __align__(8) uint64_t ringbar;
   __shared__ int s_abort, s_abort_pair[2][2];       // [pair][buf]
-  __shared__ int s_cnt[WNST], s_iss[WNST];
+  __shared__ int s_iss[WNST];
   __shared__ float s_bmax[2][2][2][MG];              // [pair][buf][half][head]
   __shared__ float s_p[2][2][64][MG];                // [pair][buf][token][head]
   __shared__ float s_m[2][MG], s_l[2][2][MG], s_mn[2][2][MG][4];
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
     for (int s = 0; s < WNST; ++s) s_iss[s] = 0;
     for (int s = 0; s < WNST && s < nb && blk0 + s < p.early_blk; ++s) {
       mbar_expect_tx(&full[s], (uint32_t)bb);
-      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 205);
+      cache_bulk_load(stage + (size_t)s * bb, region + (blk0 + s) * bb, (uint32_t)bb, &full[s], p.base, g.total_bytes, 209);
       s_iss[s] = 1;
     }
   }
@@ -126,7 +126,6 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
   const uint4* fr = reinterpret_cast<const uint4*>(p.ws.frag + (int64_t)unit * ((KSM + KSQ) * 128)) + lane;
   const float* qc = p.ws.qconst + ((int64_t)unit * MG + tig) * 4;
   const float kM = qc[0], CM = qc[1], kQ = qc[2], CQ = qc[3];
-  if (tid < WNST) s_cnt[tid] = 0;
   __syncthreads();
 
   const uint32_t maskA = 0x01010101u << tig, maskB = 0x10101010u << tig;
@@ -363,22 +362,15 @@ __global__ void __launch_bounds__(WT, WCTAS) k_decode_partial_wide(MParams p) {
         }
       }
     }
-    // Release the stage: the second warp of the pair to finish it refills it with
-    // block j + WNST (same parity, so the same pair consumes it).
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      const int done = atomicAdd(&s_cnt[st], 1);
-      if (done == 1) {
-        __threadfence_block();
-        s_cnt[st] = 0;
-        if (j + WNST < nb && !s_abort) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_expect_tx(&full[st], (uint32_t)bb);
-          cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + WNST) * bb, (uint32_t)bb, &full[st], p.base, g.total_bytes, 205);
-          s_iss[st] += 1;
-        }
-      }
+    // Release the stage: once both warps of the pair are past this barrier, the
+    // pair's first warp refills it with block j + WNST (same parity, so the same
+    // pair consumes it).
+    pair_sync(pair);
+    if (pair_ok && half == 0 && lane == 0 && j + WNST < nb && !s_abort) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&full[st], (uint32_t)bb);
+      cache_bulk_load(stage + (size_t)st * bb, region + (blk0 + j + WNST) * bb, (uint32_t)bb, &full[st], p.base, g.total_bytes, 205);
+      s_iss[st] += 1;
     }
     if (!pair_ok) break;       // both warps of the pair read the same flag after the same barrier
   }

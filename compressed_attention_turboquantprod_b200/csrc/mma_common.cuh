@@ -177,6 +177,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// Named barrier of warp pair `pair` (barrier 1 + pair, 64 threads) that returns the
+// OR of `stop` over both warps: the pair's warps take the same decision, so a loop
+// that leaves on it keeps every later barrier of the pair matched.
+__device__ __forceinline__ bool pair_release(int pair, bool stop) {
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred pa, pb;\n setp.ne.u32 pa, %1, 0;\n bar.red.or.pred pb, %2, 64, pa;\n"
+      " selp.u32 %0, 1, 0, pb;\n}\n"
+      : "=r"(any)
+      : "r"((uint32_t)stop), "r"(1 + pair)
+      : "memory");
+  return any != 0;
+}
+
 // The output of a unit from its splits' (m, l, o), run by the CTA of the split that
 // finishes last (NT = 32 MG threads, at most 32 splits: a lane per split).  Every
 // warp reads the (m, l) of all MG heads, lane s those of split s, and turns them
